@@ -1,0 +1,219 @@
+/*
+ * metis_fp8.h — C ABI of the B200 (sm_100a) FP8 "fast-math" linear layer.
+ *
+ * What it computes, from the Metis-1.6 model cards:
+ *  - "Lernex/Metis-1.6-Logos-FP8", section "What --fast-math does": every
+ *    quantized layer's BF16 input is rounded to FP8 per token and multiplied
+ *    with the FP8 weights on FP8 tensor cores (fast-math); by default the FP8
+ *    weights are instead widened to 16 bits and the maths is done in 16-bit
+ *    precision, so only the weights are rounded.
+ *  - same card, section "What is in FP8": E4M3 weights with one scale per
+ *    output channel, activations quantized per token at run time; the routed
+ *    experts are among the FP8 matrices.
+ *  - "Lernex/Metis-1.6-Praxis-NVFP4", section "What --fast-math does": the
+ *    fast maths only changes steps that handle many tokens at once; one
+ *    stream's decode always uses the default maths.
+ *
+ * The cards print no formula. The readings this library implements:
+ *  - per-token scale  s[m] = amax_k |x[m,k]| / 448          (binary32 IEEE)
+ *  - codes            q[m,k] = E4M3_rn_satfinite(x[m,k] * (448 / amax))
+ *                     with 448/amax in binary32, clamped to FLT_MAX, and 0
+ *                     when amax = 0 (then s = 0 and every code is +-0);
+ *  - W8A8             y[m,n] = bf16_rn( s_tok[m] * s_w[n] * sum_k D(q)[m,k] D(w)[n,k] ),
+ *                     FP32 accumulation on the tensor cores;
+ *  - W8A16            y[m,n] = bf16_rn( s_w[n] * sum_k x[m,k] D(w)[n,k] ), FP32 accumulation;
+ *  - routed experts   per routed slot (t, j) with expert e: h = W8A8(x[t], w_up[e]),
+ *                     no activation, h re-quantized per row, o = W8A8(h, w_down[e]),
+ *                     y[t] = bf16_rn( sum_j topk_w[t,j] * o[t,j] ) in FP32, j ascending.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers, owned by the caller. The library
+ *    never allocates, frees or synchronises; it only launches kernels,
+ *    asynchronously, on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *  - BF16 tensors are 16-bit bit patterns (`const void*`), E4M3 tensors bytes.
+ *  - Matrices are row-major. Unless a leading dimension is passed, rows are
+ *    dense (leading dimension = number of columns).
+ *  - Return value: METIS_OK (0) or a negative metis_status. Argument errors are
+ *    detected on the host BEFORE anything is launched and leave all outputs
+ *    untouched; metis_last_error() then returns a message for this thread.
+ *  - Device-side watchdog: every wait inside a kernel is bounded. A wait that
+ *    runs out sets a sticky device error word and the kernel returns early
+ *    with incomplete output; metis_check_device_status() reports it.
+ *  - Results are bitwise reproducible run to run (no floating-point atomics).
+ */
+#ifndef METIS_FP8_H
+#define METIS_FP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define METIS_API __attribute__((visibility("default")))
+#else
+#define METIS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    METIS_OK = 0,
+    METIS_ERR_INVALID_ARG = -1, /* bad pointer, size, alignment or layout */
+    METIS_ERR_UNSUPPORTED = -2, /* valid request this build does not implement */
+    METIS_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed */
+    METIS_ERR_TIMEOUT = -4      /* a device-side bounded wait ran out */
+} metis_status;
+
+/* Opaque CUDA stream (cudaStream_t). */
+typedef void* metis_stream_t;
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+METIS_API int metis_version(void);
+
+/* Message describing the last error returned on the calling thread ("" if none).
+ * The pointer stays valid until the next library call on this thread. */
+METIS_API const char* metis_last_error(void);
+
+/* Reads (and, if `clear` != 0, clears) the sticky device error word on the
+ * current device, synchronising `stream` first. Returns METIS_OK,
+ * METIS_ERR_TIMEOUT if a kernel's bounded wait ran out, or METIS_ERR_CUDA.
+ * This is the one entry point that synchronises. */
+METIS_API int metis_check_device_status(metis_stream_t stream, int clear);
+
+/* Sets the per-wait limit of the device watchdog in nanoseconds (default
+ * 2e9 = 2 s; 0 restores the default). Affects kernels launched afterwards. */
+METIS_API int metis_set_watchdog_ns(uint64_t ns);
+
+/* Per-token FP8 quantization of BF16 activations.
+ * Source: "Lernex/Metis-1.6-Logos-FP8", "What --fast-math does" (each layer's
+ * input rounded to FP8 per token) and "What is in FP8" (activations quantized
+ * per token at run time).
+ *   x_bf16 [M, ldx] BF16 (K valid columns), xq [M, ldq] E4M3 out, s_tok [M] FP32 out.
+ *   Requires M >= 0, K > 0, K % 8 == 0, ldx >= K, ldq >= K, ldx % 8 == 0,
+ *   ldq % 8 == 0, x_bf16 16-byte aligned, xq 8-byte aligned, s_tok 4-byte
+ *   aligned. (Codes that feed metis_fp8_gemm need K % 16 == 0 and dense rows.)
+ *   M == 0 launches nothing. */
+METIS_API int metis_quant_fp8_per_token(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                              uint8_t* xq, int64_t ldq, float* s_tok, metis_stream_t stream);
+
+/* Per-output-channel FP8 quantization of FP32 weights, the same rule as the
+ * per-token quantizer applied to each weight row (one scale per output
+ * channel, "Lernex/Metis-1.6-Logos-FP8", "What is in FP8"). Prepares the
+ * weight operand of the GEMMs.
+ *   w [N, ldw] FP32, wq [N, ldq] E4M3 out, s_w [N] FP32 out.
+ *   Requires K % 4 == 0, ldw % 4 == 0, ldq % 4 == 0, ldw >= K, ldq >= K,
+ *   w 16-byte aligned, wq 4-byte aligned. */
+METIS_API int metis_quant_fp8_per_channel(const float* w, int64_t N, int64_t K, int64_t ldw,
+                                uint8_t* wq, int64_t ldq, float* s_w, metis_stream_t stream);
+
+/* Fast-math W8A8 GEMM with the per-token x per-channel scale epilogue on
+ * tcgen05 tensor cores ("Lernex/Metis-1.6-Logos-FP8", "What --fast-math does").
+ *   a_kind = METIS_A_E4M3: `a` is E4M3 [M, K] (dense rows), s_tok [M] is an input.
+ *   a_kind = METIS_A_BF16: `a` is BF16 [M, K] (dense rows); the per-token
+ *            quantization is fused into the GEMM (an amax pre-pass writes
+ *            s_tok [M] as an OUTPUT, identical to metis_quant_fp8_per_token,
+ *            and the E4M3 codes are produced in shared memory, never in HBM).
+ *            Needs `workspace` of metis_workspace_size(METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0)
+ *            bytes (16-byte aligned).
+ *   wq [N, K] E4M3 (one row per output channel), s_w [N] FP32, y [M, N] BF16 out.
+ *   Requires K % 16 == 0, N % 8 == 0, K >= 16, N >= 8, M >= 0; a, wq, y
+ *   16-byte aligned. */
+#define METIS_A_E4M3 0
+#define METIS_A_BF16 1
+METIS_API int metis_fp8_gemm(const void* a, int a_kind, float* s_tok, const uint8_t* wq,
+                   const float* s_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                   void* workspace, size_t ws_bytes, metis_stream_t stream);
+
+/* Default-maths weight-only GEMM for decode (M <= 8): the E4M3 weights are
+ * streamed from HBM and widened exactly to 16 bits in registers, products
+ * accumulate in FP32, the per-channel scale is applied to the sum
+ * ("Lernex/Metis-1.6-Logos-FP8", "What --fast-math does": the default maths,
+ * which single-stream decode always uses).
+ *   x [M, K] BF16, wq [N, K] E4M3, s_w [N] FP32, y [M, N] BF16 out.
+ *   Requires 1 <= M <= 8, K % 16 == 0, 16 <= K <= 12288, N >= 1; x, wq
+ *   16-byte aligned. */
+METIS_API int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
+                     int64_t M, int64_t N, int64_t K, metis_stream_t stream);
+
+/* Routed-expert W8A8 layer ("Lernex/Metis-1.6-Logos-FP8", "What is in FP8":
+ * the routed experts are FP8 with per-channel scales and per-token
+ * activations). Steps, all on the device, no host synchronisation:
+ * routing histogram -> exclusive prefix sum -> stable permutation of the
+ * slots (t, j) by expert -> per-token quantization of x (once per token) ->
+ * gather into expert-contiguous rows -> grouped up-projection (W8A8) ->
+ * per-row re-quantization -> grouped down-projection (W8A8) -> weighted
+ * un-permute y[t] = sum_j topk_w[t,j] o[t,j] (FP32, j ascending) -> BF16.
+ *   x [T, H] BF16, topk_ids [T, topk] int32 in [0, E), topk_w [T, topk] FP32,
+ *   w_up [E, I, H] E4M3, s_up [E, I], w_down [E, H, I] E4M3, s_down [E, H],
+ *   y [T, H] BF16 out.
+ *   act must be METIS_ACT_NONE (the cards do not state the experts' activation).
+ *   Requires H % 16 == 0, I % 16 == 0, H >= 16, I >= 16, 1 <= topk <= E <= 1024;
+ *   ids outside [0, E) are a caller error (not checked on the device).
+ *   Needs `workspace` of metis_workspace_size(METIS_OP_MOE, T, I, H, topk, E)
+ *   bytes (256-byte aligned); its regions are given by metis_moe_workspace_offset. */
+#define METIS_ACT_NONE 0
+METIS_API int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* topk_ids, const float* topk_w,
+                               int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
+                               const uint8_t* w_up, const float* s_up,
+                               const uint8_t* w_down, const float* s_down, int act,
+                               void* y_bf16, void* workspace, size_t ws_bytes,
+                               metis_stream_t stream);
+
+/* Workspace sizes in bytes.
+ *   METIS_OP_FP8_GEMM_FUSED: (M, N, K) of metis_fp8_gemm with a_kind = METIS_A_BF16.
+ *   METIS_OP_MOE:            (T, I, H, topk, E) of metis_moe_fp8_grouped_gemm.
+ *   Other ops need none (0). Returns 0 for invalid arguments. */
+#define METIS_OP_FP8_GEMM 0
+#define METIS_OP_FP8_GEMM_FUSED 1
+#define METIS_OP_W8A16 2
+#define METIS_OP_MOE 3
+METIS_API size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, int64_t K_or_H,
+                            int64_t topk, int64_t E);
+
+/* Byte offset of one region inside the routed-expert workspace, so callers
+ * and tests can read the intermediates (S = T * topk slots):
+ *   METIS_MOE_WS_COUNTS      int32 [E]      slots per expert
+ *   METIS_MOE_WS_OFFSETS     int32 [E + 1]  exclusive prefix sum of COUNTS
+ *   METIS_MOE_WS_SLOT_TO_ROW int32 [S]      row of slot s = t*topk + j in expert order
+ *   METIS_MOE_WS_ROW_TO_SLOT int32 [S]      inverse permutation
+ *   METIS_MOE_WS_XQ          E4M3  [T, H]   per-token codes of x
+ *   METIS_MOE_WS_SX          FP32  [T]      per-token scales of x
+ *   METIS_MOE_WS_AQ          E4M3  [S, H]   XQ rows gathered into expert order
+ *   METIS_MOE_WS_SA          FP32  [S]      their scales
+ *   METIS_MOE_WS_H           BF16  [S, I]   up-projection output, expert order
+ *   METIS_MOE_WS_HQ          E4M3  [S, I]   its per-row codes
+ *   METIS_MOE_WS_SH          FP32  [S]      their scales
+ *   METIS_MOE_WS_O           BF16  [S, H]   down-projection output, expert order
+ * Returns -1 for an unknown region or invalid sizes. */
+#define METIS_MOE_WS_COUNTS 0
+#define METIS_MOE_WS_OFFSETS 1
+#define METIS_MOE_WS_SLOT_TO_ROW 2
+#define METIS_MOE_WS_ROW_TO_SLOT 3
+#define METIS_MOE_WS_XQ 4
+#define METIS_MOE_WS_SX 5
+#define METIS_MOE_WS_AQ 6
+#define METIS_MOE_WS_SA 7
+#define METIS_MOE_WS_H 8
+#define METIS_MOE_WS_HQ 9
+#define METIS_MOE_WS_SH 10
+#define METIS_MOE_WS_O 11
+METIS_API int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk, int64_t E,
+                                   int64_t H, int64_t I);
+
+/* The dispatch rule of the cards ("Lernex/Metis-1.6-Praxis-NVFP4", "What
+ * --fast-math does"): M <= 8 tokens always take the default maths
+ * (metis_w8a16_gemm); more tokens take the fast-math W8A8 path when
+ * fast_math != 0 (quantizing x per token, fused: a_kind = METIS_A_BF16), and
+ * otherwise the large-M default path, which this build does not implement
+ * (METIS_ERR_UNSUPPORTED). s_tok [M] receives the per-token scales on the
+ * fast-math path. `workspace` as for metis_fp8_gemm with METIS_A_BF16. */
+METIS_API int metis_linear(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
+                 int64_t M, int64_t N, int64_t K, int fast_math, float* s_tok,
+                 void* workspace, size_t ws_bytes, metis_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* METIS_FP8_H */

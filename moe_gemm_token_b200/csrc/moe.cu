@@ -1,0 +1,268 @@
+// Routed-expert W8A8 layer: the FP8 linear layer grouped over top-k routed
+// experts ("Lernex/Metis-1.6-Logos-FP8", "What is in FP8": the routed experts
+// are FP8, E4M3 with one scale per output channel, activations quantized per
+// token at run time).
+//
+// Device pipeline (no host synchronisation; segment sizes stay on the GPU):
+//   1. per-token quantization of x            (quantizer kernel, once per token)
+//   2. routing histogram per chunk of slots    (shared-memory integer atomics)
+//   3. prefix sums: per-expert offsets and per-(chunk, expert) bases
+//   4. stable scatter: row of slot s = t*topk + j in expert order, via warp
+//      match + per-warp counts (no atomics in the ordering), and gather of
+//      the token's codes and scale into expert-contiguous rows
+//   5. grouped up-projection (tcgen05 W8A8 GEMM, tile schedule from offsets)
+//   6. per-row re-quantization of h
+//   7. grouped down-projection
+//   8. weighted un-permute y[t] = sum_j w[t,j] * o[row(t,j)], FP32, j ascending.
+#include "common.cuh"
+
+namespace metis {
+
+template <typename T>
+int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                      float* s, cudaStream_t st);
+int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b, const float* s_b,
+                            __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
+                            int K, cudaStream_t st);
+int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
+                          int64_t* total);
+
+namespace moe {
+
+constexpr int CHUNK = 256;   // slots per routing CTA (one per thread)
+constexpr int MAX_E = 1024;
+
+// chunk_counts[c][e] = number of slots of chunk c routed to expert e.
+// Ids outside [0, E) are dropped and flagged in the device status word.
+__global__ void __launch_bounds__(CHUNK) count_kernel(const int32_t* __restrict__ ids, int S, int E,
+                                                      int32_t* __restrict__ chunk_counts,
+                                                      uint32_t* status) {
+    __shared__ int cnt[MAX_E];
+    for (int e = threadIdx.x; e < E; e += CHUNK) cnt[e] = 0;
+    __syncthreads();
+    const int s = blockIdx.x * CHUNK + threadIdx.x;
+    if (s < S) {
+        const int e = ids[s];
+        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+        else atomicOr(status, kDevErrBadIndex);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += CHUNK)
+        chunk_counts[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
+}
+
+// counts[e], offsets[e] (exclusive, E + 1 entries) and, in place,
+// chunk_counts[c][e] -> base row of chunk c's slots of expert e.
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_counts, int C, int E,
+                                                    int32_t* __restrict__ counts,
+                                                    int32_t* __restrict__ offsets) {
+    __shared__ int warp_tot[32];
+    const int e = threadIdx.x;
+    int total = 0;
+    if (e < E)
+        for (int c = 0; c < C; ++c) total += chunk_counts[static_cast<size_t>(c) * E + e];
+    // block-wide exclusive scan of total over e
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = total;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_tot[lane];
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += v;
+        }
+        warp_tot[lane] = wi - w;  // exclusive prefix of warp totals
+    }
+    __syncthreads();
+    const int excl = warp_tot[warp] + incl - total;
+    if (e < E) {
+        counts[e] = total;
+        offsets[e] = excl;
+        int run = excl;
+        for (int c = 0; c < C; ++c) {
+            const size_t i = static_cast<size_t>(c) * E + e;
+            const int v = chunk_counts[i];
+            chunk_counts[i] = run;
+            run += v;
+        }
+        if (e == E - 1) offsets[E] = run;
+    }
+}
+
+// Stable rank of each slot within its expert, then gather of the token's
+// codes into the slot's row.
+__global__ void __launch_bounds__(CHUNK) scatter_gather_kernel(
+    const int32_t* __restrict__ ids, int S, int E, int topk, const int32_t* __restrict__ chunk_base,
+    int32_t* __restrict__ slot_to_row, int32_t* __restrict__ row_to_slot,
+    const uint8_t* __restrict__ xq, const float* __restrict__ sx, int H, uint8_t* __restrict__ aq,
+    float* __restrict__ sa) {
+    constexpr int WARPS = CHUNK / 32;
+    __shared__ int wcnt[WARPS][MAX_E];  // per-warp counts, then exclusive prefix over warps
+    __shared__ int rows[CHUNK];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int i = threadIdx.x; i < WARPS * E; i += CHUNK) wcnt[i / E][i % E] = 0;
+    __syncthreads();
+    const int s = blockIdx.x * CHUNK + threadIdx.x;
+    int e = s < S ? ids[s] : -1;
+    if (e >= E) e = -1;
+    const bool ok = e >= 0;
+    if (s < S && !ok) slot_to_row[s] = -1;  // dropped: never read by the combine
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(peers & ((1u << lane) - 1u));
+    if (ok && rank_w == 0) wcnt[warp][e] = __popc(peers);
+    __syncthreads();
+    // exclusive prefix over warps, per expert
+    for (int x = threadIdx.x; x < E; x += CHUNK) {
+        int run = 0;
+        for (int w = 0; w < WARPS; ++w) {
+            const int v = wcnt[w][x];
+            wcnt[w][x] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    int row = -1;
+    if (ok) {
+        row = chunk_base[static_cast<size_t>(blockIdx.x) * E + e] + wcnt[warp][e] + rank_w;
+        slot_to_row[s] = row;
+        row_to_slot[row] = s;
+        sa[row] = sx[s / topk];
+    }
+    rows[threadIdx.x] = row;
+    __syncthreads();
+    // gather: each warp copies whole rows, 16 bytes per lane per step
+    const int first = blockIdx.x * CHUNK;
+    for (int i = warp; i < CHUNK; i += WARPS) {
+        const int r = rows[i];
+        if (r < 0) continue;
+        const uint4* src = reinterpret_cast<const uint4*>(xq + static_cast<size_t>((first + i) / topk) * H);
+        uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<size_t>(r) * H);
+        for (int v = lane; v < H / 16; v += 32) dst[v] = src[v];
+    }
+}
+
+// y[t, n..n+7] = bf16( sum_j w[t, j] * o[slot_to_row[t*topk + j], n..n+7] ).
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ o,
+                                                      const float* __restrict__ w,
+                                                      const int32_t* __restrict__ slot_to_row,
+                                                      int T, int topk, int H,
+                                                      __nv_bfloat16* __restrict__ y) {
+    const int groups = H / 8;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<int64_t>(T) * groups) return;
+    const int t = static_cast<int>(idx / groups);
+    const int n = static_cast<int>(idx - static_cast<int64_t>(t) * groups) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < topk; ++j) {
+        const int s = t * topk + j;
+        const float wj = w[s];
+        const int r = slot_to_row[s];
+        if (r < 0) continue;
+        const uint4 c = *reinterpret_cast<const uint4*>(o + static_cast<size_t>(r) * H + n);
+        const uint32_t v[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = fmaf(wj, bf16_lo(v[i]), acc[2 * i]);
+            acc[2 * i + 1] = fmaf(wj, bf16_hi(v[i]), acc[2 * i + 1]);
+        }
+    }
+    uint4 out;
+    out.x = pack_bf16x2(acc[0], acc[1]);
+    out.y = pack_bf16x2(acc[2], acc[3]);
+    out.z = pack_bf16x2(acc[4], acc[5]);
+    out.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + n) = out;
+}
+
+}  // namespace moe
+}  // namespace metis
+
+using namespace metis;
+
+extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* topk_ids,
+                                          const float* topk_w, int64_t T, int64_t topk, int64_t E,
+                                          int64_t H, int64_t I, const uint8_t* w_up,
+                                          const float* s_up, const uint8_t* w_down,
+                                          const float* s_down, int act, void* y_bf16,
+                                          void* workspace, size_t ws_bytes,
+                                          metis_stream_t stream) {
+    using namespace moe;
+    clear_error();
+    if (act != METIS_ACT_NONE)
+        return fail(METIS_ERR_UNSUPPORTED, "moe: act=%d; only METIS_ACT_NONE is built", act);
+    if (T < 0 || topk < 1 || E < topk || E > MAX_E)
+        return fail(METIS_ERR_INVALID_ARG, "moe: need T >= 0 and 1 <= topk <= E <= %d (T=%lld topk=%lld E=%lld)",
+                    MAX_E, (long long)T, (long long)topk, (long long)E);
+    if (H < 16 || I < 16 || H % 16 || I % 16 || H > (1 << 20) || I > (1 << 20))
+        return fail(METIS_ERR_INVALID_ARG, "moe: need H, I >= 16 and multiples of 16 (H=%lld I=%lld)",
+                    (long long)H, (long long)I);
+    const int64_t S = T * topk;
+    if (S > (1ll << 30)) return fail(METIS_ERR_INVALID_ARG, "moe: T*topk too large");
+    const size_t need = metis_workspace_size(METIS_OP_MOE, T, I, H, topk, E);
+    if (T == 0) return METIS_OK;
+    if (!x_bf16 || !topk_ids || !topk_w || !w_up || !s_up || !w_down || !s_down || !y_bf16 || !workspace)
+        return fail(METIS_ERR_INVALID_ARG, "moe: null pointer");
+    if (ws_bytes < need)
+        return fail(METIS_ERR_INVALID_ARG, "moe: workspace of %zu bytes, need %zu", ws_bytes, need);
+    if (!aligned(workspace, 256) || !aligned(x_bf16, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
+        !aligned(y_bf16, 16) || !aligned(s_up, 16) || !aligned(s_down, 16))
+        return fail(METIS_ERR_INVALID_ARG,
+                    "moe: workspace must be 256-byte aligned; x, weights, scales and y 16-byte aligned");
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto region = [&](int r) { return ws + moe_region_offset(r, T, topk, E, H, I, nullptr); };
+    int32_t* counts = reinterpret_cast<int32_t*>(region(METIS_MOE_WS_COUNTS));
+    int32_t* offsets = reinterpret_cast<int32_t*>(region(METIS_MOE_WS_OFFSETS));
+    int32_t* s2r = reinterpret_cast<int32_t*>(region(METIS_MOE_WS_SLOT_TO_ROW));
+    int32_t* r2s = reinterpret_cast<int32_t*>(region(METIS_MOE_WS_ROW_TO_SLOT));
+    uint8_t* xq = region(METIS_MOE_WS_XQ);
+    float* sx = reinterpret_cast<float*>(region(METIS_MOE_WS_SX));
+    uint8_t* aq = region(METIS_MOE_WS_AQ);
+    float* sa = reinterpret_cast<float*>(region(METIS_MOE_WS_SA));
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(region(METIS_MOE_WS_H));
+    uint8_t* hq = region(METIS_MOE_WS_HQ);
+    float* sh = reinterpret_cast<float*>(region(METIS_MOE_WS_SH));
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(region(METIS_MOE_WS_O));
+    // the per-(chunk, expert) table reuses the H region, which is written
+    // only later by the up-projection
+    const int C = static_cast<int>((S + CHUNK - 1) / CHUNK);
+    int32_t* chunk_tab = reinterpret_cast<int32_t*>(h);
+    if (static_cast<int64_t>(C) * E * 4 > 2 * S * I)
+        return fail(METIS_ERR_UNSUPPORTED, "moe: routing table does not fit the workspace (E too large for T*topk*I)");
+
+    if ((rc = launch_quant_rows<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_bf16), T, H, H, xq, H,
+                                               sx, st)))
+        return rc;
+    uint32_t* status = nullptr;
+    if ((rc = device_status_word(&status))) return rc;
+    count_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
+                                      status);
+    scan_kernel<<<1, 1024, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets);
+    scatter_gather_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E),
+                                               static_cast<int>(topk), chunk_tab, s2r, r2s, xq, sx,
+                                               static_cast<int>(H), aq, sa);
+    if ((rc = cuda_check(cudaGetLastError(), "moe routing launch"))) return rc;
+    if ((rc = launch_fp8_gemm_grouped(aq, sa, w_up, s_up, h, offsets, static_cast<int>(E),
+                                      static_cast<int>(S), static_cast<int>(I), static_cast<int>(H), st)))
+        return rc;
+    if ((rc = launch_quant_rows<__nv_bfloat16>(h, S, I, I, hq, I, sh, st))) return rc;
+    if ((rc = launch_fp8_gemm_grouped(hq, sh, w_down, s_down, o, offsets, static_cast<int>(E),
+                                      static_cast<int>(S), static_cast<int>(H), static_cast<int>(I), st)))
+        return rc;
+    const int64_t work = T * (H / 8);
+    combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
+        o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
+        static_cast<__nv_bfloat16*>(y_bf16));
+    return cuda_check(cudaGetLastError(), "moe combine launch");
+}

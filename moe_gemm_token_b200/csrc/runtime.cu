@@ -1,0 +1,239 @@
+// Host runtime of libmetis_fp8: per-thread error messages, cached device
+// properties, the device watchdog word, TMA descriptor encoding, workspace
+// layout, and the dispatch entry point.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+
+namespace metis {
+
+namespace {
+thread_local std::string g_last_error;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DeviceInfo g_info[kMaxDevices];
+uint32_t* g_status_ptr[kMaxDevices];
+uint64_t g_watchdog_ns = 2000000000ull;
+
+// Sticky error word, one per device that loads the library.
+__device__ uint32_t g_device_status;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+}  // namespace
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+void clear_error() { g_last_error.clear(); }
+
+int cuda_check(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return METIS_OK;
+    return fail(METIS_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+int current_device_info(DeviceInfo* out) {
+    int dev = 0;
+    int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+    if (rc) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return fail(METIS_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_info[dev];
+    if (d.device < 0) {
+        DeviceInfo n;
+        n.device = dev;
+        if ((rc = cuda_check(cudaDeviceGetAttribute(&n.num_sms, cudaDevAttrMultiProcessorCount, dev),
+                             "cudaDeviceGetAttribute(SMs)")))
+            return rc;
+        if ((rc = cuda_check(cudaDeviceGetAttribute(&n.max_smem_optin,
+                                                    cudaDevAttrMaxSharedMemoryPerBlockOptin, dev),
+                             "cudaDeviceGetAttribute(smem)")))
+            return rc;
+        if ((rc = cuda_check(cudaDeviceGetAttribute(&n.cc_major, cudaDevAttrComputeCapabilityMajor, dev),
+                             "cudaDeviceGetAttribute(cc)")))
+            return rc;
+        if ((rc = cuda_check(cudaDeviceGetAttribute(&n.cc_minor, cudaDevAttrComputeCapabilityMinor, dev),
+                             "cudaDeviceGetAttribute(cc)")))
+            return rc;
+        if (n.cc_major != 10 || n.cc_minor != 0)
+            return fail(METIS_ERR_UNSUPPORTED,
+                        "libmetis_fp8 is built for sm_100a (B200); device %d is sm_%d%d", dev,
+                        n.cc_major, n.cc_minor);
+        d = n;
+    }
+    *out = d;
+    return METIS_OK;
+}
+
+int device_status_word(uint32_t** out) {
+    int dev = 0;
+    int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+    if (rc) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return fail(METIS_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        rc = cuda_check(cudaGetSymbolAddress(&p, g_device_status), "cudaGetSymbolAddress(status)");
+        if (rc) return rc;
+        g_status_ptr[dev] = static_cast<uint32_t*>(p);
+    }
+    *out = g_status_ptr[dev];
+    return METIS_OK;
+}
+
+uint64_t watchdog_ns() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_watchdog_ns;
+}
+
+int make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                 uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    if (!g_encode) return fail(METIS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    CUtensorMapDataType dt;
+    switch (elem_bytes) {
+        case 1: dt = CU_TENSOR_MAP_DATA_TYPE_UINT8; break;
+        case 2: dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; break;
+        case 4: dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; break;
+        default: return fail(METIS_ERR_INVALID_ARG, "tensor map element size %d", elem_bytes);
+    }
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "cuTensorMapEncodeTiled failed (%d): cols=%llu rows=%llu pitch=%llu box=%ux%u",
+                    static_cast<int>(r), (unsigned long long)cols, (unsigned long long)rows,
+                    (unsigned long long)row_bytes, box_cols, box_rows);
+    return METIS_OK;
+}
+
+// Routed-expert workspace layout (regions 256-byte aligned).
+static int64_t align256(int64_t v) { return (v + 255) & ~static_cast<int64_t>(255); }
+
+int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
+                          int64_t* total) {
+    const int64_t S = T * topk;
+    const int64_t sizes[12] = {
+        4 * E,        // COUNTS
+        4 * (E + 1),  // OFFSETS
+        4 * S,        // SLOT_TO_ROW
+        4 * S,        // ROW_TO_SLOT
+        T * H,        // XQ
+        4 * T,        // SX
+        S * H,        // AQ
+        4 * S,        // SA
+        2 * S * I,    // H
+        S * I,        // HQ
+        4 * S,        // SH
+        2 * S * H,    // O
+    };
+    int64_t off = 0, at = -1;
+    for (int r = 0; r < 12; ++r) {
+        if (r == region) at = off;
+        off = align256(off + sizes[r]);
+    }
+    if (total) *total = off;
+    return at;
+}
+
+}  // namespace metis
+
+using namespace metis;
+
+extern "C" int metis_version(void) { return 100; }
+
+extern "C" const char* metis_last_error(void) { return g_last_error.c_str(); }
+
+extern "C" int metis_set_watchdog_ns(uint64_t ns) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_watchdog_ns = ns ? ns : 2000000000ull;
+    return METIS_OK;
+}
+
+extern "C" int metis_check_device_status(metis_stream_t stream, int clear) {
+    clear_error();
+    uint32_t* word = nullptr;
+    int rc = device_status_word(&word);
+    if (rc) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((rc = cuda_check(cudaStreamSynchronize(s), "cudaStreamSynchronize"))) return rc;
+    uint32_t v = 0;
+    if ((rc = cuda_check(cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost), "read status")))
+        return rc;
+    if (clear && v) {
+        uint32_t z = 0;
+        if ((rc = cuda_check(cudaMemcpy(word, &z, sizeof z, cudaMemcpyHostToDevice), "clear status")))
+            return rc;
+    }
+    if (v & kDevErrTimeout)
+        return fail(METIS_ERR_TIMEOUT, "a device-side bounded wait ran out (status word 0x%x)", v);
+    if (v & kDevErrBadIndex)
+        return fail(METIS_ERR_INVALID_ARG, "a routing id outside [0, E) was dropped (status word 0x%x)", v);
+    return METIS_OK;
+}
+
+extern "C" size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, int64_t K_or_H,
+                                       int64_t topk, int64_t E) {
+    if (M_or_T < 0 || N_or_I < 0 || K_or_H < 0) return 0;
+    switch (op) {
+        case METIS_OP_FP8_GEMM_FUSED:
+            // per-token reciprocal scales 448/amax, one FP32 per row
+            return static_cast<size_t>(align256(4 * (M_or_T > 0 ? M_or_T : 1)));
+        case METIS_OP_MOE: {
+            if (topk < 1 || E < 1) return 0;
+            int64_t total = 0;
+            moe_region_offset(0, M_or_T, topk, E, K_or_H, N_or_I, &total);
+            return static_cast<size_t>(total);
+        }
+        default:
+            return 0;
+    }
+}
+
+extern "C" int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk, int64_t E,
+                                              int64_t H, int64_t I) {
+    if (region < 0 || region > 11 || T < 0 || topk < 1 || E < 1 || H < 0 || I < 0) return -1;
+    return moe_region_offset(region, T, topk, E, H, I, nullptr);
+}
+
+extern "C" int metis_linear(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
+                            int64_t M, int64_t N, int64_t K, int fast_math, float* s_tok,
+                            void* workspace, size_t ws_bytes, metis_stream_t stream) {
+    clear_error();
+    if (M >= 1 && M <= 8) return metis_w8a16_gemm(x_bf16, wq, s_w, y_bf16, M, N, K, stream);
+    if (!fast_math)
+        return fail(METIS_ERR_UNSUPPORTED,
+                    "metis_linear: the default (16-bit) maths for M > 8 tokens is not built; "
+                    "pass fast_math=1");
+    return metis_fp8_gemm(x_bf16, METIS_A_BF16, s_tok, wq, s_w, y_bf16, M, N, K, workspace,
+                          ws_bytes, stream);
+}

@@ -1,0 +1,191 @@
+"""Thin Python binding of libmetis_fp8 (the C ABI in ``include/metis_fp8.h``).
+
+Every function here has the name of the C entry point it calls and only
+marshals arguments: torch CUDA tensors become device pointers, shapes become
+sizes, the current torch stream becomes the ``cudaStream_t``. All arithmetic
+runs in the library's CUDA kernels. There is no fallback: if the library is
+missing, :func:`load` raises.
+
+BF16 tensors may be ``torch.bfloat16`` or ``torch.int16``/``uint16`` bit
+patterns; E4M3 tensors ``torch.uint8`` or ``torch.float8_e4m3fn``.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmetis_fp8.so")
+
+METIS_OK = 0
+METIS_ERR_INVALID_ARG = -1
+METIS_ERR_UNSUPPORTED = -2
+METIS_ERR_CUDA = -3
+METIS_ERR_TIMEOUT = -4
+
+METIS_A_E4M3 = 0
+METIS_A_BF16 = 1
+METIS_ACT_NONE = 0
+METIS_OP_FP8_GEMM = 0
+METIS_OP_FP8_GEMM_FUSED = 1
+METIS_OP_W8A16 = 2
+METIS_OP_MOE = 3
+
+MOE_WS = dict(COUNTS=0, OFFSETS=1, SLOT_TO_ROW=2, ROW_TO_SLOT=3, XQ=4, SX=5, AQ=6, SA=7, H=8,
+              HQ=9, SH=10, O=11)
+
+_lib = None
+
+
+class MetisError(RuntimeError):
+    def __init__(self, name, code, msg):
+        super().__init__(f"{name} returned {code}: {msg}")
+        self.code = code
+
+
+def load():
+    """Loads libmetis_fp8.so (built in-tree by ``moe_gemm_token_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m moe_gemm_token_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    sz = ctypes.c_size_t
+    sig = {
+        "metis_version": ([], i32),
+        "metis_last_error": ([], ctypes.c_char_p),
+        "metis_check_device_status": ([p, i32], i32),
+        "metis_set_watchdog_ns": ([ctypes.c_uint64], i32),
+        "metis_quant_fp8_per_token": ([p, i64, i64, i64, p, i64, p, p], i32),
+        "metis_quant_fp8_per_channel": ([p, i64, i64, i64, p, i64, p, p], i32),
+        "metis_fp8_gemm": ([p, i32, p, p, p, p, i64, i64, i64, p, sz, p], i32),
+        "metis_w8a16_gemm": ([p, p, p, p, i64, i64, i64, p], i32),
+        "metis_moe_fp8_grouped_gemm": ([p, p, p, i64, i64, i64, i64, i64, p, p, p, p, i32, p, p,
+                                        sz, p], i32),
+        "metis_workspace_size": ([i32, i64, i64, i64, i64, i64], sz),
+        "metis_moe_workspace_offset": ([i32, i64, i64, i64, i64, i64], i64),
+        "metis_linear": ([p, p, p, p, i64, i64, i64, i32, p, p, sz, p], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(name, rc):
+    if rc != METIS_OK:
+        raise MetisError(name, rc, load().metis_last_error().decode())
+    return rc
+
+
+def _rows(t):
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+def metis_version():
+    return load().metis_version()
+
+
+def metis_check_device_status(stream=None, clear=True):
+    """Synchronises the stream and returns the sticky device status (0 = OK)."""
+    return load().metis_check_device_status(_s(stream), int(bool(clear)))
+
+
+def metis_set_watchdog_ns(ns):
+    return _check("metis_set_watchdog_ns", load().metis_set_watchdog_ns(int(ns)))
+
+
+def metis_quant_fp8_per_token(x, xq, s_tok, stream=None):
+    """x [M, K] BF16 -> xq [M, K] E4M3 codes, s_tok [M] FP32."""
+    M, K, ldx = _rows(x)
+    return _check("metis_quant_fp8_per_token", load().metis_quant_fp8_per_token(
+        _p(x), M, K, ldx, _p(xq), xq.stride(0), _p(s_tok), _s(stream)))
+
+
+def metis_quant_fp8_per_channel(w, wq, s_w, stream=None):
+    """w [N, K] FP32 -> wq [N, K] E4M3 codes, s_w [N] FP32."""
+    N, K, ldw = _rows(w)
+    return _check("metis_quant_fp8_per_channel", load().metis_quant_fp8_per_channel(
+        _p(w), N, K, ldw, _p(wq), wq.stride(0), _p(s_w), _s(stream)))
+
+
+def metis_fp8_gemm(a, a_kind, s_tok, wq, s_w, y, workspace=None, stream=None):
+    """y [M, N] = W8A8(a, wq); a is E4M3 (a_kind 0) or BF16 (a_kind 1, fused quantization)."""
+    M, K = a.shape
+    N = wq.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return _check("metis_fp8_gemm", load().metis_fp8_gemm(
+        _p(a), int(a_kind), _p(s_tok), _p(wq), _p(s_w), _p(y), M, N, K, _p(workspace), ws_bytes,
+        _s(stream)))
+
+
+def metis_w8a16_gemm(x, wq, s_w, y, stream=None):
+    """y [M, N] = W8A16(x, wq) for M <= 8."""
+    M, K = x.shape
+    N = wq.shape[0]
+    return _check("metis_w8a16_gemm", load().metis_w8a16_gemm(
+        _p(x), _p(wq), _p(s_w), _p(y), M, N, K, _s(stream)))
+
+
+def metis_moe_fp8_grouped_gemm(x, topk_ids, topk_w, w_up, s_up, w_down, s_down, y, workspace,
+                               act=METIS_ACT_NONE, stream=None):
+    """Routed-expert W8A8 layer; see the C header for shapes."""
+    T, H = x.shape
+    topk = topk_ids.shape[1]
+    E, I, H2 = w_up.shape
+    assert H2 == H
+    ws_bytes = workspace.numel() * workspace.element_size()
+    return _check("metis_moe_fp8_grouped_gemm", load().metis_moe_fp8_grouped_gemm(
+        _p(x), _p(topk_ids), _p(topk_w), T, topk, E, H, I, _p(w_up), _p(s_up), _p(w_down),
+        _p(s_down), int(act), _p(y), _p(workspace), ws_bytes, _s(stream)))
+
+
+def metis_workspace_size(op, m_or_t, n_or_i, k_or_h, topk=0, num_experts=0):
+    return int(load().metis_workspace_size(int(op), int(m_or_t), int(n_or_i), int(k_or_h),
+                                           int(topk), int(num_experts)))
+
+
+def metis_moe_workspace_offset(region, T, topk, E, H, I):
+    if isinstance(region, str):
+        region = MOE_WS[region]
+    return int(load().metis_moe_workspace_offset(int(region), int(T), int(topk), int(E), int(H),
+                                                 int(I)))
+
+
+def metis_linear(x, wq, s_w, y, fast_math=True, s_tok=None, workspace=None, stream=None):
+    """Dispatch rule: M <= 8 -> W8A16; otherwise W8A8 (fast_math) with fused quantization."""
+    M, K = x.shape
+    N = wq.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return _check("metis_linear", load().metis_linear(
+        _p(x), _p(wq), _p(s_w), _p(y), M, N, K, int(bool(fast_math)), _p(s_tok), _p(workspace),
+        ws_bytes, _s(stream)))
+
+
+def metis_internal_w8a16_variant(v):
+    """Tuning hook: selects how the W8A16 kernel widens E4M3 weights (0, 1, 2)."""
+    fn = load().metis_internal_w8a16_variant
+    fn.argtypes = [ctypes.c_int]
+    fn.restype = ctypes.c_int
+    return fn(int(v))

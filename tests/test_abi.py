@@ -1,0 +1,116 @@
+"""The C ABI library loads, exports every entry point its header declares,
+and rejects bad arguments on the host before touching the GPU (these calls
+need no GPU). Also checks that the product path never falls back to the CPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from moe_gemm_token_b200 import build as libbuild
+from moe_gemm_token_b200 import metis
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return metis.load()
+
+
+def _declared():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"METIS_API\s+[\w\s\*]+?\b(metis_\w+)\s*\(", text)
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    dyn = os.popen(f"nm -D --defined-only {metis.LIB_PATH}").read()
+    for n in names:
+        assert re.search(rf"\bT {n}\b", dyn), n
+
+
+def test_build_targets_sm100a_only():
+    assert libbuild.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert "--use_fast_math" not in libbuild.FLAGS
+
+
+def test_version(lib):
+    assert metis.metis_version() == 100
+
+
+def _rc(fn, *args):
+    return fn(*args)
+
+
+def test_host_validation_without_gpu(lib):
+    p = ctypes.c_void_p(0x1000)
+    null = None
+    # quantizer: K not a multiple of 8, bad leading dimensions
+    assert lib.metis_quant_fp8_per_token(p, 4, 12, 12, p, 16, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert b"K % 8" in lib.metis_last_error()
+    assert lib.metis_quant_fp8_per_token(p, 4, 16, 8, p, 16, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_quant_fp8_per_token(p, 4, 16, 16, p, 20, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_quant_fp8_per_token(p, 0, 16, 16, p, 16, p, null) == metis.METIS_OK  # nothing to do
+    assert lib.metis_quant_fp8_per_token(null, 4, 16, 16, p, 16, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_quant_fp8_per_token(ctypes.c_void_p(0x1008), 4, 16, 16, p, 16, p, null) == \
+        metis.METIS_ERR_INVALID_ARG  # misaligned x
+    assert lib.metis_quant_fp8_per_channel(p, 4, 6, 8, p, 16, p, null) == metis.METIS_ERR_INVALID_ARG
+    # GEMM: K % 16, N % 8, bad kind
+    assert lib.metis_fp8_gemm(p, 0, p, p, p, p, 16, 512, 40, null, 0, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_fp8_gemm(p, 0, p, p, p, p, 16, 500, 256, null, 0, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_fp8_gemm(p, 7, p, p, p, p, 16, 512, 256, null, 0, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_fp8_gemm(p, 0, p, p, p, p, 0, 512, 256, null, 0, null) == metis.METIS_OK
+    # W8A16: M > 8, K too large
+    assert lib.metis_w8a16_gemm(p, p, p, p, 9, 128, 256, null) == metis.METIS_ERR_INVALID_ARG
+    assert b"M <= 8" in lib.metis_last_error()
+    assert lib.metis_w8a16_gemm(p, p, p, p, 4, 128, 16384, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_w8a16_gemm(p, p, p, p, 4, 128, 264, null) == metis.METIS_ERR_INVALID_ARG
+    # MoE: activation, topk > E, H % 16, small workspace
+    assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 2, 4, 64, 32, p, p, p, p, 1, p, p, 1 << 30,
+                                          null) == metis.METIS_ERR_UNSUPPORTED
+    assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 5, 4, 64, 32, p, p, p, p, 0, p, p, 1 << 30,
+                                          null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 2, 4, 72, 32, p, p, p, p, 0, p, p, 1 << 30,
+                                          null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 2, 4, 64, 32, p, p, p, p, 0, p, p, 16,
+                                          null) == metis.METIS_ERR_INVALID_ARG
+    assert b"workspace" in lib.metis_last_error()
+    # dispatch: large M default maths is not built
+    assert lib.metis_linear(p, p, p, p, 64, 128, 256, 0, p, p, 1 << 20, null) == metis.METIS_ERR_UNSUPPORTED
+
+
+def test_valid_call_without_gpu_fails_loudly(lib):
+    """No CPU fallback: a well-formed call on a machine without a GPU returns
+    METIS_ERR_CUDA instead of computing anything."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    p = ctypes.c_void_p(0x1000)
+    rc = lib.metis_quant_fp8_per_token(p, 4, 16, 16, p, 16, p, None)
+    assert rc == metis.METIS_ERR_CUDA
+    assert lib.metis_last_error()
+
+
+def test_workspace_layout(lib):
+    T, k, E, H, I = 4096, 8, 64, 2048, 1024
+    total = metis.metis_workspace_size(metis.METIS_OP_MOE, T, I, H, k, E)
+    offs = [metis.metis_moe_workspace_offset(r, T, k, E, H, I) for r in range(12)]
+    assert offs[0] == 0 and all(o % 256 == 0 for o in offs)
+    assert all(b > a for a, b in zip(offs, offs[1:]))
+    S = T * k
+    sizes = [4 * E, 4 * (E + 1), 4 * S, 4 * S, T * H, 4 * T, S * H, 4 * S, 2 * S * I, S * I, 4 * S,
+             2 * S * H]
+    for o, s, nxt in zip(offs, sizes, offs[1:] + [total]):
+        assert o + s <= nxt
+    assert metis.metis_moe_workspace_offset(12, T, k, E, H, I) == -1
+    assert metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, 4096, 2048, 2048) >= 4 * 4096
+    assert metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM, 4096, 2048, 2048) == 0

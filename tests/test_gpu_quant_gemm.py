@@ -1,0 +1,177 @@
+"""GPU parity of the quantizers, the W8A8 GEMM and the W8A16 GEMM against the
+CPU oracle, through the C ABI. Bytes and scales bit-exact; BF16 outputs within
+1e-2 * (1 + |ref|)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_gemm_token_b200 import synth
+from gpu_helpers import assert_bytes_equal, assert_close, bf16_dev, bf16_host, dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _quant_gpu(m, x_bits, ldx=None):
+    M, K = x_bits.shape
+    if ldx is None:
+        xd = bf16_dev(x_bits)
+    else:
+        big = np.zeros((M, ldx), dtype=np.uint16)
+        big[:, :K] = x_bits
+        xd = bf16_dev(big)[:, :K]
+    xq = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty((M,), dtype=torch.float32, device="cuda")
+    m.metis_quant_fp8_per_token(xd, xq, s)
+    torch.cuda.synchronize()
+    return xq.cpu().numpy(), s.cpu().numpy()
+
+
+@pytest.mark.parametrize("M,K,seed", [(16, 256, 0), (37, 264, 1), (5, 6144, 2), (3, 20480, 3),
+                                      (1, 8, 4), (200, 2048, 5), (9, 16384, 6), (130, 1024, 7)])
+def test_quant_per_token_bit_exact(metis, M, K, seed):
+    d = synth.linear(seed, M, K, 8, outlier_channels=min(4, K), outlier_scale=25.0,
+                     zero_rows=(M // 2,), row_magnitude_log10=(-3, 3))
+    q, s = _quant_gpu(metis, d["x"])
+    qr, sr = oracle.quant_per_token(d["x"])
+    assert_bytes_equal(s.view(np.uint32), sr.view(np.uint32), "scales")
+    assert_bytes_equal(q, qr, "codes")
+
+
+def test_quant_per_token_extremes(metis):
+    """BF16 subnormal rows (448/amax overflows and is clamped), huge rows,
+    negative zeros, exact ties of the E4M3 grid."""
+    K = 64
+    rows = [
+        np.full(K, 2.0 ** -130, np.float32),                       # subnormal BF16
+        np.linspace(-3e38, 3e38, K).astype(np.float32),           # near BF16 max
+        np.where(np.arange(K) % 2 == 0, -0.0, 0.0).astype(np.float32),
+        (np.arange(K) - 32).astype(np.float32) * 0.5,              # many exact ties after scaling
+        np.r_[448.0, np.full(K - 1, 1.0625, np.float32)].astype(np.float32),
+        np.r_[np.full(K - 1, 1e-8, np.float32), 1.0].astype(np.float32),
+    ]
+    x = synth.f32_to_bf16_bits(np.stack(rows))
+    q, s = _quant_gpu(metis, x)
+    qr, sr = oracle.quant_per_token(x)
+    assert_bytes_equal(s.view(np.uint32), sr.view(np.uint32), "scales")
+    assert_bytes_equal(q, qr, "codes")
+
+
+def test_quant_per_token_strided(metis):
+    d = synth.linear(3, 50, 1000, 8, outlier_channels=3, outlier_scale=30.0)
+    q, s = _quant_gpu(metis, d["x"], ldx=1032)
+    qr, sr = oracle.quant_per_token(d["x"])
+    assert_bytes_equal(q, qr, "codes")
+    assert_bytes_equal(s.view(np.uint32), sr.view(np.uint32), "scales")
+
+
+@pytest.mark.parametrize("N,K", [(512, 256), (33, 100), (7, 20484), (1000, 4096)])
+def test_quant_per_channel_bit_exact(metis, N, K):
+    rng = np.random.default_rng(N + K)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    w[N // 3] = 0.0
+    wd = dev(w)
+    wq = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty((N,), dtype=torch.float32, device="cuda")
+    metis.metis_quant_fp8_per_channel(wd, wq, s)
+    torch.cuda.synchronize()
+    qr, sr = oracle.quant_per_channel(w)
+    assert_bytes_equal(s.cpu().numpy().view(np.uint32), sr.view(np.uint32), "scales")
+    assert_bytes_equal(wq.cpu().numpy(), qr, "codes")
+
+
+def _prep_weights(metis, w):
+    N, K = w.shape
+    wq = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty((N,), dtype=torch.float32, device="cuda")
+    metis.metis_quant_fp8_per_channel(dev(w), wq, s)
+    return wq, s
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 272), (1, 8, 16), (129, 264, 1040),
+                                   (520, 784, 1024), (257, 1024, 2048)])
+def test_fp8_gemm_parity(metis, M, N, K):
+    d = synth.linear(M * 7 + N, M, K, N, outlier_channels=4, outlier_scale=20.0, zero_rows=(M // 3,))
+    wq, s_w = _prep_weights(metis, d["w"])
+    xd = bf16_dev(d["x"])
+    xq = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    s_tok = torch.empty((M,), dtype=torch.float32, device="cuda")
+    metis.metis_quant_fp8_per_token(xd, xq, s_tok)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_fp8_gemm(xq, metis.METIS_A_E4M3, s_tok, wq, s_w, y)
+    assert metis.metis_check_device_status() == 0
+    wq_r, sw_r = oracle.quant_per_channel(d["w"])
+    assert_bytes_equal(wq.cpu().numpy(), wq_r, "weight codes")
+    y_r, y64, xq_r, st_r = oracle.linear_w8a8(d["x"], wq_r, sw_r)
+    assert_bytes_equal(xq.cpu().numpy(), xq_r, "activation codes")
+    assert_close(bf16_host(y), y64, f"y {M}x{N}x{K}")
+
+
+def test_fp8_gemm_exact_integer_products(metis):
+    """Codes whose products and sums are small integers: the FP32 accumulation
+    is exact, so with unit scales the output equals the oracle's BF16 bits."""
+    rng = np.random.default_rng(11)
+    M, N, K = 200, 272, 512
+    vals = np.array([0x38, 0x40, 0x44, 0xB8, 0xC0, 0x00, 0x30], np.uint8)  # 1,2,3,-1,-2,0,0.5
+    a = vals[rng.integers(0, vals.size, (M, K))]
+    b = vals[rng.integers(0, vals.size, (N, K))]
+    one_m, one_n = np.ones(M, np.float32), np.ones(N, np.float32)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_fp8_gemm(dev(a), 0, dev(one_m), dev(b), dev(one_n), y)
+    yr, _ = oracle.gemm_w8a8(a, one_m, b, one_n)
+    assert_bytes_equal(bf16_host(y), yr, "bf16 bits")
+
+
+@pytest.mark.parametrize("variant", [0, 1, 2])
+@pytest.mark.parametrize("M,N,K", [(1, 1000, 4096), (2, 37, 272), (3, 300, 12288), (4, 1000, 4096),
+                                   (5, 48, 1024), (8, 1000, 4096), (8, 16, 16)])
+def test_w8a16_parity(metis, variant, M, N, K):
+    d = synth.linear(M + 13 * N + K, M, K, N)
+    wq, s_w = _prep_weights(metis, d["w"])
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    old = metis.metis_internal_w8a16_variant(variant)
+    try:
+        metis.metis_w8a16_gemm(bf16_dev(d["x"]), wq, s_w, y)
+        torch.cuda.synchronize()
+    finally:
+        metis.metis_internal_w8a16_variant(old)
+    wq_r, sw_r = oracle.quant_per_channel(d["w"])
+    assert_bytes_equal(wq.cpu().numpy(), wq_r, "weight codes")
+    _, y64 = oracle.gemm_w8a16(d["x"], wq_r, sw_r)
+    assert_close(bf16_host(y), y64, f"w8a16 v{variant} {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("variant", [0, 1, 2])
+def test_w8a16_subnormal_weights_and_wide_x(metis, variant):
+    """Weight rows with many E4M3 subnormal codes and tokens whose elements
+    span many binades: the widening and the per-token shift stay exact."""
+    rng = np.random.default_rng(5)
+    M, N, K = 8, 96, 512
+    w = (rng.standard_normal((N, K)) * np.power(10.0, rng.uniform(-5, 0, (N, K)))).astype(np.float32)
+    x = (rng.standard_normal((M, K)) * np.power(10.0, rng.uniform(-4, 4, (M, K)))).astype(np.float32)
+    x[3] = 0.0
+    xb = synth.f32_to_bf16_bits(x)
+    wq, s_w = _prep_weights(metis, w)
+    wq_r, sw_r = oracle.quant_per_channel(w)
+    assert np.mean((wq_r & 0x78) == 0) > 0.2  # plenty of subnormal / zero codes
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    old = metis.metis_internal_w8a16_variant(variant)
+    try:
+        metis.metis_w8a16_gemm(bf16_dev(xb), wq, s_w, y)
+        torch.cuda.synchronize()
+    finally:
+        metis.metis_internal_w8a16_variant(old)
+    _, y64 = oracle.gemm_w8a16(xb, wq_r, sw_r)
+    assert_close(bf16_host(y), y64, f"w8a16 subnormal v{variant}")
+
+
+def test_linear_dispatch(metis):
+    """M <= 8 takes the default maths (W8A16), bit-identical to the direct call."""
+    d = synth.linear(21, 4, 512, 64)
+    wq, s_w = _prep_weights(metis, d["w"])
+    y1 = torch.empty((4, 64), dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty_like(y1)
+    metis.metis_w8a16_gemm(bf16_dev(d["x"]), wq, s_w, y1)
+    metis.metis_linear(bf16_dev(d["x"]), wq, s_w, y2, fast_math=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
