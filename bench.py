@@ -1,0 +1,490 @@
+#!/usr/bin/env python3
+"""Benchmark of the FP8 fast-math linear layer on B200.
+
+Headline workload: a 4096-token prompt read through two chained FP8 linear
+layers (K=2048 -> N=6144 -> 2048), each one per-token FP8 quantization of its
+BF16 input followed by the tcgen05 W8A8 GEMM with the per-token x
+per-channel scale epilogue. One step = q1 + G1 + q2 + G2 over one batch;
+value = whole-job tokens per second (N GPUs run independent replicas with
+their own token batches: weak scaling, no collective on the data path).
+
+Inputs are seeded synthetic data of the workload's shapes and distributions
+(BF16 activations ~N(0,1) with 1% outlier channels x30, FP32 weights ~N(0,0.02)
+quantized per output channel on the GPU before timing). Four layer sets
+(x, W1, W2) rotate from step to step so the working set (169 MB) exceeds the
+126 MB L2.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl metis|reference]
+Prints one JSON line (rank 0).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 W8A8 GEMM TFLOP/s & % FP8 peak; 4096-tok prefill tok/s; decode GB/s %HBM"
+M_TOK, K_HID, N_FF = 4096, 2048, 6144
+SETS = 4
+FP8_PER_BF16 = 2.0  # nominal dense FP8 : BF16 tensor throughput (4.5 : 2.25 PFLOP/s)
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["metis", "reference"], default="metis")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the context figures")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK, "fallback"
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_prefill_tokens(d, wq, tokens):
+    """The oracle's prefill chain on the given tokens (rows are independent)."""
+    import oracle
+    (w1q, s1), (w2q, s2) = wq
+    xq, st = oracle.quant_per_token(d["x"][tokens])
+    y1, _ = oracle.gemm_w8a8(xq, st, w1q, s1)
+    xq2, st2 = oracle.quant_per_token(y1)
+    y2, _ = oracle.gemm_w8a8(xq2, st2, w2q, s2)
+    return y2
+
+
+def cpu_baseline(budget_s, batch=256):
+    """Times the oracle (as it stands) on as many tokens of the workload as fit
+    in about `budget_s` seconds, in batches of `batch` tokens."""
+    import oracle
+    from moe_gemm_token_b200 import synth
+    d = synth.prefill_chain()
+    wq = (oracle.quant_per_channel(d["w1"]), oracle.quant_per_channel(d["w2"]))
+    done, t0 = 0, time.perf_counter()
+    while done < M_TOK:
+        toks = np.arange(done, min(M_TOK, done + batch))
+        oracle_prefill_tokens(d, wq, toks)
+        done += toks.size
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tok/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{done} of the {M_TOK} tokens of the prefill chain (quantize, GEMM "
+                      f"2048->6144, quantize, GEMM 6144->2048), float64 oracle, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return 0
+    import oracle
+    from moe_gemm_token_b200 import synth
+    d = synth.prefill_chain()
+    wq = (oracle.quant_per_channel(d["w1"]), oracle.quant_per_channel(d["w2"]))
+    t0 = time.perf_counter()
+    oracle_prefill_tokens(d, wq, np.arange(8))
+    per_tok = (time.perf_counter() - t0) / 8
+    budget = 150.0  # seconds for warm-up + timed steps
+    per_step = max(1, min(M_TOK, int(budget / max(1, args.steps + args.warmup) / per_tok)))
+    step_tokens = lambda i: (np.arange(per_step) + i * per_step) % M_TOK
+    for i in range(args.warmup):
+        oracle_prefill_tokens(d, wq, step_tokens(i))
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_prefill_tokens(d, wq, step_tokens(args.warmup + i))
+    dt = time.perf_counter() - t0
+    value = args.steps * per_step / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill_chain_4096tok_2048x6144x2048", "tokens_per_step": per_step,
+                   "note": "each step is a bounded sample of the 4096-token batch"},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"{per_step} tokens per step of the prefill chain"},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------- clock sampler
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only)."""
+
+    def __init__(self, device_index, period=0.02):
+        self.samples = []
+        self.period = period
+        self.ok = False
+        try:
+            import pynvml as nv
+            import torch
+            nv.nvmlInit()
+            self.nv = nv
+            # NVML ignores CUDA_VISIBLE_DEVICES: find this device by its UUID
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = nv.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, r))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        nv = self.nv
+        names = {
+            nv.nvmlClocksEventReasonGpuIdle: "gpu_idle",
+            nv.nvmlClocksEventReasonApplicationsClocksSetting: "applications_clocks",
+            nv.nvmlClocksEventReasonSwPowerCap: "sw_power_cap",
+            nv.nvmlClocksEventReasonHwSlowdown: "hw_slowdown",
+            nv.nvmlClocksEventReasonSyncBoost: "sync_boost",
+            nv.nvmlClocksEventReasonSwThermalSlowdown: "sw_thermal_slowdown",
+            nv.nvmlClocksEventReasonHwThermalSlowdown: "hw_thermal_slowdown",
+            nv.nvmlClocksEventReasonHwPowerBrakeSlowdown: "hw_power_brake_slowdown",
+        }
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in names.items():
+                if r & bit:
+                    reasons.add(name)
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------- metis arm
+
+def gemm_traffic_from_profile():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "fp8_gemm_prefill_4096x6144x2048.md")
+    src = os.path.join(ROOT, "moe_gemm_token_b200", "csrc", "gemm_fp8.cu")
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel source sha256[:16]") != sha:
+        return None
+    try:
+        return float(vals["dram bytes per launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_metis(args):
+    import torch
+    import torch.distributed as dist
+    from moe_gemm_token_b200 import metis, synth
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+    metis.load()
+    stream = torch.cuda.current_stream()
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    # ---- inputs: SETS layer sets, weights quantized per channel on the GPU
+    sets = []
+    for r in range(SETS):
+        d = synth.prefill_chain(seed=1 + 100 * r + 10000 * rank)
+        ws = []
+        for w in (d["w1"], d["w2"]):
+            wd = torch.from_numpy(w).to(dev)
+            wq = torch.empty(w.shape, dtype=torch.uint8, device=dev)
+            sw = torch.empty((w.shape[0],), dtype=torch.float32, device=dev)
+            metis.metis_quant_fp8_per_channel(wd, wq, sw)
+            ws.append((wq, sw))
+            del wd
+        sets.append({"x": bf16(d["x"]), "x_host": d["x"], "w": ws})
+    xq1 = torch.empty((M_TOK, K_HID), dtype=torch.uint8, device=dev)
+    st1 = torch.empty((M_TOK,), dtype=torch.float32, device=dev)
+    y1 = torch.empty((M_TOK, N_FF), dtype=torch.bfloat16, device=dev)
+    xq2 = torch.empty((M_TOK, N_FF), dtype=torch.uint8, device=dev)
+    st2 = torch.empty((M_TOK,), dtype=torch.float32, device=dev)
+    y2 = torch.empty((M_TOK, K_HID), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+
+    def step(i, ev=None):
+        s = sets[i % SETS]
+        (w1, s1), (w2, s2) = s["w"]
+        metis.metis_quant_fp8_per_token(s["x"], xq1, st1, stream)
+        if ev is not None:
+            ev[0].record(stream)
+        metis.metis_fp8_gemm(xq1, metis.METIS_A_E4M3, st1, w1, s1, y1, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        metis.metis_quant_fp8_per_token(y1, xq2, st2, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        metis.metis_fp8_gemm(xq2, metis.METIS_A_E4M3, st2, w2, s2, y2, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    launches_per_step = 4
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if metis.metis_check_device_status(stream) != 0:
+        raise RuntimeError("device status error after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(i, evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * M_TOK / (ms_per_step * 1e-3)
+
+    # ---- roofline of the dominant kernel (the W8A8 GEMM), from the live events
+    g1 = [e[0].elapsed_time(e[1]) for e in evs]
+    g2 = [e[2].elapsed_time(e[3]) for e in evs]
+    gemm_ms = (statistics.mean(g1) + statistics.mean(g2)) / 2
+    flops = 2.0 * M_TOK * K_HID * N_FF
+    achieved = flops / (gemm_ms * 1e-3) / 1e12
+    pk, pk_kind = peaks()
+    peak = pk["bf16_tflops"] * FP8_PER_BF16
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": gemm_traffic_from_profile(),
+                "kernel": "fp8_gemm_kernel (tcgen05 kind::f8f6f4, 128x256 tiles)",
+                "peak_source": f"{pk_kind} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP8_PER_BF16} "
+                               "(nominal FP8:BF16 dense ratio)",
+                "gemm_share_of_step": 2 * gemm_ms / ms_per_step,
+                "gemm_ms": [statistics.mean(g1), statistics.mean(g2)]}
+
+    # ---- end to end through the C ABI with host buffers
+    e2e_steps = min(args.steps, 200)
+    x_host = torch.from_numpy(sets[0]["x_host"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((M_TOK, K_HID), dtype=torch.bfloat16).pin_memory()
+    x_dev = sets[0]["x"]
+    (w1, s1), (w2, s2) = sets[0]["w"]
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        metis.metis_quant_fp8_per_token(x_dev, xq1, st1, stream)
+        metis.metis_fp8_gemm(xq1, 0, st1, w1, s1, y1, stream=stream)
+        metis.metis_quant_fp8_per_token(y1, xq2, st2, stream)
+        metis.metis_fp8_gemm(xq2, 0, st2, w2, s2, y2, stream=stream)
+        y_host.copy_(y2, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * M_TOK / (e2e_ms * 1e-3), "unit": "tok/s",
+           "h2d_bytes_per_step": M_TOK * K_HID * 2, "d2h_bytes_per_step": M_TOK * K_HID * 2,
+           "steps": e2e_steps}
+
+    secondary = None
+    if not args.no_secondary:
+        secondary = secondary_figures(metis, dev, pk)
+    if metis.metis_check_device_status(stream) != 0:
+        raise RuntimeError("device status error after the timed region")
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline(args.cpu_budget)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic",
+            "config": {"workload": "prefill_chain_4096tok_2048x6144x2048", "global_batch": world * M_TOK,
+                       "tokens_per_gpu": M_TOK, "layers": "2048->6144 then 6144->2048, no activation",
+                       "step": "quantize+GEMM+quantize+GEMM", "parallelism": f"replicas x{world}",
+                       "l2": f"{SETS} rotating layer sets (x, W1, W2), 169 MB > 126 MB L2"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(), "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def secondary_figures(metis, dev, pk):
+    """Context figures of the other hot-path kernels (not the headline):
+    decode W8A16 GB/s, quantizer GB/s, large-M W8A8 TFLOP/s, routed experts."""
+    import torch
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+
+    def codes(n, k):
+        c = torch.randint(0, 256, (n, k), dtype=torch.uint8, device=dev, generator=g)
+        c[(c & 0x7F) == 0x7F] = 0x38
+        return c
+
+    def timeit(fn, iters):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters * 1e-3
+
+    out = {}
+    hbm = pk["hbm_gbs"]
+    peak8 = pk["bf16_tflops"] * FP8_PER_BF16
+    # decode: 4 rotating weight sets (235 MB > L2)
+    N, K = 14336, 4096
+    ws = [codes(N, K) for _ in range(4)]
+    sw = torch.rand(N, device=dev, generator=g) * 1e-3
+    for M in (1, 8):
+        x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        i = [0]
+
+        def f():
+            i[0] = (i[0] + 1) % 4
+            metis.metis_w8a16_gemm(x, ws[i[0]], sw, y)
+        t = timeit(f, 200)
+        byt = N * K + 4 * N + 2 * M * K + 2 * M * N
+        out[f"decode_w8a16_M{M}"] = {"us": t * 1e6, "GB/s": byt / t / 1e9,
+                                     "frac_of_measured_hbm": byt / t / 1e9 / hbm}
+    del ws
+    # quantizer at the prefill and large-M shapes (2 rotating inputs > L2)
+    for (M, K) in [(4096, 2048), (16384, 8192)]:
+        xs = [torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16) for _ in range(2)]
+        xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        s = torch.empty(M, device=dev)
+        i = [0]
+
+        def f():
+            i[0] ^= 1
+            metis.metis_quant_fp8_per_token(xs[i[0]], xq, s)
+        t = timeit(f, 100)
+        out[f"quant_{M}x{K}"] = {"us": t * 1e6, "GB/s": (3 * M * K + 4 * M) / t / 1e9,
+                                 "frac_of_measured_hbm": (3 * M * K + 4 * M) / t / 1e9 / hbm}
+        del xs
+    # large-M W8A8 GEMM
+    for (M, K) in [(8192, 4096), (16384, 8192)]:
+        a = codes(M, K)
+        b = codes(K, K)
+        sa = torch.rand(M, device=dev, generator=g)
+        sb = torch.rand(K, device=dev, generator=g)
+        y = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        t = timeit(lambda: metis.metis_fp8_gemm(a, 0, sa, b, sb, y), 20)
+        tf = 2 * M * K * K / t / 1e12
+        out[f"gemm_{M}x{K}x{K}"] = {"us": t * 1e6, "TFLOP/s": tf, "frac_of_fp8_peak": tf / peak8}
+        del a, b, y
+    # routed experts: 4096 tokens, hidden 2048, latent 1024, 64 experts, top-8
+    T, H, I, E, k = 4096, 2048, 1024, 64, 8
+    x = torch.randn(T, H, device=dev, generator=g).to(torch.bfloat16)
+    logits = torch.randn(T, E, device=dev, generator=g)
+    logits[:, :4] += 0.93  # skew toward four hot experts
+    top = torch.topk(logits, k, dim=1)
+    ids = top.indices.to(torch.int32).contiguous()
+    w = torch.softmax(top.values, dim=1).float().contiguous()
+    wu = codes(E * I, H).view(E, I, H)
+    su = torch.rand(E, I, device=dev, generator=g) * 1e-3
+    wd = codes(E * H, I).view(E, H, I)
+    sd = torch.rand(E, H, device=dev, generator=g) * 1e-3
+    y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    wsp = torch.empty(metis.metis_workspace_size(metis.METIS_OP_MOE, T, I, H, k, E),
+                      dtype=torch.uint8, device=dev)
+    t = timeit(lambda: metis.metis_moe_fp8_grouped_gemm(x, ids, w, wu, su, wd, sd, y, wsp), 20)
+    tf = 2 * 2 * T * k * H * I / t / 1e12
+    out["moe_4096tok_64e_top8"] = {"us": t * 1e6, "tok/s": T / t, "TFLOP/s": tf,
+                                   "frac_of_fp8_peak": tf / peak8}
+    return out
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_metis(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -33,7 +33,7 @@ constexpr int XROW_PAD = 8;       // bytes; row pitch = 2K + 8 (bank-conflict fr
 
 // Weight widening variants (selected once, see metis_internal_w8a16_variant).
 enum Conv { kCvt = 0, kAluMul = 1, kAluFold = 2 };
-int g_variant = kCvt;
+int g_variant = kAluFold;
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     uint4 v;
@@ -137,7 +137,21 @@ __global__ void __launch_bounds__(THREADS, 1) w8a16_kernel(const Args a) {
     const int cpw = (nchunks + WARPS - 1) / WARPS;  // chunks per warp per tile
     const int units = ntl * cpw;
 
-    // -------- start the weight stream before staging x
+    // -------- stage x: issue this thread's x loads, then the first weight
+    // units, so both are in flight together. x is kept raw (BF16) in shared
+    // memory while the per-token amax is reduced, then widened in place.
+    constexpr int XB = 8;  // x chunks (16 bytes) per thread per batch
+    const int xchunks = a.M * (a.K / 8);
+    const int kc = a.K / 8;  // chunks per row
+    unsigned* row_amax = reinterpret_cast<unsigned*>(shift);  // reused before shift is set
+    if (threadIdx.x < 8) row_amax[threadIdx.x] = 0u;
+    uint4 xb[XB];
+#pragma unroll
+    for (int j = 0; j < XB; ++j) {
+        const int c = threadIdx.x + THREADS * j;
+        xb[j] = c < xchunks ? *reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(c) * 8)
+                            : make_uint4(0, 0, 0, 0);
+    }
     uint4 ra[DEPTH], rb[DEPTH];
     auto load_unit = [&](int u, uint4& A, uint4& B) {
         A = make_uint4(0, 0, 0, 0);
@@ -155,38 +169,49 @@ __global__ void __launch_bounds__(THREADS, 1) w8a16_kernel(const Args a) {
     };
 #pragma unroll
     for (int d = 0; d < DEPTH; ++d) load_unit(d, ra[d], rb[d]);
-
-    // -------- per-token power-of-two shift so amax lands in [2^14, 2^15)
-    if (warp < 8) {
-        float amax = 0.0f;
-        if (warp < a.M) {
-            const __nv_bfloat16* xr = a.x + static_cast<size_t>(warp) * a.K;
-            for (int k = lane * 8; k < a.K; k += 256) {
-                const uint4 c = *reinterpret_cast<const uint4*>(xr + k);
-                const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+    __syncthreads();  // row_amax cleared
+    for (int j0 = 0; j0 * THREADS < xchunks; j0 += XB) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(wv[i])), fabsf(bf16_hi(wv[i]))));
+        for (int j = 0; j < XB; ++j) {
+            const int c = threadIdx.x + THREADS * (j0 + j);
+            if (j0 > 0)
+                xb[j] = c < xchunks ? *reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(c) * 8)
+                                    : make_uint4(0, 0, 0, 0);
+            const int m = c < xchunks ? c / kc : -1;
+            const uint32_t wv[4] = {xb[j].x, xb[j].y, xb[j].z, xb[j].w};
+            float ca = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ca = fmaxf(ca, fmaxf(fabsf(bf16_lo(wv[i])), fabsf(bf16_hi(wv[i]))));
+            const unsigned peers = __match_any_sync(0xffffffffu, m);
+            const unsigned mx = __reduce_max_sync(peers, __float_as_uint(ca));
+            if (m >= 0) {
+                if ((peers & ((1u << lane) - 1u)) == 0) atomicMax(&row_amax[m], mx);
+                const int k = (c - m * kc) * 8;
+                uint2* dst = reinterpret_cast<uint2*>(xs + m * xpitch + 2 * k);
+                dst[0] = make_uint2(xb[j].x, xb[j].y);
+                dst[1] = make_uint2(xb[j].z, xb[j].w);
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        }
-        if (lane == 0) {
-            const int sh = amax > 0.0f ? 14 - ilogbf(amax) : 0;
-            shift[warp] = sh;
-            unshift[warp] = ldexpf(1.0f, -sh);
         }
     }
     __syncthreads();
-    // -------- stage x as FP16 rows (rows >= M are zero)
-    for (int i = threadIdx.x * 8; i < 8 * a.K; i += THREADS * 8) {
-        const int m = i / a.K;
-        const int k = i - m * a.K;
+    // per-token power-of-two shift so amax lands in [2^14, 2^15)
+    if (threadIdx.x < 8) {
+        const float amax = __uint_as_float(row_amax[threadIdx.x]);
+        const int sh = amax > 0.0f ? 14 - ilogbf(amax) : 0;
+        shift[threadIdx.x] = sh;
+        unshift[threadIdx.x] = ldexpf(1.0f, -sh);
+    }
+    __syncthreads();
+    // widen in place to FP16 (rows >= M are zero)
+    for (int c = threadIdx.x; c < 8 * kc; c += THREADS) {
+        const int m = c / kc;
+        const int k = (c - m * kc) * 8;
+        uint2* p = reinterpret_cast<uint2*>(xs + m * xpitch + 2 * k);
         uint4 out = make_uint4(0, 0, 0, 0);
         if (m < a.M) {
-            const uint4 c = *reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * a.K + k);
+            const uint2 lo = p[0], hi = p[1];
             const int sh = shift[m];
-            const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+            const uint32_t wv[4] = {lo.x, lo.y, hi.x, hi.y};
             float f[8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -208,10 +233,8 @@ __global__ void __launch_bounds__(THREADS, 1) w8a16_kernel(const Args a) {
             for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(f[2 * j], f[2 * j + 1]);
             out = *reinterpret_cast<uint4*>(h);
         }
-        // the row pitch is 8 mod 16 bytes: two 8-byte stores
-        uint2* dst = reinterpret_cast<uint2*>(xs + m * xpitch + 2 * k);
-        dst[0] = make_uint2(out.x, out.y);
-        dst[1] = make_uint2(out.z, out.w);
+        p[0] = make_uint2(out.x, out.y);
+        p[1] = make_uint2(out.z, out.w);
     }
     __syncthreads();
 

@@ -175,3 +175,26 @@ def test_linear_dispatch(metis):
     metis.metis_linear(bf16_dev(d["x"]), wq, s_w, y2, fast_math=True)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("variant", [0, 1, 2])
+def test_w8a16_all_subnormal_codes_exact(metis, variant):
+    """Every weight code is an E4M3 subnormal (+-m * 2^-9) and x holds small
+    integers, so every product and partial sum is exact in FP32: the output
+    must equal the oracle's BF16 bits. A widening or a tensor core that
+    flushed FP16 subnormals would return zeros here."""
+    rng = np.random.default_rng(8)
+    M, N, K = 8, 64, 256
+    codes = (rng.integers(1, 8, (N, K)) | (rng.integers(0, 2, (N, K)) << 7)).astype(np.uint8)
+    x = synth.f32_to_bf16_bits(rng.integers(-4, 5, (M, K)).astype(np.float32))
+    s_w = np.ones(N, np.float32)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    old = metis.metis_internal_w8a16_variant(variant)
+    try:
+        metis.metis_w8a16_gemm(bf16_dev(x), dev(codes), dev(s_w), y)
+        torch.cuda.synchronize()
+    finally:
+        metis.metis_internal_w8a16_variant(old)
+    yr, _ = oracle.gemm_w8a16(x, codes, s_w)
+    assert np.any(yr != 0)
+    assert_bytes_equal(bf16_host(y), yr, f"w8a16 v{variant} subnormal codes")
