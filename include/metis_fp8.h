@@ -160,6 +160,28 @@ METIS_API int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* topk
                                void* y_bf16, void* workspace, size_t ws_bytes,
                                metis_stream_t stream);
 
+/* Allocation-free form of metis_moe_fp8_grouped_gemm (the model cards have
+ * no counterpart: this entry point exists for callers, not for the method).
+ * Meant for callers that cannot allocate device memory themselves, such as a
+ * host program running inside an engine that planned all GPU memory up front,
+ * or a plugin given device pointers but no allocator. It takes the same inputs
+ * and output but no workspace: its scratch is a 16 MiB array built into the
+ * library, which each GPU that loads the library keeps until the process exits.
+ *   - Problems whose metis_workspace_size(METIS_OP_MOE, ...) exceeds 16 MiB are
+ *     rejected with METIS_ERR_INVALID_ARG before anything is launched (about
+ *     200 tokens at top-8 with H = 2048, I = 1024).
+ *   - The first call on each device looks up the array's device address; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents (nothing in it needs to start at zero). Calls that may
+ *     overlap on the GPU, e.g. on two streams, race on it: serialise them. */
+METIS_API int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int32_t* topk_ids,
+                                                 const float* topk_w, int64_t T, int64_t topk,
+                                                 int64_t E, int64_t H, int64_t I,
+                                                 const uint8_t* w_up, const float* s_up,
+                                                 const uint8_t* w_down, const float* s_down,
+                                                 int act, void* y_bf16, metis_stream_t stream);
+
 /* Workspace sizes in bytes.
  *   METIS_OP_FP8_GEMM_FUSED: (M, N, K) of metis_fp8_gemm with a_kind = METIS_A_BF16.
  *   METIS_OP_MOE:            (T, I, H, topk, E) of metis_moe_fp8_grouped_gemm.

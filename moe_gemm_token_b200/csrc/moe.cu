@@ -14,6 +14,8 @@
 //   6. per-row re-quantization of h
 //   7. grouped down-projection
 //   8. weighted un-permute y[t] = sum_j w[t,j] * o[row(t,j)], FP32, j ascending.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace metis {
@@ -265,4 +267,69 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
         o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
         static_cast<__nv_bfloat16*>(y_bf16));
     return cuda_check(cudaGetLastError(), "moe combine launch");
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the routed-expert entry point.
+//
+// Some callers cannot allocate device memory on their own: a host program
+// that runs inside an engine which planned all of the GPU's memory when it
+// loaded, or a plugin handed device pointers but no allocator, and callers
+// for whom a cudaMalloc (which can synchronise the whole device) would stall
+// other work. metis_moe_fp8_grouped_gemm_noalloc serves them from a fixed
+// scratch array that lives in this file, so they pass only inputs and
+// outputs. Its capacity is kMoeStaticScratchBytes; every GPU that loads the
+// library keeps that much device memory until the process exits.
+//
+// The array's name is meaningful to device code only: on the host it is a
+// stand-in, so its device address is looked up once per device with
+// cudaGetSymbolAddress (on the first call on that device, with the device
+// current) and that address is what the kernels receive.
+namespace metis {
+namespace {
+constexpr size_t kMoeStaticScratchBytes = static_cast<size_t>(16) << 20;  // 16 MiB
+static __device__ __align__(256) uint8_t g_moe_static_scratch[kMoeStaticScratchBytes];
+
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_ptr[64];
+
+int static_scratch_address(void** out) {
+    int dev = 0;
+    int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+    if (rc) return rc;
+    if (dev < 0 || dev >= 64) return fail(METIS_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lk(g_static_scratch_mu);
+    if (!g_static_scratch_ptr[dev]) {
+        void* p = nullptr;
+        rc = cuda_check(cudaGetSymbolAddress(&p, g_moe_static_scratch),
+                        "cudaGetSymbolAddress(static MoE scratch)");
+        if (rc) return rc;
+        g_static_scratch_ptr[dev] = p;
+    }
+    *out = g_static_scratch_ptr[dev];
+    return METIS_OK;
+}
+}  // namespace
+}  // namespace metis
+
+extern "C" int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int32_t* topk_ids,
+                                                  const float* topk_w, int64_t T, int64_t topk,
+                                                  int64_t E, int64_t H, int64_t I,
+                                                  const uint8_t* w_up, const float* s_up,
+                                                  const uint8_t* w_down, const float* s_down,
+                                                  int act, void* y_bf16, metis_stream_t stream) {
+    clear_error();
+    if (T == 0) return METIS_OK;
+    const size_t need = metis_workspace_size(METIS_OP_MOE, T, I, H, topk, E);
+    if (need > kMoeStaticScratchBytes)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "moe_noalloc: this problem needs %zu bytes of scratch but the built-in array "
+                    "holds %zu (16 MiB); use metis_moe_fp8_grouped_gemm with a caller workspace",
+                    need, kMoeStaticScratchBytes);
+    void* scratch = nullptr;
+    int rc = static_scratch_address(&scratch);
+    if (rc) return rc;
+    return metis_moe_fp8_grouped_gemm(x_bf16, topk_ids, topk_w, T, topk, E, H, I, w_up, s_up,
+                                      w_down, s_down, act, y_bf16, scratch,
+                                      kMoeStaticScratchBytes, stream);
 }

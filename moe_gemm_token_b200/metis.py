@@ -65,6 +65,8 @@ def load():
         "metis_w8a16_gemm": ([p, p, p, p, i64, i64, i64, p], i32),
         "metis_moe_fp8_grouped_gemm": ([p, p, p, i64, i64, i64, i64, i64, p, p, p, p, i32, p, p,
                                         sz, p], i32),
+        "metis_moe_fp8_grouped_gemm_noalloc": ([p, p, p, i64, i64, i64, i64, i64, p, p, p, p,
+                                                i32, p, p], i32),
         "metis_workspace_size": ([i32, i64, i64, i64, i64, i64], sz),
         "metis_moe_workspace_offset": ([i32, i64, i64, i64, i64, i64], i64),
         "metis_linear": ([p, p, p, p, i64, i64, i64, i32, p, p, sz, p], i32),
@@ -159,6 +161,18 @@ def metis_moe_fp8_grouped_gemm(x, topk_ids, topk_w, w_up, s_up, w_down, s_down, 
     return _check("metis_moe_fp8_grouped_gemm", load().metis_moe_fp8_grouped_gemm(
         _p(x), _p(topk_ids), _p(topk_w), T, topk, E, H, I, _p(w_up), _p(s_up), _p(w_down),
         _p(s_down), int(act), _p(y), _p(workspace), ws_bytes, _s(stream)))
+
+
+def metis_moe_fp8_grouped_gemm_noalloc(x, topk_ids, topk_w, w_up, s_up, w_down, s_down, y,
+                                       act=METIS_ACT_NONE, stream=None):
+    """Routed-expert W8A8 layer without a caller workspace (built-in 16 MiB scratch)."""
+    T, H = x.shape
+    topk = topk_ids.shape[1]
+    E, I, H2 = w_up.shape
+    assert H2 == H
+    return _check("metis_moe_fp8_grouped_gemm_noalloc", load().metis_moe_fp8_grouped_gemm_noalloc(
+        _p(x), _p(topk_ids), _p(topk_w), T, topk, E, H, I, _p(w_up), _p(s_up), _p(w_down),
+        _p(s_down), int(act), _p(y), _s(stream)))
 
 
 def metis_workspace_size(op, m_or_t, n_or_i, k_or_h, topk=0, num_experts=0):
