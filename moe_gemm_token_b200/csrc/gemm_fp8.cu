@@ -6,90 +6,100 @@
 // token and multiplied with the FP8 weights on FP8 tensor cores; "What is in
 // FP8": one scale per output channel).
 //
-// One persistent CTA per SM, 192 threads, warp-specialised:
-//   warp 0      TMA producer: 128x128-byte A tiles and 256x128-byte B tiles,
-//               128-byte swizzle, into a 4-stage shared-memory ring;
-//   warp 1      allocates 512 TMEM columns; lane 0 issues tcgen05.mma
-//               (kind::f8f6f4, M=128, N=256, K=32) and commits to mbarriers;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
-//               output row per thread), scale, round to BF16, store.
-// The accumulator is double-buffered in TMEM (2 x 256 columns), so the
-// epilogue of tile i overlaps the main loop of tile i+1.
-//
-// The same kernel runs the grouped GEMM of the routed experts: rows of A are
-// grouped by expert (offsets[e] .. offsets[e+1]), B is [E * N, K] and the
-// scale of output channel n of expert e is s_b[e * N + n]. The tile schedule
-// is built on the device from the offsets, so no host synchronisation.
-//
-// Every mbarrier wait is bounded by the device watchdog: on a timeout the
-// CTA sets the sticky error word, stops issuing work, drains what it issued,
+// Persistent, warp-specialised, 192 threads per CTA:
+//   warp 0      TMA producer into a shared-memory ring (128-byte swizzle);
+//   warp 1      allocates 512 TMEM columns (two 256-column accumulators); one
+//               lane issues tcgen05.mma kind::f8f6f4 and commits to mbarriers;
+//   warps 2..5  epilogue: per-channel scales staged in shared memory once per
+//               tile, tcgen05.ld software-pipelined, the accumulator released
+//               as soon as it is read, scaled BF16 rows staged per warp in a
+//               swizzled 32x32 block and written out as full 64-byte row pieces.
+// Two variants:
+//   CTAS = 2  a CTA pair (cluster of 2) computes a 256 x 256 tile with
+//             tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A
+//             and 128 rows of B (16 + 16 KB per 128-deep k-block, 6 stages),
+//             so each SM streams half of the B tile it would need alone. Both
+//             CTAs' TMA loads complete on the even CTA's mbarrier; its MMA
+//             commits are multicast to both CTAs. Dense GEMMs with M > 128.
+//   CTAS = 1  one CTA computes 128 x 256 (4 stages of 16 + 32 KB). Used for
+//             the grouped GEMM of the routed experts (rows of A grouped by
+//             expert, B = [E * N, K], tile schedule built on the device from
+//             the expert offsets) and for small M.
+// Every mbarrier wait is bounded by the device watchdog: on a timeout the CTA
+// sets the sticky error word, stops issuing work, drains what it issued,
 // frees TMEM and returns.
 #include "common.cuh"
 
 namespace metis {
 namespace gemm {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 128;  // bytes = E4M3 elements per stage
-constexpr int STAGES = 4;
-constexpr int A_STAGE = BM * BK;
-constexpr int B_STAGE = BN * BK;
+constexpr int BK = 128;    // bytes = E4M3 elements per k-block
+constexpr int BN = 256;    // output columns per tile
+constexpr int ROWS = 128;  // output rows per CTA per tile (TMEM lanes)
 constexpr int THREADS = 192;
-constexpr int EPI_THREADS = 128;
+constexpr int EPI_WARPS = 4;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int MAX_GROUPS = 1024;
-constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
 
-// barriers: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
-constexpr int NUM_BARS = 2 * STAGES + 5;
-constexpr size_t SMEM_TILES = static_cast<size_t>(STAGES) * (A_STAGE + B_STAGE);
-constexpr size_t SMEM_BYTES_DENSE = 1024 + SMEM_TILES + NUM_BARS * 8 + 16;
-constexpr size_t SMEM_BYTES_GROUPED = SMEM_BYTES_DENSE + 2 * (MAX_GROUPS + 1) * 4;
+template <int CTAS>
+struct Layout {
+    static constexpr int STAGES = CTAS == 2 ? 6 : 4;
+    static constexpr int B_ROWS = BN / CTAS;   // rows of B loaded by one CTA
+    static constexpr int A_STAGE = ROWS * BK;
+    static constexpr int B_STAGE = B_ROWS * BK;
+    static constexpr int TILES = STAGES * (A_STAGE + B_STAGE);
+    static constexpr int STAGING = EPI_WARPS * 32 * 64;  // a 32 x 32 BF16 block per epilogue warp
+    static constexpr int SW = 2 * BN * 4;                // per-channel scales, double-buffered
+    // full, empty, tfull[2], tempty[2], drain, epilogue sync[2]
+    static constexpr int NUM_BARS = 2 * STAGES + 7;
+    static constexpr int BAR_OFF = TILES + STAGING + SW;
+    static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+    static constexpr int GROUP_OFF = MISC_OFF + 16;
+    static constexpr size_t BYTES_DENSE = 1024 + GROUP_OFF;
+    static constexpr size_t BYTES_GROUPED = BYTES_DENSE + 2 * (MAX_GROUPS + 1) * 4;
+    static constexpr uint32_t IDESC = idesc_e4m3_f32(ROWS * CTAS, BN);
+};
 
 struct Params {
-    const float* s_a;       // [rows of A]
-    const float* s_b;       // [groups * N]
-    __nv_bfloat16* y;       // [rows of A, N]
-    const int32_t* offsets; // grouped: [E + 1] row offsets into A; dense: null
-    int M;                  // dense: rows of A
-    int N;                  // output columns (per group)
+    const float* s_a;        // [rows of A]
+    const float* s_b;        // [groups * N]
+    __nv_bfloat16* y;        // [rows of A, N]
+    const int32_t* offsets;  // grouped: [E + 1] row offsets into A; dense: null
+    int M;                   // dense: rows of A
+    int N;                   // output columns (per group)
     int K;
-    int E;                  // groups (1 for dense)
+    int E;                   // groups (1 for dense)
     uint32_t* status;
     uint64_t timeout_ns;
 };
 
 struct Tile {
-    int a_row0;   // first row of A (and y) of this tile
+    int a_row0;   // first row of A (and y) of this CTA's part of the tile
     int row_end;  // rows >= row_end belong to another group (or are past M)
-    int b_row0;   // first row of B
+    int b_row0;   // first row of B loaded by this CTA
     int n0;       // first output column
     int group;
 };
 
+template <int CTAS>
 struct Sched {
-    int num_n;
-    int num_m;          // dense only
-    int total;
+    int num_n, num_m, total, E, N, M;
+    uint32_t rank;
     const int* g_tile;  // grouped: prefix sums of tiles per group [E + 1] (smem)
     const int* g_row;   // grouped: row offsets [E + 1] (smem)
-    int E;
-    int N;
-    int M;
 
     __device__ __forceinline__ Tile get(int t) const {
         Tile ti;
         if (g_tile == nullptr) {
             const int mb = t % num_m;
             const int nb = t / num_m;
-            ti.a_row0 = mb * BM;
+            ti.a_row0 = mb * ROWS * CTAS + static_cast<int>(rank) * ROWS;
             ti.row_end = M;
-            ti.b_row0 = nb * BN;
+            ti.b_row0 = nb * BN + static_cast<int>(rank) * (BN / CTAS);
             ti.n0 = nb * BN;
             ti.group = 0;
         } else {
-            int lo = 0, hi = E;  // find e with g_tile[e] <= t < g_tile[e + 1]
+            int lo = 0, hi = E;  // e with g_tile[e] <= t < g_tile[e + 1]
             while (hi - lo > 1) {
                 const int mid = (lo + hi) >> 1;
                 if (g_tile[mid] <= t) lo = mid; else hi = mid;
@@ -97,10 +107,10 @@ struct Sched {
             const int e = lo;
             const int local = t - g_tile[e];
             const int rows = g_row[e + 1] - g_row[e];
-            const int mt = (rows + BM - 1) / BM;
+            const int mt = (rows + ROWS - 1) / ROWS;
             const int mb = local % mt;
             const int nb = local / mt;
-            ti.a_row0 = g_row[e] + mb * BM;
+            ti.a_row0 = g_row[e] + mb * ROWS;
             ti.row_end = g_row[e + 1];
             ti.b_row0 = e * N + nb * BN;
             ti.n0 = nb * BN;
@@ -114,27 +124,66 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <bool GROUPED>
+// One 32-column chunk of the epilogue: scale, round, stage in the warp's
+// swizzled block (16-byte pieces of each 64-byte row XOR-ed with (row>>1)&3,
+// so both the row-wise writes and the piece-wise reads are conflict-free),
+// then write 8 rows x 64 bytes per instruction.
+__device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, const Tile& ti, int q,
+                                            int lane, float rs, const float* sw,
+                                            uint8_t* stg, __nv_bfloat16* y, int N) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float lo = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * j]), rs), sw[c * 32 + 2 * j]);
+        const float hi = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * j + 1]), rs), sw[c * 32 + 2 * j + 1]);
+        pk[j] = pack_bf16x2(lo, hi);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int pc = 0; pc < 4; ++pc)
+        *reinterpret_cast<uint4*>(stg + lane * 64 + ((pc ^ ((lane >> 1) & 3)) * 16)) =
+            make_uint4(pk[4 * pc], pk[4 * pc + 1], pk[4 * pc + 2], pk[4 * pc + 3]);
+    __syncwarp();
+    const int n = ti.n0 + c * 32 + (lane & 3) * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int rr = (lane >> 2) + 8 * i;
+        const uint4 val =
+            *reinterpret_cast<const uint4*>(stg + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
+        const int row = ti.a_row0 + q * 32 + rr;
+        if (row < ti.row_end && n < N)
+            *reinterpret_cast<uint4*>(y + static_cast<size_t>(row) * N + n) = val;
+    }
+}
+
+template <int CTAS, bool GROUPED>
 __global__ void __launch_bounds__(THREADS, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
+    using L = Layout<CTAS>;
+    constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sA = smem;
-    uint8_t* sB = smem + STAGES * A_STAGE;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_TILES);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* g_tile = reinterpret_cast<int*>(tmem_slot + 4);
+    uint8_t* sB = smem + STAGES * L::A_STAGE;
+    uint8_t* staging = smem + L::TILES;
+    float* sw_smem = reinterpret_cast<float*>(smem + L::TILES + L::STAGING);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+    int* g_tile = reinterpret_cast<int*>(smem + L::GROUP_OFF);
     int* g_row = g_tile + (MAX_GROUPS + 1);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
+    const uint32_t rank = CTAS == 2 ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
     auto full = [&](int s) { return smem_u32(&bars[s]); };
     auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
     auto tfull = [&](int b) { return smem_u32(&bars[2 * STAGES + b]); };
     auto tempty = [&](int b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
     const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
+    auto epi_sync = [&](int b) { return smem_u32(&bars[2 * STAGES + 5 + b]); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -143,23 +192,31 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull(b), 1);
-            mbar_init(tempty(b), EPI_THREADS);
+            mbar_init(tempty(b), CTAS * EPI_WARPS);
         }
         mbar_init(drain, 1);
+        mbar_init(epi_sync(0), EPI_WARPS * 32);
+        mbar_init(epi_sync(1), EPI_WARPS * 32);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (CTAS == 2) {
+            tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+            tmem_relinquish();
+        }
     }
 
-    Sched sc;
+    Sched<CTAS> sc;
     sc.N = p.N;
     sc.M = p.M;
     sc.E = p.E;
+    sc.rank = rank;
     sc.num_n = (p.N + BN - 1) / BN;
     if constexpr (GROUPED) {
         // prefix sums of row offsets and of tiles per group, by warp 0
@@ -171,7 +228,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const int e = g0 + i;
                 if (e < p.E) {
                     const int rows = p.offsets[e + 1] - p.offsets[e];
-                    local += ((rows + BM - 1) / BM) * sc.num_n;
+                    local += ((rows + ROWS - 1) / ROWS) * sc.num_n;
                 }
             }
             int incl = local;
@@ -187,7 +244,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     const int rows = p.offsets[e + 1] - p.offsets[e];
                     g_tile[e] = run;
                     g_row[e] = p.offsets[e];
-                    run += ((rows + BM - 1) / BM) * sc.num_n;
+                    run += ((rows + ROWS - 1) / ROWS) * sc.num_n;
                 }
             }
             if (lane == 31) {
@@ -201,33 +258,42 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     } else {
         sc.g_tile = nullptr;
         sc.g_row = nullptr;
-        sc.num_m = (p.M + BM - 1) / BM;
+        sc.num_m = (p.M + ROWS * CTAS - 1) / (ROWS * CTAS);
         sc.total = sc.num_m * sc.num_n;
     }
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CTAS == 2) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     if constexpr (GROUPED) sc.total = g_tile[p.E];
     const uint32_t tmem_base = *tmem_slot;
     const int num_kb = (p.K + BK - 1) / BK;
+    const int first = CTAS == 2 ? static_cast<int>(blockIdx.x / 2) : static_cast<int>(blockIdx.x);
+    const int stride = CTAS == 2 ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------------------- producer
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued = 0;  // bit s: stage s has a load whose completion is unobserved
-            uint32_t issued_phase = 0;
-            for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+            uint32_t issued = 0, issued_phase = 0;
+            for (int t = first; t < sc.total && !*abort_flag; t += stride) {
                 const Tile ti = sc.get(t);
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(empty(stage), phase ^ 1u, p.timeout_ns, p.status)) {
                         *abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(full(stage), A_STAGE + B_STAGE);
-                    tma_load_2d(smem_u32(sA + stage * A_STAGE), &tmA, kb * BK, ti.a_row0, full(stage));
-                    tma_load_2d(smem_u32(sB + stage * B_STAGE), &tmB, kb * BK, ti.b_row0, full(stage));
+                    if constexpr (CTAS == 2) {
+                        const uint32_t fl = mapa_shared(full(stage), 0);
+                        if (leader) mbar_arrive_expect_tx(full(stage), CTAS * (L::A_STAGE + L::B_STAGE));
+                        tma_load_2d_pair(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * BK, ti.a_row0, fl);
+                        tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * BK, ti.b_row0, fl);
+                    } else {
+                        mbar_arrive_expect_tx(full(stage), L::A_STAGE + L::B_STAGE);
+                        tma_load_2d(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * BK, ti.a_row0, full(stage));
+                        tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * BK, ti.b_row0, full(stage));
+                    }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -235,19 +301,24 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             }
             if (*abort_flag) {
                 // let the copies in flight land before the CTA exits
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued & (1u << s))
-                        mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
+                if (leader) {
+                    for (int s = 0; s < STAGES; ++s)
+                        if (issued & (1u << s))
+                            mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
+                } else {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 100000ull) {}
+                }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             // --------------------------------------------------------- MMA issuer
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+            for (int t = first; t < sc.total && !*abort_flag; t += stride) {
                 if (!mbar_wait(tempty(acc), acc_phase ^ 1u, p.timeout_ns, p.status)) {
                     *abort_flag = 1;
                     break;
@@ -261,104 +332,140 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * A_STAGE));
-                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * B_STAGE));
+                    const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * L::A_STAGE));
+                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * L::B_STAGE));
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) {
                         // advance 32 bytes along K inside the swizzled 128-byte rows
-                        mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC,
-                                   (kb > 0 || k > 0) ? 1u : 0u);
+                        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                        if constexpr (CTAS == 2)
+                            mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
+                        else
+                            mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
                     }
-                    mma_commit(empty(stage));
+                    if constexpr (CTAS == 2) mma_commit_pair_mc(empty(stage), 0x3);
+                    else mma_commit(empty(stage));
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) {
                     *abort_flag = 1;
                     break;
                 }
-                mma_commit(tfull(acc));
+                if constexpr (CTAS == 2) mma_commit_pair_mc(tfull(acc), 0x3);
+                else mma_commit(tfull(acc));
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             }
             // all MMAs issued by this thread complete before TMEM is released
-            mma_commit(drain);
+            if constexpr (CTAS == 2) mma_commit_pair(drain);
+            else mma_commit(drain);
             mbar_wait(drain, 0, p.timeout_ns, p.status);
         }
     } else {
         // -------------------------------------------------------------- epilogue
-        const int q = warp & 3;  // TMEM lane quadrant this warp may access
-        const int r = q * 32 + lane;
+        const int q = warp & 3;        // TMEM lane quadrant this warp may access
+        const int et = threadIdx.x - 64;  // 0..127
+        uint8_t* stg = staging + (warp - 2) * (32 * 64);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+        for (int t = first; t < sc.total && !*abort_flag; t += stride) {
             const Tile ti = sc.get(t);
-            if (!mbar_wait(tfull(acc), acc_phase, p.timeout_ns, p.status)) {
+            // per-channel scales of this tile into shared memory
+            {
+                const float* sb = p.s_b + static_cast<size_t>(ti.group) * p.N;
+                const int n = ti.n0 + 2 * et;
+                const float2 v = n < p.N ? *reinterpret_cast<const float2*>(sb + n) : make_float2(0.f, 0.f);
+                reinterpret_cast<float2*>(sw_smem + acc * BN)[et] = v;
+            }
+            const int row = ti.a_row0 + q * 32 + lane;
+            const float rs = row < ti.row_end ? p.s_a[row] : 0.0f;
+            // all epilogue threads have written their scales (bounded wait)
+            mbar_arrive(epi_sync(acc));
+            if (!mbar_wait(epi_sync(acc), acc_phase, p.timeout_ns, p.status) ||
+                !mbar_wait(tfull(acc), acc_phase, p.timeout_ns, p.status)) {
                 *abort_flag = 1;
                 break;
             }
             tc_fence_after();
-            const int row = ti.a_row0 + r;
-            const bool row_ok = row < ti.row_end;
-            const float rs = row_ok ? p.s_a[row] : 0.0f;
-            const float* sb = p.s_b + static_cast<size_t>(ti.group) * p.N;
-            __nv_bfloat16* yrow = p.y + static_cast<size_t>(row_ok ? row : 0) * p.N;
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                       static_cast<uint32_t>(acc * BN + c),
-                                   v);
+            const float* sw = sw_smem + acc * BN;
+            const uint32_t tbase =
+                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+            uint32_t va[32], vb[32];
+            tmem_ld_32x32b_x32(tbase, va);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < BN / 32; c += 2) {
+                tmem_ld_32x32b_x32(tbase + (c + 1) * 32, vb);
+                store_chunk(va, c, ti, q, lane, rs, sw, stg, p.y, p.N);
                 tmem_ld_wait();
-                const int n = ti.n0 + c;
-                if (row_ok) {
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int ng = n + 8 * g;
-                        if (ng < p.N) {
-                            const float4 s0 = __ldg(reinterpret_cast<const float4*>(sb + ng));
-                            const float4 s1 = __ldg(reinterpret_cast<const float4*>(sb + ng + 4));
-                            const float f[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-                            uint32_t o[4];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float lo = __fmul_rn(__fmul_rn(__uint_as_float(v[8 * g + 2 * j]), rs), f[2 * j]);
-                                const float hi = __fmul_rn(__fmul_rn(__uint_as_float(v[8 * g + 2 * j + 1]), rs), f[2 * j + 1]);
-                                o[j] = pack_bf16x2(lo, hi);
-                            }
-                            *reinterpret_cast<uint4*>(yrow + ng) = make_uint4(o[0], o[1], o[2], o[3]);
-                        }
+                if (c + 2 < BN / 32) {
+                    tmem_ld_32x32b_x32(tbase + (c + 2) * 32, va);
+                } else {
+                    // every column of this accumulator has been read: release it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (CTAS == 2) mbar_arrive_cluster(mapa_shared(tempty(acc), 0));
+                        else mbar_arrive(tempty(acc));
                     }
                 }
+                store_chunk(vb, c + 1, ti, q, lane, rs, sw, stg, p.y, p.N);
+                if (c + 2 < BN / 32) tmem_ld_wait();
             }
-            tc_fence_before();
-            mbar_arrive(tempty(acc));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
     }
 
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CTAS == 2) cluster_sync_all(); else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        if constexpr (CTAS == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 
-// Per-device one-time opt-in to the large dynamic shared memory.
-int prepare(const DeviceInfo& di, bool grouped) {
-    static bool done[64][2];
-    const size_t need = grouped ? SMEM_BYTES_GROUPED : SMEM_BYTES_DENSE;
-    if (static_cast<size_t>(di.max_smem_optin) < need)
-        return fail(METIS_ERR_UNSUPPORTED, "fp8 gemm needs %zu bytes of shared memory", need);
-    if (!done[di.device][grouped]) {
-        cudaError_t e = grouped
-            ? cudaFuncSetAttribute(fp8_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need)
-            : cudaFuncSetAttribute(fp8_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need);
-        int rc = cuda_check(e, "cudaFuncSetAttribute(fp8 gemm)");
+template <int CTAS, bool GROUPED>
+int prepare(const DeviceInfo& di, size_t smem) {
+    static bool done[64];
+    if (static_cast<size_t>(di.max_smem_optin) < smem)
+        return fail(METIS_ERR_UNSUPPORTED, "fp8 gemm needs %zu bytes of shared memory", smem);
+    if (!done[di.device]) {
+        int rc = cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem)),
+                            "cudaFuncSetAttribute(fp8 gemm)");
         if (rc) return rc;
-        done[di.device][grouped] = true;
+        done[di.device] = true;
     }
+    return METIS_OK;
+}
+
+// Co-resident CTA pairs of the 2-CTA kernel (cached per device).
+int max_pairs(const DeviceInfo& di, int* out) {
+    static int cached[64];
+    if (!cached[di.device]) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (di.num_sms / 2), 1, 1);
+        cfg.blockDim = dim3(THREADS, 1, 1);
+        cfg.dynamicSmemBytes = Layout<2>::BYTES_DENSE;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, false>, &cfg),
+                            "cudaOccupancyMaxActiveClusters");
+        if (rc) return rc;
+        if (n < 1) return fail(METIS_ERR_UNSUPPORTED, "no CTA pair of the fp8 gemm fits an SM pair");
+        cached[di.device] = n;
+    }
+    *out = cached[di.device];
     return METIS_OK;
 }
 
@@ -371,16 +478,41 @@ int launch_fp8_gemm_dense(const uint8_t* a, const float* s_a, const uint8_t* b, 
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
-    if ((rc = prepare(di, false))) return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
-    CUtensorMap ta, tb;
-    if ((rc = make_tmap_2d(&ta, a, 1, K, M, K, BK, BM, true))) return rc;
-    if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, BN, true))) return rc;
     Params p{s_a, s_b, y, nullptr, M, N, K, 1, status, watchdog_ns()};
-    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int num_n = (N + BN - 1) / BN;
+    CUtensorMap ta, tb;
+    if ((rc = make_tmap_2d(&ta, a, 1, K, M, K, BK, ROWS, true))) return rc;
+    if (M > ROWS) {
+        using L = Layout<2>;
+        if ((rc = prepare<2, false>(di, L::BYTES_DENSE))) return rc;
+        int pairs = 0;
+        if ((rc = max_pairs(di, &pairs))) return rc;
+        if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
+        const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
+        const int clusters = tiles < pairs ? tiles : pairs;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * clusters, 1, 1);
+        cfg.blockDim = dim3(THREADS, 1, 1);
+        cfg.dynamicSmemBytes = L::BYTES_DENSE;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cuda_check(cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<2, false>, ta, tb, p),
+                          "fp8 gemm (CTA pair) launch");
+    }
+    using L = Layout<1>;
+    if ((rc = prepare<1, false>(di, L::BYTES_DENSE))) return rc;
+    if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
+    const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
-    fp8_gemm_kernel<false><<<grid, THREADS, SMEM_BYTES_DENSE, st>>>(ta, tb, p);
+    fp8_gemm_kernel<1, false><<<grid, THREADS, L::BYTES_DENSE, st>>>(ta, tb, p);
     return cuda_check(cudaGetLastError(), "fp8 gemm launch");
 }
 
@@ -390,18 +522,20 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
                             __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
                             int K, cudaStream_t st) {
     using namespace gemm;
+    using L = Layout<1>;
     if (E > MAX_GROUPS) return fail(METIS_ERR_UNSUPPORTED, "grouped gemm: E=%d > %d", E, MAX_GROUPS);
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
-    if ((rc = prepare(di, true))) return rc;
+    if ((rc = prepare<1, true>(di, L::BYTES_GROUPED))) return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
     CUtensorMap ta, tb;
-    if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, BM, true))) return rc;
-    if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, BN, true))) return rc;
+    if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, ROWS, true))) return rc;
+    if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
+        return rc;
     Params p{s_a, s_b, y, offsets, rows, N, K, E, status, watchdog_ns()};
-    fp8_gemm_kernel<true><<<di.num_sms, THREADS, SMEM_BYTES_GROUPED, st>>>(ta, tb, p);
+    fp8_gemm_kernel<1, true><<<di.num_sms, THREADS, L::BYTES_GROUPED, st>>>(ta, tb, p);
     return cuda_check(cudaGetLastError(), "grouped fp8 gemm launch");
 }
 
