@@ -390,7 +390,8 @@ def run_metis(args):
 
 def secondary_figures(metis, dev, pk):
     """Context figures of the other hot-path kernels (not the headline):
-    decode W8A16 GB/s, quantizer GB/s, large-M W8A8 TFLOP/s, routed experts."""
+    decode W8A16 GB/s, quantizer GB/s, large-M W8A8 TFLOP/s, routed experts.
+    Each is timed by replaying a CUDA graph of many calls."""
     import torch
     g = torch.Generator(device=dev)
     g.manual_seed(7)
@@ -401,16 +402,30 @@ def secondary_figures(metis, dev, pk):
         return c
 
     def timeit(fn, iters):
+        """GPU time per call: `iters` calls captured once in a CUDA graph and
+        replayed, so host-side launch overhead does not enter the figure."""
         for _ in range(5):
             fn()
         torch.cuda.synchronize()
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(graph, stream=stream):
+                for _ in range(iters):
+                    fn()
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
         a.record()
-        for _ in range(iters):
-            fn()
+        for _ in range(reps):
+            graph.replay()
         b.record()
         torch.cuda.synchronize()
-        return a.elapsed_time(b) / iters * 1e-3
+        del graph
+        return a.elapsed_time(b) / (reps * iters) * 1e-3
 
     out = {}
     hbm = pk["hbm_gbs"]

@@ -140,15 +140,15 @@ METIS_API int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const floa
  * the routed experts are FP8 with per-channel scales and per-token
  * activations). Steps, all on the device, no host synchronisation:
  * routing histogram -> exclusive prefix sum -> stable permutation of the
- * slots (t, j) by expert -> per-token quantization of x (once per token) ->
- * gather into expert-contiguous rows -> grouped up-projection (W8A8) ->
+ * slots (t, j) by expert -> per-token quantization of x (once per token,
+ * written into the expert-contiguous rows of its slots) -> grouped up-projection (W8A8) ->
  * per-row re-quantization -> grouped down-projection (W8A8) -> weighted
  * un-permute y[t] = sum_j topk_w[t,j] o[t,j] (FP32, j ascending) -> BF16.
  *   x [T, H] BF16, topk_ids [T, topk] int32 in [0, E), topk_w [T, topk] FP32,
  *   w_up [E, I, H] E4M3, s_up [E, I], w_down [E, H, I] E4M3, s_down [E, H],
  *   y [T, H] BF16 out.
  *   act must be METIS_ACT_NONE (the cards do not state the experts' activation).
- *   Requires H % 16 == 0, I % 16 == 0, H >= 16, I >= 16, 1 <= topk <= E <= 1024;
+ *   Requires H % 16 == 0, I % 16 == 0, 16 <= H <= 16384, I >= 16, 1 <= topk <= E <= 1024;
  *   ids outside [0, E) are a caller error (not checked on the device).
  *   Needs `workspace` of metis_workspace_size(METIS_OP_MOE, T, I, H, topk, E)
  *   bytes (256-byte aligned); its regions are given by metis_moe_workspace_offset. */
@@ -199,10 +199,8 @@ METIS_API size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, in
  *   METIS_MOE_WS_OFFSETS     int32 [E + 1]  exclusive prefix sum of COUNTS
  *   METIS_MOE_WS_SLOT_TO_ROW int32 [S]      row of slot s = t*topk + j in expert order
  *   METIS_MOE_WS_ROW_TO_SLOT int32 [S]      inverse permutation
- *   METIS_MOE_WS_XQ          E4M3  [T, H]   per-token codes of x
- *   METIS_MOE_WS_SX          FP32  [T]      per-token scales of x
- *   METIS_MOE_WS_AQ          E4M3  [S, H]   XQ rows gathered into expert order
- *   METIS_MOE_WS_SA          FP32  [S]      their scales
+ *   METIS_MOE_WS_AQ          E4M3  [S, H]   per-token codes of x, one row per slot, expert order
+ *   METIS_MOE_WS_SA          FP32  [S]      their per-token scales
  *   METIS_MOE_WS_H           BF16  [S, I]   up-projection output, expert order
  *   METIS_MOE_WS_HQ          E4M3  [S, I]   its per-row codes
  *   METIS_MOE_WS_SH          FP32  [S]      their scales
@@ -212,14 +210,12 @@ METIS_API size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, in
 #define METIS_MOE_WS_OFFSETS 1
 #define METIS_MOE_WS_SLOT_TO_ROW 2
 #define METIS_MOE_WS_ROW_TO_SLOT 3
-#define METIS_MOE_WS_XQ 4
-#define METIS_MOE_WS_SX 5
-#define METIS_MOE_WS_AQ 6
-#define METIS_MOE_WS_SA 7
-#define METIS_MOE_WS_H 8
-#define METIS_MOE_WS_HQ 9
-#define METIS_MOE_WS_SH 10
-#define METIS_MOE_WS_O 11
+#define METIS_MOE_WS_AQ 4
+#define METIS_MOE_WS_SA 5
+#define METIS_MOE_WS_H 6
+#define METIS_MOE_WS_HQ 7
+#define METIS_MOE_WS_SH 8
+#define METIS_MOE_WS_O 9
 METIS_API int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk, int64_t E,
                                    int64_t H, int64_t I);
 

@@ -4,12 +4,12 @@
 // token at run time).
 //
 // Device pipeline (no host synchronisation; segment sizes stay on the GPU):
-//   1. per-token quantization of x            (quantizer kernel, once per token)
-//   2. routing histogram per chunk of slots    (shared-memory integer atomics)
-//   3. prefix sums: per-expert offsets and per-(chunk, expert) bases
-//   4. stable scatter: row of slot s = t*topk + j in expert order, via warp
-//      match + per-warp counts (no atomics in the ordering), and gather of
-//      the token's codes and scale into expert-contiguous rows
+//   1. routing histogram per chunk of slots    (shared-memory integer atomics)
+//   2. prefix sums: per-expert offsets and per-(chunk, expert) bases
+//   3. stable ranks: row of slot s = t*topk + j in expert order, via warp
+//      match + per-warp counts (no atomics decide the order)
+//   4. per-token quantization of x, each token once, its codes and scale
+//      written straight into the expert-ordered rows it was routed to
 //   5. grouped up-projection (tcgen05 W8A8 GEMM, tile schedule from offsets)
 //   6. per-row re-quantization of h
 //   7. grouped down-projection
@@ -22,7 +22,7 @@ namespace metis {
 
 template <typename T>
 int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
-                      float* s, cudaStream_t st);
+                      float* s, cudaStream_t st, const int32_t* dst_rows, int topk);
 int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b, const float* s_b,
                             __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
                             int K, cudaStream_t st);
@@ -61,8 +61,17 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
     __shared__ int warp_tot[32];
     const int e = threadIdx.x;
     int total = 0;
-    if (e < E)
-        for (int c = 0; c < C; ++c) total += chunk_counts[static_cast<size_t>(c) * E + e];
+    if (e < E) {
+        int c = 0;
+        for (; c + 8 <= C; c += 8) {
+            int v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = chunk_counts[static_cast<size_t>(c + i) * E + e];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) total += v[i];
+        }
+        for (; c < C; ++c) total += chunk_counts[static_cast<size_t>(c) * E + e];
+    }
     // block-wide exclusive scan of total over e
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int incl = total;
@@ -89,7 +98,18 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
         counts[e] = total;
         offsets[e] = excl;
         int run = excl;
-        for (int c = 0; c < C; ++c) {
+        int c = 0;
+        for (; c + 8 <= C; c += 8) {
+            int v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = chunk_counts[static_cast<size_t>(c + i) * E + e];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                chunk_counts[static_cast<size_t>(c + i) * E + e] = run;
+                run += v[i];
+            }
+        }
+        for (; c < C; ++c) {
             const size_t i = static_cast<size_t>(c) * E + e;
             const int v = chunk_counts[i];
             chunk_counts[i] = run;
@@ -99,16 +119,14 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
     }
 }
 
-// Stable rank of each slot within its expert, then gather of the token's
-// codes into the slot's row.
-__global__ void __launch_bounds__(CHUNK) scatter_gather_kernel(
-    const int32_t* __restrict__ ids, int S, int E, int topk, const int32_t* __restrict__ chunk_base,
-    int32_t* __restrict__ slot_to_row, int32_t* __restrict__ row_to_slot,
-    const uint8_t* __restrict__ xq, const float* __restrict__ sx, int H, uint8_t* __restrict__ aq,
-    float* __restrict__ sa) {
+// Stable rank of each slot within its expert: slots of the chunk are ranked
+// by warp (match + popcount) and then by the per-warp counts of earlier warps.
+__global__ void __launch_bounds__(CHUNK) rank_kernel(const int32_t* __restrict__ ids, int S, int E,
+                                                     const int32_t* __restrict__ chunk_base,
+                                                     int32_t* __restrict__ slot_to_row,
+                                                     int32_t* __restrict__ row_to_slot) {
     constexpr int WARPS = CHUNK / 32;
     __shared__ int wcnt[WARPS][MAX_E];  // per-warp counts, then exclusive prefix over warps
-    __shared__ int rows[CHUNK];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     for (int i = threadIdx.x; i < WARPS * E; i += CHUNK) wcnt[i / E][i % E] = 0;
     __syncthreads();
@@ -116,12 +134,11 @@ __global__ void __launch_bounds__(CHUNK) scatter_gather_kernel(
     int e = s < S ? ids[s] : -1;
     if (e >= E) e = -1;
     const bool ok = e >= 0;
-    if (s < S && !ok) slot_to_row[s] = -1;  // dropped: never read by the combine
+    if (s < S && !ok) slot_to_row[s] = -1;  // dropped: never written or read again
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank_w = __popc(peers & ((1u << lane) - 1u));
     if (ok && rank_w == 0) wcnt[warp][e] = __popc(peers);
     __syncthreads();
-    // exclusive prefix over warps, per expert
     for (int x = threadIdx.x; x < E; x += CHUNK) {
         int run = 0;
         for (int w = 0; w < WARPS; ++w) {
@@ -131,23 +148,10 @@ __global__ void __launch_bounds__(CHUNK) scatter_gather_kernel(
         }
     }
     __syncthreads();
-    int row = -1;
     if (ok) {
-        row = chunk_base[static_cast<size_t>(blockIdx.x) * E + e] + wcnt[warp][e] + rank_w;
+        const int row = chunk_base[static_cast<size_t>(blockIdx.x) * E + e] + wcnt[warp][e] + rank_w;
         slot_to_row[s] = row;
         row_to_slot[row] = s;
-        sa[row] = sx[s / topk];
-    }
-    rows[threadIdx.x] = row;
-    __syncthreads();
-    // gather: each warp copies whole rows, 16 bytes per lane per step
-    const int first = blockIdx.x * CHUNK;
-    for (int i = warp; i < CHUNK; i += WARPS) {
-        const int r = rows[i];
-        if (r < 0) continue;
-        const uint4* src = reinterpret_cast<const uint4*>(xq + static_cast<size_t>((first + i) / topk) * H);
-        uint4* dst = reinterpret_cast<uint4*>(aq + static_cast<size_t>(r) * H);
-        for (int v = lane; v < H / 16; v += 32) dst[v] = src[v];
     }
 }
 
@@ -203,8 +207,9 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     if (T < 0 || topk < 1 || E < topk || E > MAX_E)
         return fail(METIS_ERR_INVALID_ARG, "moe: need T >= 0 and 1 <= topk <= E <= %d (T=%lld topk=%lld E=%lld)",
                     MAX_E, (long long)T, (long long)topk, (long long)E);
-    if (H < 16 || I < 16 || H % 16 || I % 16 || H > (1 << 20) || I > (1 << 20))
-        return fail(METIS_ERR_INVALID_ARG, "moe: need H, I >= 16 and multiples of 16 (H=%lld I=%lld)",
+    if (H < 16 || I < 16 || H % 16 || I % 16 || H > 16384 || I > (1 << 20))
+        return fail(METIS_ERR_INVALID_ARG,
+                    "moe: need 16 <= H <= 16384 and I >= 16, both multiples of 16 (H=%lld I=%lld)",
                     (long long)H, (long long)I);
     const int64_t S = T * topk;
     if (S > (1ll << 30)) return fail(METIS_ERR_INVALID_ARG, "moe: T*topk too large");
@@ -228,8 +233,6 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     int32_t* offsets = reinterpret_cast<int32_t*>(region(METIS_MOE_WS_OFFSETS));
     int32_t* s2r = reinterpret_cast<int32_t*>(region(METIS_MOE_WS_SLOT_TO_ROW));
     int32_t* r2s = reinterpret_cast<int32_t*>(region(METIS_MOE_WS_ROW_TO_SLOT));
-    uint8_t* xq = region(METIS_MOE_WS_XQ);
-    float* sx = reinterpret_cast<float*>(region(METIS_MOE_WS_SX));
     uint8_t* aq = region(METIS_MOE_WS_AQ);
     float* sa = reinterpret_cast<float*>(region(METIS_MOE_WS_SA));
     __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(region(METIS_MOE_WS_H));
@@ -243,22 +246,21 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     if (static_cast<int64_t>(C) * E * 4 > 2 * S * I)
         return fail(METIS_ERR_UNSUPPORTED, "moe: routing table does not fit the workspace (E too large for T*topk*I)");
 
-    if ((rc = launch_quant_rows<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_bf16), T, H, H, xq, H,
-                                               sx, st)))
-        return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
     count_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
                                       status);
     scan_kernel<<<1, 1024, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets);
-    scatter_gather_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E),
-                                               static_cast<int>(topk), chunk_tab, s2r, r2s, xq, sx,
-                                               static_cast<int>(H), aq, sa);
+    rank_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
+                                     s2r, r2s);
     if ((rc = cuda_check(cudaGetLastError(), "moe routing launch"))) return rc;
+    if ((rc = launch_quant_rows<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_bf16), T, H, H, aq, H,
+                                               sa, st, s2r, static_cast<int>(topk))))
+        return rc;
     if ((rc = launch_fp8_gemm_grouped(aq, sa, w_up, s_up, h, offsets, static_cast<int>(E),
                                       static_cast<int>(S), static_cast<int>(I), static_cast<int>(H), st)))
         return rc;
-    if ((rc = launch_quant_rows<__nv_bfloat16>(h, S, I, I, hq, I, sh, st))) return rc;
+    if ((rc = launch_quant_rows<__nv_bfloat16>(h, S, I, I, hq, I, sh, st, nullptr, 1))) return rc;
     if ((rc = launch_fp8_gemm_grouped(hq, sh, w_down, s_down, o, offsets, static_cast<int>(E),
                                       static_cast<int>(S), static_cast<int>(H), static_cast<int>(I), st)))
         return rc;

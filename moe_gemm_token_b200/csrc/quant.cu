@@ -51,11 +51,14 @@ struct Elem<float> {
     }
 };
 
-// Register-resident path: K <= TEAM * NV * EPC.
-template <typename T, int TEAM, int NV>
+// Register-resident path: K <= TEAM * NV * EPC. With SCATTER, row r's codes
+// and scale go to rows dst[r * topk + j] (j < topk; negative entries skipped)
+// instead of row r: the routed-expert path quantizes each token once and
+// writes it straight into the expert-ordered rows it was routed to.
+template <typename T, int TEAM, int NV, bool SCATTER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx, uint8_t* __restrict__ q,
-                  int64_t ldq, float* __restrict__ s) {
+                  int64_t ldq, float* __restrict__ s, const int32_t* __restrict__ dst, int topk) {
     constexpr int EPC = Elem<T>::kPerChunk;
     constexpr int TEAMS = kQuantThreads / TEAM;
     constexpr int WARPS_PER_TEAM = TEAM / 32;
@@ -100,25 +103,35 @@ quant_rows_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx, uint8_
 
     float sc, inv;
     row_scales(amax, &sc, &inv);
-    if (tid == 0) s[row] = sc;
-    uint8_t* qr = q + row * ldq;
+    // this thread's codes: 8 (BF16 input) or 4 (FP32 input) bytes per chunk
+    uint2 out[NV];
 #pragma unroll
     for (int c = 0; c < NV; ++c) {
-        const int e0 = (c * TEAM + tid) * EPC;
-        if (e0 >= K) continue;
         float v[EPC];
         Elem<T>::unpack(buf[c], v);
         if constexpr (EPC == 8) {
-            uint2 out;
-            out.x = f32x2_to_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv)) |
-                    (f32x2_to_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv)) << 16);
-            out.y = f32x2_to_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv)) |
-                    (f32x2_to_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv)) << 16);
-            *reinterpret_cast<uint2*>(qr + e0) = out;
+            out[c].x = f32x2_to_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv)) |
+                       (f32x2_to_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv)) << 16);
+            out[c].y = f32x2_to_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv)) |
+                       (f32x2_to_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv)) << 16);
         } else {
-            uint32_t out = f32x2_to_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv)) |
-                           (f32x2_to_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv)) << 16);
-            *reinterpret_cast<uint32_t*>(qr + e0) = out;
+            out[c].x = f32x2_to_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv)) |
+                       (f32x2_to_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv)) << 16);
+            out[c].y = 0;
+        }
+    }
+    const int ndst = SCATTER ? topk : 1;
+    for (int j = 0; j < ndst; ++j) {
+        const int64_t r = SCATTER ? static_cast<int64_t>(dst[row * topk + j]) : row;
+        if (r < 0) continue;
+        if (tid == 0) s[r] = sc;
+        uint8_t* qr = q + r * ldq;
+#pragma unroll
+        for (int c = 0; c < NV; ++c) {
+            const int e0 = (c * TEAM + tid) * EPC;
+            if (e0 >= K) continue;
+            if constexpr (EPC == 8) *reinterpret_cast<uint2*>(qr + e0) = out[c];
+            else *reinterpret_cast<uint32_t*>(qr + e0) = out[c].x;
         }
     }
 }
@@ -171,39 +184,51 @@ quant_rows_long_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx,
     }
 }
 
+struct Dest {
+    const int32_t* rows;  // null: row r -> row r; else row r -> rows[r * topk + j]
+    int topk;
+};
+
 template <typename T, int TEAM, int NV>
 cudaError_t launch_fixed(const T* x, int64_t M, int K, int64_t ldx, uint8_t* q, int64_t ldq,
-                         float* s, cudaStream_t st) {
+                         float* s, Dest d, cudaStream_t st) {
     constexpr int TEAMS = kQuantThreads / TEAM;
-    const int64_t grid = (M + TEAMS - 1) / TEAMS;
-    quant_rows_kernel<T, TEAM, NV><<<static_cast<unsigned>(grid), kQuantThreads, 0, st>>>(
-        x, M, K, ldx, q, ldq, s);
+    const unsigned grid = static_cast<unsigned>((M + TEAMS - 1) / TEAMS);
+    if (d.rows)
+        quant_rows_kernel<T, TEAM, NV, true><<<grid, kQuantThreads, 0, st>>>(x, M, K, ldx, q, ldq, s,
+                                                                             d.rows, d.topk);
+    else
+        quant_rows_kernel<T, TEAM, NV, false><<<grid, kQuantThreads, 0, st>>>(x, M, K, ldx, q, ldq, s,
+                                                                              nullptr, 1);
     return cudaGetLastError();
 }
 
 template <typename T, int TEAM>
 cudaError_t launch_team(int nv, const T* x, int64_t M, int K, int64_t ldx, uint8_t* q,
-                        int64_t ldq, float* s, cudaStream_t st) {
+                        int64_t ldq, float* s, Dest d, cudaStream_t st) {
     switch (nv) {
-        case 1: return launch_fixed<T, TEAM, 1>(x, M, K, ldx, q, ldq, s, st);
-        case 2: return launch_fixed<T, TEAM, 2>(x, M, K, ldx, q, ldq, s, st);
-        case 3: return launch_fixed<T, TEAM, 3>(x, M, K, ldx, q, ldq, s, st);
-        case 4: return launch_fixed<T, TEAM, 4>(x, M, K, ldx, q, ldq, s, st);
-        case 5: return launch_fixed<T, TEAM, 5>(x, M, K, ldx, q, ldq, s, st);
-        case 6: return launch_fixed<T, TEAM, 6>(x, M, K, ldx, q, ldq, s, st);
-        case 7: return launch_fixed<T, TEAM, 7>(x, M, K, ldx, q, ldq, s, st);
-        default: return launch_fixed<T, TEAM, 8>(x, M, K, ldx, q, ldq, s, st);
+        case 1: return launch_fixed<T, TEAM, 1>(x, M, K, ldx, q, ldq, s, d, st);
+        case 2: return launch_fixed<T, TEAM, 2>(x, M, K, ldx, q, ldq, s, d, st);
+        case 3: return launch_fixed<T, TEAM, 3>(x, M, K, ldx, q, ldq, s, d, st);
+        case 4: return launch_fixed<T, TEAM, 4>(x, M, K, ldx, q, ldq, s, d, st);
+        case 5: return launch_fixed<T, TEAM, 5>(x, M, K, ldx, q, ldq, s, d, st);
+        case 6: return launch_fixed<T, TEAM, 6>(x, M, K, ldx, q, ldq, s, d, st);
+        case 7: return launch_fixed<T, TEAM, 7>(x, M, K, ldx, q, ldq, s, d, st);
+        default: return launch_fixed<T, TEAM, 8>(x, M, K, ldx, q, ldq, s, d, st);
     }
 }
 
 }  // namespace
 
 // Launches the per-row quantizer for T = bf16 or float (arguments already
-// validated). Exposed to the other translation units of the library.
+// validated). Exposed to the other translation units of the library. With
+// `dst_rows` non-null, row r is written to rows dst_rows[r * topk + j]
+// (register-resident row lengths only: K <= 256 * 8 * chunk elements).
 template <typename T>
 int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
-                      float* s, cudaStream_t st) {
+                      float* s, cudaStream_t st, const int32_t* dst_rows, int topk) {
     if (M == 0) return METIS_OK;
+    const Dest d{dst_rows, topk};
     constexpr int EPC = Elem<T>::kPerChunk;
     const int64_t chunks = K / EPC;
     cudaError_t e;
@@ -213,6 +238,8 @@ int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
         if ((chunks + teams[i] - 1) / teams[i] <= 8) { pick = i; break; }
     if (pick < 0 || M > (int64_t)0x7fffffff * (kQuantThreads / teams[pick])) {
         if (M > 0x7fffffff) return fail(METIS_ERR_UNSUPPORTED, "quantizer: M=%lld too large", (long long)M);
+        if (d.rows) return fail(METIS_ERR_UNSUPPORTED, "quantizer: scattered rows need K <= %d",
+                                256 * 8 * EPC);
         quant_rows_long_kernel<T><<<static_cast<unsigned>(M), kQuantThreads, 0, st>>>(
             x, M, static_cast<int>(K), ldx, q, ldq, s);
         e = cudaGetLastError();
@@ -220,19 +247,20 @@ int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
         const int team = teams[pick];
         const int nv = static_cast<int>((chunks + team - 1) / team);
         switch (team) {
-            case 32: e = launch_team<T, 32>(nv, x, M, (int)K, ldx, q, ldq, s, st); break;
-            case 64: e = launch_team<T, 64>(nv, x, M, (int)K, ldx, q, ldq, s, st); break;
-            case 128: e = launch_team<T, 128>(nv, x, M, (int)K, ldx, q, ldq, s, st); break;
-            default: e = launch_team<T, 256>(nv, x, M, (int)K, ldx, q, ldq, s, st); break;
+            case 32: e = launch_team<T, 32>(nv, x, M, (int)K, ldx, q, ldq, s, d, st); break;
+            case 64: e = launch_team<T, 64>(nv, x, M, (int)K, ldx, q, ldq, s, d, st); break;
+            case 128: e = launch_team<T, 128>(nv, x, M, (int)K, ldx, q, ldq, s, d, st); break;
+            default: e = launch_team<T, 256>(nv, x, M, (int)K, ldx, q, ldq, s, d, st); break;
         }
     }
     return cuda_check(e, "quantizer launch");
 }
 
 template int launch_quant_rows<__nv_bfloat16>(const __nv_bfloat16*, int64_t, int64_t, int64_t,
-                                              uint8_t*, int64_t, float*, cudaStream_t);
+                                              uint8_t*, int64_t, float*, cudaStream_t,
+                                              const int32_t*, int);
 template int launch_quant_rows<float>(const float*, int64_t, int64_t, int64_t, uint8_t*, int64_t,
-                                      float*, cudaStream_t);
+                                      float*, cudaStream_t, const int32_t*, int);
 
 }  // namespace metis
 
@@ -259,7 +287,7 @@ extern "C" int metis_quant_fp8_per_token(const void* x_bf16, int64_t M, int64_t 
     int rc = current_device_info(&di);
     if (rc) return rc;
     return launch_quant_rows<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_bf16), M, K, ldx,
-                                            xq, ldq, s_tok, static_cast<cudaStream_t>(stream));
+                                            xq, ldq, s_tok, static_cast<cudaStream_t>(stream), nullptr, 1);
 }
 
 extern "C" int metis_quant_fp8_per_channel(const float* w, int64_t N, int64_t K, int64_t ldw,
@@ -279,5 +307,6 @@ extern "C" int metis_quant_fp8_per_channel(const float* w, int64_t N, int64_t K,
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
-    return launch_quant_rows<float>(w, N, K, ldw, wq, ldq, s_w, static_cast<cudaStream_t>(stream));
+    return launch_quant_rows<float>(w, N, K, ldw, wq, ldq, s_w, static_cast<cudaStream_t>(stream),
+                                    nullptr, 1);
 }

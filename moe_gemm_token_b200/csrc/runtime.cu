@@ -136,19 +136,35 @@ int make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t co
     return METIS_OK;
 }
 
+int make_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+    CUtensorMap probe;
+    int rc = make_tmap_2d(&probe, base, 1, 16, 1, 16, 16, 1, false);  // resolves the encoder
+    if (rc) return rc;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {s1, s2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(METIS_ERR_INVALID_ARG, "cuTensorMapEncodeTiled (3-D) failed (%d)", static_cast<int>(r));
+    return METIS_OK;
+}
+
 // Routed-expert workspace layout (regions 256-byte aligned).
 static int64_t align256(int64_t v) { return (v + 255) & ~static_cast<int64_t>(255); }
 
 int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
                           int64_t* total) {
     const int64_t S = T * topk;
-    const int64_t sizes[12] = {
+    const int64_t sizes[10] = {
         4 * E,        // COUNTS
         4 * (E + 1),  // OFFSETS
         4 * S,        // SLOT_TO_ROW
         4 * S,        // ROW_TO_SLOT
-        T * H,        // XQ
-        4 * T,        // SX
         S * H,        // AQ
         4 * S,        // SA
         2 * S * I,    // H
@@ -156,8 +172,9 @@ int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_
         4 * S,        // SH
         2 * S * H,    // O
     };
+    (void)T;
     int64_t off = 0, at = -1;
-    for (int r = 0; r < 12; ++r) {
+    for (int r = 0; r < 10; ++r) {
         if (r == region) at = off;
         off = align256(off + sizes[r]);
     }
@@ -221,7 +238,7 @@ extern "C" size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, i
 
 extern "C" int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk, int64_t E,
                                               int64_t H, int64_t I) {
-    if (region < 0 || region > 11 || T < 0 || topk < 1 || E < 1 || H < 0 || I < 0) return -1;
+    if (region < 0 || region > 9 || T < 0 || topk < 1 || E < 1 || H < 0 || I < 0) return -1;
     return moe_region_offset(region, T, topk, E, H, I, nullptr);
 }
 

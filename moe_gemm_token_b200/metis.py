@@ -31,8 +31,8 @@ METIS_OP_FP8_GEMM_FUSED = 1
 METIS_OP_W8A16 = 2
 METIS_OP_MOE = 3
 
-MOE_WS = dict(COUNTS=0, OFFSETS=1, SLOT_TO_ROW=2, ROW_TO_SLOT=3, XQ=4, SX=5, AQ=6, SA=7, H=8,
-              HQ=9, SH=10, O=11)
+MOE_WS = dict(COUNTS=0, OFFSETS=1, SLOT_TO_ROW=2, ROW_TO_SLOT=3, AQ=4, SA=5, H=6, HQ=7, SH=8,
+              O=9)
 
 _lib = None
 
@@ -197,8 +197,9 @@ def metis_linear(x, wq, s_w, y, fast_math=True, s_tok=None, workspace=None, stre
         ws_bytes, _s(stream)))
 
 
+
 def metis_internal_w8a16_variant(v):
-    """Tuning hook: selects how the W8A16 kernel widens E4M3 weights (0, 1, 2)."""
+    """Tuning hook: E4M3 widening of the W8A16 kernel (0: cvt, 1: bit placement)."""
     fn = load().metis_internal_w8a16_variant
     fn.argtypes = [ctypes.c_int]
     fn.restype = ctypes.c_int

@@ -38,7 +38,6 @@ def run_moe(metis, d):
     out = dict(
         counts=R("COUNTS", (E,), torch.int32), offsets=R("OFFSETS", (E + 1,), torch.int32),
         s2r=R("SLOT_TO_ROW", (S,), torch.int32), r2s=R("ROW_TO_SLOT", (S,), torch.int32),
-        xq=R("XQ", (T, H), torch.uint8), sx=R("SX", (T,), torch.float32),
         aq=R("AQ", (S, H), torch.uint8), sa=R("SA", (S,), torch.float32),
         h=R("H", (S, I), torch.int16).view(np.uint16), hq=R("HQ", (S, I), torch.uint8),
         sh=R("SH", (S,), torch.float32), o=R("O", (S, H), torch.int16).view(np.uint16),
@@ -55,13 +54,11 @@ def check_moe(d, g, tokens=None):
     assert_bytes_equal(g["offsets"], offsets, "offsets")
     assert_bytes_equal(g["s2r"], s2r, "slot_to_row")
     assert_bytes_equal(g["r2s"], r2s, "row_to_slot")
-    # per-token codes of x and their gather
+    # per-token codes of x, written into every row the token was routed to
     xq, sx = oracle.quant_per_token(d["x"])
-    assert_bytes_equal(g["xq"], xq, "x codes")
-    assert_bytes_equal(g["sx"].view(np.uint32), sx.view(np.uint32), "x scales")
     tok_of_row = r2s // k
-    assert_bytes_equal(g["aq"], xq[tok_of_row], "gathered codes")
-    assert_bytes_equal(g["sa"].view(np.uint32), sx[tok_of_row].view(np.uint32), "gathered scales")
+    assert_bytes_equal(g["aq"], xq[tok_of_row], "x codes in expert order")
+    assert_bytes_equal(g["sa"].view(np.uint32), sx[tok_of_row].view(np.uint32), "x scales in expert order")
     slots = np.arange(T * k) if tokens is None else \
         (np.asarray(tokens)[:, None] * k + np.arange(k)).reshape(-1)
     rows = s2r[slots]

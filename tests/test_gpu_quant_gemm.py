@@ -122,27 +122,29 @@ def test_fp8_gemm_exact_integer_products(metis):
     assert_bytes_equal(bf16_host(y), yr, "bf16 bits")
 
 
-@pytest.mark.parametrize("variant", [0, 1, 2])
+@pytest.fixture(params=[0, 1], ids=["cvt", "place"])
+def widening(request, metis):
+    old = metis.metis_internal_w8a16_variant(request.param)
+    yield request.param
+    metis.metis_internal_w8a16_variant(old)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 1000, 4096), (2, 37, 272), (3, 300, 12288), (4, 1000, 4096),
-                                   (5, 48, 1024), (8, 1000, 4096), (8, 16, 16)])
-def test_w8a16_parity(metis, variant, M, N, K):
+                                   (5, 48, 1024), (8, 1000, 4096), (8, 16, 16), (7, 2333, 1040),
+                                   (6, 148 * 16 * 7 + 5, 2048)])
+def test_w8a16_parity(metis, widening, M, N, K):
     d = synth.linear(M + 13 * N + K, M, K, N)
     wq, s_w = _prep_weights(metis, d["w"])
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    old = metis.metis_internal_w8a16_variant(variant)
-    try:
-        metis.metis_w8a16_gemm(bf16_dev(d["x"]), wq, s_w, y)
-        torch.cuda.synchronize()
-    finally:
-        metis.metis_internal_w8a16_variant(old)
+    metis.metis_w8a16_gemm(bf16_dev(d["x"]), wq, s_w, y)
+    torch.cuda.synchronize()
     wq_r, sw_r = oracle.quant_per_channel(d["w"])
     assert_bytes_equal(wq.cpu().numpy(), wq_r, "weight codes")
     _, y64 = oracle.gemm_w8a16(d["x"], wq_r, sw_r)
-    assert_close(bf16_host(y), y64, f"w8a16 v{variant} {M}x{N}x{K}")
+    assert_close(bf16_host(y), y64, f"w8a16 {M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("variant", [0, 1, 2])
-def test_w8a16_subnormal_weights_and_wide_x(metis, variant):
+def test_w8a16_subnormal_weights_and_wide_x(metis, widening):
     """Weight rows with many E4M3 subnormal codes and tokens whose elements
     span many binades: the widening and the per-token shift stay exact."""
     rng = np.random.default_rng(5)
@@ -155,14 +157,10 @@ def test_w8a16_subnormal_weights_and_wide_x(metis, variant):
     wq_r, sw_r = oracle.quant_per_channel(w)
     assert np.mean((wq_r & 0x78) == 0) > 0.2  # plenty of subnormal / zero codes
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    old = metis.metis_internal_w8a16_variant(variant)
-    try:
-        metis.metis_w8a16_gemm(bf16_dev(xb), wq, s_w, y)
-        torch.cuda.synchronize()
-    finally:
-        metis.metis_internal_w8a16_variant(old)
+    metis.metis_w8a16_gemm(bf16_dev(xb), wq, s_w, y)
+    torch.cuda.synchronize()
     _, y64 = oracle.gemm_w8a16(xb, wq_r, sw_r)
-    assert_close(bf16_host(y), y64, f"w8a16 subnormal v{variant}")
+    assert_close(bf16_host(y), y64, "w8a16 subnormal weights")
 
 
 def test_linear_dispatch(metis):
@@ -177,8 +175,7 @@ def test_linear_dispatch(metis):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
-@pytest.mark.parametrize("variant", [0, 1, 2])
-def test_w8a16_all_subnormal_codes_exact(metis, variant):
+def test_w8a16_all_subnormal_codes_exact(metis, widening):
     """Every weight code is an E4M3 subnormal (+-m * 2^-9) and x holds small
     integers, so every product and partial sum is exact in FP32: the output
     must equal the oracle's BF16 bits. A widening or a tensor core that
@@ -189,12 +186,8 @@ def test_w8a16_all_subnormal_codes_exact(metis, variant):
     x = synth.f32_to_bf16_bits(rng.integers(-4, 5, (M, K)).astype(np.float32))
     s_w = np.ones(N, np.float32)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    old = metis.metis_internal_w8a16_variant(variant)
-    try:
-        metis.metis_w8a16_gemm(bf16_dev(x), dev(codes), dev(s_w), y)
-        torch.cuda.synchronize()
-    finally:
-        metis.metis_internal_w8a16_variant(old)
+    metis.metis_w8a16_gemm(bf16_dev(x), dev(codes), dev(s_w), y)
+    torch.cuda.synchronize()
     yr, _ = oracle.gemm_w8a16(x, codes, s_w)
     assert np.any(yr != 0)
-    assert_bytes_equal(bf16_host(y), yr, f"w8a16 v{variant} subnormal codes")
+    assert_bytes_equal(bf16_host(y), yr, "w8a16 subnormal codes")
