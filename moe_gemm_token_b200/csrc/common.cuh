@@ -47,6 +47,15 @@ int make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t co
 int make_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                     uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
 
+// Per-row E4M3 quantizer (quant.cu), for T = __nv_bfloat16 or float; the
+// arguments are validated by the caller. dst_rows non-null: row r's codes
+// and scale go to rows dst_rows[r * topk + j] (negative entries skipped).
+// q null: scales only, s[r] and inv_out[r] = 448/amax.
+template <typename T>
+int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                      float* s, cudaStream_t st, const int32_t* dst_rows, int topk,
+                      float* inv_out = nullptr);
+
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Device error word bits.
@@ -136,6 +145,24 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
+}
+
+// Prefetches a 3-D tensor box into L2 (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int32_t x, int32_t y,
+                                                   int32_t z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+// Programmatic dependent launch: wait until the grids this launch depends on
+// have completed and their memory is visible; allow dependents to launch.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_shared() {

@@ -25,6 +25,11 @@
 //             the grouped GEMM of the routed experts (rows of A grouped by
 //             expert, B = [E * N, K], tile schedule built on the device from
 //             the expert offsets) and for small M.
+// Fused quantization (ABF16): A arrives as BF16. An amax pre-pass has written
+// each row's 448/amax; the producer TMA-loads BF16 A tiles into a 2-slot
+// staging ring, and 8 converter warps turn each into the swizzled E4M3 tile
+// the MMA reads (x * (448/amax), cvt.rn.satfinite: the standalone quantizer's
+// bytes), so the codes never go through HBM.
 // Every mbarrier wait is bounded by the device watchdog: on a timeout the CTA
 // sets the sticky error word, stops issuing work, drains what it issued,
 // frees TMEM and returns.
@@ -41,17 +46,22 @@ constexpr int EPI_WARPS = 4;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int MAX_GROUPS = 1024;
 
-template <int CTAS>
+constexpr int CONV_WARPS = 8;                  // fused-quantization converter warps
+constexpr int ASTG_SLOT = ROWS * BK * 2;       // one BF16 A tile (two 64-column boxes)
+
+template <int CTAS, bool ABF16 = false>
 struct Layout {
-    static constexpr int STAGES = CTAS == 2 ? 6 : 4;
+    static constexpr int STAGES = CTAS == 2 ? (ABF16 ? 4 : 6) : (ABF16 ? 3 : 4);
+    static constexpr int ASTG = ABF16 ? 2 : 0;  // BF16 staging slots
+    static constexpr int THREADS_ = ABF16 ? THREADS + CONV_WARPS * 32 : THREADS;
     static constexpr int B_ROWS = BN / CTAS;   // rows of B loaded by one CTA
     static constexpr int A_STAGE = ROWS * BK;
     static constexpr int B_STAGE = B_ROWS * BK;
-    static constexpr int TILES = STAGES * (A_STAGE + B_STAGE);
+    static constexpr int TILES = STAGES * (A_STAGE + B_STAGE) + ASTG * ASTG_SLOT;
     static constexpr int STAGING = EPI_WARPS * 32 * 64;  // a 32 x 32 BF16 block per epilogue warp
     static constexpr int SW = 2 * BN * 4;                // per-channel scales, double-buffered
-    // full, empty, tfull[2], tempty[2], drain, epilogue sync[2]
-    static constexpr int NUM_BARS = 2 * STAGES + 7;
+    // full, empty, tfull[2], tempty[2], drain, epilogue sync[2], staging full/empty
+    static constexpr int NUM_BARS = 2 * STAGES + 7 + 2 * ASTG;
     static constexpr int BAR_OFF = TILES + STAGING + SW;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int GROUP_OFF = MISC_OFF + 16;
@@ -62,6 +72,7 @@ struct Layout {
 
 struct Params {
     const float* s_a;        // [rows of A]
+    const float* inv;        // fused quantization: 448/amax per row of A
     const float* s_b;        // [groups * N]
     __nv_bfloat16* y;        // [rows of A, N]
     const int32_t* offsets;  // grouped: [E + 1] row offsets into A; dense: null
@@ -156,16 +167,17 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, cons
     }
 }
 
-template <int CTAS, bool GROUPED>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int CTAS, bool GROUPED, bool ABF16>
+__global__ void __launch_bounds__(Layout<CTAS, ABF16>::THREADS_, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
-    using L = Layout<CTAS>;
+    using L = Layout<CTAS, ABF16>;
     constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * L::A_STAGE;
+    uint8_t* astg = smem + STAGES * (L::A_STAGE + L::B_STAGE);  // BF16 staging slots
     uint8_t* staging = smem + L::TILES;
     float* sw_smem = reinterpret_cast<float*>(smem + L::TILES + L::STAGING);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
@@ -184,11 +196,19 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     auto tempty = [&](int b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
     const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
     auto epi_sync = [&](int b) { return smem_u32(&bars[2 * STAGES + 5 + b]); };
+    auto bfull = [&](int j) { return smem_u32(&bars[2 * STAGES + 7 + j]); };
+    auto bempty = [&](int j) { return smem_u32(&bars[2 * STAGES + 7 + L::ASTG + j]); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full(s), 1);
+            // fused quantization: the stage is full when B has landed and every
+            // converter warp of both CTAs has written its part of A
+            mbar_init(full(s), ABF16 ? 1 + CTAS * CONV_WARPS : 1);
             mbar_init(empty(s), 1);
+        }
+        for (int j = 0; j < L::ASTG; ++j) {
+            mbar_init(bfull(j), 1);
+            mbar_init(bempty(j), CONV_WARPS);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull(b), 1);
@@ -276,6 +296,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             // ---------------------------------------------------------- producer
             int stage = 0;
             uint32_t phase = 0;
+            int slot = 0;
+            uint32_t sphase = 0;
             uint32_t issued = 0, issued_phase = 0;
             for (int t = first; t < sc.total && !*abort_flag; t += stride) {
                 const Tile ti = sc.get(t);
@@ -284,7 +306,27 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         *abort_flag = 1;
                         break;
                     }
-                    if constexpr (CTAS == 2) {
+                    if constexpr (ABF16) {
+                        // B into the stage (counted on the even CTA's barrier);
+                        // BF16 A into a staging slot for the converter warps
+                        if constexpr (CTAS == 2) {
+                            const uint32_t fl = mapa_shared(full(stage), 0);
+                            if (leader) mbar_arrive_expect_tx(full(stage), CTAS * L::B_STAGE);
+                            tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * BK, ti.b_row0, fl);
+                        } else {
+                            mbar_arrive_expect_tx(full(stage), L::B_STAGE);
+                            tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * BK, ti.b_row0, full(stage));
+                        }
+                        if (!mbar_wait(bempty(slot), sphase ^ 1u, p.timeout_ns, p.status)) {
+                            *abort_flag = 1;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(bfull(slot), ASTG_SLOT);
+                        const uint32_t dst = smem_u32(astg + slot * ASTG_SLOT);
+                        tma_load_2d(dst, &tmA, kb * BK, ti.a_row0, bfull(slot));
+                        tma_load_2d(dst + ASTG_SLOT / 2, &tmA, kb * BK + BK / 2, ti.a_row0, bfull(slot));
+                        if (++slot == L::ASTG) { slot = 0; sphase ^= 1u; }
+                    } else if constexpr (CTAS == 2) {
                         const uint32_t fl = mapa_shared(full(stage), 0);
                         if (leader) mbar_arrive_expect_tx(full(stage), CTAS * (L::A_STAGE + L::B_STAGE));
                         tma_load_2d_pair(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * BK, ti.a_row0, fl);
@@ -301,7 +343,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             }
             if (*abort_flag) {
                 // let the copies in flight land before the CTA exits
-                if (leader) {
+                if (ABF16) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 100000ull) {}
+                } else if (leader) {
                     for (int s = 0; s < STAGES; ++s)
                         if (issued & (1u << s))
                             mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
@@ -361,7 +406,71 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             else mma_commit(drain);
             mbar_wait(drain, 0, p.timeout_ns, p.status);
         }
-    } else {
+    } else if (ABF16 && warp >= 2 + EPI_WARPS) {
+        // ------------------------------------------------- converters (fused)
+        const int ct = threadIdx.x - 32 * (2 + EPI_WARPS);  // 0 .. 255
+        int stage = 0;
+        uint32_t phase = 0;
+        int slot = 0;
+        uint32_t sphase = 0;
+        for (int t = first; t < sc.total && !*abort_flag; t += stride) {
+            const Tile ti = sc.get(t);
+            float invr[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = ti.a_row0 + (ct >> 3) + 32 * i;
+                invr[i] = row < ti.row_end ? p.inv[row] : 0.0f;
+            }
+            bool ok = true;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!mbar_wait(bfull(slot), sphase, p.timeout_ns, p.status) ||
+                    !mbar_wait(empty(stage), phase ^ 1u, p.timeout_ns, p.status)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* src0 = astg + slot * ASTG_SLOT;
+                uint8_t* dst0 = sA + stage * L::A_STAGE;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    // 16 elements: row r, E4M3 chunk c (k = 16c .. 16c+15)
+                    const int task = ct + 256 * i;
+                    const int r = task >> 3, c = task & 7;
+                    const uint8_t* src = src0 + (c >> 2) * (ASTG_SLOT / 2) + r * 128;
+                    // the two BF16 pieces; the second box's threads take the odd
+                    // piece first so that 8 threads of a row hit 8 bank groups
+                    const int hb = c >> 2;
+                    const int cc = 2 * (c & 3);
+                    const uint4 va = *reinterpret_cast<const uint4*>(src + (((cc + hb) ^ (r & 7)) << 4));
+                    const uint4 vb = *reinterpret_cast<const uint4*>(src + (((cc + 1 - hb) ^ (r & 7)) << 4));
+                    const uint4 v0 = hb ? vb : va;
+                    const uint4 v1 = hb ? va : vb;
+                    const float inv = invr[i];
+                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2)
+                        o[q2] = f32x2_to_e4m3x2(__fmul_rn(bf16_lo(w[2 * q2]), inv), __fmul_rn(bf16_hi(w[2 * q2]), inv)) |
+                                (f32x2_to_e4m3x2(__fmul_rn(bf16_lo(w[2 * q2 + 1]), inv),
+                                                 __fmul_rn(bf16_hi(w[2 * q2 + 1]), inv)) << 16);
+                    *reinterpret_cast<uint4*>(dst0 + r * 128 + ((c ^ (r & 7)) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                fence_proxy_async_shared();  // generic-proxy writes -> tensor-core reads
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bempty(slot));
+                    if constexpr (CTAS == 2) mbar_arrive_cluster(mapa_shared(full(stage), 0));
+                    else mbar_arrive(full(stage));
+                }
+                if (++slot == L::ASTG) { slot = 0; sphase ^= 1u; }
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                break;
+            }
+        }
+    } else if (warp < 2 + EPI_WARPS) {
         // -------------------------------------------------------------- epilogue
         const int q = warp & 3;        // TMEM lane quadrant this warp may access
         const int et = threadIdx.x - 64;  // 0..127
@@ -427,13 +536,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
 }
 
-template <int CTAS, bool GROUPED>
+template <int CTAS, bool GROUPED, bool ABF16 = false>
 int prepare(const DeviceInfo& di, size_t smem) {
     static bool done[64];
     if (static_cast<size_t>(di.max_smem_optin) < smem)
         return fail(METIS_ERR_UNSUPPORTED, "fp8 gemm needs %zu bytes of shared memory", smem);
     if (!done[di.device]) {
-        int rc = cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED>,
+        int rc = cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED, ABF16>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(smem)),
                             "cudaFuncSetAttribute(fp8 gemm)");
@@ -444,13 +553,14 @@ int prepare(const DeviceInfo& di, size_t smem) {
 }
 
 // Co-resident CTA pairs of the 2-CTA kernel (cached per device).
+template <bool ABF16 = false>
 int max_pairs(const DeviceInfo& di, int* out) {
     static int cached[64];
     if (!cached[di.device]) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (di.num_sms / 2), 1, 1);
-        cfg.blockDim = dim3(THREADS, 1, 1);
-        cfg.dynamicSmemBytes = Layout<2>::BYTES_DENSE;
+        cfg.blockDim = dim3(Layout<2, ABF16>::THREADS_, 1, 1);
+        cfg.dynamicSmemBytes = Layout<2, ABF16>::BYTES_DENSE;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -459,7 +569,7 @@ int max_pairs(const DeviceInfo& di, int* out) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, false>, &cfg),
+        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, false, ABF16>, &cfg),
                             "cudaOccupancyMaxActiveClusters");
         if (rc) return rc;
         if (n < 1) return fail(METIS_ERR_UNSUPPORTED, "no CTA pair of the fp8 gemm fits an SM pair");
@@ -480,7 +590,7 @@ int launch_fp8_gemm_dense(const uint8_t* a, const float* s_a, const uint8_t* b, 
     if (rc) return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
-    Params p{s_a, s_b, y, nullptr, M, N, K, 1, status, watchdog_ns()};
+    Params p{s_a, nullptr, s_b, y, nullptr, M, N, K, 1, status, watchdog_ns()};
     const int num_n = (N + BN - 1) / BN;
     CUtensorMap ta, tb;
     if ((rc = make_tmap_2d(&ta, a, 1, K, M, K, BK, ROWS, true))) return rc;
@@ -504,7 +614,7 @@ int launch_fp8_gemm_dense(const uint8_t* a, const float* s_a, const uint8_t* b, 
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cuda_check(cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<2, false>, ta, tb, p),
+        return cuda_check(cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<2, false, false>, ta, tb, p),
                           "fp8 gemm (CTA pair) launch");
     }
     using L = Layout<1>;
@@ -512,7 +622,7 @@ int launch_fp8_gemm_dense(const uint8_t* a, const float* s_a, const uint8_t* b, 
     if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
     const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
-    fp8_gemm_kernel<1, false><<<grid, THREADS, L::BYTES_DENSE, st>>>(ta, tb, p);
+    fp8_gemm_kernel<1, false, false><<<grid, THREADS, L::BYTES_DENSE, st>>>(ta, tb, p);
     return cuda_check(cudaGetLastError(), "fp8 gemm launch");
 }
 
@@ -534,9 +644,56 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, ROWS, true))) return rc;
     if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
         return rc;
-    Params p{s_a, s_b, y, offsets, rows, N, K, E, status, watchdog_ns()};
-    fp8_gemm_kernel<1, true><<<di.num_sms, THREADS, L::BYTES_GROUPED, st>>>(ta, tb, p);
+    Params p{s_a, nullptr, s_b, y, offsets, rows, N, K, E, status, watchdog_ns()};
+    fp8_gemm_kernel<1, true, false><<<di.num_sms, THREADS, L::BYTES_GROUPED, st>>>(ta, tb, p);
     return cuda_check(cudaGetLastError(), "grouped fp8 gemm launch");
+}
+
+// Fused-quantization W8A8 GEMM launch: a is BF16 [M, K]; inv [M] holds
+// 448/amax per row (written by the scales-only quantizer pass).
+int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float* inv,
+                          const uint8_t* b, const float* s_b, __nv_bfloat16* y, int M, int N, int K,
+                          cudaStream_t st) {
+    using namespace gemm;
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    uint32_t* status = nullptr;
+    if ((rc = device_status_word(&status))) return rc;
+    Params p{s_a, inv, s_b, y, nullptr, M, N, K, 1, status, watchdog_ns()};
+    const int num_n = (N + BN - 1) / BN;
+    CUtensorMap ta, tb;
+    if ((rc = make_tmap_2d(&ta, a, 2, K, M, static_cast<uint64_t>(K) * 2, BK / 2, ROWS, true))) return rc;
+    if (M > ROWS) {
+        using L = Layout<2, true>;
+        if ((rc = prepare<2, false, true>(di, L::BYTES_DENSE))) return rc;
+        int pairs = 0;
+        if ((rc = max_pairs<true>(di, &pairs))) return rc;
+        if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
+        const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
+        const int clusters = tiles < pairs ? tiles : pairs;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * clusters, 1, 1);
+        cfg.blockDim = dim3(L::THREADS_, 1, 1);
+        cfg.dynamicSmemBytes = L::BYTES_DENSE;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cuda_check(cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<2, false, true>, ta, tb, p),
+                          "fused fp8 gemm (CTA pair) launch");
+    }
+    using L = Layout<1, true>;
+    if ((rc = prepare<1, false, true>(di, L::BYTES_DENSE))) return rc;
+    if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
+    const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
+    const int grid = tiles < di.num_sms ? tiles : di.num_sms;
+    fp8_gemm_kernel<1, false, true><<<grid, L::THREADS_, L::BYTES_DENSE, st>>>(ta, tb, p);
+    return cuda_check(cudaGetLastError(), "fused fp8 gemm launch");
 }
 
 }  // namespace metis
@@ -565,7 +722,18 @@ extern "C" int metis_fp8_gemm(const void* a, int a_kind, float* s_tok, const uin
         return launch_fp8_gemm_dense(static_cast<const uint8_t*>(a), s_tok, wq, s_w,
                                      static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(M),
                                      static_cast<int>(N), static_cast<int>(K), st);
-    (void)workspace;
-    (void)ws_bytes;
-    return fail(METIS_ERR_UNSUPPORTED, "fp8_gemm: the fused BF16 prologue is not built yet");
+    // fused quantization: scales pass (s_tok out, 448/amax into the workspace),
+    // then the GEMM that quantizes A tiles in shared memory
+    const size_t need = metis_workspace_size(METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 16))
+        return fail(METIS_ERR_INVALID_ARG,
+                    "fp8_gemm (BF16 A): needs a 16-byte aligned workspace of %zu bytes (got %zu)",
+                    need, ws_bytes);
+    float* inv = static_cast<float*>(workspace);
+    int rc = launch_quant_rows<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(a), M, K, K, nullptr,
+                                              K, s_tok, st, nullptr, 1, inv);
+    if (rc) return rc;
+    return launch_fp8_gemm_fused(static_cast<const __nv_bfloat16*>(a), s_tok, inv, wq, s_w,
+                                 static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(M),
+                                 static_cast<int>(N), static_cast<int>(K), st);
 }

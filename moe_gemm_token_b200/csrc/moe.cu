@@ -20,9 +20,6 @@
 
 namespace metis {
 
-template <typename T>
-int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
-                      float* s, cudaStream_t st, const int32_t* dst_rows, int topk);
 int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b, const float* s_b,
                             __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
                             int K, cudaStream_t st);

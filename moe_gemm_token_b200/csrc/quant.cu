@@ -55,10 +55,13 @@ struct Elem<float> {
 // and scale go to rows dst[r * topk + j] (j < topk; negative entries skipped)
 // instead of row r: the routed-expert path quantizes each token once and
 // writes it straight into the expert-ordered rows it was routed to.
+// With q == null only the scales are written: s[r] and inv_out[r] = 448/amax
+// (the prologue of the fused-quantization GEMM).
 template <typename T, int TEAM, int NV, bool SCATTER>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx, uint8_t* __restrict__ q,
-                  int64_t ldq, float* __restrict__ s, const int32_t* __restrict__ dst, int topk) {
+                  int64_t ldq, float* __restrict__ s, const int32_t* __restrict__ dst, int topk,
+                  float* __restrict__ inv_out) {
     constexpr int EPC = Elem<T>::kPerChunk;
     constexpr int TEAMS = kQuantThreads / TEAM;
     constexpr int WARPS_PER_TEAM = TEAM / 32;
@@ -103,6 +106,13 @@ quant_rows_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx, uint8_
 
     float sc, inv;
     row_scales(amax, &sc, &inv);
+    if (q == nullptr) {
+        if (tid == 0) {
+            s[row] = sc;
+            inv_out[row] = inv;
+        }
+        return;
+    }
     // this thread's codes: 8 (BF16 input) or 4 (FP32 input) bytes per chunk
     uint2 out[NV];
 #pragma unroll
@@ -141,7 +151,8 @@ quant_rows_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx, uint8_
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_long_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx,
-                       uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ s) {
+                       uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ s,
+                       float* __restrict__ inv_out) {
     constexpr int EPC = Elem<T>::kPerChunk;
     __shared__ float red[kQuantThreads / 32];
     const int64_t row = blockIdx.x;
@@ -163,7 +174,11 @@ quant_rows_long_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx,
     for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, red[w]);
     float sc, inv;
     row_scales(amax, &sc, &inv);
-    if (threadIdx.x == 0) s[row] = sc;
+    if (threadIdx.x == 0) {
+        s[row] = sc;
+        if (q == nullptr) inv_out[row] = inv;
+    }
+    if (q == nullptr) return;
     uint8_t* qr = q + row * ldq;
     for (int e0 = threadIdx.x * EPC; e0 < K; e0 += kQuantThreads * EPC) {
         float v[EPC];
@@ -187,6 +202,7 @@ quant_rows_long_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx,
 struct Dest {
     const int32_t* rows;  // null: row r -> row r; else row r -> rows[r * topk + j]
     int topk;
+    float* inv;           // scales only (q null): 448/amax per row
 };
 
 template <typename T, int TEAM, int NV>
@@ -194,12 +210,12 @@ cudaError_t launch_fixed(const T* x, int64_t M, int K, int64_t ldx, uint8_t* q, 
                          float* s, Dest d, cudaStream_t st) {
     constexpr int TEAMS = kQuantThreads / TEAM;
     const unsigned grid = static_cast<unsigned>((M + TEAMS - 1) / TEAMS);
-    if (d.rows)
+    if (d.rows && q)
         quant_rows_kernel<T, TEAM, NV, true><<<grid, kQuantThreads, 0, st>>>(x, M, K, ldx, q, ldq, s,
-                                                                             d.rows, d.topk);
+                                                                             d.rows, d.topk, nullptr);
     else
         quant_rows_kernel<T, TEAM, NV, false><<<grid, kQuantThreads, 0, st>>>(x, M, K, ldx, q, ldq, s,
-                                                                              nullptr, 1);
+                                                                              nullptr, 1, d.inv);
     return cudaGetLastError();
 }
 
@@ -224,11 +240,15 @@ cudaError_t launch_team(int nv, const T* x, int64_t M, int K, int64_t ldx, uint8
 // validated). Exposed to the other translation units of the library. With
 // `dst_rows` non-null, row r is written to rows dst_rows[r * topk + j]
 // (register-resident row lengths only: K <= 256 * 8 * chunk elements).
+// With q == nullptr no codes are written: s receives the scales and inv_out
+// 448/amax per row.
 template <typename T>
 int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
-                      float* s, cudaStream_t st, const int32_t* dst_rows, int topk) {
+                      float* s, cudaStream_t st, const int32_t* dst_rows, int topk, float* inv_out) {
     if (M == 0) return METIS_OK;
-    const Dest d{dst_rows, topk};
+    if (q == nullptr && (inv_out == nullptr || dst_rows != nullptr))
+        return fail(METIS_ERR_INVALID_ARG, "quantizer: scales-only needs inv_out and no row map");
+    const Dest d{dst_rows, topk, inv_out};
     constexpr int EPC = Elem<T>::kPerChunk;
     const int64_t chunks = K / EPC;
     cudaError_t e;
@@ -241,7 +261,7 @@ int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
         if (d.rows) return fail(METIS_ERR_UNSUPPORTED, "quantizer: scattered rows need K <= %d",
                                 256 * 8 * EPC);
         quant_rows_long_kernel<T><<<static_cast<unsigned>(M), kQuantThreads, 0, st>>>(
-            x, M, static_cast<int>(K), ldx, q, ldq, s);
+            x, M, static_cast<int>(K), ldx, q, ldq, s, inv_out);
         e = cudaGetLastError();
     } else {
         const int team = teams[pick];
@@ -258,9 +278,9 @@ int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
 
 template int launch_quant_rows<__nv_bfloat16>(const __nv_bfloat16*, int64_t, int64_t, int64_t,
                                               uint8_t*, int64_t, float*, cudaStream_t,
-                                              const int32_t*, int);
+                                              const int32_t*, int, float*);
 template int launch_quant_rows<float>(const float*, int64_t, int64_t, int64_t, uint8_t*, int64_t,
-                                      float*, cudaStream_t, const int32_t*, int);
+                                      float*, cudaStream_t, const int32_t*, int, float*);
 
 }  // namespace metis
 

@@ -13,22 +13,23 @@
 //    3-D view of the weights, {64 bytes, rows (stride K), 64-byte k-groups},
 //    one 16 x 16 x 64-byte box (16 KB: 16 rows x a 1024-byte k-window) per
 //    ring stage, laid out as one 16-row x 64-byte block per consumer warp;
-//    6 stages keep ~100 KB per SM in flight without occupying registers. 16 consumer
-//    warps read their box (rows g and g+8, 16 bytes per thread, conflict-free),
-//    widen E4M3 to FP16 and issue mma.sync.m16n8k16 with the weights as the
-//    M = 16 operand and the <= 8 tokens as n = 8 (four independent FP32
-//    accumulators).
+//    the deepest ring that fits (up to 12 stages, ~190 KB per SM in flight)
+//    without occupying registers. 16 consumer warps read their box (rows g and
+//    g+8, 16 bytes per thread, conflict-free), widen E4M3 to FP16 and issue
+//    mma.sync.m16n8k16 with the weights as the M = 16 operand and the <= 8
+//    tokens as n = 8 (four independent FP32 accumulators). A reducer warp
+//    adds each finished tile's partial sums (double-buffered) and stores it
+//    while the stream goes on. Launched as a programmatic dependent: barrier
+//    set-up and an L2 prefetch of the first ring's worth of weights overlap
+//    the previous kernel; x is read, y written and shared memory filled only
+//    after the grid dependency is resolved.
 //  * register kernel (K % 64 != 0, or when x plus a ring do not fit in
 //    shared memory): 16 warps stream 128-byte chunks of the rows straight
 //    into registers, 4 chunks in flight per thread.
 //
-// Both widen exactly (every E4M3 value is an FP16 normal):
-//    CONV_CVT   cvt.rn.f16x2.e4m3x2 on byte pairs (0,1) and (2,3);
-//    CONV_PLACE the E4M3 bits placed directly in FP16 bit positions, which is
-//               exactly the value times 2^-8 (FP16 bias 15, E4M3 bias 7; both
-//               subnormal ranges scale alike), the 2^8 folded into the
-//               epilogue; bytes (0,2) and (1,3) form the pairs, so x is staged
-//               with k permuted 0,2,1,3 inside every group of four.
+// Both widen with cvt.rn.f16x2.e4m3x2 (exact: every E4M3 value is an FP16
+// normal), which measured faster here than placing the E4M3 bits into FP16
+// positions with integer operations.
 // x is staged as FP16 after an exact per-token power-of-two shift that puts
 // the token's amax in [2^14, 2^15): every element within a factor 2^29 of the
 // amax keeps its BF16 value exactly, so the products are those of the BF16
@@ -42,12 +43,9 @@ namespace w8a16 {
 constexpr int WARPS = 16;             // consumer warps
 constexpr int CTHREADS = WARPS * 32;  // consumer threads
 constexpr int MAX_K = 12288;
-enum Conv { CONV_CVT = 0, CONV_PLACE = 1 };
-int g_conv = CONV_CVT;
-int g_layout = -1;  // -1: preferred view if the encoder accepts it, else 1; 0/1: forced
+
 
 // TMA kernel geometry
-constexpr int TMA_THREADS = CTHREADS + 32;  // + producer warp
 constexpr int BOX_K = 64;                   // bytes of K per box (one consumer warp)
 constexpr int WIN = WARPS * BOX_K;          // k-window per stage: 1024
 constexpr int STAGE_BYTES = 16 * WIN;       // 16 rows x 1024 = 16 KB
@@ -62,14 +60,6 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
-}
-
-// E4M3 bytes (b0, b2) resp. (b1, b3) of q as an FP16 pair equal to value * 2^-8.
-__device__ __forceinline__ uint32_t place_even(uint32_t q) {
-    return ((q << 8) & 0x80008000u) | ((q << 7) & 0x3F803F80u);
-}
-__device__ __forceinline__ uint32_t place_odd(uint32_t q) {
-    return (q & 0x80008000u) | ((q >> 1) & 0x3F803F80u);
 }
 
 // Two E4M3 byte pairs of w, (0,1) and (2,3), to two FP16 pairs (exact).
@@ -91,7 +81,6 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
 
 // 16 rows x 16 bytes of K (rows g and g + 8 of this thread: words A, B)
 // against the thread's x fragment (8 words, 4 k-steps), into acc[4].
-template <int CONV>
 __device__ __forceinline__ void piece_mma(float (&acc)[4][4], const uint4& A, const uint4& B,
                                           const uint4& xa, const uint4& xc) {
     const uint32_t wa[4] = {A.x, A.y, A.z, A.w};
@@ -100,15 +89,8 @@ __device__ __forceinline__ void piece_mma(float (&acc)[4][4], const uint4& A, co
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
         uint32_t a0, a1, a2, a3;
-        if constexpr (CONV == CONV_PLACE) {
-            a0 = place_even(wa[s]);
-            a2 = place_odd(wa[s]);
-            a1 = place_even(wb[s]);
-            a3 = place_odd(wb[s]);
-        } else {
-            cvt_pairs(wa[s], a0, a2);
-            cvt_pairs(wb[s], a1, a3);
-        }
+        cvt_pairs(wa[s], a0, a2);
+        cvt_pairs(wb[s], a1, a3);
         mma_16816(acc[s], a0, a1, a2, a3, bx[2 * s], bx[2 * s + 1]);
     }
 }
@@ -134,30 +116,55 @@ struct Smem {
     int xpitch;    // bytes per staged x row (2 * KP + 16: 16 mod 128 -> conflict-free)
     int x_off;     // [M][xpitch] FP16
     int misc_off;  // unshift[8] f32, shift/amax[8], pow2[8]
-    int part_off;  // [max_tpc][16 warps][32 lanes][4] f32
+    int part_off;  // [part_tiles][16 warps][32 lanes][4] f32
     int ring_off;  // TMA ring
-    int bar_off;   // full[stages], empty[stages]
+    int bar_off;   // full[stages], empty[stages], tfull[2], tfree[2]
     int total;
 };
 
-__host__ __device__ inline Smem smem_layout(int M, int KP, int max_tpc, int stages) {
+__host__ __device__ inline Smem smem_layout(int M, int KP, int part_tiles, int stages) {
     Smem s;
     s.xpitch = 2 * KP + 16;
     s.x_off = 0;
     s.misc_off = M * s.xpitch;  // 16-byte aligned
     s.part_off = s.misc_off + 128;
-    s.ring_off = s.part_off + max_tpc * WARPS * 32 * 16;
+    s.ring_off = s.part_off + part_tiles * WARPS * 32 * 16;
     s.ring_off = (s.ring_off + 127) & ~127;  // TMA destination alignment
     s.bar_off = s.ring_off + stages * STAGE_BYTES;
-    s.total = s.bar_off + 2 * stages * 8;
+    s.total = s.bar_off + (2 * stages + 4) * 8;
     return s;
 }
 
-// Stages x [M][K] BF16 into shared memory as FP16 rows of KP elements (k
-// permuted per CONV, zero-padded) with the per-token power-of-two shift.
+// Stages x [M][K] BF16 into shared memory as FP16 rows of KP elements
+// (zero-padded) with the per-token power-of-two shift.
 // Executed by the CTHREADS consumer threads, synchronised on named barrier 1
-// (no other thread takes part, and nothing here waits on an mbarrier).
-template <int CONV>
+// (no other thread takes part, and nothing here waits on an mbarrier). When
+// all of x fits in the threads' registers (M*K <= 32768) each element is
+// read once from global memory and written once to shared memory.
+__device__ __forceinline__ void widen8(const uint4& raw, int sh, float p2, uint4& out) {
+    const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+    float f[8];
+    if (p2 != 0.0f) {  // 2^sh is a binary32: one exact multiply per element
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            f[2 * j] = bf16_lo(wv[j]) * p2;
+            f[2 * j + 1] = bf16_hi(wv[j]) * p2;
+        }
+    } else {  // extreme token magnitudes only
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            f[2 * j] = ldexpf(bf16_lo(wv[j]), sh);
+            f[2 * j + 1] = ldexpf(bf16_hi(wv[j]), sh);
+        }
+    }
+    const __half2 h0 = __floats2half2_rn(f[0], f[1]);
+    const __half2 h1 = __floats2half2_rn(f[2], f[3]);
+    const __half2 h2 = __floats2half2_rn(f[4], f[5]);
+    const __half2 h3 = __floats2half2_rn(f[6], f[7]);
+    out = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                     *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+}
+
 __device__ __forceinline__ void stage_x(const Args& a, uint8_t* smem, const Smem& L, int tid) {
     uint8_t* xs = smem + L.x_off;
     float* unshift = reinterpret_cast<float*>(smem + L.misc_off);
@@ -168,6 +175,7 @@ __device__ __forceinline__ void stage_x(const Args& a, uint8_t* smem, const Smem
     constexpr int XB = 8;
     const int kc = a.K / 8;
     const int xchunks = a.M * kc;
+    const bool in_regs = xchunks <= XB * CTHREADS;
     if (tid < 8) row_amax[tid] = 0u;
     uint4 xb[XB];
 #pragma unroll
@@ -193,8 +201,10 @@ __device__ __forceinline__ void stage_x(const Args& a, uint8_t* smem, const Smem
             const unsigned mx = __reduce_max_sync(peers, __float_as_uint(ca));
             if (m >= 0) {
                 if ((peers & ((1u << lane) - 1u)) == 0) atomicMax(&row_amax[m], mx);
-                const int k = (c - m * kc) * 8;
-                *reinterpret_cast<uint4*>(xs + m * L.xpitch + 2 * k) = xb[j];
+                if (!in_regs) {
+                    const int k = (c - m * kc) * 8;
+                    *reinterpret_cast<uint4*>(xs + m * L.xpitch + 2 * k) = xb[j];
+                }
             }
         }
     }
@@ -210,31 +220,34 @@ __device__ __forceinline__ void stage_x(const Args& a, uint8_t* smem, const Smem
     }
     named_barrier(1, CTHREADS);
     const int kpc = a.KP / 8;
-    for (int c = tid; c < a.M * kpc; c += CTHREADS) {
-        const int m = c / kpc;
-        const int k = (c - m * kpc) * 8;
-        uint4* p = reinterpret_cast<uint4*>(xs + m * L.xpitch + 2 * k);
-        uint4 out = make_uint4(0, 0, 0, 0);
-        if (k < a.K) {
-            const uint4 raw = *p;
-            const int sh = shift[m];
-            const float p2 = pow2[m];
-            const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-            float f[8];
+    if (in_regs) {
+        // widen the chunks held in registers; then zero the padding [K, KP)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                f[2 * j] = p2 != 0.0f ? bf16_lo(wv[j]) * p2 : ldexpf(bf16_lo(wv[j]), sh);
-                f[2 * j + 1] = p2 != 0.0f ? bf16_hi(wv[j]) * p2 : ldexpf(bf16_hi(wv[j]), sh);
+        for (int j = 0; j < XB; ++j) {
+            const int c = tid + CTHREADS * j;
+            if (c < xchunks) {
+                const int m = c / kc;
+                const int k = (c - m * kc) * 8;
+                uint4 out;
+                widen8(xb[j], shift[m], pow2[m], out);
+                *reinterpret_cast<uint4*>(xs + m * L.xpitch + 2 * k) = out;
             }
-            constexpr bool perm = CONV == CONV_PLACE;  // pairs (0,2), (1,3)
-            const __half2 h0 = __floats2half2_rn(f[0], perm ? f[2] : f[1]);
-            const __half2 h1 = __floats2half2_rn(perm ? f[1] : f[2], f[3]);
-            const __half2 h2 = __floats2half2_rn(f[4], perm ? f[6] : f[5]);
-            const __half2 h3 = __floats2half2_rn(perm ? f[5] : f[6], f[7]);
-            out = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
-                             *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
         }
-        *p = out;
+        const int pad = kpc - kc;
+        for (int c = tid; c < a.M * pad; c += CTHREADS) {
+            const int m = c / pad;
+            const int k = a.K + (c - m * pad) * 8;
+            *reinterpret_cast<uint4*>(xs + m * L.xpitch + 2 * k) = make_uint4(0, 0, 0, 0);
+        }
+    } else {
+        for (int c = tid; c < a.M * kpc; c += CTHREADS) {
+            const int m = c / kpc;
+            const int k = (c - m * kpc) * 8;
+            uint4* p = reinterpret_cast<uint4*>(xs + m * L.xpitch + 2 * k);
+            uint4 out = make_uint4(0, 0, 0, 0);
+            if (k < a.K) widen8(*p, shift[m], pow2[m], out);
+            *p = out;
+        }
     }
     named_barrier(1, CTHREADS);
 }
@@ -264,13 +277,11 @@ __device__ __forceinline__ void flush(float (&acc)[4][4], float* partial, int ct
 }
 
 // Fixed-order reduction of the warps' partial sums, scale, round, store.
-template <int CONV>
 __device__ __forceinline__ void reduce_store(const Args& a, const uint8_t* smem, const Smem& L,
                                              int t0, int ntl, int tid) {
     const float* partial = reinterpret_cast<const float*>(smem + L.part_off);
     const float* unshift = reinterpret_cast<const float*>(smem + L.misc_off);
     const int per_tok = ntl * 16;
-    const float fold = CONV == CONV_PLACE ? 256.0f : 1.0f;
     for (int idx = tid; idx < per_tok * a.M; idx += CTHREADS) {
         const int m = idx / per_tok;
         const int nl = idx - m * per_tok;
@@ -284,23 +295,26 @@ __device__ __forceinline__ void reduce_store(const Args& a, const uint8_t* smem,
         float sum = 0.f;
 #pragma unroll
         for (int w = 0; w < WARPS; ++w) sum += src[w * 32 * 4];
-        const float v = __fmul_rn(__fmul_rn(__fmul_rn(sum, unshift[m]), fold), a.s_w[n]);
+        const float v = __fmul_rn(__fmul_rn(sum, unshift[m]), a.s_w[n]);
         a.y[static_cast<size_t>(m) * a.N + n] = __float2bfloat16_rn(v);
     }
 }
 
 // ------------------------------------------------------------- TMA kernel
 
-template <int CONV>
+constexpr int TMA_THREADS = CTHREADS + 64;  // + producer warp + reducer warp
+
 __global__ void __launch_bounds__(TMA_THREADS, 1)
 w8a16_tma_kernel(const __grid_constant__ CUtensorMap tmW, const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const Smem L = smem_layout(a.M, a.KP, a.max_tpc, a.stages);
+    const Smem L = smem_layout(a.M, a.KP, 2, a.stages);
     uint8_t* ring = smem + L.ring_off;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
     const int S = a.stages;
     auto full = [&](int s) { return smem_u32(&bars[s]); };
     auto empty = [&](int s) { return smem_u32(&bars[S + s]); };
+    auto tfull = [&](int b) { return smem_u32(&bars[2 * S + b]); };
+    auto tfree = [&](int b) { return smem_u32(&bars[2 * S + 2 + b]); };
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -309,42 +323,92 @@ w8a16_tma_kernel(const __grid_constant__ CUtensorMap tmW, const Args a) {
     const int ntl = t1 - t0;
     const int kwin = a.KP / WIN;    // k-windows per tile
     const int nstage = ntl * kwin;  // stages this CTA streams
+    auto box_coords = [&](int i, int& x, int& y, int& z) {
+        const int tl = i / kwin;
+        const int kw = i - tl * kwin;
+        x = 0;
+        y = a.wlayout == 0 ? (t0 + tl) * 16 : kw * WARPS;
+        z = a.wlayout == 0 ? kw * WARPS : (t0 + tl) * 16;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), WARPS);
         }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), WARPS);
+            mbar_init(tfree(b), 1);
+        }
         fence_mbar_init();
         tma_prefetch_desc(&tmW);
     }
     __syncthreads();
+    grid_launch_dependents();
 
     if (warp == WARPS) {
         // ---------------------------------------------------------- producer
-        // Consumers wait for every stage issued here before the CTA ends, so
-        // no copy can land after the CTA exits; a timeout stops the stream.
+        // Warm L2 with the first ring's worth of weights while the previous
+        // kernel may still run (a prefetch reads through the coherent L2, so
+        // it is safe whatever that kernel writes), then stream into shared
+        // memory once the grid dependency is resolved. Consumers wait for
+        // every stage issued here before the CTA ends.
         if (lane == 0) {
+            for (int i = 0; i < nstage && i < S; ++i) {
+                int x, y, z;
+                box_coords(i, x, y, z);
+                tma_prefetch_l2_3d(&tmW, x, y, z);
+            }
+            grid_dependency_wait();
             int s = 0;
             uint32_t ph = 0;
             for (int i = 0; i < nstage; ++i) {
-                const int tl = i / kwin;
-                const int kw = i - tl * kwin;
                 if (!mbar_wait(empty(s), ph ^ 1u, a.timeout_ns, a.status)) break;
                 mbar_arrive_expect_tx(full(s), STAGE_BYTES);
-                if (a.wlayout == 0)
-                    tma_load_3d(smem_u32(ring + s * STAGE_BYTES), &tmW, 0, (t0 + tl) * 16, kw * WARPS, full(s));
-                else
-                    tma_load_3d(smem_u32(ring + s * STAGE_BYTES), &tmW, 0, kw * WARPS, (t0 + tl) * 16, full(s));
+                int x, y, z;
+                box_coords(i, x, y, z);
+                tma_load_3d(smem_u32(ring + s * STAGE_BYTES), &tmW, x, y, z, full(s));
                 if (++s == S) { s = 0; ph ^= 1u; }
             }
+        }
+        return;
+    }
+    if (warp == WARPS + 1) {
+        // ----------------------------------------------------------- reducer
+        // Adds the 16 warps' partial sums of each finished tile in a fixed
+        // order, scales, rounds and stores it; frees the partial buffer.
+        grid_dependency_wait();
+        const float* partial = reinterpret_cast<const float*>(smem + L.part_off);
+        const float* unshift = reinterpret_cast<const float*>(smem + L.misc_off);
+        for (int tl = 0; tl < ntl; ++tl) {
+            const int b = tl & 1;
+            if (!mbar_wait(tfull(b), (tl >> 1) & 1u, a.timeout_ns, a.status)) break;
+            const float* pb = partial + b * WARPS * 32 * 4;
+            for (int o = lane; o < 16 * a.M; o += 32) {
+                const int m = o >> 4;
+                const int row = o & 15;
+                const int n = (t0 + tl) * 16 + row;
+                const int ln = (row & 7) * 4 + (m >> 1);
+                const int comp = (row >> 3) * 2 + (m & 1);
+                const float* src = pb + ln * 4 + comp;
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < WARPS; ++w) sum += src[w * 32 * 4];
+                if (n < a.N) {
+                    const float v = __fmul_rn(__fmul_rn(sum, unshift[m]), a.s_w[n]);
+                    a.y[static_cast<size_t>(m) * a.N + n] = __float2bfloat16_rn(v);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tfree(b));
         }
         return;
     }
 
     // -------------------------------------------------------------- consumers
     const int tid = threadIdx.x;
-    stage_x<CONV>(a, smem, L, tid);
+    grid_dependency_wait();
+    stage_x(a, smem, L, tid);
     const int g = lane >> 2, t = lane & 3;
     const uint8_t* xrow = smem + L.x_off + g * L.xpitch;
     const bool xok = g < a.M;
@@ -366,21 +430,22 @@ w8a16_tma_kernel(const __grid_constant__ CUtensorMap tmW, const Args a) {
         if (lane == 0) mbar_arrive(empty(s));  // the box is in registers: free the slot
         uint4 xa, xc;
         load_x(xrow, xok, kw * WIN + warp * BOX_K + 16 * t, xa, xc);
-        piece_mma<CONV>(acc, A, B, xa, xc);
+        piece_mma(acc, A, B, xa, xc);
         if (++kw == kwin) {
-            flush(acc, partial, ct, warp, lane);
+            const int b = ct & 1;
+            if (!mbar_wait(tfree(b), ((ct >> 1) & 1u) ^ 1u, a.timeout_ns, a.status)) break;
+            flush(acc, partial + b * WARPS * 32 * 4, 0, warp, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tfull(b));
             kw = 0;
             ++ct;
         }
         if (++s == S) { s = 0; ph ^= 1u; }
     }
-    named_barrier(1, CTHREADS);
-    reduce_store<CONV>(a, smem, L, t0, ntl, tid);
 }
 
 // -------------------------------------------------------- register kernel
 
-template <int CONV>
 __global__ void __launch_bounds__(CTHREADS, 1) w8a16_reg_kernel(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const Smem L = smem_layout(a.M, a.KP, a.max_tpc, 0);
@@ -430,7 +495,7 @@ __global__ void __launch_bounds__(CTHREADS, 1) w8a16_reg_kernel(const Args a) {
 #pragma unroll
     for (int d = 0; d < DEPTH; ++d) load_next(ra[d], rb[d]);
 
-    stage_x<CONV>(a, smem, L, threadIdx.x);
+    stage_x(a, smem, L, threadIdx.x);
     const uint8_t* xrow = smem + L.x_off + g * L.xpitch;
     const bool xok = g < a.M;
     float* partial = reinterpret_cast<float*>(smem + L.part_off);
@@ -447,7 +512,7 @@ __global__ void __launch_bounds__(CTHREADS, 1) w8a16_reg_kernel(const Args a) {
                 for (int h = 0; h < 2; ++h) {
                     uint4 xa, xc;
                     load_x(xrow, xok, k0 + 64 * h, xa, xc);
-                    piece_mma<CONV>(acc, ra[d][h], rb[d][h], xa, xc);
+                    piece_mma(acc, ra[d][h], rb[d][h], xa, xc);
                 }
                 load_next(ra[d], rb[d]);
                 k0 += 16 * CHUNK;
@@ -461,7 +526,7 @@ __global__ void __launch_bounds__(CTHREADS, 1) w8a16_reg_kernel(const Args a) {
         }
     }
     __syncthreads();
-    reduce_store<CONV>(a, smem, L, t0, ntl, threadIdx.x);
+    reduce_store(a, smem, L, t0, ntl, threadIdx.x);
 }
 
 }  // namespace w8a16
@@ -490,11 +555,9 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
     if (rc) return rc;
     static bool attr_done[64];
     if (!attr_done[di.device]) {
-        const cudaError_t es[4] = {
-            cudaFuncSetAttribute(w8a16_tma_kernel<CONV_CVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin),
-            cudaFuncSetAttribute(w8a16_tma_kernel<CONV_PLACE>, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin),
-            cudaFuncSetAttribute(w8a16_reg_kernel<CONV_CVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin),
-            cudaFuncSetAttribute(w8a16_reg_kernel<CONV_PLACE>, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin)};
+        const cudaError_t es[2] = {
+            cudaFuncSetAttribute(w8a16_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin),
+            cudaFuncSetAttribute(w8a16_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin)};
         for (cudaError_t e : es)
             if ((rc = cuda_check(e, "cudaFuncSetAttribute(w8a16)"))) return rc;
         attr_done[di.device] = true;
@@ -514,7 +577,6 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
     a.timeout_ns = watchdog_ns();
     const int budget = di.max_smem_optin;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool cvt = g_conv == CONV_CVT;
 
     // TMA path (K % 64 == 0, so the 3-D view never reaches past a row): x rows
     // cover whole 1024-byte windows; as many ring stages (12 down to 3) as fit
@@ -522,22 +584,20 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
     a.cpw = 0;
     if (K % BOX_K == 0) {
         // one CTA per SM; the deepest ring (12 down to 3 stages) that fits next
-        // to x and the partial sums; more CTAs only if even 3 stages do not fit
-        for (int grid = a.tiles < di.num_sms ? a.tiles : di.num_sms; grid <= a.tiles; ++grid) {
-            const int max_tpc = (a.tiles + grid - 1) / grid;
-            int stages = 12;
-            Smem L = smem_layout(a.M, a.KP, max_tpc, stages);
-            while (L.total > budget && stages > 3) L = smem_layout(a.M, a.KP, max_tpc, --stages);
-            if (L.total > budget) continue;
-            a.max_tpc = max_tpc;
+        // to x and the double-buffered partial sums
+        const int grid = a.tiles < di.num_sms ? a.tiles : di.num_sms;
+        int stages = 12;
+        Smem L = smem_layout(a.M, a.KP, 2, stages);
+        while (L.total > budget && stages > 3) L = smem_layout(a.M, a.KP, 2, --stages);
+        if (L.total <= budget) {
+            a.max_tpc = (a.tiles + grid - 1) / grid;
             a.stages = stages;
             // preferred view {64 B, rows, k-groups}: the box lands as one 16-row
             // block per consumer warp (conflict-free reads); if the encoder wants
             // monotonic strides, the view {64 B, k-groups, rows} (row-major box)
             CUtensorMap tm;
             a.wlayout = 0;
-            if (g_layout == 1 ||
-                make_tmap_3d_u8(&tm, wq, BOX_K, static_cast<uint64_t>(N), static_cast<uint64_t>(K / BOX_K),
+            if (make_tmap_3d_u8(&tm, wq, BOX_K, static_cast<uint64_t>(N), static_cast<uint64_t>(K / BOX_K),
                                 static_cast<uint64_t>(K), BOX_K, BOX_K, 16, WARPS) != METIS_OK) {
                 clear_error();
                 a.wlayout = 1;
@@ -546,9 +606,17 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
                                           BOX_K, WARPS, 16)))
                     return rc;
             }
-            if (cvt) w8a16_tma_kernel<CONV_CVT><<<grid, TMA_THREADS, L.total, st>>>(tm, a);
-            else w8a16_tma_kernel<CONV_PLACE><<<grid, TMA_THREADS, L.total, st>>>(tm, a);
-            return cuda_check(cudaGetLastError(), "w8a16 launch");
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(grid, 1, 1);
+            cfg.blockDim = dim3(TMA_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = L.total;
+            cfg.stream = st;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            return cuda_check(cudaLaunchKernelEx(&cfg, w8a16_tma_kernel, tm, a), "w8a16 launch");
         }
     }
     // register path
@@ -565,19 +633,6 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
     }
     if (L.total > budget) return fail(METIS_ERR_UNSUPPORTED, "w8a16_gemm: K too large");
     a.max_tpc = max_tpc;
-    if (cvt) w8a16_reg_kernel<CONV_CVT><<<grid, CTHREADS, L.total, st>>>(a);
-    else w8a16_reg_kernel<CONV_PLACE><<<grid, CTHREADS, L.total, st>>>(a);
+    w8a16_reg_kernel<<<grid, CTHREADS, L.total, st>>>(a);
     return cuda_check(cudaGetLastError(), "w8a16 launch");
-}
-
-// Tuning hook: bit 0 selects the E4M3 -> FP16 widening of metis_w8a16_gemm
-// (0: cvt instruction, 1: bit placement); bit 1 forces the row-major weight
-// box layout. Returns the previous setting.
-extern "C" METIS_API int metis_internal_w8a16_variant(int v) {
-    const int old = w8a16::g_conv | (w8a16::g_layout == 1 ? 2 : 0);
-    if (v >= 0 && v <= 3) {
-        w8a16::g_conv = v & 1;
-        w8a16::g_layout = (v & 2) ? 1 : -1;
-    }
-    return old;
 }

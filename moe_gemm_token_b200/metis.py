@@ -197,10 +197,3 @@ def metis_linear(x, wq, s_w, y, fast_math=True, s_tok=None, workspace=None, stre
         ws_bytes, _s(stream)))
 
 
-
-def metis_internal_w8a16_variant(v):
-    """Tuning hook: E4M3 widening of the W8A16 kernel (0: cvt, 1: bit placement)."""
-    fn = load().metis_internal_w8a16_variant
-    fn.argtypes = [ctypes.c_int]
-    fn.restype = ctypes.c_int
-    return fn(int(v))

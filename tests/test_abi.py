@@ -69,6 +69,15 @@ def test_host_validation_without_gpu(lib):
     assert lib.metis_fp8_gemm(p, 0, p, p, p, p, 16, 500, 256, null, 0, null) == metis.METIS_ERR_INVALID_ARG
     assert lib.metis_fp8_gemm(p, 7, p, p, p, p, 16, 512, 256, null, 0, null) == metis.METIS_ERR_INVALID_ARG
     assert lib.metis_fp8_gemm(p, 0, p, p, p, p, 0, 512, 256, null, 0, null) == metis.METIS_OK
+    # fused quantization (BF16 A): a workspace of align256(4 * M) bytes, 16-byte aligned
+    need = lib.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, 300, 512, 256, 0, 0)
+    assert need == 1280
+    assert lib.metis_fp8_gemm(p, 1, p, p, p, p, 300, 512, 256, null, 0, null) == metis.METIS_ERR_INVALID_ARG
+    assert b"workspace" in lib.metis_last_error()
+    assert lib.metis_fp8_gemm(p, 1, p, p, p, p, 300, 512, 256, p, need - 4, null) == \
+        metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_fp8_gemm(p, 1, p, p, p, p, 300, 512, 256, ctypes.c_void_p(0x1004), need,
+                              null) == metis.METIS_ERR_INVALID_ARG
     # W8A16: M > 8, K too large
     assert lib.metis_w8a16_gemm(p, p, p, p, 9, 128, 256, null) == metis.METIS_ERR_INVALID_ARG
     assert b"M <= 8" in lib.metis_last_error()

@@ -122,17 +122,90 @@ def test_fp8_gemm_exact_integer_products(metis):
     assert_bytes_equal(bf16_host(y), yr, "bf16 bits")
 
 
-@pytest.fixture(params=[0, 1], ids=["cvt", "place"])
-def widening(request, metis):
-    old = metis.metis_internal_w8a16_variant(request.param)
-    yield request.param
-    metis.metis_internal_w8a16_variant(old)
+def _fused(metis, xd, wq, s_w, M, N, K):
+    ws = torch.empty((metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0),),
+                     dtype=torch.uint8, device="cuda")
+    s_tok = torch.full((M,), float("nan"), dtype=torch.float32, device="cuda")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_fp8_gemm(xd, metis.METIS_A_BF16, s_tok, wq, s_w, y, workspace=ws)
+    assert metis.metis_check_device_status() == 0
+    return y, s_tok
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 16), (16, 512, 256), (100, 264, 208), (128, 256, 128),
+                                   (129, 264, 1040), (300, 520, 272), (520, 784, 1024),
+                                   (257, 1024, 2048), (300, 264, 20480)])
+def test_fp8_gemm_fused_parity(metis, M, N, K):
+    """BF16 A quantized inside the GEMM (a_kind = BF16): the scales equal the
+    standalone quantizer's and the oracle's bit for bit; y is within tolerance
+    of the oracle and identical to the unfused GEMM on the standalone codes
+    (same codes in shared memory, same accumulation order)."""
+    d = synth.linear(M * 5 + N + K, M, K, N, outlier_channels=4, outlier_scale=20.0,
+                     zero_rows=(M // 3,))
+    wq, s_w = _prep_weights(metis, d["w"])
+    xd = bf16_dev(d["x"])
+    xq = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    s1 = torch.empty((M,), dtype=torch.float32, device="cuda")
+    metis.metis_quant_fp8_per_token(xd, xq, s1)
+    y1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_fp8_gemm(xq, metis.METIS_A_E4M3, s1, wq, s_w, y1)
+    y2, s2 = _fused(metis, xd, wq, s_w, M, N, K)
+    wq_r, sw_r = oracle.quant_per_channel(d["w"])
+    _, y64, _, st_r = oracle.linear_w8a8(d["x"], wq_r, sw_r)
+    assert_bytes_equal(s2.cpu().numpy().view(np.uint32), st_r.view(np.uint32), "fused s_tok")
+    assert_close(bf16_host(y2), y64, f"fused y {M}x{N}x{K}")
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), "fused != unfused"
+
+
+def test_fp8_gemm_fused_extremes(metis):
+    """Rows near the ends of the BF16 range, all-zero rows and rows with one
+    non-zero element go through the in-kernel quantization like the
+    standalone quantizer (saturation, zero scale)."""
+    rng = np.random.default_rng(23)
+    M, N, K = 160, 264, 384
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[0] *= 1.0e35 / np.abs(x[0]).max()        # huge scale, y still representable in BF16
+    x[1] *= 1.0e-38                            # tiny, partly subnormal after scaling
+    x[2] = 0.0
+    x[3] = 0.0
+    x[3, 17] = -2.5
+    x[150:] *= 1000.0                          # the second 128-row block
+    xb = synth.f32_to_bf16_bits(x)
+    w = rng.standard_normal((N, K)).astype(np.float32)
+    wq, s_w = _prep_weights(metis, w)
+    y2, s2 = _fused(metis, bf16_dev(xb), wq, s_w, M, N, K)
+    wq_r, sw_r = oracle.quant_per_channel(w)
+    _, y64, _, st_r = oracle.linear_w8a8(xb, wq_r, sw_r)
+    assert_bytes_equal(s2.cpu().numpy().view(np.uint32), st_r.view(np.uint32), "fused s_tok")
+    assert np.all(bf16_host(y2)[2] == 0)
+    assert_close(bf16_host(y2), y64, "fused extremes")
+
+
+def test_linear_fast_math_is_the_fused_gemm(metis):
+    """M > 8 with fast_math takes the fused-quantization W8A8 GEMM."""
+    M, N, K = 64, 256, 512
+    d = synth.linear(22, M, K, N)
+    wq, s_w = _prep_weights(metis, d["w"])
+    xd = bf16_dev(d["x"])
+    y1, s1 = _fused(metis, xd, wq, s_w, M, N, K)
+    ws = torch.empty((metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0),),
+                     dtype=torch.uint8, device="cuda")
+    s2 = torch.empty((M,), dtype=torch.float32, device="cuda")
+    y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_linear(xd, wq, s_w, y2, fast_math=True, s_tok=s2, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(s1, s2)
+    with pytest.raises(metis.MetisError) as ei:
+        metis.metis_linear(xd, wq, s_w, y2, fast_math=False, s_tok=s2, workspace=ws)
+    assert ei.value.code == metis.METIS_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 1000, 4096), (2, 37, 272), (3, 300, 12288), (4, 1000, 4096),
                                    (5, 48, 1024), (8, 1000, 4096), (8, 16, 16), (7, 2333, 1040),
-                                   (6, 148 * 16 * 7 + 5, 2048)])
-def test_w8a16_parity(metis, widening, M, N, K):
+                                   (6, 148 * 16 * 7 + 5, 2048), (8, 3000, 8192), (1, 64, 12288),
+                                   (8, 57344, 4096)])
+def test_w8a16_parity(metis, M, N, K):
     d = synth.linear(M + 13 * N + K, M, K, N)
     wq, s_w = _prep_weights(metis, d["w"])
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -144,7 +217,7 @@ def test_w8a16_parity(metis, widening, M, N, K):
     assert_close(bf16_host(y), y64, f"w8a16 {M}x{N}x{K}")
 
 
-def test_w8a16_subnormal_weights_and_wide_x(metis, widening):
+def test_w8a16_subnormal_weights_and_wide_x(metis):
     """Weight rows with many E4M3 subnormal codes and tokens whose elements
     span many binades: the widening and the per-token shift stay exact."""
     rng = np.random.default_rng(5)
@@ -175,11 +248,11 @@ def test_linear_dispatch(metis):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
-def test_w8a16_all_subnormal_codes_exact(metis, widening):
+def test_w8a16_all_subnormal_codes_exact(metis):
     """Every weight code is an E4M3 subnormal (+-m * 2^-9) and x holds small
     integers, so every product and partial sum is exact in FP32: the output
-    must equal the oracle's BF16 bits. A widening or a tensor core that
-    flushed FP16 subnormals would return zeros here."""
+    must equal the oracle's BF16 bits. A widening that lost E4M3 subnormals
+    would return zeros here."""
     rng = np.random.default_rng(8)
     M, N, K = 8, 64, 256
     codes = (rng.integers(1, 8, (N, K)) | (rng.integers(0, 2, (N, K)) << 7)).astype(np.uint8)
