@@ -113,8 +113,12 @@ METIS_API int metis_quant_fp8_per_channel(const float* w, int64_t N, int64_t K, 
  *   a_kind = METIS_A_BF16: `a` is BF16 [M, K] (dense rows); the per-token
  *            quantization is fused into the GEMM (an amax pre-pass writes
  *            s_tok [M] as an OUTPUT, identical to metis_quant_fp8_per_token,
- *            and the E4M3 codes are produced in shared memory, never in HBM).
- *            Needs `workspace` of metis_workspace_size(METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0)
+ *            and the E4M3 codes are produced in shared memory, never in HBM;
+ *            the output is bit-identical to quantizer + E4M3 GEMM). Each A
+ *            tile is converted once per 256-column output tile, so for wide
+ *            N this variant is slower than the two separate calls, which is
+ *            what metis_linear uses. Needs `workspace` of
+ *            metis_workspace_size(METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0)
  *            bytes (16-byte aligned).
  *   wq [N, K] E4M3 (one row per output channel), s_w [N] FP32, y [M, N] BF16 out.
  *   Requires K % 16 == 0, N % 8 == 0, K >= 16, N >= 8, M >= 0; a, wq, y
@@ -185,11 +189,13 @@ METIS_API int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int32
 /* Workspace sizes in bytes.
  *   METIS_OP_FP8_GEMM_FUSED: (M, N, K) of metis_fp8_gemm with a_kind = METIS_A_BF16.
  *   METIS_OP_MOE:            (T, I, H, topk, E) of metis_moe_fp8_grouped_gemm.
+ *   METIS_OP_LINEAR:         (M, N, K) of metis_linear with fast_math != 0.
  *   Other ops need none (0). Returns 0 for invalid arguments. */
 #define METIS_OP_FP8_GEMM 0
 #define METIS_OP_FP8_GEMM_FUSED 1
 #define METIS_OP_W8A16 2
 #define METIS_OP_MOE 3
+#define METIS_OP_LINEAR 4
 METIS_API size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, int64_t K_or_H,
                             int64_t topk, int64_t E);
 
@@ -222,10 +228,12 @@ METIS_API int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk
 /* The dispatch rule of the cards ("Lernex/Metis-1.6-Praxis-NVFP4", "What
  * --fast-math does"): M <= 8 tokens always take the default maths
  * (metis_w8a16_gemm); more tokens take the fast-math W8A8 path when
- * fast_math != 0 (quantizing x per token, fused: a_kind = METIS_A_BF16), and
- * otherwise the large-M default path, which this build does not implement
- * (METIS_ERR_UNSUPPORTED). s_tok [M] receives the per-token scales on the
- * fast-math path. `workspace` as for metis_fp8_gemm with METIS_A_BF16. */
+ * fast_math != 0 (metis_quant_fp8_per_token into the workspace, then
+ * metis_fp8_gemm with a_kind = METIS_A_E4M3), and otherwise the large-M
+ * default path, which this build does not implement (METIS_ERR_UNSUPPORTED).
+ * s_tok [M] receives the per-token scales on the fast-math path; `workspace`
+ * holds the E4M3 codes: metis_workspace_size(METIS_OP_LINEAR, M, N, K, 0, 0)
+ * bytes, 16-byte aligned (0 for M <= 8). */
 METIS_API int metis_linear(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
                  int64_t M, int64_t N, int64_t K, int fast_math, float* s_tok,
                  void* workspace, size_t ws_bytes, metis_stream_t stream);

@@ -225,6 +225,9 @@ extern "C" size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, i
         case METIS_OP_FP8_GEMM_FUSED:
             // per-token reciprocal scales 448/amax, one FP32 per row
             return static_cast<size_t>(align256(4 * (M_or_T > 0 ? M_or_T : 1)));
+        case METIS_OP_LINEAR:
+            // E4M3 codes of x for the W8A8 path (nothing for the M <= 8 path)
+            return M_or_T <= 8 ? 0 : static_cast<size_t>(align256(M_or_T * K_or_H));
         case METIS_OP_MOE: {
             if (topk < 1 || E < 1) return 0;
             int64_t total = 0;
@@ -251,6 +254,17 @@ extern "C" int metis_linear(const void* x_bf16, const uint8_t* wq, const float* 
         return fail(METIS_ERR_UNSUPPORTED,
                     "metis_linear: the default (16-bit) maths for M > 8 tokens is not built; "
                     "pass fast_math=1");
-    return metis_fp8_gemm(x_bf16, METIS_A_BF16, s_tok, wq, s_w, y_bf16, M, N, K, workspace,
-                          ws_bytes, stream);
+    if (M > 0 && M * K > 0 && K % 16 == 0) {
+        const size_t need = metis_workspace_size(METIS_OP_LINEAR, M, N, K, 0, 0);
+        if (!workspace || ws_bytes < need || !aligned(workspace, 16))
+            return fail(METIS_ERR_INVALID_ARG,
+                        "metis_linear: needs a 16-byte aligned workspace of %zu bytes (got %zu)",
+                        need, ws_bytes);
+    }
+    // the separate quantizer: cheaper than converting each A tile once per
+    // output tile inside the GEMM (see metis_fp8_gemm with METIS_A_BF16)
+    uint8_t* xq = static_cast<uint8_t*>(workspace);
+    int rc = metis_quant_fp8_per_token(x_bf16, M, K, K, xq, K, s_tok, stream);
+    if (rc) return rc;
+    return metis_fp8_gemm(xq, METIS_A_E4M3, s_tok, wq, s_w, y_bf16, M, N, K, nullptr, 0, stream);
 }

@@ -12,17 +12,21 @@
 //  * TMA kernel (K % 64 == 0): a producer thread streams each tile through a
 //    3-D view of the weights, {64 bytes, rows (stride K), 64-byte k-groups},
 //    one 16 x 16 x 64-byte box (16 KB: 16 rows x a 1024-byte k-window) per
-//    ring stage, laid out as one 16-row x 64-byte block per consumer warp;
-//    the deepest ring that fits (up to 12 stages, ~190 KB per SM in flight)
-//    without occupying registers. 16 consumer warps read their box (rows g and
-//    g+8, 16 bytes per thread, conflict-free), widen E4M3 to FP16 and issue
-//    mma.sync.m16n8k16 with the weights as the M = 16 operand and the <= 8
-//    tokens as n = 8 (four independent FP32 accumulators). A reducer warp
-//    adds each finished tile's partial sums (double-buffered) and stores it
-//    while the stream goes on. Launched as a programmatic dependent: barrier
-//    set-up and an L2 prefetch of the first ring's worth of weights overlap
-//    the previous kernel; x is read, y written and shared memory filled only
-//    after the grid dependency is resolved.
+//    ring stage, laid out as one 16-row x 64-byte block per consumer warp,
+//    8 stages (128 KB per SM in flight). 16 consumer warps read their box
+//    (rows g and g+8, 16 bytes per thread, conflict-free), widen E4M3 to
+//    FP16 and issue mma.sync.m16n8k16 with the weights as the M = 16 operand
+//    and the <= 8 tokens as n = 8 (four independent FP32 accumulators). For
+//    K <= 4096 each thread keeps the x fragments it needs for every k-window
+//    in registers (32 registers at K = 4096), so x is read once per CTA and
+//    never staged; larger K stages x in shared memory. The rows of W are
+//    split over the CTAs in 8-row units (at most 8 rows of imbalance); a
+//    CTA walks its rows as 16-row tiles. A reducer warp adds each finished
+//    tile's partial sums (double-buffered) and stores it while the stream
+//    goes on. Launched as a programmatic dependent: barrier set-up and an L2
+//    prefetch of the first 4 stages of weights overlap the previous kernel;
+//    x is read, y written and shared memory filled only after the grid
+//    dependency is resolved.
 //  * register kernel (K % 64 != 0, or when x plus a ring do not fit in
 //    shared memory): 16 warps stream 128-byte chunks of the rows straight
 //    into registers, 4 chunks in flight per thread.
@@ -49,6 +53,14 @@ constexpr int MAX_K = 12288;
 constexpr int BOX_K = 64;                   // bytes of K per box (one consumer warp)
 constexpr int WIN = WARPS * BOX_K;          // k-window per stage: 1024
 constexpr int STAGE_BYTES = 16 * WIN;       // 16 rows x 1024 = 16 KB
+// Ring depth and L2 warm-up: measured on B200 (K = 4096, N = 14336, cold
+// weights, calls back to back), 8 stages with the first 4 prefetched beat
+// deeper rings (12 stages: +1 us) and prefetching a CTA's whole range (+3 us).
+constexpr int MAX_STAGES = 8;
+constexpr int L2_PREFETCH = 4;
+
+constexpr int MISC_BYTES = 128 + WARPS * 8 * 4;
+constexpr int MAX_REG_KWIN = 4;             // x held in registers up to K = 4096
 
 // register kernel geometry
 constexpr int DEPTH = 4;    // chunks in flight per thread
@@ -104,6 +116,7 @@ struct Args {
     int KP;       // K rounded up to the k-range the warps visit (zero-padded in x)
     int cpw;      // register kernel: 128-byte chunks per warp per tile
     int tiles;    // ceil(N / 16)
+    int units;    // TMA kernel: ceil(N / 8), split evenly over the CTAs
     int max_tpc;  // max tiles per CTA (sizes the partial-sum buffer)
     int stages;   // TMA kernel: ring stages
     int wlayout;  // TMA kernel box layout: 0 = [k-group][row][64 B], 1 = [row][k-group][64 B]
@@ -115,19 +128,20 @@ struct Args {
 struct Smem {
     int xpitch;    // bytes per staged x row (2 * KP + 16: 16 mod 128 -> conflict-free)
     int x_off;     // [M][xpitch] FP16
-    int misc_off;  // unshift[8] f32, shift/amax[8], pow2[8]
+    int misc_off;  // unshift[8] f32, shift/amax[8], pow2[8], per-warp amax [16][8]
     int part_off;  // [part_tiles][16 warps][32 lanes][4] f32
     int ring_off;  // TMA ring
     int bar_off;   // full[stages], empty[stages], tfull[2], tfree[2]
     int total;
 };
 
-__host__ __device__ inline Smem smem_layout(int M, int KP, int part_tiles, int stages) {
+// x_rows = 0: x is not staged in shared memory (the register-resident path).
+__host__ __device__ inline Smem smem_layout(int x_rows, int KP, int part_tiles, int stages) {
     Smem s;
     s.xpitch = 2 * KP + 16;
     s.x_off = 0;
-    s.misc_off = M * s.xpitch;  // 16-byte aligned
-    s.part_off = s.misc_off + 128;
+    s.misc_off = x_rows * s.xpitch;  // 16-byte aligned
+    s.part_off = s.misc_off + MISC_BYTES;
     s.ring_off = s.part_off + part_tiles * WARPS * 32 * 16;
     s.ring_off = (s.ring_off + 127) & ~127;  // TMA destination alignment
     s.bar_off = s.ring_off + stages * STAGE_BYTES;
@@ -304,10 +318,71 @@ __device__ __forceinline__ void reduce_store(const Args& a, const uint8_t* smem,
 
 constexpr int TMA_THREADS = CTHREADS + 64;  // + producer warp + reducer warp
 
+// x fragments of this thread held in registers, KWIN k-windows: token g,
+// elements kw * 1024 + warp * 64 + 16 t + [0, 16) as FP16 after the
+// per-token power-of-two shift (the same shift as stage_x). The per-token
+// amax comes from the four lanes that share g and a per-warp table in shared
+// memory (one named barrier over the consumer threads).
+template <int KWIN>
+__device__ __forceinline__ void x_to_regs(const Args& a, uint8_t* smem, const Smem& L, int warp,
+                                          int lane, uint32_t (&xr)[KWIN][8]) {
+    const int g = lane >> 2, t = lane & 3;
+    float* unshift = reinterpret_cast<float*>(smem + L.misc_off);
+    unsigned* wmax = reinterpret_cast<unsigned*>(smem + L.misc_off + 128);  // [16 warps][8]
+    uint4 raw[KWIN][2];
+    float mx = 0.0f;
+#pragma unroll
+    for (int kw = 0; kw < KWIN; ++kw) {
+        const int k0 = kw * WIN + warp * BOX_K + 16 * t;
+        if (g < a.M && k0 < a.K) {
+            const uint4* p = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(g) * a.K + k0);
+            raw[kw][0] = p[0];
+            raw[kw][1] = p[1];
+        } else {
+            raw[kw][0] = raw[kw][1] = make_uint4(0, 0, 0, 0);
+        }
+    }
+#pragma unroll
+    for (int kw = 0; kw < KWIN; ++kw)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t wv[4] = {raw[kw][h].x, raw[kw][h].y, raw[kw][h].z, raw[kw][h].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fmaxf(fabsf(bf16_lo(wv[i])), fabsf(bf16_hi(wv[i]))));
+        }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if (t == 0) wmax[warp * 8 + g] = __float_as_uint(mx);
+    named_barrier(1, CTHREADS);
+    unsigned am = 0;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) am = max(am, wmax[w * 8 + g]);
+    const float amax = __uint_as_float(am);
+    const int sh = amax > 0.0f ? 14 - ilogbf(amax) : 0;
+    const float p2 = (sh >= -126 && sh <= 127) ? __uint_as_float(static_cast<uint32_t>(sh + 127) << 23) : 0.0f;
+    if (warp == 0 && t == 0) unshift[g] = ldexpf(1.0f, -sh);
+#pragma unroll
+    for (int kw = 0; kw < KWIN; ++kw)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint4 out;
+            widen8(raw[kw][h], sh, p2, out);
+            xr[kw][4 * h] = out.x;
+            xr[kw][4 * h + 1] = out.y;
+            xr[kw][4 * h + 2] = out.z;
+            xr[kw][4 * h + 3] = out.w;
+        }
+}
+
+// KWIN > 0: K <= KWIN * 1024 and x lives in registers; KWIN == 0: any K up
+// to MAX_K, x staged in shared memory. Each CTA owns the rows
+// [8 u0, 8 u1) of W (8-row units split evenly over the grid), walked as
+// 16-row tiles; rows past 8 u1 that the last tile loads are not stored.
+template <int KWIN>
 __global__ void __launch_bounds__(TMA_THREADS, 1)
 w8a16_tma_kernel(const __grid_constant__ CUtensorMap tmW, const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const Smem L = smem_layout(a.M, a.KP, 2, a.stages);
+    const Smem L = smem_layout(KWIN > 0 ? 0 : a.M, a.KP, 2, a.stages);
     uint8_t* ring = smem + L.ring_off;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
     const int S = a.stages;
@@ -318,17 +393,19 @@ w8a16_tma_kernel(const __grid_constant__ CUtensorMap tmW, const Args a) {
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int t0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * a.tiles / gridDim.x);
-    const int t1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * a.tiles / gridDim.x);
-    const int ntl = t1 - t0;
+    const int u0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * a.units / gridDim.x);
+    const int u1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * a.units / gridDim.x);
+    const int row0 = 8 * u0;                             // first row of this CTA
+    const int row_end = 8 * u1 < a.N ? 8 * u1 : a.N;     // rows it stores
+    const int ntl = (u1 - u0 + 1) / 2;                   // 16-row tiles
     const int kwin = a.KP / WIN;    // k-windows per tile
     const int nstage = ntl * kwin;  // stages this CTA streams
     auto box_coords = [&](int i, int& x, int& y, int& z) {
         const int tl = i / kwin;
         const int kw = i - tl * kwin;
         x = 0;
-        y = a.wlayout == 0 ? (t0 + tl) * 16 : kw * WARPS;
-        z = a.wlayout == 0 ? kw * WARPS : (t0 + tl) * 16;
+        y = a.wlayout == 0 ? row0 + 16 * tl : kw * WARPS;
+        z = a.wlayout == 0 ? kw * WARPS : row0 + 16 * tl;
     };
 
     if (threadIdx.x == 0) {
@@ -354,7 +431,7 @@ w8a16_tma_kernel(const __grid_constant__ CUtensorMap tmW, const Args a) {
         // memory once the grid dependency is resolved. Consumers wait for
         // every stage issued here before the CTA ends.
         if (lane == 0) {
-            for (int i = 0; i < nstage && i < S; ++i) {
+            for (int i = 0; i < nstage && i < S && i < L2_PREFETCH; ++i) {
                 int x, y, z;
                 box_coords(i, x, y, z);
                 tma_prefetch_l2_3d(&tmW, x, y, z);
@@ -387,14 +464,14 @@ w8a16_tma_kernel(const __grid_constant__ CUtensorMap tmW, const Args a) {
             for (int o = lane; o < 16 * a.M; o += 32) {
                 const int m = o >> 4;
                 const int row = o & 15;
-                const int n = (t0 + tl) * 16 + row;
+                const int n = row0 + 16 * tl + row;
                 const int ln = (row & 7) * 4 + (m >> 1);
                 const int comp = (row >> 3) * 2 + (m & 1);
                 const float* src = pb + ln * 4 + comp;
                 float sum = 0.f;
 #pragma unroll
                 for (int w = 0; w < WARPS; ++w) sum += src[w * 32 * 4];
-                if (n < a.N) {
+                if (n < row_end) {
                     const float v = __fmul_rn(__fmul_rn(sum, unshift[m]), a.s_w[n]);
                     a.y[static_cast<size_t>(m) * a.N + n] = __float2bfloat16_rn(v);
                 }
@@ -408,39 +485,64 @@ w8a16_tma_kernel(const __grid_constant__ CUtensorMap tmW, const Args a) {
     // -------------------------------------------------------------- consumers
     const int tid = threadIdx.x;
     grid_dependency_wait();
-    stage_x(a, smem, L, tid);
     const int g = lane >> 2, t = lane & 3;
-    const uint8_t* xrow = smem + L.x_off + g * L.xpitch;
-    const bool xok = g < a.M;
     float* partial = reinterpret_cast<float*>(smem + L.part_off);
     float acc[4][4];
 #pragma unroll
     for (int s = 0; s < 4; ++s) acc[s][0] = acc[s][1] = acc[s][2] = acc[s][3] = 0.f;
+    const uint8_t* box0 = ring + 16 * t + (a.wlayout == 0 ? warp * 16 * BOX_K + g * BOX_K : g * WIN + warp * BOX_K);
+    const int rstep = a.wlayout == 0 ? 8 * BOX_K : 8 * WIN;  // rows g -> g + 8
     int s = 0;
     uint32_t ph = 0;
-    int kw = 0, ct = 0;
-    for (int i = 0; i < nstage; ++i) {
-        if (!mbar_wait(full(s), ph, a.timeout_ns, a.status)) break;
-        const uint8_t* box = ring + s * STAGE_BYTES + 16 * t +
-                             (a.wlayout == 0 ? warp * 16 * BOX_K + g * BOX_K : g * WIN + warp * BOX_K);
-        const int rstep = a.wlayout == 0 ? 8 * BOX_K : 8 * WIN;  // rows g -> g + 8
-        const uint4 A = *reinterpret_cast<const uint4*>(box);
-        const uint4 B = *reinterpret_cast<const uint4*>(box + rstep);
+    // one ring stage: this warp's 16 x 64-byte block into registers, slot freed
+    auto take = [&](uint4& A, uint4& B) -> bool {
+        if (!mbar_wait(full(s), ph, a.timeout_ns, a.status)) return false;
+        const uint8_t* box = box0 + s * STAGE_BYTES;
+        A = *reinterpret_cast<const uint4*>(box);
+        B = *reinterpret_cast<const uint4*>(box + rstep);
         __syncwarp();
-        if (lane == 0) mbar_arrive(empty(s));  // the box is in registers: free the slot
-        uint4 xa, xc;
-        load_x(xrow, xok, kw * WIN + warp * BOX_K + 16 * t, xa, xc);
-        piece_mma(acc, A, B, xa, xc);
-        if (++kw == kwin) {
-            const int b = ct & 1;
-            if (!mbar_wait(tfree(b), ((ct >> 1) & 1u) ^ 1u, a.timeout_ns, a.status)) break;
-            flush(acc, partial + b * WARPS * 32 * 4, 0, warp, lane);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tfull(b));
-            kw = 0;
-            ++ct;
-        }
+        if (lane == 0) mbar_arrive(empty(s));
         if (++s == S) { s = 0; ph ^= 1u; }
+        return true;
+    };
+    // a finished tile: partial sums to the reducer (double-buffered)
+    auto tile_done = [&](int ct) -> bool {
+        const int b = ct & 1;
+        if (!mbar_wait(tfree(b), ((ct >> 1) & 1u) ^ 1u, a.timeout_ns, a.status)) return false;
+        flush(acc, partial + b * WARPS * 32 * 4, 0, warp, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tfull(b));
+        return true;
+    };
+    if constexpr (KWIN > 0) {
+        uint32_t xr[KWIN][8];
+        x_to_regs<KWIN>(a, smem, L, warp, lane, xr);
+        bool ok = true;
+        for (int ct = 0; ct < ntl && ok; ++ct) {
+#pragma unroll
+            for (int kw = 0; kw < KWIN; ++kw) {
+                uint4 A, B;
+                if (!take(A, B)) { ok = false; break; }
+                piece_mma(acc, A, B, make_uint4(xr[kw][0], xr[kw][1], xr[kw][2], xr[kw][3]),
+                          make_uint4(xr[kw][4], xr[kw][5], xr[kw][6], xr[kw][7]));
+            }
+            if (ok) ok = tile_done(ct);
+        }
+    } else {
+        stage_x(a, smem, L, tid);
+        const uint8_t* xrow = smem + L.x_off + g * L.xpitch;
+        const bool xok = g < a.M;
+        bool ok = true;
+        for (int ct = 0; ct < ntl && ok; ++ct) {
+            for (int kw = 0; kw < kwin; ++kw) {
+                uint4 A, B;
+                if (!take(A, B)) { ok = false; break; }
+                uint4 xa, xc;
+                load_x(xrow, xok, kw * WIN + warp * BOX_K + 16 * t, xa, xc);
+                piece_mma(acc, A, B, xa, xc);
+            }
+            if (ok) ok = tile_done(ct);
+        }
     }
 }
 
@@ -555,9 +657,14 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
     if (rc) return rc;
     static bool attr_done[64];
     if (!attr_done[di.device]) {
-        const cudaError_t es[2] = {
-            cudaFuncSetAttribute(w8a16_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin),
-            cudaFuncSetAttribute(w8a16_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin)};
+        const int sm = di.max_smem_optin;
+        const cudaError_t es[6] = {
+            cudaFuncSetAttribute(w8a16_tma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm),
+            cudaFuncSetAttribute(w8a16_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm),
+            cudaFuncSetAttribute(w8a16_tma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm),
+            cudaFuncSetAttribute(w8a16_tma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm),
+            cudaFuncSetAttribute(w8a16_tma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm),
+            cudaFuncSetAttribute(w8a16_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm)};
         for (cudaError_t e : es)
             if ((rc = cuda_check(e, "cudaFuncSetAttribute(w8a16)"))) return rc;
         attr_done[di.device] = true;
@@ -585,12 +692,16 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
     if (K % BOX_K == 0) {
         // one CTA per SM; the deepest ring (12 down to 3 stages) that fits next
         // to x and the double-buffered partial sums
-        const int grid = a.tiles < di.num_sms ? a.tiles : di.num_sms;
-        int stages = 12;
-        Smem L = smem_layout(a.M, a.KP, 2, stages);
-        while (L.total > budget && stages > 3) L = smem_layout(a.M, a.KP, 2, --stages);
+        // x in registers for K <= 4096 (KWIN k-windows), else staged
+        const int kwin_reg = a.KP / WIN <= MAX_REG_KWIN ? a.KP / WIN : 0;
+        a.units = static_cast<int>((N + 7) / 8);
+        const int grid = a.units < di.num_sms ? a.units : di.num_sms;
+        const int x_rows = kwin_reg > 0 ? 0 : a.M;
+        int stages = MAX_STAGES;
+        Smem L = smem_layout(x_rows, a.KP, 2, stages);
+        while (L.total > budget && stages > 3) L = smem_layout(x_rows, a.KP, 2, --stages);
         if (L.total <= budget) {
-            a.max_tpc = (a.tiles + grid - 1) / grid;
+            a.max_tpc = 0;
             a.stages = stages;
             // preferred view {64 B, rows, k-groups}: the box lands as one 16-row
             // block per consumer warp (conflict-free reads); if the encoder wants
@@ -616,7 +727,15 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
             attr[0].val.programmaticStreamSerializationAllowed = 1;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
-            return cuda_check(cudaLaunchKernelEx(&cfg, w8a16_tma_kernel, tm, a), "w8a16 launch");
+            cudaError_t e;
+            switch (kwin_reg) {
+                case 1: e = cudaLaunchKernelEx(&cfg, w8a16_tma_kernel<1>, tm, a); break;
+                case 2: e = cudaLaunchKernelEx(&cfg, w8a16_tma_kernel<2>, tm, a); break;
+                case 3: e = cudaLaunchKernelEx(&cfg, w8a16_tma_kernel<3>, tm, a); break;
+                case 4: e = cudaLaunchKernelEx(&cfg, w8a16_tma_kernel<4>, tm, a); break;
+                default: e = cudaLaunchKernelEx(&cfg, w8a16_tma_kernel<0>, tm, a); break;
+            }
+            return cuda_check(e, "w8a16 launch");
         }
     }
     // register path

@@ -30,6 +30,7 @@ METIS_OP_FP8_GEMM = 0
 METIS_OP_FP8_GEMM_FUSED = 1
 METIS_OP_W8A16 = 2
 METIS_OP_MOE = 3
+METIS_OP_LINEAR = 4
 
 MOE_WS = dict(COUNTS=0, OFFSETS=1, SLOT_TO_ROW=2, ROW_TO_SLOT=3, AQ=4, SA=5, H=6, HQ=7, SH=8,
               O=9)
@@ -188,7 +189,8 @@ def metis_moe_workspace_offset(region, T, topk, E, H, I):
 
 
 def metis_linear(x, wq, s_w, y, fast_math=True, s_tok=None, workspace=None, stream=None):
-    """Dispatch rule: M <= 8 -> W8A16; otherwise W8A8 (fast_math) with fused quantization."""
+    """Dispatch rule: M <= 8 -> W8A16; otherwise W8A8 (fast_math): per-token
+    quantizer into `workspace`, then the E4M3 GEMM."""
     M, K = x.shape
     N = wq.shape[0]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -95,6 +95,12 @@ def test_host_validation_without_gpu(lib):
     assert b"workspace" in lib.metis_last_error()
     # dispatch: large M default maths is not built
     assert lib.metis_linear(p, p, p, p, 64, 128, 256, 0, p, p, 1 << 20, null) == metis.METIS_ERR_UNSUPPORTED
+    # fast-math dispatch needs room for the codes of x
+    assert lib.metis_workspace_size(metis.METIS_OP_LINEAR, 64, 128, 256, 0, 0) == 64 * 256
+    assert lib.metis_workspace_size(metis.METIS_OP_LINEAR, 8, 128, 256, 0, 0) == 0
+    assert lib.metis_linear(p, p, p, p, 64, 128, 256, 1, p, p, 64 * 256 - 16, null) == \
+        metis.METIS_ERR_INVALID_ARG
+    assert b"workspace" in lib.metis_last_error()
 
 
 def test_valid_call_without_gpu_fails_loudly(lib):

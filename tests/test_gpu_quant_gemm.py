@@ -181,21 +181,29 @@ def test_fp8_gemm_fused_extremes(metis):
     assert_close(bf16_host(y2), y64, "fused extremes")
 
 
-def test_linear_fast_math_is_the_fused_gemm(metis):
-    """M > 8 with fast_math takes the fused-quantization W8A8 GEMM."""
+def test_linear_fast_math(metis):
+    """M > 8 with fast_math: the per-token quantizer, then the E4M3 GEMM; the
+    result equals the two direct calls and the fused variant bit for bit."""
     M, N, K = 64, 256, 512
     d = synth.linear(22, M, K, N)
     wq, s_w = _prep_weights(metis, d["w"])
     xd = bf16_dev(d["x"])
     y1, s1 = _fused(metis, xd, wq, s_w, M, N, K)
-    ws = torch.empty((metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0),),
+    ws = torch.empty((metis.metis_workspace_size(metis.METIS_OP_LINEAR, M, N, K, 0, 0),),
                      dtype=torch.uint8, device="cuda")
     s2 = torch.empty((M,), dtype=torch.float32, device="cuda")
     y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     metis.metis_linear(xd, wq, s_w, y2, fast_math=True, s_tok=s2, workspace=ws)
+    xq = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    s3 = torch.empty((M,), dtype=torch.float32, device="cuda")
+    y3 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_quant_fp8_per_token(xd, xq, s3)
+    metis.metis_fp8_gemm(xq, metis.METIS_A_E4M3, s3, wq, s_w, y3)
     torch.cuda.synchronize()
+    assert torch.equal(y2.view(torch.int16), y3.view(torch.int16))
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
-    assert torch.equal(s1, s2)
+    assert torch.equal(s1, s2) and torch.equal(s2, s3)
+    assert torch.equal(ws[:M * K].view(M, K), xq)
     with pytest.raises(metis.MetisError) as ei:
         metis.metis_linear(xd, wq, s_w, y2, fast_math=False, s_tok=s2, workspace=ws)
     assert ei.value.code == metis.METIS_ERR_UNSUPPORTED
@@ -204,7 +212,8 @@ def test_linear_fast_math_is_the_fused_gemm(metis):
 @pytest.mark.parametrize("M,N,K", [(1, 1000, 4096), (2, 37, 272), (3, 300, 12288), (4, 1000, 4096),
                                    (5, 48, 1024), (8, 1000, 4096), (8, 16, 16), (7, 2333, 1040),
                                    (6, 148 * 16 * 7 + 5, 2048), (8, 3000, 8192), (1, 64, 12288),
-                                   (8, 57344, 4096)])
+                                   (8, 57344, 4096), (3, 777, 2560), (8, 100, 3072), (1, 5, 1024),
+                                   (8, 9, 2048), (2, 148 * 8 + 3, 4096)])
 def test_w8a16_parity(metis, M, N, K):
     d = synth.linear(M + 13 * N + K, M, K, N)
     wq, s_w = _prep_weights(metis, d["w"])
