@@ -216,8 +216,8 @@ def gemm_traffic_from_profile():
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     vals = {}
     for line in open(path):
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
+        if ": " in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(": ", 1)
             vals[k.strip()] = v.strip().strip("`")
     if vals.get("kernel source sha256[:16]") != sha:
         return None
