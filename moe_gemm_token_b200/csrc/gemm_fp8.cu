@@ -124,12 +124,12 @@ struct Sched {
             const int e = lo;
             const int local = t - g_tile[e];
             const int rows = g_row[e + 1] - g_row[e];
-            const int mt = (rows + ROWS - 1) / ROWS;
+            const int mt = (rows + ROWS * CTAS - 1) / (ROWS * CTAS);
             const int mb = local % mt;
             const int nb = local / mt;
-            ti.a_row0 = g_row[e] + mb * ROWS;
+            ti.a_row0 = g_row[e] + mb * ROWS * CTAS + static_cast<int>(rank) * ROWS;
             ti.row_end = g_row[e + 1];
-            ti.b_row0 = e * N + nb * BN;
+            ti.b_row0 = e * N + nb * BN + static_cast<int>(rank) * (BN / CTAS);
             ti.n0 = nb * BN;
             ti.group = e;
         }
@@ -255,7 +255,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const int e = g0 + i;
                 if (e < p.E) {
                     const int rows = p.offsets[e + 1] - p.offsets[e];
-                    local += ((rows + ROWS - 1) / ROWS) * sc.num_n;
+                    local += ((rows + ROWS * CTAS - 1) / (ROWS * CTAS)) * sc.num_n;
                 }
             }
             int incl = local;
@@ -271,7 +271,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     const int rows = p.offsets[e + 1] - p.offsets[e];
                     g_tile[e] = run;
                     g_row[e] = p.offsets[e];
-                    run += ((rows + ROWS - 1) / ROWS) * sc.num_n;
+                    run += ((rows + ROWS * CTAS - 1) / (ROWS * CTAS)) * sc.num_n;
                 }
             }
             if (lane == 31) {
@@ -563,14 +563,15 @@ int prepare(const DeviceInfo& di, size_t smem) {
 }
 
 // Co-resident CTA pairs of the 2-CTA kernel (cached per device).
-template <bool ABF16 = false, int BN = BN_MAX>
+template <bool ABF16 = false, int BN = BN_MAX, bool GROUPED = false>
 int max_pairs(const DeviceInfo& di, int* out) {
     static int cached[64];
     if (!cached[di.device]) {
+        using L = Layout<2, ABF16, BN>;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (di.num_sms / 2), 1, 1);
-        cfg.blockDim = dim3(Layout<2, ABF16, BN>::THREADS_, 1, 1);
-        cfg.dynamicSmemBytes = Layout<2, ABF16, BN>::BYTES_DENSE;
+        cfg.blockDim = dim3(L::THREADS_, 1, 1);
+        cfg.dynamicSmemBytes = GROUPED ? L::BYTES_GROUPED : L::BYTES_DENSE;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -579,7 +580,7 @@ int max_pairs(const DeviceInfo& di, int* out) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, false, ABF16, BN>, &cfg),
+        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, GROUPED, ABF16, BN>, &cfg),
                             "cudaOccupancyMaxActiveClusters");
         if (rc) return rc;
         if (n < 1) return fail(METIS_ERR_UNSUPPORTED, "no CTA pair of the fp8 gemm fits an SM pair");
@@ -655,21 +656,47 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
                             __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
                             int K, cudaStream_t st) {
     using namespace gemm;
-    using L = Layout<1>;
     if (E > MAX_GROUPS) return fail(METIS_ERR_UNSUPPORTED, "grouped gemm: E=%d > %d", E, MAX_GROUPS);
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
-    if ((rc = prepare<1, true>(di, L::BYTES_GROUPED))) return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
+    Params p{s_a, nullptr, s_b, y, offsets, rows, N, K, E, status, watchdog_ns()};
     CUtensorMap ta, tb;
     if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, ROWS, true))) return rc;
+    if (K < 2048) {
+        // short k-loops: 128-row single-CTA tiles (measured faster for the
+        // routed down-projection, K = 1024, than CTA pairs)
+        using L = Layout<1>;
+        if ((rc = prepare<1, true>(di, L::BYTES_GROUPED))) return rc;
+        if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
+            return rc;
+        fp8_gemm_kernel<1, true, false, BN_MAX><<<di.num_sms, L::THREADS_, L::BYTES_GROUPED, st>>>(ta, tb, p);
+        return cuda_check(cudaGetLastError(), "grouped fp8 gemm launch");
+    }
+    // CTA pairs on 256-row tiles: each SM streams half of B (routed
+    // up-projection, K = 2048: 72 -> 66 us)
+    using L = Layout<2>;
+    if ((rc = prepare<2, true>(di, L::BYTES_GROUPED))) return rc;
+    int pairs = 0;
+    if ((rc = max_pairs<false, BN_MAX, true>(di, &pairs))) return rc;
     if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
         return rc;
-    Params p{s_a, nullptr, s_b, y, offsets, rows, N, K, E, status, watchdog_ns()};
-    fp8_gemm_kernel<1, true, false, BN_MAX><<<di.num_sms, L::THREADS_, L::BYTES_GROUPED, st>>>(ta, tb, p);
-    return cuda_check(cudaGetLastError(), "grouped fp8 gemm launch");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(L::THREADS_, 1, 1);
+    cfg.dynamicSmemBytes = L::BYTES_GROUPED;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_check(cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<2, true, false, BN_MAX>, ta, tb, p),
+                      "grouped fp8 gemm (CTA pair) launch");
 }
 
 // Fused-quantization W8A8 GEMM launch: a is BF16 [M, K]; inv [M] holds

@@ -52,24 +52,46 @@ __global__ void __launch_bounds__(CHUNK) count_kernel(const int32_t* __restrict_
 
 // counts[e], offsets[e] (exclusive, E + 1 entries) and, in place,
 // chunk_counts[c][e] -> base row of chunk c's slots of expert e.
-__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_counts, int C, int E,
-                                                    int32_t* __restrict__ counts,
-                                                    int32_t* __restrict__ offsets) {
+// One CTA of 1024 threads: G = 1024 / Ep threads per expert (Ep = E rounded
+// up to a power of two) each own a contiguous run of chunks, so the counts
+// are read in one batch of loads per thread rather than C sequential ones.
+constexpr int SCAN_THREADS = 1024;
+constexpr int SCAN_BATCH = 8;
+__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict__ chunk_counts, int C,
+                                                            int E, int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets) {
+    __shared__ int part[SCAN_THREADS];  // [g][e]: sums, then prefix over g
     __shared__ int warp_tot[32];
-    const int e = threadIdx.x;
-    int total = 0;
+    __shared__ int excl_e[MAX_E];
+    int Ep = 1;
+    while (Ep < E) Ep <<= 1;
+    const int G = SCAN_THREADS / Ep;
+    const int e = threadIdx.x % Ep, g = threadIdx.x / Ep;
+    const int c0 = static_cast<int>(static_cast<int64_t>(g) * C / G);
+    const int c1 = static_cast<int>(static_cast<int64_t>(g + 1) * C / G);
+    int local = 0;
     if (e < E) {
-        int c = 0;
-        for (; c + 8 <= C; c += 8) {
-            int v[8];
+        for (int c = c0; c < c1; c += SCAN_BATCH) {
+            int v[SCAN_BATCH];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = chunk_counts[static_cast<size_t>(c + i) * E + e];
+            for (int i = 0; i < SCAN_BATCH; ++i)
+                v[i] = c + i < c1 ? chunk_counts[static_cast<size_t>(c + i) * E + e] : 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) total += v[i];
+            for (int i = 0; i < SCAN_BATCH; ++i) local += v[i];
         }
-        for (; c < C; ++c) total += chunk_counts[static_cast<size_t>(c) * E + e];
     }
-    // block-wide exclusive scan of total over e
+    part[g * Ep + e] = local;
+    __syncthreads();
+    // thread t < Ep: expert t's total, and the exclusive prefix of its parts over g
+    int total = 0;
+    if (threadIdx.x < Ep) {
+        for (int gg = 0; gg < G; ++gg) {
+            const int v = part[gg * Ep + threadIdx.x];
+            part[gg * Ep + threadIdx.x] = total;
+            total += v;
+        }
+    }
+    // block-wide exclusive scan of the totals over e (thread t holds expert t)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int incl = total;
 #pragma unroll
@@ -80,7 +102,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
     if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int w = warp_tot[lane];
+        const int w = warp_tot[lane];
         int wi = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -90,29 +112,29 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
         warp_tot[lane] = wi - w;  // exclusive prefix of warp totals
     }
     __syncthreads();
-    const int excl = warp_tot[warp] + incl - total;
+    if (threadIdx.x < E) {
+        const int excl = warp_tot[warp] + incl - total;
+        counts[threadIdx.x] = total;
+        offsets[threadIdx.x] = excl;
+        excl_e[threadIdx.x] = excl;
+        if (threadIdx.x == E - 1) offsets[E] = excl + total;
+    }
+    __syncthreads();
+    // chunk bases: this thread's run of chunks, from its expert's offset plus
+    // the counts of the runs before it
     if (e < E) {
-        counts[e] = total;
-        offsets[e] = excl;
-        int run = excl;
-        int c = 0;
-        for (; c + 8 <= C; c += 8) {
-            int v[8];
+        int run = excl_e[e] + part[g * Ep + e];
+        for (int c = c0; c < c1; c += SCAN_BATCH) {
+            int v[SCAN_BATCH];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = chunk_counts[static_cast<size_t>(c + i) * E + e];
+            for (int i = 0; i < SCAN_BATCH; ++i)
+                v[i] = c + i < c1 ? chunk_counts[static_cast<size_t>(c + i) * E + e] : 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                chunk_counts[static_cast<size_t>(c + i) * E + e] = run;
+            for (int i = 0; i < SCAN_BATCH; ++i) {
+                if (c + i < c1) chunk_counts[static_cast<size_t>(c + i) * E + e] = run;
                 run += v[i];
             }
         }
-        for (; c < C; ++c) {
-            const size_t i = static_cast<size_t>(c) * E + e;
-            const int v = chunk_counts[i];
-            chunk_counts[i] = run;
-            run += v;
-        }
-        if (e == E - 1) offsets[E] = run;
     }
 }
 
@@ -247,7 +269,7 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     if ((rc = device_status_word(&status))) return rc;
     count_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
                                       status);
-    scan_kernel<<<1, 1024, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets);
+    scan_kernel<<<1, SCAN_THREADS, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets);
     rank_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
                                      s2r, r2s);
     if ((rc = cuda_check(cudaGetLastError(), "moe routing launch"))) return rc;

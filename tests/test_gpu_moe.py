@@ -86,7 +86,8 @@ def check_moe(d, g, tokens=None):
 
 @pytest.mark.parametrize("T,H,I,E,k,seed", [(200, 256, 128, 8, 2, 11), (300, 512, 256, 64, 8, 12),
                                             (37, 128, 272, 5, 3, 13), (1, 64, 32, 4, 4, 14),
-                                            (513, 256, 512, 16, 1, 15)])
+                                            (513, 256, 512, 16, 1, 15),
+                                            (96, 2048, 256, 16, 4, 18)])  # K = 2048: CTA-pair tiles
 def test_moe_parity(metis, T, H, I, E, k, seed):
     d = synth.moe(seed=seed, T=T, H=H, I=I, E=E, topk=k, hot=min(2, E), load_ratio=2.0)
     g = run_moe(metis, d)
