@@ -239,6 +239,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
     }
 
+    // Everything above touches only this CTA's shared and tensor memory. The
+    // operands, scales and group offsets may be the previous kernel's
+    // outputs (PDL launch): wait for it here.
+    grid_launch_dependents();
+    grid_dependency_wait();
+
     Sched<CTAS, BN> sc;
     sc.N = p.N;
     sc.M = p.M;
@@ -606,19 +612,8 @@ int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, 
         if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
         const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
         const int clusters = tiles < pairs ? tiles : pairs;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * clusters, 1, 1);
-        cfg.blockDim = dim3(L::THREADS_, 1, 1);
-        cfg.dynamicSmemBytes = L::BYTES_DENSE;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cuda_check(cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<2, false, false, BN>, ta, tb, p),
+        return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, false, BN>, dim3(2 * clusters), dim3(L::THREADS_),
+                                     L::BYTES_DENSE, st, 2, ta, tb, p),
                           "fp8 gemm (CTA pair) launch");
     }
     using L = Layout<1, false, BN>;
@@ -626,8 +621,9 @@ int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, 
     if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
     const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
-    fp8_gemm_kernel<1, false, false, BN><<<grid, L::THREADS_, L::BYTES_DENSE, st>>>(ta, tb, p);
-    return cuda_check(cudaGetLastError(), "fp8 gemm launch");
+    return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, false, BN>, dim3(grid), dim3(L::THREADS_),
+                                 L::BYTES_DENSE, st, 1, ta, tb, p),
+                      "fp8 gemm launch");
 }
 
 }  // namespace gemm
@@ -672,8 +668,9 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
         if ((rc = prepare<1, true>(di, L::BYTES_GROUPED))) return rc;
         if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
             return rc;
-        fp8_gemm_kernel<1, true, false, BN_MAX><<<di.num_sms, L::THREADS_, L::BYTES_GROUPED, st>>>(ta, tb, p);
-        return cuda_check(cudaGetLastError(), "grouped fp8 gemm launch");
+        return cuda_check(launch_pdl(fp8_gemm_kernel<1, true, false, BN_MAX>, dim3(di.num_sms), dim3(L::THREADS_),
+                                     L::BYTES_GROUPED, st, 1, ta, tb, p),
+                          "grouped fp8 gemm launch");
     }
     // CTA pairs on 256-row tiles: each SM streams half of B (routed
     // up-projection, K = 2048: 72 -> 66 us)
@@ -683,19 +680,8 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     if ((rc = max_pairs<false, BN_MAX, true>(di, &pairs))) return rc;
     if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
         return rc;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(L::THREADS_, 1, 1);
-    cfg.dynamicSmemBytes = L::BYTES_GROUPED;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cuda_check(cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<2, true, false, BN_MAX>, ta, tb, p),
+    return cuda_check(launch_pdl(fp8_gemm_kernel<2, true, false, BN_MAX>, dim3(2 * pairs), dim3(L::THREADS_),
+                                 L::BYTES_GROUPED, st, 2, ta, tb, p),
                       "grouped fp8 gemm (CTA pair) launch");
 }
 
@@ -722,19 +708,8 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
         if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
         const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
         const int clusters = tiles < pairs ? tiles : pairs;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * clusters, 1, 1);
-        cfg.blockDim = dim3(L::THREADS_, 1, 1);
-        cfg.dynamicSmemBytes = L::BYTES_DENSE;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cuda_check(cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<2, false, true, BN_MAX>, ta, tb, p),
+        return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, true, BN_MAX>, dim3(2 * clusters), dim3(L::THREADS_),
+                                     L::BYTES_DENSE, st, 2, ta, tb, p),
                           "fused fp8 gemm (CTA pair) launch");
     }
     using L = Layout<1, true>;
@@ -742,8 +717,9 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
     if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
     const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
-    fp8_gemm_kernel<1, false, true, BN_MAX><<<grid, L::THREADS_, L::BYTES_DENSE, st>>>(ta, tb, p);
-    return cuda_check(cudaGetLastError(), "fused fp8 gemm launch");
+    return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, true, BN_MAX>, dim3(grid), dim3(L::THREADS_),
+                                 L::BYTES_DENSE, st, 1, ta, tb, p),
+                      "fused fp8 gemm launch");
 }
 
 }  // namespace metis

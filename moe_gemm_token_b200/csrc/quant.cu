@@ -67,6 +67,8 @@ quant_rows_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx, uint8_
     constexpr int WARPS_PER_TEAM = TEAM / 32;
     __shared__ float red[kQuantThreads / 32];
 
+    grid_dependency_wait();  // x may be the previous kernel's output (PDL launch)
+    grid_launch_dependents();
     const int team = threadIdx.x / TEAM;
     const int tid = threadIdx.x % TEAM;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * TEAMS + team;
@@ -155,6 +157,8 @@ quant_rows_long_kernel(const T* __restrict__ x, int64_t M, int K, int64_t ldx,
                        float* __restrict__ inv_out) {
     constexpr int EPC = Elem<T>::kPerChunk;
     __shared__ float red[kQuantThreads / 32];
+    grid_dependency_wait();
+    grid_launch_dependents();
     const int64_t row = blockIdx.x;
     if (row >= M) return;
     const T* xr = x + row * ldx;
@@ -211,12 +215,10 @@ cudaError_t launch_fixed(const T* x, int64_t M, int K, int64_t ldx, uint8_t* q, 
     constexpr int TEAMS = kQuantThreads / TEAM;
     const unsigned grid = static_cast<unsigned>((M + TEAMS - 1) / TEAMS);
     if (d.rows && q)
-        quant_rows_kernel<T, TEAM, NV, true><<<grid, kQuantThreads, 0, st>>>(x, M, K, ldx, q, ldq, s,
-                                                                             d.rows, d.topk, nullptr);
-    else
-        quant_rows_kernel<T, TEAM, NV, false><<<grid, kQuantThreads, 0, st>>>(x, M, K, ldx, q, ldq, s,
-                                                                              nullptr, 1, d.inv);
-    return cudaGetLastError();
+        return launch_pdl(quant_rows_kernel<T, TEAM, NV, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1,
+                          x, M, K, ldx, q, ldq, s, d.rows, d.topk, static_cast<float*>(nullptr));
+    return launch_pdl(quant_rows_kernel<T, TEAM, NV, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1,
+                      x, M, K, ldx, q, ldq, s, static_cast<const int32_t*>(nullptr), 1, d.inv);
 }
 
 template <typename T, int TEAM>
@@ -260,9 +262,8 @@ int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
         if (M > 0x7fffffff) return fail(METIS_ERR_UNSUPPORTED, "quantizer: M=%lld too large", (long long)M);
         if (d.rows) return fail(METIS_ERR_UNSUPPORTED, "quantizer: scattered rows need K <= %d",
                                 256 * 8 * EPC);
-        quant_rows_long_kernel<T><<<static_cast<unsigned>(M), kQuantThreads, 0, st>>>(
-            x, M, static_cast<int>(K), ldx, q, ldq, s, inv_out);
-        e = cudaGetLastError();
+        e = launch_pdl(quant_rows_long_kernel<T>, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), 0, st,
+                       1, x, M, static_cast<int>(K), ldx, q, ldq, s, inv_out);
     } else {
         const int team = teams[pick];
         const int nv = static_cast<int>((chunks + team - 1) / team);
