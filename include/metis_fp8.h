@@ -129,14 +129,18 @@ METIS_API int metis_fp8_gemm(const void* a, int a_kind, float* s_tok, const uint
                    const float* s_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
                    void* workspace, size_t ws_bytes, metis_stream_t stream);
 
-/* Default-maths weight-only GEMM for decode (M <= 8): the E4M3 weights are
- * streamed from HBM and widened exactly to 16 bits in registers, products
- * accumulate in FP32, the per-channel scale is applied to the sum
- * ("Lernex/Metis-1.6-Logos-FP8", "What --fast-math does": the default maths,
- * which single-stream decode always uses).
+/* Default-maths weight-only GEMM: the E4M3 weights are widened exactly to
+ * 16 bits as they are multiplied, products accumulate in FP32 and the
+ * per-channel scale is applied to the sum ("Lernex/Metis-1.6-Logos-FP8",
+ * "What --fast-math does": the default maths, which single-stream decode
+ * always uses and prefill uses without fast-math).
  *   x [M, K] BF16, wq [N, K] E4M3, s_w [N] FP32, y [M, N] BF16 out.
- *   Requires 1 <= M <= 8, K % 16 == 0, 16 <= K <= 12288, N >= 1; x, wq
- *   16-byte aligned. */
+ *   M <= 8 (decode): an HBM-bound weight stream with mma.sync on FP16
+ *   operands; requires K % 16 == 0, 16 <= K <= 12288, N >= 1; x, wq
+ *   16-byte aligned.
+ *   M > 8: tcgen05 BF16 maths with the widened weights in tensor memory;
+ *   requires K % 16 == 0, K >= 16, N % 8 == 0, N >= 8; x, wq, y 16-byte
+ *   aligned. */
 METIS_API int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
                      int64_t M, int64_t N, int64_t K, metis_stream_t stream);
 
@@ -229,8 +233,8 @@ METIS_API int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk
  * --fast-math does"): M <= 8 tokens always take the default maths
  * (metis_w8a16_gemm); more tokens take the fast-math W8A8 path when
  * fast_math != 0 (metis_quant_fp8_per_token into the workspace, then
- * metis_fp8_gemm with a_kind = METIS_A_E4M3), and otherwise the large-M
- * default path, which this build does not implement (METIS_ERR_UNSUPPORTED).
+ * metis_fp8_gemm with a_kind = METIS_A_E4M3), and the default maths
+ * (metis_w8a16_gemm, tensor-core path) otherwise.
  * s_tok [M] receives the per-token scales on the fast-math path; `workspace`
  * holds the E4M3 codes: metis_workspace_size(METIS_OP_LINEAR, M, N, K, 0, 0)
  * bytes, 16-byte aligned (0 for M <= 8). */

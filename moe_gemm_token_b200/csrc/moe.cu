@@ -175,6 +175,11 @@ __global__ void __launch_bounds__(CHUNK) rank_kernel(const int32_t* __restrict__
 }
 
 // y[t, n..n+7] = bf16( sum_j w[t, j] * o[slot_to_row[t*topk + j], n..n+7] ).
+// HBM-bound: the row indices and weights of the token are read first, then
+// every row load is issued before the first add (for topk <= COMBINE_MAXK),
+// so a thread has topk 16-byte loads in flight. The sum runs over j in
+// ascending order in FP32 either way.
+constexpr int COMBINE_MAXK = 8;
 __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const float* __restrict__ w,
                                                       const int32_t* __restrict__ slot_to_row,
@@ -186,17 +191,37 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
     const int t = static_cast<int>(idx / groups);
     const int n = static_cast<int>(idx - static_cast<int64_t>(t) * groups) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < topk; ++j) {
-        const int s = t * topk + j;
-        const float wj = w[s];
-        const int r = slot_to_row[s];
-        if (r < 0) continue;
-        const uint4 c = *reinterpret_cast<const uint4*>(o + static_cast<size_t>(r) * H + n);
+    auto add = [&](float wj, const uint4& c) {
         const uint32_t v[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             acc[2 * i] = fmaf(wj, bf16_lo(v[i]), acc[2 * i]);
             acc[2 * i + 1] = fmaf(wj, bf16_hi(v[i]), acc[2 * i + 1]);
+        }
+    };
+    if (topk <= COMBINE_MAXK) {
+        int r[COMBINE_MAXK];
+        float wj[COMBINE_MAXK];
+        uint4 c[COMBINE_MAXK];
+#pragma unroll
+        for (int j = 0; j < COMBINE_MAXK; ++j) {
+            if (j < topk) {
+                r[j] = slot_to_row[static_cast<int64_t>(t) * topk + j];
+                wj[j] = w[static_cast<int64_t>(t) * topk + j];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < COMBINE_MAXK; ++j)
+            if (j < topk && r[j] >= 0) c[j] = *reinterpret_cast<const uint4*>(o + static_cast<size_t>(r[j]) * H + n);
+#pragma unroll
+        for (int j = 0; j < COMBINE_MAXK; ++j)
+            if (j < topk && r[j] >= 0) add(wj[j], c[j]);
+    } else {
+        for (int j = 0; j < topk; ++j) {
+            const int64_t s = static_cast<int64_t>(t) * topk + j;
+            const int rj = slot_to_row[s];
+            if (rj < 0) continue;
+            add(w[s], *reinterpret_cast<const uint4*>(o + static_cast<size_t>(rj) * H + n));
         }
     }
     uint4 out;

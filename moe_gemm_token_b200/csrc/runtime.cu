@@ -249,11 +249,9 @@ extern "C" int metis_linear(const void* x_bf16, const uint8_t* wq, const float* 
                             int64_t M, int64_t N, int64_t K, int fast_math, float* s_tok,
                             void* workspace, size_t ws_bytes, metis_stream_t stream) {
     clear_error();
-    if (M >= 1 && M <= 8) return metis_w8a16_gemm(x_bf16, wq, s_w, y_bf16, M, N, K, stream);
-    if (!fast_math)
-        return fail(METIS_ERR_UNSUPPORTED,
-                    "metis_linear: the default (16-bit) maths for M > 8 tokens is not built; "
-                    "pass fast_math=1");
+    // M <= 8 tokens always take the default maths; more tokens take it unless fast_math
+    if ((M >= 1 && M <= 8) || (M > 8 && !fast_math))
+        return metis_w8a16_gemm(x_bf16, wq, s_w, y_bf16, M, N, K, stream);
     if (M > 0 && M * K > 0 && K % 16 == 0) {
         const size_t need = metis_workspace_size(METIS_OP_LINEAR, M, N, K, 0, 0);
         if (!workspace || ws_bytes < need || !aligned(workspace, 16))

@@ -1,0 +1,366 @@
+// Default-maths weight-only GEMM for many tokens (M > 8) on the fifth-
+// generation tensor cores:
+//   y[m, n] = bf16_rn( s_w[n] * sum_k x[m, k] * D(w[n, k]) ),  FP32 accumulation,
+// with the E4M3 weights widened exactly to BF16 and BF16 x BF16 products
+// ("Lernex/Metis-1.6-Logos-FP8", "What --fast-math does": by default the FP8
+// weights are expanded to 16 bits as they are multiplied, so the weights are
+// the only thing rounded).
+//
+// Computed as y^T = W x^T so that the widened weights never pass through
+// shared memory: a 128-channel x 128-token tile per CTA, the channels on the
+// 128 TMEM lanes.
+//   warp 0      TMA producer of the x tiles (BF16, 128 tokens x 64 elements,
+//               128-byte swizzle) into an 8-stage shared-memory ring;
+//   warp 1      allocates all 512 TMEM columns (two 128-column FP32
+//               accumulators, eight 32-column weight stages); one lane issues
+//               tcgen05.mma.kind::f16 with A = the widened weights in TMEM and
+//               B = the x tile in shared memory;
+//   warps 2..9  converters, two per TMEM lane quadrant: each thread streams
+//               32 bytes of its weight row per k-block from global memory
+//               (eight k-blocks ahead in registers), widens E4M3 to BF16
+//               exactly (through FP16 and FP32: every E4M3 value is a BF16
+//               value) and writes the 16 packed words into its lane of a TMEM
+//               weight stage (tcgen05.st);
+//   warps 10..13 epilogue: tcgen05.ld of 32 channels x 32 tokens, x s_w[n],
+//               BF16 RNE, transposed through a 32x32 shared-memory block and
+//               stored as 64-byte token rows.
+// Every mbarrier wait is bounded by the device watchdog.
+#include "common.cuh"
+
+namespace metis {
+namespace w16 {
+
+constexpr int BKE = 64;          // K elements per k-block (128 bytes of BF16 x)
+constexpr int TILE_N = 128;      // channels per tile (TMEM lanes)
+constexpr int TILE_M = 128;      // tokens per tile (accumulator columns)
+constexpr int STAGES = 8;        // x ring and TMEM weight stages
+constexpr int X_STAGE = TILE_M * BKE * 2;  // 16 KB
+constexpr int A_COLS = BKE / 2;  // TMEM columns per weight stage (two BF16 per column)
+constexpr int ACC_COLS = TILE_M;
+constexpr int TMEM_COLS = 512;   // 2 x 128 accumulator + 8 x 32 weight columns
+constexpr int A_COL0 = 2 * ACC_COLS;
+constexpr int CONV_WARPS = 8;   // two per TMEM lane quadrant, each on half of a k-block
+constexpr int PF = 8;           // k-blocks of weight bytes in flight per converter thread
+constexpr int THREADS = 64 + CONV_WARPS * 32 + 4 * 32;
+constexpr uint32_t IDESC = idesc_bf16_f32(TILE_N, TILE_M);
+
+static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+
+// shared memory: x ring | epilogue staging (4 warps x 2 KB) | barriers | misc
+constexpr int STG_OFF = STAGES * X_STAGE;
+constexpr int BAR_OFF = STG_OFF + 4 * 2048;
+// xfull[S], xempty[S], afull[S], aempty[S], tfull[2], tempty[2], drain
+constexpr int NUM_BARS = 4 * STAGES + 5;
+constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+constexpr size_t SMEM_BYTES = 1024 + MISC_OFF + 16;
+
+struct Params {
+    const uint8_t* w;     // [N, K] E4M3
+    const float* s_w;     // [N]
+    __nv_bfloat16* y;     // [M, N]
+    int M, N, K;
+    uint32_t* status;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ uint4 ld_w16(const uint8_t* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Four E4M3 bytes -> two BF16 pairs (bytes 0,1 and 2,3), exactly: E4M3 ->
+// FP16 (cvt.rn.f16x2.e4m3x2, exact) -> FP32 (exact) -> BF16 (exact, every
+// E4M3 value being a BF16 value). Eight instructions per four elements.
+__device__ __forceinline__ void e4m3x4_to_bf16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t"
+        ".reg .b16 q0, q1, a, b, c, d;\n\t"
+        ".reg .b32 h0, h1;\n\t"
+        ".reg .f32 fa, fb, fc, fd;\n\t"
+        "mov.b32 {q0, q1}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h0, q0;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h1, q1;\n\t"
+        "mov.b32 {a, b}, h0;\n\t"
+        "mov.b32 {c, d}, h1;\n\t"
+        "cvt.f32.f16 fa, a;\n\t"
+        "cvt.f32.f16 fb, b;\n\t"
+        "cvt.f32.f16 fc, c;\n\t"
+        "cvt.f32.f16 fd, d;\n\t"
+        "cvt.rn.bf16x2.f32 %0, fb, fa;\n\t"
+        "cvt.rn.bf16x2.f32 %1, fd, fc;\n\t"
+        "}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* ring = smem;
+    uint8_t* staging = smem + STG_OFF;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);
+    auto xfull = [&](int s) { return smem_u32(&bars[s]); };
+    auto xempty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+    auto afull = [&](int s) { return smem_u32(&bars[2 * STAGES + s]); };
+    auto aempty = [&](int s) { return smem_u32(&bars[3 * STAGES + s]); };
+    auto tfull = [&](int b) { return smem_u32(&bars[4 * STAGES + b]); };
+    auto tempty = [&](int b) { return smem_u32(&bars[4 * STAGES + 2 + b]); };
+    const uint32_t drain = smem_u32(&bars[4 * STAGES + 4]);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(xfull(s), 1);
+            mbar_init(xempty(s), 1);
+            mbar_init(afull(s), CONV_WARPS);
+            mbar_init(aempty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 1);
+            mbar_init(tempty(b), 4);  // the four epilogue warps
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    grid_launch_dependents();
+    grid_dependency_wait();  // x may be the previous kernel's output
+    const uint32_t tmem_base = *tmem_slot;
+    const int num_m = (p.M + TILE_M - 1) / TILE_M;
+    const int total = num_m * ((p.N + TILE_N - 1) / TILE_N);
+    const int num_kb = (p.K + BKE - 1) / BKE;
+    // tiles: token block fastest, so CTAs running together share weight rows
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------- producer
+            int s = 0;
+            uint32_t ph = 0;
+            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+                const int m0 = (t % num_m) * TILE_M;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(xempty(s), ph ^ 1u, p.timeout_ns, p.status)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(xfull(s), X_STAGE);
+                    tma_load_2d(smem_u32(ring + s * X_STAGE), &tmX, kb * BKE, m0, xfull(s));
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (*abort_flag) {
+                // let copies in flight land before the CTA exits
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 100000ull) {}
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------------------------------------------- MMA issuer
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t acc_ph = 0;
+            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+                if (!mbar_wait(tempty(acc), acc_ph ^ 1u, p.timeout_ns, p.status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(xfull(s), ph, p.timeout_ns, p.status) ||
+                        !mbar_wait(afull(s), ph, p.timeout_ns, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(ring + s * X_STAGE));
+                    const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
+#pragma unroll
+                    for (int k = 0; k < BKE / 16; ++k)  // K = 16 per MMA: 8 columns, 32 bytes
+                        mma_f16_tmem_a(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(xempty(s));
+                    mma_commit(aempty(s));
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) {
+                    *abort_flag = 1;
+                    break;
+                }
+                mma_commit(tfull(acc));
+                acc ^= 1;
+                if (acc == 0) acc_ph ^= 1u;
+            }
+            mma_commit(drain);
+            mbar_wait(drain, 0, p.timeout_ns, p.status);
+        }
+    } else if (warp < 2 + CONV_WARPS) {
+        // -------------------------------------------------------- converters
+        const int q = warp & 3;
+        const int half = (warp - 2) / 4;   // which 32 elements of the k-block
+        const int lane_base = q * 32;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+            const int row = (t / num_m) * TILE_N + lane_base + lane;  // weight row = output channel
+            const bool row_ok = row < p.N;
+            const uint8_t* wrow = p.w + static_cast<size_t>(row_ok ? row : 0) * p.K + 32 * half;
+            auto load_kb = [&](int kb, uint4 (&r)[2]) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int k = kb * BKE + 32 * half + 16 * j;
+                    r[j] = (row_ok && k < p.K) ? ld_w16(wrow + kb * BKE + 16 * j) : make_uint4(0, 0, 0, 0);
+                }
+            };
+            // PF k-blocks of weight bytes in flight per thread (L2 latency)
+            uint4 buf[PF][2];
+#pragma unroll
+            for (int d = 0; d < PF; ++d) load_kb(d, buf[d]);
+            bool ok = true;
+            for (int kb0 = 0; kb0 < num_kb && ok; kb0 += PF) {
+#pragma unroll
+                for (int d = 0; d < PF; ++d) {
+                    const int kb = kb0 + d;
+                    if (kb >= num_kb || !ok) break;
+                    uint32_t words[16];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const uint32_t v[4] = {buf[d][j].x, buf[d][j].y, buf[d][j].z, buf[d][j].w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            e4m3x4_to_bf16x2x2(v[i], words[8 * j + 2 * i], words[8 * j + 2 * i + 1]);
+                    }
+                    load_kb(kb + PF, buf[d]);  // zeros past the end of K
+                    if (!mbar_wait(aempty(s), ph ^ 1u, p.timeout_ns, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    tmem_st_32x32b_x16(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
+                                           static_cast<uint32_t>(A_COL0 + s * A_COLS + 16 * half),
+                                       words);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(afull(s));
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                break;
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;  // warps 10..13 -> quadrants 2, 3, 0, 1
+        uint8_t* stg = staging + (warp - 2 - CONV_WARPS) * 2048;  // [32 tokens][32 channels] BF16
+        int acc = 0;
+        uint32_t acc_ph = 0;
+        for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+            const int m0 = (t % num_m) * TILE_M;
+            const int n_lane = (t / num_m) * TILE_N + q * 32 + lane;  // this thread's channel
+            const float sw = n_lane < p.N ? p.s_w[n_lane] : 0.0f;
+            if (!mbar_wait(tfull(acc), acc_ph, p.timeout_ns, p.status)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tbase =
+                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_COLS);
+            const int nq0 = (t / num_m) * TILE_N + q * 32;  // first channel of this warp
+            for (int c = 0; c < TILE_M / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tbase + c * 32, v);
+                tmem_ld_wait();
+                if (c == TILE_M / 32 - 1) {
+                    // the accumulator has been read: release it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty(acc));
+                }
+                // lane = channel, j = token: transpose into [token][channel]
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__uint_as_float(v[j]), sw));
+                    *reinterpret_cast<__nv_bfloat16*>(stg + j * 64 + lane * 2) = b;
+                }
+                __syncwarp();
+                // 8 tokens x 64 bytes per instruction
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int tk = (lane >> 2) + 8 * i;
+                    const int m = m0 + c * 32 + tk;
+                    const int n = nq0 + (lane & 3) * 8;
+                    const uint4 val = *reinterpret_cast<const uint4*>(stg + tk * 64 + (lane & 3) * 16);
+                    if (m < p.M && n < p.N)
+                        *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(m) * p.N + n) = val;
+                }
+            }
+            acc ^= 1;
+            if (acc == 0) acc_ph ^= 1u;
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace w16
+
+// Weight-only W8A16 GEMM for M > 8 tokens (arguments validated by the
+// caller): x BF16 [M, K], wq E4M3 [N, K], N % 8 == 0, K % 16 == 0.
+int launch_w8a16_tensor(const __nv_bfloat16* x, const uint8_t* wq, const float* s_w,
+                        __nv_bfloat16* y, int M, int N, int K, cudaStream_t st) {
+    using namespace w16;
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    static bool attr_done[64];
+    if (!attr_done[di.device]) {
+        if (static_cast<size_t>(di.max_smem_optin) < SMEM_BYTES)
+            return fail(METIS_ERR_UNSUPPORTED, "w8a16 tensor-core GEMM needs %zu bytes of shared memory",
+                        SMEM_BYTES);
+        if ((rc = cuda_check(cudaFuncSetAttribute(w16_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(SMEM_BYTES)),
+                             "cudaFuncSetAttribute(w16 gemm)")))
+            return rc;
+        attr_done[di.device] = true;
+    }
+    uint32_t* status = nullptr;
+    if ((rc = device_status_word(&status))) return rc;
+    CUtensorMap tx;
+    if ((rc = make_tmap_2d(&tx, x, 2, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                           static_cast<uint64_t>(K) * 2, BKE, TILE_M, true)))
+        return rc;
+    Params p{wq, s_w, y, M, N, K, status, watchdog_ns()};
+    const int tiles = ((M + TILE_M - 1) / TILE_M) * ((N + TILE_N - 1) / TILE_N);
+    const int grid = tiles < di.num_sms ? tiles : di.num_sms;
+    return cuda_check(launch_pdl(w16_gemm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, st, 1, tx, p),
+                      "w8a16 tensor-core GEMM launch");
+}
+
+}  // namespace metis

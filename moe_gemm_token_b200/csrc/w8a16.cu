@@ -641,8 +641,21 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
                                 metis_stream_t stream) {
     using namespace w8a16;
     clear_error();
-    if (M < 1 || M > 8)
-        return fail(METIS_ERR_INVALID_ARG, "w8a16_gemm: M=%lld, need 1 <= M <= 8", (long long)M);
+    if (M < 1 || M > 0x7fffffff)
+        return fail(METIS_ERR_INVALID_ARG, "w8a16_gemm: M=%lld, need M >= 1", (long long)M);
+    if (M > 8) {
+        // many tokens: the tensor-core path (weights widened into TMEM)
+        if (N < 8 || N % 8 != 0 || N > 0x7fffffff || K < 16 || K % 16 != 0 || K > 0x7fffffff)
+            return fail(METIS_ERR_INVALID_ARG,
+                        "w8a16_gemm (M > 8): need N >= 8 with N %% 8 == 0, K >= 16 with K %% 16 == 0 "
+                        "(N=%lld K=%lld)", (long long)N, (long long)K);
+        if (!x_bf16 || !wq || !s_w || !y_bf16) return fail(METIS_ERR_INVALID_ARG, "w8a16_gemm: null pointer");
+        if (!aligned(x_bf16, 16) || !aligned(wq, 16) || !aligned(s_w, 4) || !aligned(y_bf16, 16))
+            return fail(METIS_ERR_INVALID_ARG, "w8a16_gemm (M > 8): x, wq and y must be 16-byte aligned");
+        return launch_w8a16_tensor(static_cast<const __nv_bfloat16*>(x_bf16), wq, s_w,
+                                   static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(M), static_cast<int>(N),
+                                   static_cast<int>(K), static_cast<cudaStream_t>(stream));
+    }
     if (K < 16 || K % 16 != 0 || K > MAX_K)
         return fail(METIS_ERR_INVALID_ARG, "w8a16_gemm: K=%lld, need 16 <= K <= %d and K %% 16 == 0",
                     (long long)K, MAX_K);

@@ -6,6 +6,7 @@ only the device status word.
     python -m moe_gemm_token_b200.drive gemm  M N K [--calls N]
     python -m moe_gemm_token_b200.drive fused M N K [--calls N]
     python -m moe_gemm_token_b200.drive decode M [--calls N]
+    python -m moe_gemm_token_b200.drive w16 M N K [--calls N]
     python -m moe_gemm_token_b200.drive quant M K [--calls N]
 
 Each call is enqueued on the current stream; the script synchronises once at
@@ -27,7 +28,7 @@ def _codes(n, k, g):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["moe", "gemm", "fused", "decode", "quant"])
+    ap.add_argument("op", choices=["moe", "gemm", "fused", "decode", "w16", "quant"])
     ap.add_argument("dims", nargs="*", type=int)
     ap.add_argument("--calls", type=int, default=3)
     a = ap.parse_args(argv)
@@ -66,6 +67,13 @@ def main(argv=None):
             ws = torch.empty(metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0),
                              dtype=torch.uint8, device=dev)
             call = lambda: metis.metis_fp8_gemm(x, metis.METIS_A_BF16, s, b, sb, y, workspace=ws)
+    elif a.op == "w16":
+        M, N, K = a.dims
+        x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+        wq = _codes(N, K, g)
+        sw = torch.rand(N, device=dev, generator=g) * 1e-3
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        call = lambda: metis.metis_w8a16_gemm(x, wq, sw, y)
     elif a.op == "decode":
         (M,) = a.dims
         N, K = 14336, 4096

@@ -144,7 +144,8 @@ def metis_fp8_gemm(a, a_kind, s_tok, wq, s_w, y, workspace=None, stream=None):
 
 
 def metis_w8a16_gemm(x, wq, s_w, y, stream=None):
-    """y [M, N] = W8A16(x, wq) for M <= 8."""
+    """y [M, N] = W8A16(x, wq): the default maths (decode kernel for M <= 8,
+    tensor-core kernel for M > 8)."""
     M, K = x.shape
     N = wq.shape[0]
     return _check("metis_w8a16_gemm", load().metis_w8a16_gemm(
@@ -189,8 +190,8 @@ def metis_moe_workspace_offset(region, T, topk, E, H, I):
 
 
 def metis_linear(x, wq, s_w, y, fast_math=True, s_tok=None, workspace=None, stream=None):
-    """Dispatch rule: M <= 8 -> W8A16; otherwise W8A8 (fast_math): per-token
-    quantizer into `workspace`, then the E4M3 GEMM."""
+    """Dispatch rule: M <= 8 -> W8A16; otherwise W8A8 with fast_math (per-token
+    quantizer into `workspace`, then the E4M3 GEMM) and W8A16 without."""
     M, K = x.shape
     N = wq.shape[0]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

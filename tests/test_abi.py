@@ -78,9 +78,11 @@ def test_host_validation_without_gpu(lib):
         metis.METIS_ERR_INVALID_ARG
     assert lib.metis_fp8_gemm(p, 1, p, p, p, p, 300, 512, 256, ctypes.c_void_p(0x1004), need,
                               null) == metis.METIS_ERR_INVALID_ARG
-    # W8A16: M > 8, K too large
-    assert lib.metis_w8a16_gemm(p, p, p, p, 9, 128, 256, null) == metis.METIS_ERR_INVALID_ARG
-    assert b"M <= 8" in lib.metis_last_error()
+    # W8A16: M = 0; M > 8 needs N % 8; K too large for the decode kernel
+    assert lib.metis_w8a16_gemm(p, p, p, p, 0, 128, 256, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_w8a16_gemm(p, p, p, p, 9, 100, 256, null) == metis.METIS_ERR_INVALID_ARG
+    assert b"N % 8" in lib.metis_last_error()
+    assert lib.metis_w8a16_gemm(p, p, p, p, 9, 128, 250, null) == metis.METIS_ERR_INVALID_ARG
     assert lib.metis_w8a16_gemm(p, p, p, p, 4, 128, 16384, null) == metis.METIS_ERR_INVALID_ARG
     assert lib.metis_w8a16_gemm(p, p, p, p, 4, 128, 264, null) == metis.METIS_ERR_INVALID_ARG
     # MoE: activation, topk > E, H % 16, small workspace
@@ -93,8 +95,8 @@ def test_host_validation_without_gpu(lib):
     assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 2, 4, 64, 32, p, p, p, p, 0, p, p, 16,
                                           null) == metis.METIS_ERR_INVALID_ARG
     assert b"workspace" in lib.metis_last_error()
-    # dispatch: large M default maths is not built
-    assert lib.metis_linear(p, p, p, p, 64, 128, 256, 0, p, p, 1 << 20, null) == metis.METIS_ERR_UNSUPPORTED
+    # dispatch: the default maths for M > 8 validates like metis_w8a16_gemm
+    assert lib.metis_linear(p, p, p, p, 64, 100, 256, 0, p, p, 1 << 20, null) == metis.METIS_ERR_INVALID_ARG
     # fast-math dispatch needs room for the codes of x
     assert lib.metis_workspace_size(metis.METIS_OP_LINEAR, 64, 128, 256, 0, 0) == 64 * 256
     assert lib.metis_workspace_size(metis.METIS_OP_LINEAR, 8, 128, 256, 0, 0) == 0

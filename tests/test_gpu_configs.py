@@ -80,6 +80,27 @@ def test_prefill_chain_full_size(metis):
     assert_close(bf16_host(y2)[rows], y2_64, "layer 2")
 
 
+def test_prefill_chain_default_maths_full_size(metis):
+    """The same 4096-token chain through the default maths (metis_linear
+    without fast-math: W8A16, weights widened to BF16 on the tensor cores)."""
+    d = synth.prefill_chain()
+    M, K, N = d["M"], d["K"], d["N"]
+    w1, s1, w1r, s1r = _weights(metis, d["w1"])
+    w2, s2, w2r, s2r = _weights(metis, d["w2"])
+    y1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    s_tok = torch.empty((M,), dtype=torch.float32, device="cuda")
+    metis.metis_linear(bf16_dev(d["x"]), w1, s1, y1, fast_math=False, s_tok=s_tok)
+    metis.metis_linear(y1, w2, s2, y2, fast_math=False, s_tok=s_tok)
+    assert metis.metis_check_device_status() == 0
+    rows = _sample_rows(M, d["x"])
+    _, y1_64 = oracle.gemm_w8a16(d["x"][rows], w1r, s1r)
+    y1h = bf16_host(y1)
+    assert_close(y1h[rows], y1_64, "layer 1 (default maths)")
+    _, y2_64 = oracle.gemm_w8a16(y1h[rows], w2r, s2r)
+    assert_close(bf16_host(y2)[rows], y2_64, "layer 2 (default maths)")
+
+
 @pytest.mark.parametrize("M", [1, 2, 4, 8])
 def test_decode_full_size(metis, M):
     d = synth.decode(M=M)

@@ -204,9 +204,13 @@ def test_linear_fast_math(metis):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     assert torch.equal(s1, s2) and torch.equal(s2, s3)
     assert torch.equal(ws[:M * K].view(M, K), xq)
-    with pytest.raises(metis.MetisError) as ei:
-        metis.metis_linear(xd, wq, s_w, y2, fast_math=False, s_tok=s2, workspace=ws)
-    assert ei.value.code == metis.METIS_ERR_UNSUPPORTED
+    # without fast-math the default maths (W8A16) runs, bit-identical to the direct call
+    y4 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    y5 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_linear(xd, wq, s_w, y4, fast_math=False, s_tok=s2, workspace=ws)
+    metis.metis_w8a16_gemm(xd, wq, s_w, y5)
+    torch.cuda.synchronize()
+    assert torch.equal(y4.view(torch.int16), y5.view(torch.int16))
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 1000, 4096), (2, 37, 272), (3, 300, 12288), (4, 1000, 4096),
@@ -224,6 +228,41 @@ def test_w8a16_parity(metis, M, N, K):
     assert_bytes_equal(wq.cpu().numpy(), wq_r, "weight codes")
     _, y64 = oracle.gemm_w8a16(d["x"], wq_r, sw_r)
     assert_close(bf16_host(y), y64, f"w8a16 {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(9, 264, 512), (64, 256, 128), (100, 520, 272), (128, 128, 64),
+                                   (200, 1000, 1040), (300, 6144, 2048), (513, 136, 4096)])
+def test_w8a16_tensor_core_parity(metis, M, N, K):
+    """M > 8: the default maths on the tensor cores (weights widened to BF16
+    in tensor memory, x BF16 from shared memory), ragged in M, N and K."""
+    d = synth.linear(M * 3 + N + 7 * K, M, K, N, outlier_channels=2, outlier_scale=20.0)
+    wq, s_w = _prep_weights(metis, d["w"])
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_w8a16_gemm(bf16_dev(d["x"]), wq, s_w, y)
+    assert metis.metis_check_device_status() == 0
+    wq_r, sw_r = oracle.quant_per_channel(d["w"])
+    _, y64 = oracle.gemm_w8a16(d["x"], wq_r, sw_r)
+    assert_close(bf16_host(y), y64, f"w8a16 tensor {M}x{N}x{K}")
+
+
+def test_w8a16_tensor_core_exact_products(metis):
+    """Every weight code an E4M3 subnormal or small normal and x small
+    integers: products and partial sums are exact in FP32, so the output
+    equals the oracle's BF16 bits. A widening that lost subnormals, or a
+    wrong lane/column layout of the weights in tensor memory, fails here."""
+    rng = np.random.default_rng(9)
+    M, N, K = 160, 264, 320
+    codes = (rng.integers(1, 8, (N, K)) | (rng.integers(0, 2, (N, K)) << 7)).astype(np.uint8)
+    codes[:, ::5] = 0x38  # 1.0
+    codes[::3, 1::7] = 0xC0  # -2.0
+    x = synth.f32_to_bf16_bits(rng.integers(-4, 5, (M, K)).astype(np.float32))
+    s_w = np.ones(N, np.float32)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_w8a16_gemm(bf16_dev(x), dev(codes), dev(s_w), y)
+    assert metis.metis_check_device_status() == 0
+    yr, _ = oracle.gemm_w8a16(x, codes, s_w)
+    assert np.any(yr != 0)
+    assert_bytes_equal(bf16_host(y), yr, "w8a16 tensor exact")
 
 
 def test_w8a16_subnormal_weights_and_wide_x(metis):
