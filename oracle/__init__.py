@@ -213,6 +213,22 @@ def moe_route(topk_ids, num_experts):
     return counts, offsets, s2r, r2s
 
 
+def route_topk(logits, topk, bias=None):
+    """Router top-k on binary32 logits [T, E] (+ optional binary32 balance bias
+    [E] that only decides the choice): ids [T, k] int32 in descending score
+    order (ties to the lower expert), weights [T, k] float64, a softmax over
+    the chosen experts' own logits."""
+    lib = _load()
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    b = None if bias is None else _c(bias, np.float32)
+    ids = np.empty((T, topk), dtype=np.int32)
+    w = np.empty((T, topk), dtype=np.float64)
+    _check(lib.metis_oracle_route_topk(_ptr(lg), _ptr(b), T, E, int(topk), _ptr(ids), _ptr(w)),
+           "route_topk")
+    return ids, w
+
+
 def moe_combine(o_slots_bf16, topk_w):
     """y[t] = bf16(sum_j w[t,j] o[t,j]) with o in slot order [T, k, H] (bf16 bits)."""
     lib = _load()

@@ -283,6 +283,50 @@ int metis_oracle_moe_route(const int32_t* ids, int64_t T, int64_t topk, int64_t 
     return ORACLE_OK;
 }
 
+/* Router top-k. The cards keep "the routers and their balance bias" in FP32
+ * ("Lernex/Metis-1.6-Logos-FP8", "What is in FP8") and route each token to
+ * a few experts; they print no formula. Reading: the balance bias only
+ * decides which experts are chosen, and the chosen experts' weights are a
+ * softmax over their own (unbiased) logits. Choice j of token t is the j-th
+ * largest binary32 score logit + bias (the binary32 sum decides, as the
+ * logits are binary32), ties going to the lower expert index; its weight is
+ * exp(l_j - m) / sum_i exp(l_i - m) over the chosen experts, m their largest
+ * logit, evaluated in float64. bias may be NULL (no bias). */
+int metis_oracle_route_topk(const float* logits, const float* bias, int64_t T, int64_t E,
+                            int64_t topk, int32_t* ids, double* w) {
+    int64_t t;
+    if (topk < 1 || topk > E) return ORACLE_BAD_INDEX;
+    for (t = 0; t < T; ++t) {
+        const float* l = logits + t * E;
+        int64_t j, e;
+        double m, sum;
+        for (j = 0; j < topk; ++j) {
+            int64_t best = -1;
+            float best_s = 0.0f;
+            for (e = 0; e < E; ++e) {
+                int64_t i, taken = 0;
+                float s;
+                for (i = 0; i < j; ++i)
+                    if (ids[t * topk + i] == e) taken = 1;
+                if (taken) continue;
+                s = bias ? l[e] + bias[e] : l[e];
+                if (best < 0 || s > best_s) { /* strict: ties keep the lower index */
+                    best = e;
+                    best_s = s;
+                }
+            }
+            ids[t * topk + j] = (int32_t)best;
+        }
+        m = l[ids[t * topk]];
+        for (j = 1; j < topk; ++j)
+            if (l[ids[t * topk + j]] > m) m = l[ids[t * topk + j]];
+        sum = 0.0;
+        for (j = 0; j < topk; ++j) sum += exp((double)l[ids[t * topk + j]] - m);
+        for (j = 0; j < topk; ++j) w[t * topk + j] = exp((double)l[ids[t * topk + j]] - m) / sum;
+    }
+    return ORACLE_OK;
+}
+
 /* Routing-weighted combine: y[t][n] = bf16( sum_j w[t][j] * o[t][j][n] ),
  * o given in slot order as BF16, float64 sum over j in order 0..topk-1. */
 int metis_oracle_moe_combine(const uint16_t* o, const float* w, int64_t T, int64_t topk,

@@ -109,3 +109,87 @@ def test_expert_gemm_uses_each_slots_own_expert():
     exp = d["topk_ids"].reshape(-1)
     changed = np.any(base["h"] != sw["h"], axis=1)
     assert np.array_equal(changed, np.isin(exp, [0, 1]))
+
+
+# ---------------------------------------------------------------- router top-k
+
+def _route_reference(logits32, k, bias32=None):
+    """Independent restatement: sort by (-score, expert) with the score formed
+    by numpy binary32 addition; softmax over the chosen unbiased logits."""
+    T, E = logits32.shape
+    score = logits32 if bias32 is None else (logits32 + bias32[None, :]).astype(np.float32)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-float(score[t, e]), e))[:k]
+        ids[t] = order
+        z = logits32[t, order].astype(np.float64)
+        p = np.exp(z - z.max())
+        w[t] = p / p.sum()
+    return ids, w
+
+
+def test_route_topk_all_experts_is_the_softmax():
+    """k = E: every expert chosen in descending order; the weights are the
+    plain softmax of the logits (closed form)."""
+    rng = np.random.default_rng(40)
+    lg = rng.standard_normal((50, 12)).astype(np.float32)
+    ids, w = oracle.route_topk(lg, 12)
+    order = np.argsort(-lg.astype(np.float64), axis=1, kind="stable")
+    assert np.array_equal(ids, order)
+    z = lg.astype(np.float64)
+    soft = np.exp(z - z.max(axis=1, keepdims=True))
+    soft /= soft.sum(axis=1, keepdims=True)
+    assert np.allclose(w, np.take_along_axis(soft, order, axis=1), rtol=1e-13, atol=0)
+
+
+def test_route_topk_one_expert_gets_weight_one():
+    rng = np.random.default_rng(41)
+    lg = rng.integers(-3, 4, (200, 16)).astype(np.float32)  # many ties
+    ids, w = oracle.route_topk(lg, 1)
+    assert np.array_equal(ids[:, 0], np.argmax(lg, axis=1))  # first maximum = lower index
+    assert np.all(w == 1.0)
+
+
+@pytest.mark.parametrize("seed,T,E,k,with_bias", [(42, 64, 6, 3, False), (43, 64, 9, 4, True),
+                                                  (44, 32, 16, 8, True), (45, 16, 5, 5, True)])
+def test_route_topk_matches_an_independent_sort(seed, T, E, k, with_bias):
+    """Small-integer logits and biases force ties; halves make binary32 sums
+    exact or rounded. Ids must match a plain sort by (-score, expert)."""
+    rng = np.random.default_rng(seed)
+    lg = (rng.integers(-4, 5, (T, E)) * 0.5).astype(np.float32)
+    lg[:, 0] = lg[:, 1]  # guaranteed ties
+    b = (rng.integers(-2, 3, E) * 0.25).astype(np.float32) if with_bias else None
+    ids, w = oracle.route_topk(lg, k, b)
+    ids_r, w_r = _route_reference(lg, k, b)
+    assert np.array_equal(ids, ids_r)
+    assert np.allclose(w, w_r, rtol=1e-14, atol=0)
+
+
+def test_route_topk_bias_decides_the_choice_not_the_weights():
+    lg = np.array([[3.0, 2.0, 1.0, 0.5]], np.float32)
+    ids, w = oracle.route_topk(lg, 2)
+    assert ids.tolist() == [[0, 1]]
+    bias = np.array([0.0, 0.0, 5.0, 0.0], np.float32)  # expert 2 overtakes both
+    ids_b, w_b = oracle.route_topk(lg, 2, bias)
+    assert ids_b.tolist() == [[2, 0]]
+    z = np.array([1.0, 3.0])  # unbiased logits of experts 2 and 0
+    assert np.allclose(w_b[0], np.exp(z - 3.0) / np.exp(z - 3.0).sum(), rtol=1e-15)
+    # a bias that keeps the choice leaves the weights unchanged
+    ids_c, w_c = oracle.route_topk(lg, 2, np.array([0.1, 0.1, 0.0, 0.0], np.float32))
+    assert ids_c.tolist() == [[0, 1]] and np.array_equal(w_c, w)
+
+
+def test_route_topk_invariants():
+    rng = np.random.default_rng(46)
+    lg = rng.standard_normal((300, 64)).astype(np.float32)
+    b = (rng.standard_normal(64) * 0.3).astype(np.float32)
+    ids, w = oracle.route_topk(lg, 8, b)
+    score = lg + b
+    for t in range(300):
+        assert len(set(ids[t].tolist())) == 8
+        chosen = score[t, ids[t]]
+        assert np.all(np.diff(chosen) <= 0)  # descending
+        others = np.delete(score[t], ids[t])
+        assert chosen.min() >= others.max()
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-12)
