@@ -1,9 +1,11 @@
 """Pins of the oracle's routed-expert path: routing bookkeeping against
-numpy's stable sort, the combine against exact rationals, and the whole
-layer against its degenerate cases (one expert; identical experts)."""
+numpy's stable sort, the combine against exact rationals, the whole layer
+against its degenerate cases (one expert; identical experts), and the router
+top-k against an independent sort, the plain softmax and its invariants."""
 from fractions import Fraction
 
 import numpy as np
+import pytest
 
 import oracle
 from moe_gemm_token_b200 import synth
