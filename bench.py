@@ -576,6 +576,11 @@ def secondary_figures(metis, dev, pk):
     y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     wsp = torch.empty(metis.metis_workspace_size(metis.METIS_OP_MOE, T, I, H, k, E),
                       dtype=torch.uint8, device=dev)
+    ids_g = torch.empty_like(ids)
+    w_g = torch.empty_like(w)
+    t_r = timeit(lambda: metis.metis_moe_route_topk(logits, ids_g, w_g), 50)
+    out["router_topk_4096tok_64e_top8"] = {"us": t_r * 1e6,
+                                           "GB/s": (T * E * 4 + T * k * 8) / t_r / 1e9}
     t = timeit(lambda: metis.metis_moe_fp8_grouped_gemm(x, ids, w, wu, su, wd, sd, y, wsp), 20)
     tf = 2 * 2 * T * k * H * I / t / 1e12
     out["moe_4096tok_64e_top8"] = {"us": t * 1e6, "tok/s": T / t, "TFLOP/s": tf,

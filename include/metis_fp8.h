@@ -144,6 +144,22 @@ METIS_API int metis_fp8_gemm(const void* a, int a_kind, float* s_tok, const uint
 METIS_API int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
                      int64_t M, int64_t N, int64_t K, metis_stream_t stream);
 
+/* Router top-k feeding the routed-expert layer. The cards keep "the routers
+ * and their balance bias" in FP32 and route each token to a few experts
+ * ("Lernex/Metis-1.6-Logos-FP8", "What is in FP8"; four per token in
+ * "Lernex/Metis-1.6-Praxis-Base"); they print no formula. Reading: choice j
+ * of token t is the expert with the j-th largest binary32 score
+ * logits[t, e] + bias[e] (ties to the lower expert index); the weights are a
+ * softmax over the chosen experts' own logits (the bias decides the choice
+ * only), computed in FP32.
+ *   logits [T, E] FP32, bias [E] FP32 or NULL; topk_ids [T, topk] int32 out
+ *   (descending score), topk_w [T, topk] FP32 out.
+ *   Requires 1 <= E <= 1024, 1 <= topk <= min(E, 32); 4-byte aligned
+ *   pointers. NaN scores are never preferred to other scores. */
+METIS_API int metis_moe_route_topk(const float* logits, const float* bias, int64_t T, int64_t E,
+                                   int64_t topk, int32_t* topk_ids, float* topk_w,
+                                   metis_stream_t stream);
+
 /* Routed-expert W8A8 layer ("Lernex/Metis-1.6-Logos-FP8", "What is in FP8":
  * the routed experts are FP8 with per-channel scales and per-token
  * activations). Steps, all on the device, no host synchronisation:

@@ -232,6 +232,76 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
     *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + n) = out;
 }
 
+// Router top-k, one warp per token (the reading of the cards' FP32 router
+// and balance bias): choice j = the j-th largest binary32 score logit + bias,
+// ties to the lower expert index; weight = softmax over the chosen experts'
+// own logits. Lane l keeps the scores of experts l, l + 32, ...; each round
+// takes the warp's best (score, expert) pair, the owning lane marks it taken.
+constexpr int ROUTE_WARPS = 8;
+constexpr int ROUTE_PER_LANE = 32;   // E <= 1024
+constexpr int ROUTE_MAX_K = 32;      // one chosen expert per lane
+__device__ __forceinline__ bool route_better(float v, int e, float bv, int be) {
+    return v > bv || (v == bv && e < be);
+}
+__global__ void __launch_bounds__(ROUTE_WARPS * 32) route_topk_kernel(const float* __restrict__ logits,
+                                                                      const float* __restrict__ bias,
+                                                                      int T, int E, int k,
+                                                                      int32_t* __restrict__ ids,
+                                                                      float* __restrict__ w) {
+    grid_dependency_wait();  // the logits may be the previous kernel's output
+    grid_launch_dependents();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * ROUTE_WARPS + warp;
+    if (t >= T) return;
+    const float* l = logits + t * E;
+    const int per = (E + 31) / 32;
+    float sc[ROUTE_PER_LANE];
+#pragma unroll
+    for (int i = 0; i < ROUTE_PER_LANE; ++i) {
+        const int e = lane + 32 * i;
+        const float v = (i < per && e < E) ? (bias ? __fadd_rn(l[e], bias[e]) : l[e]) : 0.0f;
+        sc[i] = v != v ? -INFINITY : v;  // a NaN score counts as -inf, so every round finds an expert
+    }
+    uint32_t taken = 0;
+    int my_id = -1;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < ROUTE_PER_LANE; ++i) {
+            const int e = lane + 32 * i;
+            if (i < per && e < E && !(taken & (1u << i)) && route_better(sc[i], e, bv, be)) {
+                bv = sc[i];
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (route_better(ov, oe, bv, be)) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == j) my_id = be;
+    }
+    // weights: a softmax over the chosen experts' logits (lanes 0 .. k-1)
+    const float lv = lane < k ? l[my_id] : -INFINITY;
+    float m = lv;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ex = lane < k ? expf(lv - m) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < k) {
+        ids[t * k + lane] = my_id;
+        w[t * k + lane] = __fdiv_rn(ex, sum);
+    }
+}
+
 }  // namespace moe
 }  // namespace metis
 
@@ -378,4 +448,29 @@ extern "C" int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int3
     return metis_moe_fp8_grouped_gemm(x_bf16, topk_ids, topk_w, T, topk, E, H, I, w_up, s_up,
                                       w_down, s_down, act, y_bf16, scratch,
                                       kMoeStaticScratchBytes, stream);
+}
+
+extern "C" int metis_moe_route_topk(const float* logits, const float* bias, int64_t T, int64_t E,
+                                    int64_t topk, int32_t* topk_ids, float* topk_w,
+                                    metis_stream_t stream) {
+    using namespace moe;
+    clear_error();
+    if (T < 0 || T > 0x7fffffff || E < 1 || E > 32 * ROUTE_PER_LANE || topk < 1 || topk > E ||
+        topk > ROUTE_MAX_K)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "moe_route_topk: need T >= 0, 1 <= E <= %d, 1 <= topk <= min(E, %d) "
+                    "(T=%lld E=%lld topk=%lld)", 32 * ROUTE_PER_LANE, ROUTE_MAX_K, (long long)T,
+                    (long long)E, (long long)topk);
+    if (T == 0) return METIS_OK;
+    if (!logits || !topk_ids || !topk_w) return fail(METIS_ERR_INVALID_ARG, "moe_route_topk: null pointer");
+    if (!aligned(logits, 4) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) || (bias && !aligned(bias, 4)))
+        return fail(METIS_ERR_INVALID_ARG, "moe_route_topk: pointers must be 4-byte aligned");
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    const unsigned grid = static_cast<unsigned>((T + ROUTE_WARPS - 1) / ROUTE_WARPS);
+    return cuda_check(launch_pdl(route_topk_kernel, dim3(grid), dim3(ROUTE_WARPS * 32), 0,
+                                 static_cast<cudaStream_t>(stream), 1, logits, bias, static_cast<int>(T),
+                                 static_cast<int>(E), static_cast<int>(topk), topk_ids, topk_w),
+                      "moe_route_topk launch");
 }

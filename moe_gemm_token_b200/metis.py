@@ -64,6 +64,7 @@ def load():
         "metis_quant_fp8_per_channel": ([p, i64, i64, i64, p, i64, p, p], i32),
         "metis_fp8_gemm": ([p, i32, p, p, p, p, i64, i64, i64, p, sz, p], i32),
         "metis_w8a16_gemm": ([p, p, p, p, i64, i64, i64, p], i32),
+        "metis_moe_route_topk": ([p, p, i64, i64, i64, p, p, p], i32),
         "metis_moe_fp8_grouped_gemm": ([p, p, p, i64, i64, i64, i64, i64, p, p, p, p, i32, p, p,
                                         sz, p], i32),
         "metis_moe_fp8_grouped_gemm_noalloc": ([p, p, p, i64, i64, i64, i64, i64, p, p, p, p,
@@ -150,6 +151,14 @@ def metis_w8a16_gemm(x, wq, s_w, y, stream=None):
     N = wq.shape[0]
     return _check("metis_w8a16_gemm", load().metis_w8a16_gemm(
         _p(x), _p(wq), _p(s_w), _p(y), M, N, K, _s(stream)))
+
+
+def metis_moe_route_topk(logits, topk_ids, topk_w, bias=None, stream=None):
+    """Router top-k: logits [T, E] FP32 (+ bias [E]) -> topk_ids [T, k], topk_w [T, k]."""
+    T, E = logits.shape
+    k = topk_ids.shape[1]
+    return _check("metis_moe_route_topk", load().metis_moe_route_topk(
+        _p(logits), _p(bias), T, E, k, _p(topk_ids), _p(topk_w), _s(stream)))
 
 
 def metis_moe_fp8_grouped_gemm(x, topk_ids, topk_w, w_up, s_up, w_down, s_down, y, workspace,

@@ -95,6 +95,11 @@ def test_host_validation_without_gpu(lib):
     assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 2, 4, 64, 32, p, p, p, p, 0, p, p, 16,
                                           null) == metis.METIS_ERR_INVALID_ARG
     assert b"workspace" in lib.metis_last_error()
+    # router top-k: topk > E, E > 1024, topk > 32
+    assert lib.metis_moe_route_topk(p, null, 8, 4, 5, p, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_moe_route_topk(p, null, 8, 1025, 4, p, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_moe_route_topk(p, null, 8, 64, 33, p, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_moe_route_topk(p, null, 0, 64, 8, p, p, null) == metis.METIS_OK
     # dispatch: the default maths for M > 8 validates like metis_w8a16_gemm
     assert lib.metis_linear(p, p, p, p, 64, 100, 256, 0, p, p, 1 << 20, null) == metis.METIS_ERR_INVALID_ARG
     # fast-math dispatch needs room for the codes of x

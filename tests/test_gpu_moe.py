@@ -112,3 +112,61 @@ def test_moe_deterministic(metis):
     b = run_moe(metis, d)
     for key in ("y", "h", "o", "s2r"):
         assert np.array_equal(a[key], b[key]), key
+
+
+# ---------------------------------------------------------------- router top-k
+
+def _route_gpu(metis, logits32, k, bias32=None):
+    T, E = logits32.shape
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    metis.metis_moe_route_topk(dev(logits32), ids, w, bias=None if bias32 is None else dev(bias32))
+    assert metis.metis_check_device_status() == 0
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("T,E,k,seed,with_bias", [(4096, 64, 8, 20, False), (4096, 64, 8, 21, True),
+                                                  (333, 100, 4, 22, True), (64, 7, 7, 23, False),
+                                                  (50, 1024, 32, 24, True), (257, 192, 4, 25, True)])
+def test_route_topk_parity(metis, T, E, k, seed, with_bias):
+    """Ids bit-exact against the oracle (the same binary32 scores decide);
+    weights within 1e-5 (FP32 softmax against float64)."""
+    rng = np.random.default_rng(seed)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    b = (rng.standard_normal(E) * 0.5).astype(np.float32) if with_bias else None
+    ids, w = _route_gpu(metis, lg, k, b)
+    ids_r, w_r = oracle.route_topk(lg, k, b)
+    assert_bytes_equal(ids, ids_r, "router ids")
+    assert np.max(np.abs(w.astype(np.float64) - w_r)) <= 1e-5
+
+
+def test_route_topk_ties_and_infinities(metis):
+    """Integer logits (ties everywhere) and -inf logits: the lower expert
+    index wins ties; -inf experts are chosen last."""
+    rng = np.random.default_rng(26)
+    lg = rng.integers(-2, 3, (512, 40)).astype(np.float32)
+    lg[:, 5] = -np.inf
+    lg[::7, :] = 1.0  # whole rows tied
+    b = (rng.integers(-1, 2, 40) * 0.5).astype(np.float32)
+    cases = [(lg, 1, None), (lg, 8, None), (lg, 8, b), (lg, 32, b),
+             (np.ascontiguousarray(lg[:, :20]), 20, b[:20].copy())]  # all chosen: -inf last
+    for lgc, k, bias in cases:
+        ids, w = _route_gpu(metis, lgc, k, bias)
+        ids_r, w_r = oracle.route_topk(lgc, k, bias)
+        assert_bytes_equal(ids, ids_r, f"router ids k={k}")
+        assert np.max(np.abs(w.astype(np.float64) - w_r)) <= 1e-5
+
+
+def test_route_topk_feeds_the_layer(metis):
+    """The routed-expert layer fed by the GPU router equals the oracle layer
+    fed by the oracle router (same ids; weights within 1e-5)."""
+    d = synth.moe(seed=27, T=192, H=256, I=128, E=16, topk=4, hot=2, load_ratio=2.0)
+    lg = d["logits"].astype(np.float32)
+    ids, w = _route_gpu(metis, lg, 4)
+    ids_r, w_r = oracle.route_topk(lg, 4)
+    assert_bytes_equal(ids, ids_r, "router ids")
+    d["topk_ids"], d["topk_w"] = ids, w
+    g = run_moe(metis, d)
+    ref = oracle.moe_forward(d["x"], ids_r, w_r.astype(np.float32), g["wq_up"], g["s_up"], g["wq_dn"],
+                             g["s_dn"])
+    assert_close(g["y"], ref["y64"], "layer fed by the GPU router")
