@@ -243,6 +243,7 @@ constexpr int ROUTE_MAX_K = 32;      // one chosen expert per lane
 __device__ __forceinline__ bool route_better(float v, int e, float bv, int be) {
     return v > bv || (v == bv && e < be);
 }
+template <int P>  // scores per lane: E <= 32 P
 __global__ void __launch_bounds__(ROUTE_WARPS * 32) route_topk_kernel(const float* __restrict__ logits,
                                                                       const float* __restrict__ bias,
                                                                       int T, int E, int k,
@@ -254,12 +255,11 @@ __global__ void __launch_bounds__(ROUTE_WARPS * 32) route_topk_kernel(const floa
     const int64_t t = static_cast<int64_t>(blockIdx.x) * ROUTE_WARPS + warp;
     if (t >= T) return;
     const float* l = logits + t * E;
-    const int per = (E + 31) / 32;
-    float sc[ROUTE_PER_LANE];
+    float sc[P];
 #pragma unroll
-    for (int i = 0; i < ROUTE_PER_LANE; ++i) {
+    for (int i = 0; i < P; ++i) {
         const int e = lane + 32 * i;
-        const float v = (i < per && e < E) ? (bias ? __fadd_rn(l[e], bias[e]) : l[e]) : 0.0f;
+        const float v = e < E ? (bias ? __fadd_rn(l[e], bias[e]) : l[e]) : 0.0f;
         sc[i] = v != v ? -INFINITY : v;  // a NaN score counts as -inf, so every round finds an expert
     }
     uint32_t taken = 0;
@@ -268,9 +268,9 @@ __global__ void __launch_bounds__(ROUTE_WARPS * 32) route_topk_kernel(const floa
         float bv = -INFINITY;
         int be = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < ROUTE_PER_LANE; ++i) {
+        for (int i = 0; i < P; ++i) {
             const int e = lane + 32 * i;
-            if (i < per && e < E && !(taken & (1u << i)) && route_better(sc[i], e, bv, be)) {
+            if (e < E && !(taken & (1u << i)) && route_better(sc[i], e, bv, be)) {
                 bv = sc[i];
                 be = e;
             }
@@ -469,8 +469,17 @@ extern "C" int metis_moe_route_topk(const float* logits, const float* bias, int6
     int rc = current_device_info(&di);
     if (rc) return rc;
     const unsigned grid = static_cast<unsigned>((T + ROUTE_WARPS - 1) / ROUTE_WARPS);
-    return cuda_check(launch_pdl(route_topk_kernel, dim3(grid), dim3(ROUTE_WARPS * 32), 0,
-                                 static_cast<cudaStream_t>(stream), 1, logits, bias, static_cast<int>(T),
-                                 static_cast<int>(E), static_cast<int>(topk), topk_ids, topk_w),
-                      "moe_route_topk launch");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int iT = static_cast<int>(T), iE = static_cast<int>(E), ik = static_cast<int>(topk);
+    auto go = [&](auto kernel) {
+        return cuda_check(launch_pdl(kernel, dim3(grid), dim3(ROUTE_WARPS * 32), 0, st, 1, logits, bias, iT, iE,
+                                     ik, topk_ids, topk_w),
+                          "moe_route_topk launch");
+    };
+    if (E <= 32) return go(route_topk_kernel<1>);
+    if (E <= 64) return go(route_topk_kernel<2>);
+    if (E <= 128) return go(route_topk_kernel<4>);
+    if (E <= 256) return go(route_topk_kernel<8>);
+    if (E <= 512) return go(route_topk_kernel<16>);
+    return go(route_topk_kernel<32>);
 }
