@@ -65,6 +65,28 @@ def env_rank():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def rank_seed(set_index, rank):
+    """Seed of layer set `set_index` on `rank`: every rank draws its own
+    token batch and weights (weak scaling, independent replicas)."""
+    return 1 + 100 * set_index + 10000 * rank
+
+
+def max_over_ranks(value, dist, device, world):
+    """The slowest rank's device time (all ranks take part; rank order of the
+    collective is the same on every rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_rank, ms_per_step):
+    """Whole-job tokens per second: every rank processes its own batch per step."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_prefill_tokens(d, wq, tokens):
@@ -247,7 +269,7 @@ def run_metis(args):
     # ---- inputs: SETS layer sets, weights quantized per channel on the GPU
     sets = []
     for r in range(SETS):
-        d = synth.prefill_chain(seed=1 + 100 * r + 10000 * rank)
+        d = synth.prefill_chain(seed=rank_seed(r, rank))
         ws = []
         for w in (d["w1"], d["w2"]):
             wd = torch.from_numpy(w).to(dev)
@@ -316,13 +338,9 @@ def run_metis(args):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    elapsed_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dist, dev, world)
     ms_per_step = elapsed_ms / args.steps
-    value = world * M_TOK / (ms_per_step * 1e-3)
+    value = job_throughput(world, M_TOK, ms_per_step)
 
     # ---- roofline of the dominant kernel (the W8A8 GEMM), from the live events
     g1 = [e[0].elapsed_time(e[1]) for e in evs.values()]
@@ -396,12 +414,8 @@ def run_metis(args):
     stream.wait_stream(s_d2h)
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * M_TOK / (e2e_ms * 1e-3), "unit": "tok/s",
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, dist, dev, world)
+    e2e = {"value": job_throughput(world, M_TOK, e2e_ms), "unit": "tok/s",
            "h2d_bytes_per_step": M_TOK * K_HID * 2, "d2h_bytes_per_step": M_TOK * K_HID * 2,
            "steps": e2e_steps, "api": "metis_linear x 2 per step",
            "pipelined": "upload of step i+1 and download of step i-1 overlap step i "

@@ -75,6 +75,15 @@ METIS_API int metis_version(void);
  * The pointer stays valid until the next library call on this thread. */
 METIS_API const char* metis_last_error(void);
 
+/* Self-test of the device watchdog; the pages have no counterpart. One
+ * thread waits on an mbarrier that nothing ever completes, bounded by
+ * `limit_ns` (1 .. 1e9 ns); when the limit runs out the kernel sets the
+ * sticky device error word and returns, exactly as a stalled wait in any
+ * other kernel would. metis_check_device_status() then reports
+ * METIS_ERR_TIMEOUT and the CUDA context stays usable. The kernel touches no
+ * global memory other than the status word, and no tensor memory or TMA. */
+METIS_API int metis_watchdog_selftest(uint64_t limit_ns, metis_stream_t stream);
+
 /* Reads (and, if `clear` != 0, clears) the sticky device error word on the
  * current device, synchronising `stream` first. Returns METIS_OK,
  * METIS_ERR_TIMEOUT if a kernel's bounded wait ran out, or METIS_ERR_CUDA.

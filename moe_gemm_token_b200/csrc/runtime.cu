@@ -196,6 +196,32 @@ extern "C" int metis_set_watchdog_ns(uint64_t ns) {
     return METIS_OK;
 }
 
+namespace metis {
+// A wait that nothing satisfies: the bounded mbarrier wait gives up after
+// limit_ns and records the timeout in the status word.
+__global__ void __launch_bounds__(32) watchdog_selftest_kernel(uint64_t limit_ns, uint32_t* status) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, limit_ns, status);
+}
+}  // namespace metis
+
+extern "C" int metis_watchdog_selftest(uint64_t limit_ns, metis_stream_t stream) {
+    clear_error();
+    if (limit_ns < 1 || limit_ns > 1000000000ull)
+        return fail(METIS_ERR_INVALID_ARG, "watchdog_selftest: limit_ns=%llu, need 1 .. 1e9",
+                    (unsigned long long)limit_ns);
+    uint32_t* status = nullptr;
+    int rc = device_status_word(&status);
+    if (rc) return rc;
+    watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, status);
+    return cuda_check(cudaGetLastError(), "watchdog self-test launch");
+}
+
 extern "C" int metis_check_device_status(metis_stream_t stream, int clear) {
     clear_error();
     uint32_t* word = nullptr;

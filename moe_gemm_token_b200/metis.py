@@ -60,6 +60,7 @@ def load():
         "metis_last_error": ([], ctypes.c_char_p),
         "metis_check_device_status": ([p, i32], i32),
         "metis_set_watchdog_ns": ([ctypes.c_uint64], i32),
+        "metis_watchdog_selftest": ([ctypes.c_uint64, p], i32),
         "metis_quant_fp8_per_token": ([p, i64, i64, i64, p, i64, p, p], i32),
         "metis_quant_fp8_per_channel": ([p, i64, i64, i64, p, i64, p, p], i32),
         "metis_fp8_gemm": ([p, i32, p, p, p, p, i64, i64, i64, p, sz, p], i32),
@@ -114,6 +115,11 @@ def metis_version():
 def metis_check_device_status(stream=None, clear=True):
     """Synchronises the stream and returns the sticky device status (0 = OK)."""
     return load().metis_check_device_status(_s(stream), int(bool(clear)))
+
+
+def metis_watchdog_selftest(limit_ns, stream=None):
+    """Launches a wait that nothing satisfies, bounded by limit_ns (see the header)."""
+    return _check("metis_watchdog_selftest", load().metis_watchdog_selftest(int(limit_ns), _s(stream)))
 
 
 def metis_set_watchdog_ns(ns):

@@ -95,6 +95,9 @@ def test_host_validation_without_gpu(lib):
     assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 2, 4, 64, 32, p, p, p, p, 0, p, p, 16,
                                           null) == metis.METIS_ERR_INVALID_ARG
     assert b"workspace" in lib.metis_last_error()
+    # watchdog self-test: the limit must be 1 .. 1e9 ns
+    assert lib.metis_watchdog_selftest(0, null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_watchdog_selftest(2000000000, null) == metis.METIS_ERR_INVALID_ARG
     # router top-k: topk > E, E > 1024, topk > 32
     assert lib.metis_moe_route_topk(p, null, 8, 4, 5, p, p, null) == metis.METIS_ERR_INVALID_ARG
     assert lib.metis_moe_route_topk(p, null, 8, 1025, 4, p, p, null) == metis.METIS_ERR_INVALID_ARG
