@@ -50,6 +50,15 @@ def _load():
         lib.metis_oracle_e4m3_encode_array.argtypes = [p, i64, p]
         lib.metis_oracle_e4m3_decode_array.argtypes = [p, i64, p]
         lib.metis_oracle_bf16_from_double_array.argtypes = [p, i64, p]
+        lib.metis_oracle_route_topk.argtypes = [p, p, i64, i64, i64, p, p]
+        lib.metis_oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.metis_oracle_e2m1_decode.restype = ctypes.c_double
+        lib.metis_oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.metis_oracle_e2m1_encode.restype = ctypes.c_uint8
+        lib.metis_oracle_nvfp4_quant.argtypes = [p, i64, i64, ctypes.c_int, p, p, p]
+        lib.metis_oracle_nvfp4_gemm.argtypes = [p, p, p, p, p, ctypes.c_float, i64, i64, i64, p, p]
+        for name in ("route_topk", "nvfp4_quant", "nvfp4_gemm"):
+            getattr(lib, "metis_oracle_" + name).restype = ctypes.c_int
         for name in ("e4m3_encode_array", "e4m3_decode_array", "bf16_from_double_array"):
             getattr(lib, "metis_oracle_" + name).restype = None
         for name in ("quant_rows_bf16", "quant_rows_f32", "gemm_w8a8", "gemm_w8a16",
@@ -292,3 +301,137 @@ def moe_forward(x_bf16, topk_ids, topk_w, w_up, s_up, w_down, s_down, tokens=Non
     y, y64 = moe_combine(o.reshape(nt, k, -1), w[tokens])
     return dict(xq=xq, s_x=s_x, h=h, h64=h64, hq=hq, s_h=s_h, o=o, o64=o64, y=y, y64=y64,
                 tokens=tokens)
+
+
+# ------------------------------------------------------------------ NVFP4
+# "Lernex/Metis-1.6-Praxis-NVFP4", "What is in NVFP4": routed experts hold
+# 4-bit E2M1 values, one E4M3 scale per 16 inputs and one FP32 scale per
+# expert; "What --fast-math does": with fast-math their inputs are rounded to
+# FP4 as well. The scale rule (global scale amax/2688 = amax/(6 * 448), block
+# scale E4M3(block amax * (2688/amax) / 6)) is this oracle's reading; the
+# pages print none. Codes are carried one per byte here; the library's packed
+# form (two codes per byte, the even k in the low nibble) is converted by
+# e2m1_pack / e2m1_unpack, which do no arithmetic.
+
+def e2m1_decode(c):
+    """Exact value of each E2M1 code (low 4 bits), as float64."""
+    lib = _load()
+    c = np.asarray(c, dtype=np.uint8)
+    return np.vectorize(lambda b: lib.metis_oracle_e2m1_decode(int(b)), otypes=[np.float64])(c) \
+        if c.size else np.zeros(c.shape)
+
+
+def e2m1_encode(v):
+    """binary32 -> E2M1 code: nearest of +-{0, .5, 1, 1.5, 2, 3, 4, 6}, ties to
+    the even mantissa, saturating to +-6."""
+    lib = _load()
+    v = _c(v, np.float32)
+    return np.vectorize(lambda x: lib.metis_oracle_e2m1_encode(float(x)), otypes=[np.uint8])(v) \
+        if v.size else np.zeros(v.shape, dtype=np.uint8)
+
+
+def e2m1_pack(q):
+    """[R, K] codes (one per byte) -> [R, K/2] bytes, code of k = 2i in the low nibble."""
+    q = np.asarray(q, dtype=np.uint8)
+    return (q[..., 0::2] & 0xF) | ((q[..., 1::2] & 0xF) << 4)
+
+
+def e2m1_unpack(b):
+    """[R, K/2] packed bytes -> [R, K] codes."""
+    b = np.asarray(b, dtype=np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = b & 0xF
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def nvfp4_quant(x, per_row=True):
+    """NVFP4 quantization of rows [R, K] (K % 16 == 0) given as float32, or as
+    BF16 bit patterns (uint16, widened exactly).
+
+    per_row: one global scale per row (activations, per token); otherwise one
+    for the whole matrix (an expert's weights). Returns (codes uint8 [R, K],
+    block scales uint8 E4M3 codes [R, K/16], g float32 [R] or [1])."""
+    lib = _load()
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        x = bf16_to_float(x)
+    x = _c(x, np.float32)
+    R, K = x.shape
+    q = np.empty((R, K), dtype=np.uint8)
+    sb = np.empty((R, K // 16), dtype=np.uint8)
+    g = np.empty((R if per_row else 1,), dtype=np.float32)
+    _check(lib.metis_oracle_nvfp4_quant(_ptr(x), R, K, int(bool(per_row)), _ptr(q), _ptr(sb),
+                                        _ptr(g)), "nvfp4_quant")
+    return q, sb, g
+
+
+def nvfp4_dequant(q, sb, g):
+    """D2(q) * D(sb) * g as float64 ([R, K]); g has one entry per row or one."""
+    q = np.asarray(q, dtype=np.uint8)
+    R, K = q.shape
+    v = e2m1_decode(q) * np.repeat(e4m3_decode(sb), 16, axis=1)
+    g = np.asarray(g, dtype=np.float64)
+    return v * (g.reshape(-1, 1) if g.size == R else g.reshape(1, 1))
+
+
+def nvfp4_gemm(qa, sa, ga, qb, sbb, gb, rows=None):
+    """y[m, n] = bf16(ga[m] gb sum_k D2(qa) D(sa) D2(qb) D(sbb)), float64 sum.
+
+    qa [M, K] codes, sa [M, K/16], ga [M]; qb [N, K], sbb [N, K/16], gb one
+    float. ``rows`` selects rows of A (default all). Returns (bf16 bits,
+    float64 before rounding)."""
+    lib = _load()
+    if rows is not None:
+        rows = np.asarray(rows, dtype=np.int64)
+        qa, sa, ga = np.asarray(qa)[rows], np.asarray(sa)[rows], np.asarray(ga)[rows]
+    qa, sa, ga = _c(qa, np.uint8), _c(sa, np.uint8), _c(ga, np.float32)
+    qb, sbb = _c(qb, np.uint8), _c(sbb, np.uint8)
+    M, K = qa.shape
+    N = qb.shape[0]
+    y = np.empty((M, N), dtype=np.uint16)
+    y64 = np.empty((M, N), dtype=np.float64)
+    _check(lib.metis_oracle_nvfp4_gemm(_ptr(qa), _ptr(sa), _ptr(ga), _ptr(qb), _ptr(sbb),
+                                       float(np.float32(gb)), M, N, K, _ptr(y), _ptr(y64)),
+           "nvfp4_gemm")
+    return y, y64
+
+
+def moe_forward_nvfp4(x_bf16, topk_ids, topk_w, up, down, tokens=None):
+    """Routed-expert layer with NVFP4 experts under fast-math.
+
+    ``up`` / ``down`` are (codes [E, N, K], block scales [E, N, K/16], g [E])
+    per projection. Steps: x quantized to NVFP4 per token; per routed slot
+    (t, j), e = ids[t, j]: h = bf16(g_x[t] g_up[e] sum ...); h quantized to
+    NVFP4 per slot row; o = bf16(g_h g_dn[e] sum ...); y[t] = bf16(sum_j
+    w[t, j] o[t, j]) in float64. Returns every intermediate, rows ordered by
+    selected token, then j."""
+    x = _c(x_bf16, np.uint16)
+    ids = _c(topk_ids, np.int32)
+    w = _c(topk_w, np.float32)
+    T, k = ids.shape
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    qx, sx, gx = nvfp4_quant(x[tokens], per_row=True)
+    nt = tokens.size
+    slot_tok = np.repeat(np.arange(nt), k)
+    slot_exp = ids[tokens].reshape(-1)
+
+    def expert_gemm(qa, sa, ga, wts):
+        qw, sw, gw = wts
+        N = qw.shape[1]
+        y = np.empty((qa.shape[0], N), dtype=np.uint16)
+        y64 = np.empty((qa.shape[0], N), dtype=np.float64)
+        for e in np.unique(slot_exp):
+            sel = np.nonzero(slot_exp == e)[0]
+            ye, y64e = nvfp4_gemm(qa[sel], sa[sel], ga[sel], qw[e], sw[e], gw[e])
+            y[sel] = ye
+            y64[sel] = y64e
+        return y, y64
+
+    h, h64 = expert_gemm(qx[slot_tok], sx[slot_tok], gx[slot_tok], up)
+    qh, sh, gh = nvfp4_quant(h, per_row=True)
+    o, o64 = expert_gemm(qh, sh, gh, down)
+    y, y64 = moe_combine(o.reshape(nt, k, -1), w[tokens])
+    return dict(qx=qx, sx=sx, gx=gx, h=h, h64=h64, qh=qh, sh=sh, gh=gh, o=o, o64=o64, y=y,
+                y64=y64, tokens=tokens)
+

@@ -283,6 +283,118 @@ int metis_oracle_moe_route(const int32_t* ids, int64_t T, int64_t topk, int64_t 
     return ORACLE_OK;
 }
 
+/* ------------------------------------------------------------------ NVFP4
+ * "Lernex/Metis-1.6-Praxis-NVFP4", "What is in NVFP4": the routed experts are
+ * "4-bit E2M1 values with one FP8 (E4M3) scale per 16 inputs and an FP32
+ * scale per expert"; with --fast-math "the 4-bit experts multiply in FP4",
+ * their inputs rounded to FP4 too (section "What --fast-math does"). The card
+ * prints no rounding rule. Reading, for a row (a token, or an output channel
+ * of an expert) and its scale owner (the token itself, or the whole expert):
+ *   g     = amax_owner / 2688            (binary32; 2688 = 6 * 448)
+ *   inv_g = 2688 / amax_owner, 0 if amax_owner = 0 (binary32, FLT_MAX clamp)
+ *   per 16-element block with block amax b:
+ *     sb  = E4M3( (b * inv_g) / 6 )      (each step binary32, nearest-even,
+ *                                         saturating; a non-negative code)
+ *     q_i = E2M1( (x_i * inv_g) * (1 / D(sb)) ), 0 when sb decodes to 0
+ *   value_i = D2(q_i) * D(sb) * g.
+ * E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit: magnitudes
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6; nearest-even, saturating to 6, no NaN. */
+double metis_oracle_e2m1_decode(uint8_t c) {
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    double v = mag[c & 7];
+    return (c & 8) ? -v : v;
+}
+
+uint8_t metis_oracle_e2m1_encode(float v) {
+    /* nearest of the 8 magnitudes, ties to the even mantissa (codes 0, 2, 4, 6) */
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    uint8_t sign = signbit(v) ? 8 : 0;
+    double a = fabs((double)v);
+    uint8_t best = 0;
+    int i;
+    if (a >= 6.0) return sign | 7; /* saturate */
+    for (i = 1; i < 8; ++i) {
+        double d_best = fabs(a - mag[best]), d = fabs(a - mag[i]);
+        if (d < d_best || (d == d_best && (i & 1) == 0)) best = (uint8_t)i;
+    }
+    return sign | best;
+}
+
+/* Quantizes rows [R, K] (K % 16 == 0) to NVFP4: codes [R, K] one per byte,
+ * block scales [R, K/16] E4M3 codes, and the global scale(s): one per row
+ * when per_row != 0, else one for all rows (written to g[0]). */
+int metis_oracle_nvfp4_quant(const float* x, int64_t R, int64_t K, int per_row, uint8_t* q,
+                             uint8_t* sb, float* g) {
+    int64_t r, k, b;
+    float amax_all = 0.0f;
+    if (K % 16 != 0) return ORACLE_BAD_INDEX;
+    if (!per_row) {
+        for (r = 0; r < R * K; ++r) {
+            float a = fabsf(x[r]);
+            if (a > amax_all) amax_all = a;
+        }
+    }
+    for (r = 0; r < R; ++r) {
+        const float* row = x + r * K;
+        float amax = amax_all, inv_g;
+        if (per_row) {
+            amax = 0.0f;
+            for (k = 0; k < K; ++k)
+                if (fabsf(row[k]) > amax) amax = fabsf(row[k]);
+        }
+        inv_g = amax > 0.0f ? 2688.0f / amax : 0.0f;
+        if (inv_g > FLT_MAX) inv_g = FLT_MAX;
+        if (per_row) g[r] = amax / 2688.0f;
+        else if (r == 0) g[0] = amax / 2688.0f;
+        for (b = 0; b < K / 16; ++b) {
+            float bamax = 0.0f, t, ds, inv_s;
+            uint8_t code;
+            for (k = 0; k < 16; ++k)
+                if (fabsf(row[b * 16 + k]) > bamax) bamax = fabsf(row[b * 16 + k]);
+            t = bamax * inv_g;
+            t = t / 6.0f;
+            code = metis_oracle_e4m3_encode(t);
+            sb[r * (K / 16) + b] = code;
+            ds = (float)metis_oracle_e4m3_decode(code);
+            inv_s = ds > 0.0f ? 1.0f / ds : 0.0f;
+            for (k = 0; k < 16; ++k) {
+                float v = row[b * 16 + k] * inv_g;
+                v = v * inv_s;
+                q[r * K + b * 16 + k] = ds > 0.0f ? metis_oracle_e2m1_encode(v) : (uint8_t)(signbit(row[b * 16 + k]) ? 8 : 0);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* NVFP4 GEMM: y[m, n] = bf16( ga[m] * gb * sum_k V(a)[m, k] * V(b)[n, k] ) with
+ * V = D2(q) * D(sb) per 16-element block, float64 sum, one final rounding.
+ * ga [M] per token, gb one scale for B (the expert's). */
+int metis_oracle_nvfp4_gemm(const uint8_t* qa, const uint8_t* sa, const float* ga,
+                            const uint8_t* qb, const uint8_t* sbb, float gb, int64_t M,
+                            int64_t N, int64_t K, uint16_t* y, double* y64) {
+    int64_t m;
+    if (K % 16 != 0) return ORACLE_BAD_INDEX;
+#pragma omp parallel for schedule(static)
+    for (m = 0; m < M; ++m) {
+        int64_t n, k;
+        for (n = 0; n < N; ++n) {
+            double acc = 0.0, v;
+            for (k = 0; k < K; ++k) {
+                double av = metis_oracle_e2m1_decode(qa[m * K + k]) *
+                            metis_oracle_e4m3_decode(sa[m * (K / 16) + k / 16]);
+                double bv = metis_oracle_e2m1_decode(qb[n * K + k]) *
+                            metis_oracle_e4m3_decode(sbb[n * (K / 16) + k / 16]);
+                acc += av * bv;
+            }
+            v = (double)ga[m] * (double)gb * acc;
+            y64[m * N + n] = v;
+            y[m * N + n] = metis_oracle_bf16_from_double(v);
+        }
+    }
+    return ORACLE_OK;
+}
+
 /* Router top-k. The cards keep "the routers and their balance bias" in FP32
  * ("Lernex/Metis-1.6-Logos-FP8", "What is in FP8") and route each token to
  * a few experts; they print no formula. Reading: the balance bias only
