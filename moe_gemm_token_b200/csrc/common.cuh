@@ -61,6 +61,24 @@ int launch_quant_rows(const T* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
                       float* s, cudaStream_t st, const int32_t* dst_rows, int topk,
                       float* inv_out = nullptr);
 
+// NVFP4 quantizer (nvfp4.cu), T = __nv_bfloat16 or float; arguments
+// validated by the caller. rps > 1: rows [i*rps, (i+1)*rps) share a global
+// scale. tiled: block scales in the tensor-core atom layout. dst_rows
+// non-null: row r goes to rows dst_rows[r * topk + j] (negative skipped).
+// row_valid / nrows non-null: rows with row_valid[r] < 0, or r >= *nrows, skipped.
+template <typename T>
+int launch_nvfp4_quant(const T* x, int64_t R, int64_t K, int64_t ldx, int64_t rps, uint8_t* q,
+                       uint8_t* sf, int tiled, float* g, const int32_t* dst_rows, int topk,
+                       const int32_t* row_valid, const int32_t* nrows, cudaStream_t st);
+
+// NVFP4 block-scaled GEMM (nvfp4.cu). a_rows: rows of A's code buffer (a
+// multiple of 128); offsets/counts null: dense with M rows, else grouped
+// (expert e's rows start at offsets[e], a multiple of 128, counts[e] real).
+int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, int64_t a_rows,
+                      const uint8_t* qb, const uint8_t* sfb, const float* gb, int64_t b_rows,
+                      __nv_bfloat16* y, const int32_t* offsets, const int32_t* counts, int E, int M,
+                      int N, int K, cudaStream_t st);
+
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Device error word bits.

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "../../include/metis_nvfp4.h"
 
 namespace metis {
 
@@ -25,6 +26,9 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
                             int K, cudaStream_t st);
 int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
                           int64_t* total);
+int64_t moe4_padded_rows(int64_t T, int64_t topk, int64_t E);
+int64_t moe4_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
+                           int64_t* total);
 
 namespace moe {
 
@@ -57,9 +61,12 @@ __global__ void __launch_bounds__(CHUNK) count_kernel(const int32_t* __restrict_
 // are read in one batch of loads per thread rather than C sequential ones.
 constexpr int SCAN_THREADS = 1024;
 constexpr int SCAN_BATCH = 8;
+// pad > 1: each expert's first row is a multiple of pad (its rows padded up
+// to one); row_to_slot of the pad rows is set to -1 when r2s_pad is non-null.
 __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict__ chunk_counts, int C,
                                                             int E, int32_t* __restrict__ counts,
-                                                            int32_t* __restrict__ offsets) {
+                                                            int32_t* __restrict__ offsets, int pad,
+                                                            int32_t* __restrict__ r2s_pad) {
     __shared__ int part[SCAN_THREADS];  // [g][e]: sums, then prefix over g
     __shared__ int warp_tot[32];
     __shared__ int excl_e[MAX_E];
@@ -91,9 +98,10 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
             total += v;
         }
     }
-    // block-wide exclusive scan of the totals over e (thread t holds expert t)
+    // block-wide exclusive scan of the padded totals over e (thread t holds expert t)
+    const int ptotal = (total + pad - 1) / pad * pad;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = total;
+    int incl = ptotal;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -113,11 +121,13 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
     }
     __syncthreads();
     if (threadIdx.x < E) {
-        const int excl = warp_tot[warp] + incl - total;
+        const int excl = warp_tot[warp] + incl - ptotal;
         counts[threadIdx.x] = total;
         offsets[threadIdx.x] = excl;
         excl_e[threadIdx.x] = excl;
-        if (threadIdx.x == E - 1) offsets[E] = excl + total;
+        if (threadIdx.x == E - 1) offsets[E] = excl + ptotal;
+        if (r2s_pad)
+            for (int r = excl + total; r < excl + ptotal; ++r) r2s_pad[r] = -1;
     }
     __syncthreads();
     // chunk bases: this thread's run of chunks, from its expert's offset plus
@@ -364,7 +374,8 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     if ((rc = device_status_word(&status))) return rc;
     count_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
                                       status);
-    scan_kernel<<<1, SCAN_THREADS, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets);
+    scan_kernel<<<1, SCAN_THREADS, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets, 1,
+                                            nullptr);
     rank_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
                                      s2r, r2s);
     if ((rc = cuda_check(cudaGetLastError(), "moe routing launch"))) return rc;
@@ -482,4 +493,97 @@ extern "C" int metis_moe_route_topk(const float* logits, const float* bias, int6
     if (E <= 256) return go(route_topk_kernel<8>);
     if (E <= 512) return go(route_topk_kernel<16>);
     return go(route_topk_kernel<32>);
+}
+
+// ---------------------------------------------------------------------------
+// Routed-expert layer with NVFP4 experts under fast-math ("Lernex/Metis-1.6-
+// Praxis-NVFP4", "What is in NVFP4" and "What --fast-math does"): the steps
+// of the W8A8 layer above, with each expert's rows padded to a multiple of
+// 128 so that every tile's scale atoms are whole (one bulk copy each), x and
+// h quantized to NVFP4 (per-token global scale, E4M3 scale per 16), and the
+// block-scaled tcgen05 GEMM for both projections.
+extern "C" int metis_moe_nvfp4_grouped_gemm(const void* x_bf16, const int32_t* topk_ids,
+                                            const float* topk_w, int64_t T, int64_t topk,
+                                            int64_t E, int64_t H, int64_t I, const uint8_t* w_up,
+                                            const uint8_t* sf_up, const float* g_up,
+                                            const uint8_t* w_down, const uint8_t* sf_down,
+                                            const float* g_down, int act, void* y_bf16,
+                                            void* workspace, size_t ws_bytes,
+                                            metis_stream_t stream) {
+    using namespace moe;
+    clear_error();
+    if (act != METIS_ACT_NONE)
+        return fail(METIS_ERR_UNSUPPORTED, "moe_nvfp4: act=%d; only METIS_ACT_NONE is built", act);
+    if (T < 0 || topk < 1 || E < topk || E > MAX_E)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "moe_nvfp4: need T >= 0 and 1 <= topk <= E <= %d (T=%lld topk=%lld E=%lld)", MAX_E,
+                    (long long)T, (long long)topk, (long long)E);
+    if (H < 128 || I < 128 || H % 128 || I % 128 || H > 16384 || I > 65536)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "moe_nvfp4: need H and I multiples of 128, H <= 16384, I <= 65536 (H=%lld I=%lld)",
+                    (long long)H, (long long)I);
+    const int64_t S = T * topk;
+    if (S > (1ll << 28)) return fail(METIS_ERR_INVALID_ARG, "moe_nvfp4: T*topk too large");
+    const size_t need = metis_workspace_size(METIS_OP_MOE_NVFP4, T, I, H, topk, E);
+    if (T == 0) return METIS_OK;
+    if (!x_bf16 || !topk_ids || !topk_w || !w_up || !sf_up || !g_up || !w_down || !sf_down || !g_down ||
+        !y_bf16 || !workspace)
+        return fail(METIS_ERR_INVALID_ARG, "moe_nvfp4: null pointer");
+    if (ws_bytes < need)
+        return fail(METIS_ERR_INVALID_ARG, "moe_nvfp4: workspace of %zu bytes, need %zu", ws_bytes, need);
+    if (!aligned(workspace, 256) || !aligned(x_bf16, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
+        !aligned(sf_up, 16) || !aligned(sf_down, 16) || !aligned(y_bf16, 16) || !aligned(g_up, 4) ||
+        !aligned(g_down, 4))
+        return fail(METIS_ERR_INVALID_ARG,
+                    "moe_nvfp4: workspace 256-byte aligned; x, codes, tiled scales and y 16-byte aligned");
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto region = [&](int r) { return ws + moe4_region_offset(r, T, topk, E, H, I, nullptr); };
+    int32_t* counts = reinterpret_cast<int32_t*>(region(METIS_MOE4_WS_COUNTS));
+    int32_t* offsets = reinterpret_cast<int32_t*>(region(METIS_MOE4_WS_OFFSETS));
+    int32_t* s2r = reinterpret_cast<int32_t*>(region(METIS_MOE4_WS_SLOT_TO_ROW));
+    int32_t* r2s = reinterpret_cast<int32_t*>(region(METIS_MOE4_WS_ROW_TO_SLOT));
+    uint8_t* aq = region(METIS_MOE4_WS_AQ);
+    uint8_t* sfa = region(METIS_MOE4_WS_SFA);
+    float* ga = reinterpret_cast<float*>(region(METIS_MOE4_WS_GA));
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(region(METIS_MOE4_WS_H));
+    uint8_t* hq = region(METIS_MOE4_WS_HQ);
+    uint8_t* sfh = region(METIS_MOE4_WS_SFH);
+    float* gh = reinterpret_cast<float*>(region(METIS_MOE4_WS_GH));
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(region(METIS_MOE4_WS_O));
+    const int64_t Sp = moe4_padded_rows(T, topk, E);
+    const int C = static_cast<int>((S + CHUNK - 1) / CHUNK);
+    int32_t* chunk_tab = reinterpret_cast<int32_t*>(h);  // H is written only later
+    if (static_cast<int64_t>(C) * E * 4 > 2 * Sp * I)
+        return fail(METIS_ERR_UNSUPPORTED, "moe_nvfp4: routing table does not fit the workspace");
+
+    uint32_t* status = nullptr;
+    if ((rc = device_status_word(&status))) return rc;
+    count_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
+                                      status);
+    scan_kernel<<<1, SCAN_THREADS, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets, 128, r2s);
+    rank_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
+                                     s2r, r2s);
+    if ((rc = cuda_check(cudaGetLastError(), "moe_nvfp4 routing launch"))) return rc;
+    // x: NVFP4 per token, each token once, into the rows it was routed to
+    if ((rc = launch_nvfp4_quant(static_cast<const __nv_bfloat16*>(x_bf16), T, H, H, 1, aq, sfa, 1, ga,
+                                 s2r, static_cast<int>(topk), nullptr, nullptr, st)))
+        return rc;
+    if ((rc = launch_nvfp4_gemm(aq, sfa, ga, Sp, w_up, sf_up, g_up, E * I, h, offsets, counts,
+                                static_cast<int>(E), 0, static_cast<int>(I), static_cast<int>(H), st)))
+        return rc;
+    // h: NVFP4 per real row (pad rows and rows past offsets[E] skipped)
+    if ((rc = launch_nvfp4_quant(h, Sp, I, I, 1, hq, sfh, 1, gh, nullptr, 1, r2s, offsets + E, st)))
+        return rc;
+    if ((rc = launch_nvfp4_gemm(hq, sfh, gh, Sp, w_down, sf_down, g_down, E * H, o, offsets, counts,
+                                static_cast<int>(E), 0, static_cast<int>(H), static_cast<int>(I), st)))
+        return rc;
+    const int64_t work = T * (H / 8);
+    combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
+        o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
+        static_cast<__nv_bfloat16*>(y_bf16));
+    return cuda_check(cudaGetLastError(), "moe_nvfp4 combine launch");
 }

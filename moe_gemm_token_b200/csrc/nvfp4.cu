@@ -1,0 +1,841 @@
+// NVFP4 routed-expert maths on sm_100a ("Lernex/Metis-1.6-Praxis-NVFP4",
+// "What is in NVFP4": E2M1 values with one E4M3 scale per 16 inputs and one
+// FP32 scale per expert; "What --fast-math does": on Blackwell the 4-bit
+// experts multiply in FP4, their inputs rounded to FP4 too).
+//
+//   nvfp4_quant_kernel   one warp per row: the row's (or its set's) amax gives
+//                        the global scale g = amax/2688; each lane takes one
+//                        16-element block per pass (a warp covers 512
+//                        contiguous elements), rounds the block scale to E4M3
+//                        and the elements to E2M1 (cvt.rn.satfinite), writes
+//                        8 bytes of packed codes, and every fourth lane writes
+//                        the 4 scales of its 64-element chunk as one word, in
+//                        row-major or in the tensor cores' tiled layout.
+//   nvfp4_gemm_kernel    persistent, warp-specialised block-scaled GEMM,
+//                        128 x 256 tiles, 576 threads per CTA:
+//                          warp 0      TMA of the A and B code tiles (128-byte
+//                                      swizzle) and bulk copies of the tiled
+//                                      scale atoms into a 3-stage ring;
+//                          warp 1      TMEM owner; one lane copies each
+//                                      stage's scale atoms into TMEM
+//                                      (tcgen05.cp 32x128b.warpx4) and issues
+//                                      tcgen05.mma kind::mxf4nvf4 block16;
+//                          warps 2-17  epilogue: four warps per TMEM lane
+//                                      quadrant, 64 columns each, read the
+//                                      whole accumulator at once, release it,
+//                                      then scale (g_a[row] * g_b), round to
+//                                      BF16 and store through a swizzled
+//                                      staging block.
+//                        TMEM: one 256-column FP32 accumulator (the scale
+//                        factors need columns too, so two accumulators do not
+//                        fit in 512) and two 48-column scale buffers.
+#include "common.cuh"
+#include "../../include/metis_nvfp4.h"
+
+namespace metis {
+namespace nvfp4 {
+
+// ----------------------------------------------------------------- helpers
+
+// Eight binary32 values -> eight E2M1 codes, round-to-nearest-even and
+// saturating to +-6 (cvt.rn.satfinite.e2m1x2 puts its first source in the
+// high nibble); v[0] lands in bits 0..3 of the result.
+__device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float* v) {
+    uint32_t r;
+    asm("{\n\t"
+        ".reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+        "}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
+// Exact value of an E4M3 byte (through FP16, which holds every E4M3 value).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    float f;
+    asm("{\n\t"
+        ".reg .b16 q, lo, hi;\n\t"
+        ".reg .b32 h;\n\t"
+        "cvt.u16.u32 q, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h, q;\n\t"
+        "mov.b32 {lo, hi}, h;\n\t"
+        "cvt.f32.f16 %0, lo;\n\t"
+        "}"
+        : "=f"(f)
+        : "r"(code & 0xFFu));
+    return f;
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16 consecutive elements of a row, widened to binary32 exactly.
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[16]) {
+    const uint4 a = ld_nc_v4(p), b = ld_nc_v4(p + 8);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16_lo(w[i]);
+        v[2 * i + 1] = bf16_hi(w[i]);
+    }
+}
+__device__ __forceinline__ void load16(const float* p, float (&v)[16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 a = ld_nc_v4(p + 4 * i);
+        v[4 * i] = __uint_as_float(a.x);
+        v[4 * i + 1] = __uint_as_float(a.y);
+        v[4 * i + 2] = __uint_as_float(a.z);
+        v[4 * i + 3] = __uint_as_float(a.w);
+    }
+}
+
+// Byte offset of the 4 scales of (row r, 64-element chunk c) in the tiled
+// layout [ceil(R/128)][K/64][512]: atom (r/128, c), byte 16 (r%32) + 4 ((r%128)/32).
+__host__ __device__ __forceinline__ int64_t tiled_sf_offset(int64_t r, int64_t c, int64_t kc) {
+    return ((r >> 7) * kc + c) * 512 + 16 * (r & 31) + 4 * ((r & 127) >> 5);
+}
+
+// ----------------------------------------------------------- quantization
+
+constexpr int QWARPS = 8;
+
+struct QuantArgs {
+    const void* x;
+    int64_t R, K, ldx;        // rows, elements per row, elements between rows
+    uint8_t* q;               // packed codes, K/2 bytes per row
+    uint8_t* sf;              // block scales
+    int tiled;                // sf layout: 0 row-major [R, K/16], 1 tiled
+    float* g;                 // global scales (written when gamax is null)
+    const float* gamax;       // sets of rows: amax of the row's set, else null
+    int64_t rps;              // rows per set (gamax only)
+    const int32_t* dst_rows;  // gather: row r goes to rows dst_rows[r * topk + j]
+    int topk;
+    const int32_t* row_valid; // rows with row_valid[r] < 0 are skipped
+    const int32_t* nrows;     // device row count (rows >= *nrows are skipped)
+    int64_t pad_rows;         // tiled, no gather: rows [R, pad_rows) get zero scales
+};
+
+template <typename T>
+__global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArgs a) {
+    grid_dependency_wait();  // the rows may be the previous kernel's output
+    grid_launch_dependents();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * QWARPS + warp;
+    const int64_t kc = a.K / 64;
+    if (r >= a.R) {
+        // zero scales for the pad rows of the last 128-row atom
+        if (a.tiled && r < a.pad_rows) {
+            for (int64_t c = lane; c < kc; c += 32)
+                *reinterpret_cast<uint32_t*>(a.sf + tiled_sf_offset(r, c, kc)) = 0u;
+        }
+        return;
+    }
+    if (a.nrows && r >= *a.nrows) return;
+    if (a.row_valid && a.row_valid[r] < 0) return;
+    const T* row = static_cast<const T*>(a.x) + r * a.ldx;
+    const int nb = static_cast<int>(a.K / 16);
+    float amax;
+    if (a.gamax) {
+        amax = a.gamax[r / a.rps];
+    } else {
+        float m = 0.0f;
+        for (int b = lane; b < nb; b += 32) {
+            float v[16];
+            load16(row + 16 * b, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        amax = m;
+    }
+    const float inv_g = amax > 0.0f ? fminf(__fdiv_rn(2688.0f, amax), 3.402823466e38f) : 0.0f;
+    const int ndst = a.dst_rows ? a.topk : 1;
+    for (int b0 = 0; b0 < nb; b0 += 32) {
+        const int b = b0 + lane;
+        uint32_t lo = 0, hi = 0, sbc = 0;
+        if (b < nb) {
+            float v[16];
+            load16(row + 16 * b, v);
+            float bm = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) bm = fmaxf(bm, fabsf(v[i]));
+            sbc = f32x2_to_e4m3x2(__fdiv_rn(__fmul_rn(bm, inv_g), 6.0f), 0.0f) & 0xFFu;
+            const float ds = e4m3_to_f32(sbc);
+            const float inv_s = ds > 0.0f ? __fdiv_rn(1.0f, ds) : 0.0f;
+            float w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = __fmul_rn(__fmul_rn(v[i], inv_g), inv_s);
+            lo = f32x8_to_e2m1x8(w);
+            hi = f32x8_to_e2m1x8(w + 8);
+        }
+        // the scales of the 4 blocks of a 64-element chunk (lanes 4c .. 4c+3)
+        uint32_t s4 = sbc;
+        s4 |= __shfl_down_sync(0xffffffffu, sbc, 1) << 8;
+        s4 |= __shfl_down_sync(0xffffffffu, sbc, 2) << 16;
+        s4 |= __shfl_down_sync(0xffffffffu, sbc, 3) << 24;
+        for (int j = 0; j < ndst; ++j) {
+            const int64_t dr = a.dst_rows ? a.dst_rows[r * a.topk + j] : r;
+            if (dr < 0 || b >= nb) continue;
+            *reinterpret_cast<uint2*>(a.q + dr * (a.K / 2) + 8 * b) = make_uint2(lo, hi);
+            if ((lane & 3) == 0) {
+                const int64_t off = a.tiled ? tiled_sf_offset(dr, b / 4, kc) : dr * (a.K / 16) + b;
+                *reinterpret_cast<uint32_t*>(a.sf + off) = s4;
+            }
+            if (b0 == 0 && lane == 0 && !a.gamax) a.g[dr] = __fdiv_rn(amax, 2688.0f);
+        }
+    }
+}
+
+// amax of each set of rows, as the largest binary32 bit pattern (|x| >= 0 so
+// the integer order is the float order); gamax zeroed beforehand.
+template <typename T>
+__global__ void __launch_bounds__(QWARPS * 32) nvfp4_set_amax_kernel(const T* __restrict__ x, int64_t R,
+                                                                     int64_t K, int64_t ldx,
+                                                                     int64_t rps,
+                                                                     unsigned int* gamax) {
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * QWARPS + warp;
+    if (r >= R) return;
+    const T* row = x + r * ldx;
+    float m = 0.0f;
+    for (int64_t b = lane; b < K / 16; b += 32) {
+        float v[16];
+        load16(row + 16 * b, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) atomicMax(gamax + r / rps, __float_as_uint(m));
+}
+
+// g[i] = amax[i] / 2688, in place.
+__global__ void nvfp4_finish_scales_kernel(float* g, int64_t n) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < n) g[i] = __fdiv_rn(g[i], 2688.0f);
+}
+
+// Row-major [R, K/16] -> tiled, one thread per (row, 64-element chunk).
+__global__ void nvfp4_tile_scales_kernel(const uint8_t* __restrict__ sf, int64_t R, int64_t Rp,
+                                         int64_t K, uint8_t* __restrict__ out) {
+    const int64_t kc = K / 64;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= Rp * kc) return;
+    const int64_t r = i / kc, c = i - r * kc;
+    const uint32_t v = r < R ? *reinterpret_cast<const uint32_t*>(sf + r * (K / 16) + 4 * c) : 0u;
+    *reinterpret_cast<uint32_t*>(out + tiled_sf_offset(r, c, kc)) = v;
+}
+
+}  // namespace nvfp4
+
+// Launches the per-row quantizer (the arguments validated by the caller).
+template <typename T>
+int launch_nvfp4_quant(const T* x, int64_t R, int64_t K, int64_t ldx, int64_t rps, uint8_t* q,
+                       uint8_t* sf, int tiled, float* g, const int32_t* dst_rows, int topk,
+                       const int32_t* row_valid, const int32_t* nrows, cudaStream_t st) {
+    using namespace nvfp4;
+    nvfp4::QuantArgs a{};
+    a.x = x;
+    a.R = R;
+    a.K = K;
+    a.ldx = ldx;
+    a.q = q;
+    a.sf = sf;
+    a.tiled = tiled;
+    a.g = g;
+    a.rps = rps;
+    a.dst_rows = dst_rows;
+    a.topk = topk;
+    a.row_valid = row_valid;
+    a.nrows = nrows;
+    a.pad_rows = (tiled && !dst_rows) ? (R + 127) / 128 * 128 : R;
+    int rc;
+    if (rps > 1) {
+        // the set amax goes through g, which the last kernel turns into g = amax/2688
+        const int64_t sets = R / rps;
+        if ((rc = cuda_check(cudaMemsetAsync(g, 0, sets * sizeof(float), st), "nvfp4 amax reset"))) return rc;
+        nvfp4_set_amax_kernel<T><<<static_cast<unsigned>((R + QWARPS - 1) / QWARPS), QWARPS * 32, 0, st>>>(
+            x, R, K, ldx, rps, reinterpret_cast<unsigned int*>(g));
+        if ((rc = cuda_check(cudaGetLastError(), "nvfp4 amax launch"))) return rc;
+        a.gamax = g;
+    }
+    const int64_t rows = a.pad_rows;
+    if ((rc = cuda_check(launch_pdl(nvfp4_quant_kernel<T>, dim3(static_cast<unsigned>((rows + QWARPS - 1) / QWARPS)),
+                                    dim3(QWARPS * 32), 0, st, 1, a),
+                         "nvfp4 quant launch")))
+        return rc;
+    if (rps > 1) {
+        const int64_t sets = R / rps;
+        nvfp4_finish_scales_kernel<<<static_cast<unsigned>((sets + 255) / 256), 256, 0, st>>>(g, sets);
+        if ((rc = cuda_check(cudaGetLastError(), "nvfp4 scale launch"))) return rc;
+    }
+    return METIS_OK;
+}
+
+template int launch_nvfp4_quant<__nv_bfloat16>(const __nv_bfloat16*, int64_t, int64_t, int64_t, int64_t,
+                                               uint8_t*, uint8_t*, int, float*, const int32_t*, int,
+                                               const int32_t*, const int32_t*, cudaStream_t);
+template int launch_nvfp4_quant<float>(const float*, int64_t, int64_t, int64_t, int64_t, uint8_t*,
+                                       uint8_t*, int, float*, const int32_t*, int, const int32_t*,
+                                       const int32_t*, cudaStream_t);
+
+}  // namespace metis
+
+// ------------------------------------------------------------------- GEMM
+namespace metis {
+namespace nvfp4 {
+
+constexpr int BKB = 128;        // code bytes per row per k-block (256 elements)
+constexpr int KCH = 4;          // 64-element MMA chunks per k-block
+constexpr int ROWS = 128;       // rows of A per tile (TMEM lanes)
+constexpr int BN = 256;         // output columns per tile
+constexpr int STAGES = 3;
+constexpr int EPI_WARPS = 16;   // four per TMEM lane quadrant
+constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int ATOM = 512;       // one tiled scale atom: 128 rows x 4 scales
+constexpr int A_STAGE = ROWS * BKB;
+constexpr int B_STAGE = BN * BKB;
+constexpr int SFA_STAGE = KCH * ATOM;
+constexpr int SFB_STAGE = 2 * KCH * ATOM;   // two 128-row halves of B
+constexpr int A_OFF = 0;
+constexpr int B_OFF = A_OFF + STAGES * A_STAGE;
+constexpr int SFA_OFF = B_OFF + STAGES * B_STAGE;
+constexpr int SFB_OFF = SFA_OFF + STAGES * SFA_STAGE;
+constexpr int TILES = SFB_OFF + STAGES * SFB_STAGE;
+constexpr int STAGING = EPI_WARPS * 32 * 64;    // a 32 x 32 BF16 block per epilogue warp
+constexpr int NUM_BARS = 2 * STAGES + 3;        // full, empty, tfull, tempty, drain
+constexpr int BAR_OFF = TILES + STAGING;
+constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+constexpr int GROUP_OFF = MISC_OFF + 16;
+constexpr int MAX_GROUPS = 1024;
+constexpr size_t BYTES_DENSE = 1024 + GROUP_OFF;
+constexpr size_t BYTES_GROUPED = BYTES_DENSE + 3 * (MAX_GROUPS + 1) * 4;
+constexpr int TMEM_COLS = 512;
+constexpr int SF_COL = BN;      // two scale buffers of 48 columns after the accumulator
+constexpr int SF_BUF = 48;      // SFA: 4 chunks x 4 columns; SFB: 4 chunks x 8 columns
+
+// Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format
+// 1), K-major, UE4M3 scales (bit 23 clear), dense K = 64, N >> 3 at bit 17,
+// M >> 4 at bit 24; the scale-factor ids (bits 4-5, 29-30) stay 0.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// Shared-memory descriptor of one scale atom as the tcgen05.cp source: 32
+// rows of 16 bytes, no swizzle, 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t saddr) {
+    uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1) << 16;          // leading byte offset (one core matrix along K)
+    d |= static_cast<uint64_t>(128 >> 4) << 32;   // stride byte offset
+    d |= static_cast<uint64_t>(1) << 46;          // descriptor version (sm_100)
+    return d;
+}
+
+// Copies one 512-byte atom into TMEM columns [taddr, taddr + 4) of every lane
+// quadrant: lane l of each quadrant gets bytes 16 l .. 16 l + 15.
+__device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Non-tensor bulk copy global -> shared, completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+struct GemmParams {
+    const uint8_t* sfa;       // tiled scales of A
+    const float* ga;          // [rows of A]
+    const uint8_t* sfb;       // tiled scales of B ([groups * N] rows)
+    const float* gb;          // [groups]
+    __nv_bfloat16* y;         // [rows of A, N]
+    const int32_t* offsets;   // grouped: [E + 1] first rows (multiples of 128); dense: null
+    const int32_t* counts;    // grouped: [E] rows per group
+    int M, N, K, E;
+    uint32_t* status;
+    uint64_t timeout_ns;
+};
+
+struct Tile {
+    int a_row0, row_end, b_row0, n0, group;
+};
+
+struct Sched {
+    int num_n, num_m, total, N, M;
+    const int* g_tile;   // grouped: prefix sums of tiles per group (smem)
+    const int* g_row;    // grouped: first rows (smem)
+    const int* g_cnt;    // grouped: rows per group (smem)
+    int E;
+    __device__ __forceinline__ Tile get(int t) const {
+        Tile ti;
+        if (g_tile == nullptr) {
+            const int mb = t % num_m, nb = t / num_m;
+            ti.a_row0 = mb * ROWS;
+            ti.row_end = M;
+            ti.b_row0 = nb * BN;
+            ti.n0 = nb * BN;
+            ti.group = 0;
+        } else {
+            int lo = 0, hi = E;
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (g_tile[mid] <= t) lo = mid; else hi = mid;
+            }
+            const int e = lo;
+            const int local = t - g_tile[e];
+            const int mt = (g_cnt[e] + ROWS - 1) / ROWS;
+            const int mb = local % mt, nb = local / mt;
+            ti.a_row0 = g_row[e] + mb * ROWS;
+            ti.row_end = g_row[e] + g_cnt[e];
+            ti.b_row0 = e * N + nb * BN;
+            ti.n0 = nb * BN;
+            ti.group = e;
+        }
+        return ti;
+    }
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// One 32-column chunk: y = bf16(acc * g_a[row] * g_b), staged in the warp's
+// swizzled 32 x 64-byte block, written as 8 rows x 64 bytes per instruction.
+__device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, const Tile& ti, int q,
+                                            int lane, float ga, float gb, uint8_t* stg,
+                                            __nv_bfloat16* y, int N) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        pk[j] = pack_bf16x2(__fmul_rn(__fmul_rn(__uint_as_float(v[2 * j]), ga), gb),
+                            __fmul_rn(__fmul_rn(__uint_as_float(v[2 * j + 1]), ga), gb));
+    __syncwarp();
+#pragma unroll
+    for (int pc = 0; pc < 4; ++pc)
+        *reinterpret_cast<uint4*>(stg + lane * 64 + ((pc ^ ((lane >> 1) & 3)) * 16)) =
+            make_uint4(pk[4 * pc], pk[4 * pc + 1], pk[4 * pc + 2], pk[4 * pc + 3]);
+    __syncwarp();
+    const int n = ti.n0 + c * 32 + (lane & 3) * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int rr = (lane >> 2) + 8 * i;
+        const uint4 val =
+            *reinterpret_cast<const uint4*>(stg + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
+        const int row = ti.a_row0 + q * 32 + rr;
+        if (row < ti.row_end && n < N)
+            *reinterpret_cast<uint4*>(y + static_cast<size_t>(row) * N + n) = val;
+    }
+}
+
+template <bool GROUPED>
+__global__ void __launch_bounds__(THREADS, 1)
+nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* staging = smem + TILES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);
+    int* g_tile = reinterpret_cast<int*>(smem + GROUP_OFF);
+    int* g_row = g_tile + (MAX_GROUPS + 1);
+    int* g_cnt = g_row + (MAX_GROUPS + 1);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    auto full = [&](int s) { return smem_u32(&bars[s]); };
+    auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+    const uint32_t tfull = smem_u32(&bars[2 * STAGES]);
+    const uint32_t tempty = smem_u32(&bars[2 * STAGES + 1]);
+    const uint32_t drain = smem_u32(&bars[2 * STAGES + 2]);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, EPI_WARPS);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+
+    // operands, scales and offsets may come from the previous kernel (PDL)
+    grid_launch_dependents();
+    grid_dependency_wait();
+
+    Sched sc;
+    sc.N = p.N;
+    sc.M = p.M;
+    sc.E = p.E;
+    sc.num_n = (p.N + BN - 1) / BN;
+    if constexpr (GROUPED) {
+        if (warp == 0) {
+            const int per = (p.E + 31) / 32;
+            const int g0 = lane * per;
+            int local = 0;
+            for (int i = 0; i < per; ++i) {
+                const int e = g0 + i;
+                if (e < p.E) local += ((p.counts[e] + ROWS - 1) / ROWS) * sc.num_n;
+            }
+            int incl = local;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int run = incl - local;
+            for (int i = 0; i < per; ++i) {
+                const int e = g0 + i;
+                if (e < p.E) {
+                    g_tile[e] = run;
+                    g_row[e] = p.offsets[e];
+                    g_cnt[e] = p.counts[e];
+                    run += ((p.counts[e] + ROWS - 1) / ROWS) * sc.num_n;
+                }
+            }
+            if (lane == 31) g_tile[p.E] = incl;
+        }
+        sc.g_tile = g_tile;
+        sc.g_row = g_row;
+        sc.g_cnt = g_cnt;
+        sc.num_m = 0;
+    } else {
+        sc.g_tile = nullptr;
+        sc.g_row = nullptr;
+        sc.g_cnt = nullptr;
+        sc.num_m = (p.M + ROWS - 1) / ROWS;
+        sc.total = sc.num_m * sc.num_n;
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if constexpr (GROUPED) sc.total = g_tile[p.E];
+    const uint32_t tmem_base = *tmem_slot;
+    const int kch_total = p.K / 64;             // 64-element chunks per row
+    const int num_kb = (kch_total + KCH - 1) / KCH;
+    constexpr uint32_t IDESC = idesc_nvf4(ROWS, BN);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- producer
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_phase = 0;
+            for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+                const Tile ti = sc.get(t);
+                const int64_t rb_a = ti.a_row0 / ROWS;
+                const int64_t rb_b0 = ti.b_row0 / ROWS;
+                // the second 128-row half of B exists only when n0 + 128 < N;
+                // otherwise its scale atoms repeat the first half's (the
+                // columns it feeds are never stored)
+                const int64_t rb_b1 = ti.n0 + ROWS < p.N ? rb_b0 + 1 : rb_b0;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(empty(stage), phase ^ 1u, p.timeout_ns, p.status)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    const int nk = min(KCH, kch_total - kb * KCH);
+                    const uint32_t sfb = static_cast<uint32_t>(nk * ATOM);
+                    mbar_arrive_expect_tx(full(stage), A_STAGE + B_STAGE + 3 * sfb);
+                    tma_load_2d(smem_u32(smem + A_OFF + stage * A_STAGE), &tmA, kb * BKB, ti.a_row0, full(stage));
+                    tma_load_2d(smem_u32(smem + B_OFF + stage * B_STAGE), &tmB, kb * BKB, ti.b_row0, full(stage));
+                    const int64_t c0 = static_cast<int64_t>(kb) * KCH;
+                    bulk_load(smem_u32(smem + SFA_OFF + stage * SFA_STAGE),
+                              p.sfa + (rb_a * kch_total + c0) * ATOM, sfb, full(stage));
+                    bulk_load(smem_u32(smem + SFB_OFF + stage * SFB_STAGE),
+                              p.sfb + (rb_b0 * kch_total + c0) * ATOM, sfb, full(stage));
+                    bulk_load(smem_u32(smem + SFB_OFF + stage * SFB_STAGE + KCH * ATOM),
+                              p.sfb + (rb_b1 * kch_total + c0) * ATOM, sfb, full(stage));
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (*abort_flag) {
+                // let the copies in flight land before the CTA exits
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s))
+                        mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // --------------------------------------------------------- MMA issuer
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t acc_phase = 0;
+            uint32_t kglob = 0;
+            for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+                if (!mbar_wait(tempty, acc_phase ^ 1u, p.timeout_ns, p.status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(full(stage), phase, p.timeout_ns, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nk = min(KCH, kch_total - kb * KCH);
+                    const uint32_t sfa_t = tmem_base + SF_COL + SF_BUF * (kglob & 1u);
+                    const uint32_t sfb_t = sfa_t + 16;
+                    const uint32_t sa = smem_u32(smem + SFA_OFF + stage * SFA_STAGE);
+                    const uint32_t sb = smem_u32(smem + SFB_OFF + stage * SFB_STAGE);
+#pragma unroll
+                    for (int c = 0; c < KCH; ++c) {
+                        if (c < nk) {
+                            sf_copy(sfa_t + 4 * c, sf_atom_desc(sa + c * ATOM));
+                            sf_copy(sfb_t + 8 * c, sf_atom_desc(sb + c * ATOM));
+                            sf_copy(sfb_t + 8 * c + 4, sf_atom_desc(sb + (KCH + c) * ATOM));
+                        }
+                    }
+                    const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + A_OFF + stage * A_STAGE));
+                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + B_OFF + stage * B_STAGE));
+#pragma unroll
+                    for (int c = 0; c < KCH; ++c) {
+                        if (c < nk)
+                            mma_nvf4(tmem_base, adesc + 2 * c, bdesc + 2 * c, IDESC, sfa_t + 4 * c,
+                                     sfb_t + 8 * c, (kb > 0 || c > 0) ? 1u : 0u);
+                    }
+                    mma_commit(empty(stage));
+                    ++kglob;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) {
+                    *abort_flag = 1;
+                    break;
+                }
+                mma_commit(tfull);
+                acc_phase ^= 1u;
+            }
+            mma_commit(drain);
+            mbar_wait(drain, 0, p.timeout_ns, p.status);
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue
+        const int q = warp & 3;              // TMEM lane quadrant this warp may access
+        const int part = (warp - 2) >> 2;    // columns 64 part .. 64 part + 63
+        uint8_t* stg = staging + (warp - 2) * (32 * 64);
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+            const Tile ti = sc.get(t);
+            const int row = ti.a_row0 + q * 32 + lane;
+            const float ga = row < ti.row_end ? p.ga[row] : 0.0f;
+            const float gb = p.gb[ti.group];
+            if (!mbar_wait(tfull, acc_phase, p.timeout_ns, p.status)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(part * 64);
+            uint32_t va[32], vb[32];
+            tmem_ld_32x32b_x32(tbase, va);
+            tmem_ld_32x32b_x32(tbase + 32, vb);
+            tmem_ld_wait();
+            // the whole accumulator has been read by this warp: release it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty);
+            store_chunk(va, 2 * part, ti, q, lane, ga, gb, stg, p.y, p.N);
+            store_chunk(vb, 2 * part + 1, ti, q, lane, ga, gb, stg, p.y, p.N);
+            acc_phase ^= 1u;
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+template <bool GROUPED>
+int prepare_gemm(const DeviceInfo& di, size_t smem) {
+    static bool done[64];
+    if (static_cast<size_t>(di.max_smem_optin) < smem)
+        return fail(METIS_ERR_UNSUPPORTED, "nvfp4 gemm needs %zu bytes of shared memory", smem);
+    if (!done[di.device]) {
+        int rc = cuda_check(cudaFuncSetAttribute(nvfp4_gemm_kernel<GROUPED>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem)),
+                            "cudaFuncSetAttribute(nvfp4 gemm)");
+        if (rc) return rc;
+        done[di.device] = true;
+    }
+    return METIS_OK;
+}
+
+}  // namespace nvfp4
+
+// y = NVFP4 GEMM. a_rows: rows of A's code buffer (a multiple of 128);
+// b_rows: rows of B ([groups * N]). offsets/counts null: dense with M rows.
+// Arguments validated by the caller.
+int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, int64_t a_rows,
+                      const uint8_t* qb, const uint8_t* sfb, const float* gb, int64_t b_rows,
+                      __nv_bfloat16* y, const int32_t* offsets, const int32_t* counts, int E, int M,
+                      int N, int K, cudaStream_t st) {
+    using namespace nvfp4;
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    CUtensorMap ta, tb;
+    if ((rc = make_tmap_2d(&ta, qa, 1, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(a_rows),
+                           static_cast<uint64_t>(K / 2), BKB, ROWS, true)))
+        return rc;
+    if ((rc = make_tmap_2d(&tb, qb, 1, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(b_rows),
+                           static_cast<uint64_t>(K / 2), BKB, BN, true)))
+        return rc;
+    GemmParams p{};
+    p.sfa = sfa;
+    p.ga = ga;
+    p.sfb = sfb;
+    p.gb = gb;
+    p.y = y;
+    p.offsets = offsets;
+    p.counts = counts;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.E = offsets ? E : 1;
+    if ((rc = device_status_word(&p.status))) return rc;
+    p.timeout_ns = watchdog_ns();
+    const bool grouped = offsets != nullptr;
+    const size_t smem = grouped ? BYTES_GROUPED : BYTES_DENSE;
+    int grid = di.num_sms;
+    if (!grouped) {
+        const int64_t tiles = ((static_cast<int64_t>(M) + ROWS - 1) / ROWS) * ((N + BN - 1) / BN);
+        if (tiles == 0) return METIS_OK;
+        grid = static_cast<int>(tiles < di.num_sms ? tiles : di.num_sms);
+    }
+    if (grouped) {
+        if ((rc = prepare_gemm<true>(di, smem))) return rc;
+        return cuda_check(launch_pdl(nvfp4_gemm_kernel<true>, dim3(grid), dim3(THREADS), smem, st, 1, ta, tb, p),
+                          "nvfp4 grouped gemm launch");
+    }
+    if ((rc = prepare_gemm<false>(di, smem))) return rc;
+    return cuda_check(launch_pdl(nvfp4_gemm_kernel<false>, dim3(grid), dim3(THREADS), smem, st, 1, ta, tb, p),
+                      "nvfp4 gemm launch");
+}
+
+}  // namespace metis
+
+// ----------------------------------------------------------------- C ABI
+using namespace metis;
+
+extern "C" int metis_quant_nvfp4(const void* x, int x_kind, int64_t R, int64_t K, int64_t ldx,
+                                 int64_t rows_per_scale, uint8_t* q, uint8_t* sf, int sf_layout,
+                                 float* g, metis_stream_t stream) {
+    clear_error();
+    if (x_kind != METIS_A_BF16 && x_kind != METIS_A_F32)
+        return fail(METIS_ERR_INVALID_ARG, "quant_nvfp4: x_kind %d (need METIS_A_BF16 or METIS_A_F32)", x_kind);
+    if (sf_layout != METIS_SF_ROWMAJOR && sf_layout != METIS_SF_TILED)
+        return fail(METIS_ERR_INVALID_ARG, "quant_nvfp4: sf_layout %d", sf_layout);
+    if (R < 0 || R > 0x7fffffffll || K < 64 || K % 64 || K > 65536 || ldx < K)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "quant_nvfp4: need R >= 0, 64 <= K <= 65536 with K %% 64 == 0, ldx >= K "
+                    "(R=%lld K=%lld ldx=%lld)", (long long)R, (long long)K, (long long)ldx);
+    if (rows_per_scale < 1 || (R > 0 && R % rows_per_scale))
+        return fail(METIS_ERR_INVALID_ARG, "quant_nvfp4: rows_per_scale %lld must divide R=%lld",
+                    (long long)rows_per_scale, (long long)R);
+    if (R == 0) return METIS_OK;
+    if (!x || !q || !sf || !g) return fail(METIS_ERR_INVALID_ARG, "quant_nvfp4: null pointer");
+    const int64_t esz = x_kind == METIS_A_BF16 ? 2 : 4;
+    if (!aligned(x, 16) || (ldx * esz) % 16 || !aligned(q, 16) || !aligned(sf, 4) || !aligned(g, 4))
+        return fail(METIS_ERR_INVALID_ARG,
+                    "quant_nvfp4: x and q 16-byte aligned, ldx * element size a multiple of 16, "
+                    "sf and g 4-byte aligned");
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int tiled = sf_layout == METIS_SF_TILED;
+    if (x_kind == METIS_A_BF16)
+        return launch_nvfp4_quant(static_cast<const __nv_bfloat16*>(x), R, K, ldx, rows_per_scale, q, sf,
+                                  tiled, g, nullptr, 1, nullptr, nullptr, st);
+    return launch_nvfp4_quant(static_cast<const float*>(x), R, K, ldx, rows_per_scale, q, sf, tiled, g,
+                              nullptr, 1, nullptr, nullptr, st);
+}
+
+extern "C" int metis_nvfp4_scales_to_tiled(const uint8_t* sf, int64_t R, int64_t K,
+                                           uint8_t* sf_tiled, metis_stream_t stream) {
+    clear_error();
+    if (R < 0 || R > 0x7fffffffll || K < 64 || K % 64 || K > 65536)
+        return fail(METIS_ERR_INVALID_ARG, "nvfp4_scales_to_tiled: need R >= 0 and K a multiple of 64 "
+                    "in [64, 65536] (R=%lld K=%lld)", (long long)R, (long long)K);
+    if (R == 0) return METIS_OK;
+    if (!sf || !sf_tiled) return fail(METIS_ERR_INVALID_ARG, "nvfp4_scales_to_tiled: null pointer");
+    if (!aligned(sf, 4) || !aligned(sf_tiled, 4))
+        return fail(METIS_ERR_INVALID_ARG, "nvfp4_scales_to_tiled: pointers must be 4-byte aligned");
+    const int64_t Rp = (R + 127) / 128 * 128;
+    const uint8_t* s_end = sf + R * (K / 16);
+    const uint8_t* t_end = sf_tiled + Rp * (K / 16);
+    if (sf < t_end && sf_tiled < s_end)
+        return fail(METIS_ERR_INVALID_ARG, "nvfp4_scales_to_tiled: the buffers overlap");
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    const int64_t work = Rp * (K / 64);
+    nvfp4::nvfp4_tile_scales_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0,
+                                      static_cast<cudaStream_t>(stream)>>>(sf, R, Rp, K, sf_tiled);
+    return cuda_check(cudaGetLastError(), "nvfp4_scales_to_tiled launch");
+}
+
+extern "C" int metis_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
+                                const uint8_t* qb, const uint8_t* sfb, const float* gb, void* y,
+                                int64_t M, int64_t N, int64_t K, metis_stream_t stream) {
+    clear_error();
+    if (M < 0 || M > (1ll << 30) || N < 128 || N % 128 || N > (1 << 20) || K < 64 || K % 64 || K > 65536)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "nvfp4_gemm: need M >= 0, N a multiple of 128, K a multiple of 64 in [64, 65536] "
+                    "(M=%lld N=%lld K=%lld)", (long long)M, (long long)N, (long long)K);
+    if (M == 0) return METIS_OK;
+    if (!qa || !sfa || !ga || !qb || !sfb || !gb || !y) return fail(METIS_ERR_INVALID_ARG, "nvfp4_gemm: null pointer");
+    if (!aligned(qa, 16) || !aligned(sfa, 16) || !aligned(qb, 16) || !aligned(sfb, 16) || !aligned(y, 16) ||
+        !aligned(ga, 4) || !aligned(gb, 4))
+        return fail(METIS_ERR_INVALID_ARG, "nvfp4_gemm: codes, tiled scales and y 16-byte aligned");
+    const int64_t Mp = (M + 127) / 128 * 128;
+    return launch_nvfp4_gemm(qa, sfa, ga, Mp, qb, sfb, gb, N, static_cast<__nv_bfloat16*>(y), nullptr,
+                             nullptr, 1, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+                             static_cast<cudaStream_t>(stream));
+}

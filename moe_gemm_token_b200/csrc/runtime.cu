@@ -8,6 +8,7 @@
 #include <string>
 
 #include "common.cuh"
+#include "../../include/metis_nvfp4.h"
 
 namespace metis {
 
@@ -182,6 +183,39 @@ int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_
     return at;
 }
 
+// Rows of the NVFP4 routed-expert workspace: every expert's rows padded to a
+// multiple of 128, at most 127 pad rows per expert.
+int64_t moe4_padded_rows(int64_t T, int64_t topk, int64_t E) {
+    return (T * topk + 127 * E + 127) / 128 * 128;
+}
+
+int64_t moe4_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
+                           int64_t* total) {
+    const int64_t S = T * topk;
+    const int64_t Sp = moe4_padded_rows(T, topk, E);
+    const int64_t sizes[12] = {
+        4 * E,          // COUNTS
+        4 * (E + 1),    // OFFSETS
+        4 * S,          // SLOT_TO_ROW
+        4 * Sp,         // ROW_TO_SLOT
+        Sp * H / 2,     // AQ
+        Sp * H / 16,    // SFA (tiled)
+        4 * Sp,         // GA
+        2 * Sp * I,     // H
+        Sp * I / 2,     // HQ
+        Sp * I / 16,    // SFH (tiled)
+        4 * Sp,         // GH
+        2 * Sp * H,     // O
+    };
+    int64_t off = 0, at = -1;
+    for (int r = 0; r < 12; ++r) {
+        if (r == region) at = off;
+        off = align256(off + sizes[r]);
+    }
+    if (total) *total = off;
+    return at;
+}
+
 }  // namespace metis
 
 using namespace metis;
@@ -260,9 +294,21 @@ extern "C" size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, i
             moe_region_offset(0, M_or_T, topk, E, K_or_H, N_or_I, &total);
             return static_cast<size_t>(total);
         }
+        case METIS_OP_MOE_NVFP4: {
+            if (topk < 1 || E < 1) return 0;
+            int64_t total = 0;
+            moe4_region_offset(0, M_or_T, topk, E, K_or_H, N_or_I, &total);
+            return static_cast<size_t>(total);
+        }
         default:
             return 0;
     }
+}
+
+extern "C" int64_t metis_moe_nvfp4_workspace_offset(int region, int64_t T, int64_t topk, int64_t E,
+                                                    int64_t H, int64_t I) {
+    if (region < 0 || region > 11 || T < 0 || topk < 1 || E < 1 || H < 0 || I < 0) return -1;
+    return moe4_region_offset(region, T, topk, E, H, I, nullptr);
 }
 
 extern "C" int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk, int64_t E,

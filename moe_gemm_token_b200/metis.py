@@ -31,9 +31,16 @@ METIS_OP_FP8_GEMM_FUSED = 1
 METIS_OP_W8A16 = 2
 METIS_OP_MOE = 3
 METIS_OP_LINEAR = 4
+METIS_OP_MOE_NVFP4 = 5
+METIS_A_F32 = 2
+METIS_SF_ROWMAJOR = 0
+METIS_SF_TILED = 1
 
 MOE_WS = dict(COUNTS=0, OFFSETS=1, SLOT_TO_ROW=2, ROW_TO_SLOT=3, AQ=4, SA=5, H=6, HQ=7, SH=8,
               O=9)
+
+MOE4_WS = dict(COUNTS=0, OFFSETS=1, SLOT_TO_ROW=2, ROW_TO_SLOT=3, AQ=4, SFA=5, GA=6, H=7, HQ=8,
+               SFH=9, GH=10, O=11)
 
 _lib = None
 
@@ -73,6 +80,12 @@ def load():
         "metis_workspace_size": ([i32, i64, i64, i64, i64, i64], sz),
         "metis_moe_workspace_offset": ([i32, i64, i64, i64, i64, i64], i64),
         "metis_linear": ([p, p, p, p, i64, i64, i64, i32, p, p, sz, p], i32),
+        "metis_quant_nvfp4": ([p, i32, i64, i64, i64, i64, p, p, i32, p, p], i32),
+        "metis_nvfp4_scales_to_tiled": ([p, i64, i64, p, p], i32),
+        "metis_nvfp4_gemm": ([p, p, p, p, p, p, p, i64, i64, i64, p], i32),
+        "metis_moe_nvfp4_grouped_gemm": ([p, p, p, i64, i64, i64, i64, i64, p, p, p, p, p, p, i32,
+                                          p, p, sz, p], i32),
+        "metis_moe_nvfp4_workspace_offset": ([i32, i64, i64, i64, i64, i64], i64),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -214,4 +227,51 @@ def metis_linear(x, wq, s_w, y, fast_math=True, s_tok=None, workspace=None, stre
         _p(x), _p(wq), _p(s_w), _p(y), M, N, K, int(bool(fast_math)), _p(s_tok), _p(workspace),
         ws_bytes, _s(stream)))
 
+
+# ------------------------------------------------------------------ NVFP4
+
+def metis_quant_nvfp4(x, q, sf, g, rows_per_scale=1, tiled=False, stream=None):
+    """x [R, K] BF16 (or FP32) -> q [R, K/2] packed E2M1 codes, sf block scales
+    (row-major [R, K/16], or tiled), g [R / rows_per_scale] global scales."""
+    R, K, ldx = _rows(x)
+    kind = METIS_A_F32 if x.dtype == torch.float32 else METIS_A_BF16
+    return _check("metis_quant_nvfp4", load().metis_quant_nvfp4(
+        _p(x), kind, R, K, ldx, int(rows_per_scale), _p(q), _p(sf),
+        METIS_SF_TILED if tiled else METIS_SF_ROWMAJOR, _p(g), _s(stream)))
+
+
+def metis_nvfp4_scales_to_tiled(sf, sf_tiled, stream=None):
+    """Row-major block scales [R, K/16] -> the tiled layout."""
+    R, K16 = sf.shape
+    return _check("metis_nvfp4_scales_to_tiled", load().metis_nvfp4_scales_to_tiled(
+        _p(sf), R, K16 * 16, _p(sf_tiled), _s(stream)))
+
+
+def metis_nvfp4_gemm(qa, sfa, ga, qb, sfb, gb, y, stream=None):
+    """y [M, N] = NVFP4 GEMM; qa holds ceil(M/128)*128 rows, gb is a 1-element device tensor."""
+    M, N = y.shape
+    K = qb.shape[1] * 2
+    return _check("metis_nvfp4_gemm", load().metis_nvfp4_gemm(
+        _p(qa), _p(sfa), _p(ga), _p(qb), _p(sfb), _p(gb), _p(y), M, N, K, _s(stream)))
+
+
+def metis_moe_nvfp4_grouped_gemm(x, topk_ids, topk_w, w_up, sf_up, g_up, w_down, sf_down, g_down,
+                                 y, workspace, act=METIS_ACT_NONE, stream=None):
+    """Routed-expert layer with NVFP4 experts; see the C header for shapes."""
+    T, H = x.shape
+    topk = topk_ids.shape[1]
+    E, I, H2 = w_up.shape
+    assert H2 * 2 == H
+    ws_bytes = workspace.numel() * workspace.element_size()
+    return _check("metis_moe_nvfp4_grouped_gemm", load().metis_moe_nvfp4_grouped_gemm(
+        _p(x), _p(topk_ids), _p(topk_w), T, topk, E, H, I, _p(w_up), _p(sf_up), _p(g_up),
+        _p(w_down), _p(sf_down), _p(g_down), int(act), _p(y), _p(workspace), ws_bytes,
+        _s(stream)))
+
+
+def metis_moe_nvfp4_workspace_offset(region, T, topk, E, H, I):
+    if isinstance(region, str):
+        region = MOE4_WS[region]
+    return int(load().metis_moe_nvfp4_workspace_offset(int(region), int(T), int(topk), int(E),
+                                                       int(H), int(I)))
 

@@ -138,3 +138,47 @@ def test_workspace_layout(lib):
     assert metis.metis_moe_workspace_offset(10, T, k, E, H, I) == -1
     assert metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, 4096, 2048, 2048) >= 4 * 4096
     assert metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM, 4096, 2048, 2048) == 0
+
+
+def test_nvfp4_host_validation_without_gpu(lib):
+    p = ctypes.c_void_p(0x1000)
+    null = None
+    E = metis.METIS_ERR_INVALID_ARG
+    # quantizer: K not a multiple of 64, bad kind, rows_per_scale not dividing R
+    assert lib.metis_quant_nvfp4(p, metis.METIS_A_BF16, 4, 96, 96, 1, p, p, 0, p, null) == E
+    assert b"K" in lib.metis_last_error()
+    assert lib.metis_quant_nvfp4(p, 7, 4, 64, 64, 1, p, p, 0, p, null) == E
+    assert lib.metis_quant_nvfp4(p, metis.METIS_A_F32, 6, 64, 64, 4, p, p, 0, p, null) == E
+    assert lib.metis_quant_nvfp4(p, metis.METIS_A_BF16, 4, 64, 64, 1, p, p, 9, p, null) == E
+    assert lib.metis_quant_nvfp4(p, metis.METIS_A_BF16, 0, 64, 64, 1, p, p, 0, p, null) == metis.METIS_OK
+    # scale re-layout: K % 64, overlap
+    assert lib.metis_nvfp4_scales_to_tiled(p, 4, 80, p, null) == E
+    assert lib.metis_nvfp4_scales_to_tiled(p, 128, 64, ctypes.c_void_p(0x1100), null) == E
+    assert b"overlap" in lib.metis_last_error()
+    # GEMM: N not a multiple of 128, K not a multiple of 64, misaligned y
+    assert lib.metis_nvfp4_gemm(p, p, p, p, p, p, p, 4, 200, 256, null) == E
+    assert lib.metis_nvfp4_gemm(p, p, p, p, p, p, p, 4, 256, 96, null) == E
+    assert lib.metis_nvfp4_gemm(p, p, p, p, p, p, ctypes.c_void_p(0x1008), 4, 256, 256, null) == E
+    assert lib.metis_nvfp4_gemm(p, p, p, p, p, p, p, 0, 256, 256, null) == metis.METIS_OK
+    # routed experts: H or I not a multiple of 128, topk > E, small workspace
+    args = lambda T, k, Ex, H, I, ws: (p, p, p, T, k, Ex, H, I, p, p, p, p, p, p, 0, p, p, ws, null)
+    assert lib.metis_moe_nvfp4_grouped_gemm(*args(8, 2, 8, 192, 256, 1 << 30)) == E
+    assert lib.metis_moe_nvfp4_grouped_gemm(*args(8, 9, 8, 256, 256, 1 << 30)) == E
+    need = metis.metis_workspace_size(metis.METIS_OP_MOE_NVFP4, 8, 256, 256, 2, 8)
+    assert lib.metis_moe_nvfp4_grouped_gemm(*args(8, 2, 8, 256, 256, need - 256)) == E
+    assert b"workspace" in lib.metis_last_error()
+    assert lib.metis_moe_nvfp4_grouped_gemm(*args(0, 2, 8, 256, 256, 0)) == metis.METIS_OK
+
+
+def test_nvfp4_workspace_layout(lib):
+    T, k, E, H, I = 4096, 8, 64, 2048, 1024
+    total = metis.metis_workspace_size(metis.METIS_OP_MOE_NVFP4, T, I, H, k, E)
+    offs = [metis.metis_moe_nvfp4_workspace_offset(r, T, k, E, H, I) for r in range(12)]
+    S = T * k
+    Sp = (S + 127 * E + 127) // 128 * 128
+    sizes = [4 * E, 4 * (E + 1), 4 * S, 4 * Sp, Sp * H // 2, Sp * H // 16, 4 * Sp, 2 * Sp * I,
+             Sp * I // 2, Sp * I // 16, 4 * Sp, 2 * Sp * H]
+    assert offs[0] == 0 and all(o % 256 == 0 for o in offs)
+    for o, s, nxt in zip(offs, sizes, offs[1:] + [total]):
+        assert o + s <= nxt
+    assert metis.metis_moe_nvfp4_workspace_offset(12, T, k, E, H, I) == -1

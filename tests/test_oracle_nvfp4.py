@@ -13,7 +13,6 @@ import pytest
 import oracle
 
 
-
 def _e2m1_from_bits(c):
     # sign | 2 exponent bits (bias 1) | 1 mantissa bit; exponent 0 is subnormal
     s = -1.0 if c & 8 else 1.0
