@@ -57,7 +57,9 @@ def _load():
         lib.metis_oracle_e2m1_encode.restype = ctypes.c_uint8
         lib.metis_oracle_nvfp4_quant.argtypes = [p, i64, i64, ctypes.c_int, p, p, p]
         lib.metis_oracle_nvfp4_gemm.argtypes = [p, p, p, p, p, ctypes.c_float, i64, i64, i64, p, p]
-        for name in ("route_topk", "nvfp4_quant", "nvfp4_gemm"):
+        lib.metis_oracle_gemm_bf16.argtypes = [p, i64, p, i64, i64, i64, i64, p, p]
+        lib.metis_oracle_shared_combine.argtypes = [p, p, p, i64, i64, i64, p, p]
+        for name in ("route_topk", "nvfp4_quant", "nvfp4_gemm", "gemm_bf16", "shared_combine"):
             getattr(lib, "metis_oracle_" + name).restype = ctypes.c_int
         for name in ("e4m3_encode_array", "e4m3_decode_array", "bf16_from_double_array"):
             getattr(lib, "metis_oracle_" + name).restype = None
@@ -434,4 +436,50 @@ def moe_forward_nvfp4(x_bf16, topk_ids, topk_w, up, down, tokens=None):
     y, y64 = moe_combine(o.reshape(nt, k, -1), w[tokens])
     return dict(qx=qx, sx=sx, gx=gx, h=h, h64=h64, qh=qh, sh=sh, gh=gh, o=o, o64=o64, y=y,
                 y64=y64, tokens=tokens)
+
+
+# ------------------------------------------------------------ shared expert
+# "Lernex/Metis-1.6-Praxis" card, "Architecture": one shared expert beside
+# the routed ones in every layer; the FP8 cards ("What is in FP8") keep it in
+# BF16. Reading: it runs on every token with weight 1, with the two
+# projections of a routed expert (no activation, h rounded to BF16), and its
+# BF16 output joins the routed weighted sum before the final rounding.
+
+def gemm_bf16(x_bf16, w_bf16, rows=None):
+    """y[m, n] = bf16(sum_k x[m, k] w[n, k]) with BF16 operands, float64 sum.
+    Returns (bf16 bits, float64 before rounding)."""
+    lib = _load()
+    x = _c(x_bf16, np.uint16)
+    if rows is not None:
+        x = np.ascontiguousarray(x[np.asarray(rows)])
+    w = _c(w_bf16, np.uint16)
+    M, K = x.shape
+    N = w.shape[0]
+    y = np.empty((M, N), dtype=np.uint16)
+    y64 = np.empty((M, N), dtype=np.float64)
+    _check(lib.metis_oracle_gemm_bf16(_ptr(x), K, _ptr(w), K, M, N, K, _ptr(y), _ptr(y64)),
+           "gemm_bf16")
+    return y, y64
+
+
+def shared_combine(s_bf16, o_slots_bf16, topk_w):
+    """y[t] = bf16(s[t] + sum_j w[t, j] o[t, j]) in float64; s [T, H], o [T, k, H]."""
+    lib = _load()
+    s = _c(s_bf16, np.uint16)
+    o = _c(o_slots_bf16, np.uint16)
+    w = _c(topk_w, np.float32)
+    T, k, H = o.shape
+    y = np.empty((T, H), dtype=np.uint16)
+    y64 = np.empty((T, H), dtype=np.float64)
+    _check(lib.metis_oracle_shared_combine(_ptr(s), _ptr(o), _ptr(w), T, k, H, _ptr(y), _ptr(y64)),
+           "shared_combine")
+    return y, y64
+
+
+def shared_expert(x_bf16, w_sup_bf16, w_sdn_bf16, tokens=None):
+    """The shared expert's BF16 output: s = bf16(bf16(x W_up^T) W_down^T).
+    Returns (h bits, s bits, s float64)."""
+    h, _ = gemm_bf16(x_bf16, w_sup_bf16, rows=tokens)
+    s, s64 = gemm_bf16(h, w_sdn_bf16)
+    return h, s, s64
 

@@ -459,6 +459,53 @@ int metis_oracle_moe_combine(const uint16_t* o, const float* w, int64_t T, int64
     return ORACLE_OK;
 }
 
+/* ------------------------------------------------------- shared expert
+ * "Lernex/Metis-1.6-Praxis" card, "Architecture": every layer ends in routed
+ * experts and one shared expert; the FP8 cards ("What is in FP8") keep the
+ * shared expert as trained, in BF16. Reading: the shared expert runs on every
+ * token with weight 1 and the same two projections as a routed expert (no
+ * activation, h rounded to BF16); the layer output adds its BF16 output to
+ * the routed weighted sum before the one final rounding. */
+
+/* y[m, n] = bf16( sum_k x[m, k] w[n, k] ), BF16 operands, float64 sum. */
+int metis_oracle_gemm_bf16(const uint16_t* x, int64_t ldx, const uint16_t* w, int64_t ldw,
+                           int64_t M, int64_t N, int64_t K, uint16_t* y, double* y64) {
+    int64_t m;
+#pragma omp parallel for schedule(static)
+    for (m = 0; m < M; ++m) {
+        int64_t n, k;
+        for (n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (k = 0; k < K; ++k)
+                acc += (double)bf16_bits_to_float(x[m * ldx + k]) *
+                       (double)bf16_bits_to_float(w[n * ldw + k]);
+            if (y64) y64[m * N + n] = acc;
+            y[m * N + n] = metis_oracle_bf16_from_double(acc);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* y[t, n] = bf16( s[t, n] + sum_j w[t, j] o[t, j, n] ), s the shared
+ * expert's BF16 output [T, H], o the routed outputs in slot order [T, topk, H]. */
+int metis_oracle_shared_combine(const uint16_t* s, const uint16_t* o, const float* w, int64_t T,
+                                int64_t topk, int64_t H, uint16_t* y, double* y64) {
+    int64_t t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        int64_t n, j;
+        for (n = 0; n < H; ++n) {
+            double acc = (double)bf16_bits_to_float(s[t * H + n]);
+            for (j = 0; j < topk; ++j)
+                acc += (double)w[t * topk + j] *
+                       (double)bf16_bits_to_float(o[(t * topk + j) * H + n]);
+            if (y64) y64[t * H + n] = acc;
+            y[t * H + n] = metis_oracle_bf16_from_double(acc);
+        }
+    }
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------- array forms of the codec */
 
 void metis_oracle_e4m3_encode_array(const float* v, int64_t n, uint8_t* out) {

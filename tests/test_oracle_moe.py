@@ -195,3 +195,53 @@ def test_route_topk_invariants():
         others = np.delete(score[t], ids[t])
         assert chosen.min() >= others.max()
     assert np.allclose(w.sum(axis=1), 1.0, atol=1e-12)
+
+
+# ------------------------------------------------------------ shared expert
+
+def _bf16(a):
+    return (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_gemm_bf16_equals_float64_matmul():
+    rng = np.random.default_rng(31)
+    x = _bf16(rng.standard_normal((7, 96)))
+    w = _bf16(rng.standard_normal((5, 96)) * 0.05)
+    y, y64 = oracle.gemm_bf16(x, w)
+    # BF16 products are exact in float64 and these sums stay exact
+    want = oracle.bf16_to_float(x).astype(np.float64) @ oracle.bf16_to_float(w).astype(np.float64).T
+    assert np.array_equal(y64, want)
+    assert np.array_equal(y, oracle.bf16_from_double(want))
+    y2, _ = oracle.gemm_bf16(x, w, rows=[4, 1])
+    assert np.array_equal(y2, y[[4, 1]])
+
+
+def test_shared_combine_reduces_to_the_routed_combine_and_to_the_shared_output():
+    rng = np.random.default_rng(32)
+    T, k, H = 6, 3, 40
+    o = _bf16(rng.standard_normal((T, k, H)))
+    w = rng.uniform(0, 1, (T, k)).astype(np.float32)
+    s = _bf16(rng.standard_normal((T, H)))
+    zero = np.zeros((T, H), np.uint16)
+    # no shared output: the routed combine
+    assert np.array_equal(oracle.shared_combine(zero, o, w)[0], oracle.moe_combine(o, w)[0])
+    # no routed weight: the shared output itself, unchanged
+    assert np.array_equal(oracle.shared_combine(s, o, np.zeros_like(w))[0], s)
+    # the sum, rounded once
+    want = oracle.bf16_to_float(s).astype(np.float64) + \
+        (oracle.bf16_to_float(o).astype(np.float64) * w.astype(np.float64)[:, :, None]).sum(axis=1)
+    y, y64 = oracle.shared_combine(s, o, w)
+    assert np.allclose(y64, want, rtol=1e-15, atol=0)
+    assert np.array_equal(y, oracle.bf16_from_double(y64))
+
+
+def test_shared_expert_is_two_rounded_gemms():
+    rng = np.random.default_rng(33)
+    x = _bf16(rng.standard_normal((4, 64)))
+    wu = _bf16(rng.standard_normal((32, 64)) * 0.1)
+    wd = _bf16(rng.standard_normal((64, 32)) * 0.1)
+    h, s, s64 = oracle.shared_expert(x, wu, wd)
+    assert np.array_equal(h, oracle.gemm_bf16(x, wu)[0])
+    assert np.array_equal(s, oracle.gemm_bf16(h, wd)[0])
+    _, s_sub, _ = oracle.shared_expert(x, wu, wd, tokens=[3, 0])
+    assert np.array_equal(s_sub, s[[3, 0]])
