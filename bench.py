@@ -37,6 +37,7 @@ M_TOK, K_HID, N_FF = 4096, 2048, 6144
 SETS = 4
 EV_EVERY = 20  # GEMM timing events on every 20th step of the timed graph
 FP8_PER_BF16 = 2.0  # nominal dense FP8 : BF16 tensor throughput (4.5 : 2.25 PFLOP/s)
+FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -599,6 +600,40 @@ def secondary_figures(metis, dev, pk):
     tf = 2 * 2 * T * k * H * I / t / 1e12
     out["moe_4096tok_64e_top8"] = {"us": t * 1e6, "tok/s": T / t, "TFLOP/s": tf,
                                    "frac_of_fp8_peak": tf / peak8}
+    del wu, wd, wsp
+    # the same routed-expert layer with NVFP4 experts (E2M1 codes, E4M3 scale
+    # per 16, FP32 scale per expert; inputs rounded to NVFP4 per token)
+    peak4 = pk["bf16_tflops"] * FP4_PER_BF16
+
+    def sf_codes(n):  # E4M3 scales 2^-3 .. 2^2, no NaN code
+        return torch.randint(0x20, 0x48, (n,), dtype=torch.uint8, device=dev, generator=g)
+    wu4 = torch.randint(0, 256, (E, I, H // 2), dtype=torch.uint8, device=dev, generator=g)
+    wd4 = torch.randint(0, 256, (E, H, I // 2), dtype=torch.uint8, device=dev, generator=g)
+    sfu, sfd = sf_codes(E * I * H // 16), sf_codes(E * H * I // 16)
+    gu = torch.rand(E, device=dev, generator=g) * 1e-3 + 1e-4
+    gd = torch.rand(E, device=dev, generator=g) * 1e-3 + 1e-4
+    ws4 = torch.empty(metis.metis_workspace_size(metis.METIS_OP_MOE_NVFP4, T, I, H, k, E),
+                      dtype=torch.uint8, device=dev)
+    t = timeit(lambda: metis.metis_moe_nvfp4_grouped_gemm(x, ids, w, wu4, sfu, gu, wd4, sfd, gd,
+                                                          y, ws4), 20)
+    tf = 2 * 2 * T * k * H * I / t / 1e12
+    out["moe_nvfp4_4096tok_64e_top8"] = {"us": t * 1e6, "tok/s": T / t, "TFLOP/s": tf,
+                                         "frac_of_fp4_peak": tf / peak4}
+    del wu4, wd4, sfu, sfd, ws4
+    # dense NVFP4 GEMM (codes and tiled scales resident, 2 rotating B > L2 at the large size)
+    for (M, K) in [(8192, 4096), (16384, 8192)]:
+        qa = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        sa = sf_codes(M * K // 16)
+        ga = torch.rand(M, device=dev, generator=g) + 0.5
+        qb = torch.randint(0, 256, (K, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        sb = sf_codes(K * K // 16)
+        gb = torch.ones(1, device=dev)
+        y = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        t = timeit(lambda: metis.metis_nvfp4_gemm(qa, sa, ga, qb, sb, gb, y), 20)
+        fl = 2 * M * K * K
+        out[f"nvfp4_gemm_{M}x{K}x{K}"] = {"us": t * 1e6, "TFLOP/s": fl / t / 1e12,
+                                          "frac_of_fp4_peak": fl / t / 1e12 / peak4}
+        del qa, sa, qb, sb, y
     return out
 
 

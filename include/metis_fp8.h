@@ -179,7 +179,9 @@ METIS_API int metis_moe_route_topk(const float* logits, const float* bias, int64
  * un-permute y[t] = sum_j topk_w[t,j] o[t,j] (FP32, j ascending) -> BF16.
  *   x [T, H] BF16, topk_ids [T, topk] int32 in [0, E), topk_w [T, topk] FP32,
  *   w_up [E, I, H] E4M3, s_up [E, I], w_down [E, H, I] E4M3, s_down [E, H],
- *   y [T, H] BF16 out.
+ *   y [T, H] BF16 out, or NULL: the layer then stops after the down-projection
+ *   and leaves o and the routing in the workspace for
+ *   metis_moe_shared_fused_combine (no combine kernel runs).
  *   act must be METIS_ACT_NONE (the cards do not state the experts' activation).
  *   Requires H % 16 == 0, I % 16 == 0, 16 <= H <= 16384, I >= 16, 1 <= topk <= E <= 1024;
  *   ids outside [0, E) are a caller error (not checked on the device).
@@ -215,6 +217,37 @@ METIS_API int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int32
                                                  const uint8_t* w_down, const float* s_down,
                                                  int act, void* y_bf16, metis_stream_t stream);
 
+/* BF16 GEMM on the tensor cores (tcgen05.mma kind::f16, FP32 accumulation):
+ *   y[m, n] = bf16_rn( sum_k x[m, k] w[n, k] ).
+ * The shared expert's projections use it ("Lernex/Metis-1.6-Praxis" card,
+ * "Architecture": one shared expert in every layer; the FP8 cards keep it
+ * in BF16). x [M, K], w [N, K], y [M, N] BF16, 16-byte aligned; N and K
+ * multiples of 8. */
+METIS_API int metis_bf16_gemm(const void* x_bf16, const void* w_bf16, void* y_bf16, int64_t M,
+                              int64_t N, int64_t K, metis_stream_t stream);
+
+/* The shared expert with the routed combine fused into its down-projection.
+ * Reading of the cards (they print no formula): the shared expert runs on
+ * every token with weight 1, with the two projections of a routed expert (no
+ * activation), and the layer output adds its BF16 output s to the routed
+ * weighted sum before the one final rounding:
+ *   h_s[t] = bf16( x[t] W_sup^T )                      W_sup [I_s, H] BF16
+ *   s[t]   = bf16( h_s[t] W_sdn^T )                    W_sdn [H, I_s] BF16
+ *   y[t]   = bf16( s[t] + sum_j topk_w[t, j] o[slot_to_row[t*topk + j]] )
+ *            (FP32, j ascending; slots with slot_to_row < 0 skipped).
+ *   o_routed, slot_to_row: the routed layer's O and SLOT_TO_ROW workspace
+ *   regions after metis_moe_fp8_grouped_gemm or metis_moe_nvfp4_grouped_gemm
+ *   ran with y = NULL (o rows of H BF16 values).
+ *   Requires H and I_s multiples of 16 (H <= 16384), 1 <= topk <= 8; needs
+ *   `workspace` of metis_workspace_size(METIS_OP_SHARED, T, I_s, H, topk, 0)
+ *   bytes (16-byte aligned) for h_s. */
+METIS_API int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int64_t H, int64_t I_s,
+                                             const void* w_sup_bf16, const void* w_sdn_bf16,
+                                             const void* o_routed_bf16, const int32_t* slot_to_row,
+                                             const float* topk_w, int64_t topk, void* y_bf16,
+                                             void* workspace, size_t ws_bytes,
+                                             metis_stream_t stream);
+
 /* Workspace sizes in bytes.
  *   METIS_OP_FP8_GEMM_FUSED: (M, N, K) of metis_fp8_gemm with a_kind = METIS_A_BF16.
  *   METIS_OP_MOE:            (T, I, H, topk, E) of metis_moe_fp8_grouped_gemm.
@@ -225,6 +258,7 @@ METIS_API int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int32
 #define METIS_OP_W8A16 2
 #define METIS_OP_MOE 3
 #define METIS_OP_LINEAR 4
+#define METIS_OP_SHARED 6       /* metis_moe_shared_fused_combine: (T, I_s, H, topk, 0) */
 METIS_API size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, int64_t K_or_H,
                             int64_t topk, int64_t E);
 

@@ -113,7 +113,8 @@ METIS_API int metis_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const floa
  *           matrix; g_up [E] FP32. w_down [E, H, I/2]; sf_down tiled scales of
  *           [E*H, I]; g_down [E].
  *   act     METIS_ACT_NONE.
- *   y       [T, H] BF16.
+ *   y       [T, H] BF16, or NULL: stop after the down-projection, leaving o
+ *           and the routing for metis_moe_shared_fused_combine.
  *   workspace  metis_workspace_size(METIS_OP_MOE_NVFP4, T, I, H, topk, E)
  *           bytes, 256-byte aligned; regions by metis_moe_nvfp4_workspace_offset.
  * H and I multiples of 128, 128 <= H <= 16384, 128 <= I <= 65536;

@@ -79,6 +79,12 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
                       __nv_bfloat16* y, const int32_t* offsets, const int32_t* counts, int E, int M,
                       int N, int K, cudaStream_t st);
 
+// BF16 GEMM y = bf16(a b^T) (gemm_fp8.cu); o non-null fuses the routed
+// combine: y[t] = bf16(bf16(a b^T)[t] + sum_j topk_w[t*topk+j] o[s2r[t*topk+j]]).
+int launch_bf16_gemm(const __nv_bfloat16* a, const __nv_bfloat16* b, __nv_bfloat16* y, int M, int N,
+                     int K, const __nv_bfloat16* o, const int32_t* s2r, const float* topk_w, int topk,
+                     cudaStream_t st);
+
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Device error word bits.
@@ -409,6 +415,27 @@ __device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t adesc,
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// BF16 x BF16 -> FP32 (kind::f16) with both operands in shared memory: one
+// CTA, or the CTA pair (A and B rows split between the two CTAs as above).
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_f16_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }

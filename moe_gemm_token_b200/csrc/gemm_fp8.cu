@@ -33,6 +33,13 @@
 // staging ring, and 8 converter warps turn each into the swizzled E4M3 tile
 // the MMA reads (x * (448/amax), cvt.rn.satfinite: the standalone quantizer's
 // bytes), so the codes never go through HBM.
+// BF16 operands (W16): the same pipeline with BF16 A and B tiles (64 elements
+// = 128 bytes per k-block row, tcgen05.mma kind::f16), no scales; used by the
+// shared expert ("Lernex/Metis-1.6-Praxis" card, "Architecture": one shared
+// expert beside the routed ones; kept in BF16 by the FP8 cards). Its
+// down-projection can add the routed experts' weighted outputs in the
+// epilogue: y[t] = bf16(s[t] + sum_j w[t,j] o[row(t,j)]) with s the BF16
+// product, so the routed combine needs no kernel and s never reaches HBM.
 // Every mbarrier wait is bounded by the device watchdog: on a timeout the CTA
 // sets the sticky error word, stops issuing work, drains what it issued,
 // frees TMEM and returns.
@@ -49,11 +56,14 @@ constexpr int TMEM_COLS = 2 * BN_MAX;
 constexpr int MAX_GROUPS = 1024;
 
 constexpr int CONV_WARPS = 8;                  // fused-quantization converter warps
+constexpr int COMB_K = 8;                      // fused combine: routed slots per token
 constexpr int ASTG_SLOT = ROWS * BK * 2;       // one BF16 A tile (two 64-column boxes)
 
-template <int CTAS, bool ABF16 = false, int BN = BN_MAX>
+template <int CTAS, bool ABF16 = false, int BN = BN_MAX, bool W16 = false>
 struct Layout {
-    static constexpr int STAGES = CTAS == 2 ? (ABF16 ? 4 : 6) : (ABF16 ? 3 : 4);
+    // BF16 k-blocks take twice the MMA time of E4M3 ones: fewer stages suffice
+    static constexpr int STAGES = W16 ? (CTAS == 2 ? 4 : 3)
+                                      : (CTAS == 2 ? (ABF16 ? 4 : 6) : (ABF16 ? 3 : 4));
     static constexpr int ASTG = ABF16 ? 2 : 0;  // BF16 staging slots
     // epilogue warps: two per TMEM lane quadrant, each on half the columns
     // (one per quadrant in the fused variants, whose shared memory and
@@ -66,14 +76,17 @@ struct Layout {
     static constexpr int TILES = STAGES * (A_STAGE + B_STAGE) + ASTG * ASTG_SLOT;
     static constexpr int STAGING = EPI * 32 * 64;  // a 32 x 32 BF16 block per epilogue warp
     static constexpr int SW = 2 * BN * 4;                // per-channel scales, double-buffered
+    static constexpr int COMB = W16 ? EPI * 32 * COMB_K * 8 : 0;  // (row, weight) per routed slot
     // full, empty, tfull[2], tempty[2], drain, epilogue sync[2], staging full/empty
     static constexpr int NUM_BARS = 2 * STAGES + 7 + 2 * ASTG;
-    static constexpr int BAR_OFF = TILES + STAGING + SW;
+    static constexpr int COMB_OFF = TILES + STAGING + SW;
+    static constexpr int BAR_OFF = COMB_OFF + COMB;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int GROUP_OFF = MISC_OFF + 16;
     static constexpr size_t BYTES_DENSE = 1024 + GROUP_OFF;
     static constexpr size_t BYTES_GROUPED = BYTES_DENSE + 2 * (MAX_GROUPS + 1) * 4;
-    static constexpr uint32_t IDESC = idesc_e4m3_f32(ROWS * CTAS, BN);
+    static constexpr uint32_t IDESC = W16 ? idesc_bf16_f32(ROWS * CTAS, BN) : idesc_e4m3_f32(ROWS * CTAS, BN);
+    static constexpr int KE = W16 ? BK / 2 : BK;  // elements per k-block row
 };
 
 struct Params {
@@ -88,6 +101,11 @@ struct Params {
     int E;                   // groups (1 for dense)
     uint32_t* status;
     uint64_t timeout_ns;
+    // W16 fused combine (o null: none): y[t] += sum_j topk_w[t*topk+j] * o[s2r[t*topk+j]]
+    const __nv_bfloat16* o;  // routed outputs [rows, N]
+    const int32_t* s2r;      // [rows of A * topk]; negative: slot dropped
+    const float* topk_w;     // [rows of A * topk]
+    int topk;
 };
 
 struct Tile {
@@ -173,11 +191,66 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, cons
     }
 }
 
-template <int CTAS, bool GROUPED, bool ABF16, int BN>
-__global__ void __launch_bounds__(Layout<CTAS, ABF16, BN>::THREADS_, 1)
+// The W16 epilogue chunk: y = bf16(acc), staged as above; with the fused
+// combine each 8-column piece then gets the token's routed outputs added,
+// y = bf16(s + sum_j w_j o_j) in FP32, j ascending (all loads issued first).
+__device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, const Tile& ti, int q,
+                                                int lane, uint8_t* stg, const int2* cb,
+                                                const Params& p) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+    __syncwarp();
+#pragma unroll
+    for (int pc = 0; pc < 4; ++pc)
+        *reinterpret_cast<uint4*>(stg + lane * 64 + ((pc ^ ((lane >> 1) & 3)) * 16)) =
+            make_uint4(pk[4 * pc], pk[4 * pc + 1], pk[4 * pc + 2], pk[4 * pc + 3]);
+    __syncwarp();
+    const int n = ti.n0 + c * 32 + (lane & 3) * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int rr = (lane >> 2) + 8 * i;
+        uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
+        const int row = ti.a_row0 + q * 32 + rr;
+        if (row >= ti.row_end || n >= p.N) continue;
+        if (p.o != nullptr) {
+            const int2* e = cb + rr * COMB_K;
+            uint4 ov[COMB_K];
+#pragma unroll
+            for (int j = 0; j < COMB_K; ++j)
+                if (j < p.topk && e[j].x >= 0)
+                    ov[j] = *reinterpret_cast<const uint4*>(p.o + static_cast<size_t>(e[j].x) * p.N + n);
+            const uint32_t sv[4] = {val.x, val.y, val.z, val.w};
+            float a[8];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                a[2 * h] = bf16_lo(sv[h]);
+                a[2 * h + 1] = bf16_hi(sv[h]);
+            }
+#pragma unroll
+            for (int j = 0; j < COMB_K; ++j) {
+                if (j < p.topk && e[j].x >= 0) {
+                    const float wj = __int_as_float(e[j].y);
+                    const uint32_t ow[4] = {ov[j].x, ov[j].y, ov[j].z, ov[j].w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        a[2 * h] = fmaf(wj, bf16_lo(ow[h]), a[2 * h]);
+                        a[2 * h + 1] = fmaf(wj, bf16_hi(ow[h]), a[2 * h + 1]);
+                    }
+                }
+            }
+            val = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                             pack_bf16x2(a[6], a[7]));
+        }
+        *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.N + n) = val;
+    }
+}
+
+template <int CTAS, bool GROUPED, bool ABF16, int BN, bool W16 = false>
+__global__ void __launch_bounds__(Layout<CTAS, ABF16, BN, W16>::THREADS_, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
-    using L = Layout<CTAS, ABF16, BN>;
+    using L = Layout<CTAS, ABF16, BN, W16>;
     constexpr int STAGES = L::STAGES;
     constexpr int EPI = L::EPI;
     extern __shared__ uint8_t smem_raw[];
@@ -190,6 +263,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+    int2* comb = reinterpret_cast<int2*>(smem + L::COMB_OFF);
     int* g_tile = reinterpret_cast<int*>(smem + L::GROUP_OFF);
     int* g_row = g_tile + (MAX_GROUPS + 1);
 
@@ -300,7 +374,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     tc_fence_after();
     if constexpr (GROUPED) sc.total = g_tile[p.E];
     const uint32_t tmem_base = *tmem_slot;
-    const int num_kb = (p.K + BK - 1) / BK;
+    const int num_kb = (p.K + L::KE - 1) / L::KE;
     const int first = CTAS == 2 ? static_cast<int>(blockIdx.x / 2) : static_cast<int>(blockIdx.x);
     const int stride = CTAS == 2 ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
 
@@ -342,12 +416,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     } else if constexpr (CTAS == 2) {
                         const uint32_t fl = mapa_shared(full(stage), 0);
                         if (leader) mbar_arrive_expect_tx(full(stage), CTAS * (L::A_STAGE + L::B_STAGE));
-                        tma_load_2d_pair(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * BK, ti.a_row0, fl);
-                        tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * BK, ti.b_row0, fl);
+                        tma_load_2d_pair(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * L::KE, ti.a_row0, fl);
+                        tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * L::KE, ti.b_row0, fl);
                     } else {
                         mbar_arrive_expect_tx(full(stage), L::A_STAGE + L::B_STAGE);
-                        tma_load_2d(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * BK, ti.a_row0, full(stage));
-                        tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * BK, ti.b_row0, full(stage));
+                        tma_load_2d(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * L::KE, ti.a_row0, full(stage));
+                        tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * L::KE, ti.b_row0, full(stage));
                     }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -395,8 +469,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) {
                         // advance 32 bytes along K inside the swizzled 128-byte rows
+                        // (32 bytes: 32 E4M3 or 16 BF16 elements per instruction)
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                        if constexpr (CTAS == 2)
+                        if constexpr (W16 && CTAS == 2)
+                            mma_f16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
+                        else if constexpr (W16)
+                            mma_f16_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
+                        else if constexpr (CTAS == 2)
                             mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
                         else
                             mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
@@ -494,15 +573,28 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         uint32_t acc_phase = 0;
         for (int t = first; t < sc.total && !*abort_flag; t += stride) {
             const Tile ti = sc.get(t);
-            // per-channel scales of this tile into shared memory
-            {
+            const int2* cb = comb + (warp - 2) * 32 * COMB_K;
+            if constexpr (W16) {
+                // the fused combine's (row, weight) pairs of this warp's 32 rows
+                if (p.o != nullptr) {
+                    const int row = ti.a_row0 + q * 32 + lane;
+                    int2* mine = comb + ((warp - 2) * 32 + lane) * COMB_K;
+                    for (int j = 0; j < p.topk; ++j) {
+                        const size_t sidx = static_cast<size_t>(row) * p.topk + j;
+                        mine[j] = row < ti.row_end ? make_int2(p.s2r[sidx], __float_as_int(p.topk_w[sidx]))
+                                                   : make_int2(-1, 0);
+                    }
+                    __syncwarp();
+                }
+            } else {
+                // per-channel scales of this tile into shared memory
                 const float* sb = p.s_b + static_cast<size_t>(ti.group) * p.N;
                 const int n = ti.n0 + 2 * et;
                 const float2 v = n < p.N ? *reinterpret_cast<const float2*>(sb + n) : make_float2(0.f, 0.f);
                 if (et < BN / 2) reinterpret_cast<float2*>(sw_smem + acc * BN)[et] = v;
             }
             const int row = ti.a_row0 + q * 32 + lane;
-            const float rs = row < ti.row_end ? p.s_a[row] : 0.0f;
+            const float rs = (!W16 && row < ti.row_end) ? p.s_a[row] : 0.0f;
             // all epilogue threads have written their scales (bounded wait)
             mbar_arrive(epi_sync(acc));
             if (!mbar_wait(epi_sync(acc), acc_phase, p.timeout_ns, p.status) ||
@@ -534,7 +626,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         else mbar_arrive(tempty(acc));
                     }
                 }
-                store_chunk(cur, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N);
+                if constexpr (W16) store_chunk_w16(cur, c0 + i, ti, q, lane, stg, cb, p);
+                else store_chunk(cur, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N);
                 if (i + 1 < CPW) tmem_ld_wait();
             }
             acc ^= 1;
@@ -552,13 +645,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
 }
 
-template <int CTAS, bool GROUPED, bool ABF16 = false, int BN = BN_MAX>
+template <int CTAS, bool GROUPED, bool ABF16 = false, int BN = BN_MAX, bool W16 = false>
 int prepare(const DeviceInfo& di, size_t smem) {
     static bool done[64];
     if (static_cast<size_t>(di.max_smem_optin) < smem)
         return fail(METIS_ERR_UNSUPPORTED, "fp8 gemm needs %zu bytes of shared memory", smem);
     if (!done[di.device]) {
-        int rc = cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED, ABF16, BN>,
+        int rc = cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED, ABF16, BN, W16>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(smem)),
                             "cudaFuncSetAttribute(fp8 gemm)");
@@ -569,11 +662,11 @@ int prepare(const DeviceInfo& di, size_t smem) {
 }
 
 // Co-resident CTA pairs of the 2-CTA kernel (cached per device).
-template <bool ABF16 = false, int BN = BN_MAX, bool GROUPED = false>
+template <bool ABF16 = false, int BN = BN_MAX, bool GROUPED = false, bool W16 = false>
 int max_pairs(const DeviceInfo& di, int* out) {
     static int cached[64];
     if (!cached[di.device]) {
-        using L = Layout<2, ABF16, BN>;
+        using L = Layout<2, ABF16, BN, W16>;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (di.num_sms / 2), 1, 1);
         cfg.blockDim = dim3(L::THREADS_, 1, 1);
@@ -586,7 +679,7 @@ int max_pairs(const DeviceInfo& di, int* out) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, GROUPED, ABF16, BN>, &cfg),
+        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, GROUPED, ABF16, BN, W16>, &cfg),
                             "cudaOccupancyMaxActiveClusters");
         if (rc) return rc;
         if (n < 1) return fail(METIS_ERR_UNSUPPORTED, "no CTA pair of the fp8 gemm fits an SM pair");
@@ -722,9 +815,64 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
                       "fused fp8 gemm launch");
 }
 
+// BF16 x BF16 GEMM y = bf16(a b^T) on the tcgen05 pipeline (CTA pairs for
+// M > 128), optionally with the routed combine fused into the epilogue (o
+// non-null). Arguments validated by the caller.
+int launch_bf16_gemm(const __nv_bfloat16* a, const __nv_bfloat16* b, __nv_bfloat16* y, int M, int N,
+                     int K, const __nv_bfloat16* o, const int32_t* s2r, const float* topk_w, int topk,
+                     cudaStream_t st) {
+    using namespace gemm;
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    uint32_t* status = nullptr;
+    if ((rc = device_status_word(&status))) return rc;
+    Params p{nullptr, nullptr, nullptr, y, nullptr, M, N, K, 1, status, watchdog_ns(), o, s2r, topk_w, topk};
+    const int num_n = (N + BN_MAX - 1) / BN_MAX;
+    CUtensorMap ta, tb;
+    if ((rc = make_tmap_2d(&ta, a, 2, K, M, static_cast<uint64_t>(K) * 2, BK / 2, ROWS, true))) return rc;
+    if (M > ROWS) {
+        using L = Layout<2, false, BN_MAX, true>;
+        if ((rc = prepare<2, false, false, BN_MAX, true>(di, L::BYTES_DENSE))) return rc;
+        int pairs = 0;
+        if ((rc = max_pairs<false, BN_MAX, false, true>(di, &pairs))) return rc;
+        if ((rc = make_tmap_2d(&tb, b, 2, K, N, static_cast<uint64_t>(K) * 2, BK / 2, L::B_ROWS, true)))
+            return rc;
+        const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
+        const int clusters = tiles < pairs ? tiles : pairs;
+        return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, false, BN_MAX, true>, dim3(2 * clusters),
+                                     dim3(L::THREADS_), L::BYTES_DENSE, st, 2, ta, tb, p),
+                          "bf16 gemm (CTA pair) launch");
+    }
+    using L = Layout<1, false, BN_MAX, true>;
+    if ((rc = prepare<1, false, false, BN_MAX, true>(di, L::BYTES_DENSE))) return rc;
+    if ((rc = make_tmap_2d(&tb, b, 2, K, N, static_cast<uint64_t>(K) * 2, BK / 2, L::B_ROWS, true))) return rc;
+    const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
+    const int grid = tiles < di.num_sms ? tiles : di.num_sms;
+    return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, false, BN_MAX, true>, dim3(grid), dim3(L::THREADS_),
+                                 L::BYTES_DENSE, st, 1, ta, tb, p),
+                      "bf16 gemm launch");
+}
+
 }  // namespace metis
 
 using namespace metis;
+
+extern "C" int metis_bf16_gemm(const void* x_bf16, const void* w_bf16, void* y_bf16, int64_t M,
+                               int64_t N, int64_t K, metis_stream_t stream) {
+    clear_error();
+    if (M < 0 || N < 8 || N % 8 || K < 8 || K % 8 || M > 0x7fffffff || N > 0x7fffffff || K > 0x7fffffff)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "bf16_gemm: need M >= 0, N and K multiples of 8 (M=%lld N=%lld K=%lld)", (long long)M,
+                    (long long)N, (long long)K);
+    if (M == 0) return METIS_OK;
+    if (!x_bf16 || !w_bf16 || !y_bf16) return fail(METIS_ERR_INVALID_ARG, "bf16_gemm: null pointer");
+    if (!aligned(x_bf16, 16) || !aligned(w_bf16, 16) || !aligned(y_bf16, 16))
+        return fail(METIS_ERR_INVALID_ARG, "bf16_gemm: x, w and y must be 16-byte aligned");
+    return launch_bf16_gemm(static_cast<const __nv_bfloat16*>(x_bf16), static_cast<const __nv_bfloat16*>(w_bf16),
+                            static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(M), static_cast<int>(N),
+                            static_cast<int>(K), nullptr, nullptr, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
 
 extern "C" int metis_fp8_gemm(const void* a, int a_kind, float* s_tok, const uint8_t* wq,
                               const float* s_w, void* y_bf16, int64_t M, int64_t N, int64_t K,

@@ -339,12 +339,12 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     if (S > (1ll << 30)) return fail(METIS_ERR_INVALID_ARG, "moe: T*topk too large");
     const size_t need = metis_workspace_size(METIS_OP_MOE, T, I, H, topk, E);
     if (T == 0) return METIS_OK;
-    if (!x_bf16 || !topk_ids || !topk_w || !w_up || !s_up || !w_down || !s_down || !y_bf16 || !workspace)
+    if (!x_bf16 || !topk_ids || !topk_w || !w_up || !s_up || !w_down || !s_down || !workspace)
         return fail(METIS_ERR_INVALID_ARG, "moe: null pointer");
     if (ws_bytes < need)
         return fail(METIS_ERR_INVALID_ARG, "moe: workspace of %zu bytes, need %zu", ws_bytes, need);
     if (!aligned(workspace, 256) || !aligned(x_bf16, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
-        !aligned(y_bf16, 16) || !aligned(s_up, 16) || !aligned(s_down, 16))
+        (y_bf16 && !aligned(y_bf16, 16)) || !aligned(s_up, 16) || !aligned(s_down, 16))
         return fail(METIS_ERR_INVALID_ARG,
                     "moe: workspace must be 256-byte aligned; x, weights, scales and y 16-byte aligned");
     DeviceInfo di;
@@ -389,6 +389,7 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     if ((rc = launch_fp8_gemm_grouped(hq, sh, w_down, s_down, o, offsets, static_cast<int>(E),
                                       static_cast<int>(S), static_cast<int>(H), static_cast<int>(I), st)))
         return rc;
+    if (!y_bf16) return METIS_OK;  // the caller combines (metis_moe_shared_fused_combine)
     const int64_t work = T * (H / 8);
     combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
         o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
@@ -527,12 +528,12 @@ extern "C" int metis_moe_nvfp4_grouped_gemm(const void* x_bf16, const int32_t* t
     const size_t need = metis_workspace_size(METIS_OP_MOE_NVFP4, T, I, H, topk, E);
     if (T == 0) return METIS_OK;
     if (!x_bf16 || !topk_ids || !topk_w || !w_up || !sf_up || !g_up || !w_down || !sf_down || !g_down ||
-        !y_bf16 || !workspace)
+        !workspace)
         return fail(METIS_ERR_INVALID_ARG, "moe_nvfp4: null pointer");
     if (ws_bytes < need)
         return fail(METIS_ERR_INVALID_ARG, "moe_nvfp4: workspace of %zu bytes, need %zu", ws_bytes, need);
     if (!aligned(workspace, 256) || !aligned(x_bf16, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
-        !aligned(sf_up, 16) || !aligned(sf_down, 16) || !aligned(y_bf16, 16) || !aligned(g_up, 4) ||
+        !aligned(sf_up, 16) || !aligned(sf_down, 16) || (y_bf16 && !aligned(y_bf16, 16)) || !aligned(g_up, 4) ||
         !aligned(g_down, 4))
         return fail(METIS_ERR_INVALID_ARG,
                     "moe_nvfp4: workspace 256-byte aligned; x, codes, tiled scales and y 16-byte aligned");
@@ -581,9 +582,55 @@ extern "C" int metis_moe_nvfp4_grouped_gemm(const void* x_bf16, const int32_t* t
     if ((rc = launch_nvfp4_gemm(hq, sfh, gh, Sp, w_down, sf_down, g_down, E * H, o, offsets, counts,
                                 static_cast<int>(E), 0, static_cast<int>(H), static_cast<int>(I), st)))
         return rc;
+    if (!y_bf16) return METIS_OK;  // the caller combines (metis_moe_shared_fused_combine)
     const int64_t work = T * (H / 8);
     combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
         o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
         static_cast<__nv_bfloat16*>(y_bf16));
     return cuda_check(cudaGetLastError(), "moe_nvfp4 combine launch");
 }
+
+// ---------------------------------------------------------------------------
+// The shared expert with the routed combine in its down-projection's epilogue
+// ("Lernex/Metis-1.6-Praxis" card, "Architecture": one shared expert beside
+// the routed ones in every layer; the FP8 cards keep it in BF16):
+//   h_s = bf16(x W_sup^T)                      (BF16 tcgen05 GEMM)
+//   y   = bf16(bf16(h_s W_sdn^T) + sum_j w_j o_j)  (same GEMM, combine fused)
+extern "C" int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int64_t H, int64_t I_s,
+                                              const void* w_sup_bf16, const void* w_sdn_bf16,
+                                              const void* o_routed_bf16,
+                                              const int32_t* slot_to_row, const float* topk_w,
+                                              int64_t topk, void* y_bf16, void* workspace,
+                                              size_t ws_bytes, metis_stream_t stream) {
+    clear_error();
+    if (T < 0 || T > (1ll << 28) || topk < 1 || topk > 8)
+        return fail(METIS_ERR_INVALID_ARG, "shared_fused_combine: need T >= 0 and 1 <= topk <= 8 "
+                    "(T=%lld topk=%lld)", (long long)T, (long long)topk);
+    if (H < 16 || H % 16 || H > 16384 || I_s < 16 || I_s % 16 || I_s > 65536)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "shared_fused_combine: need H and I_s multiples of 16, H <= 16384, I_s <= 65536 "
+                    "(H=%lld I_s=%lld)", (long long)H, (long long)I_s);
+    if (T == 0) return METIS_OK;
+    if (!x_bf16 || !w_sup_bf16 || !w_sdn_bf16 || !o_routed_bf16 || !slot_to_row || !topk_w || !y_bf16 ||
+        !workspace)
+        return fail(METIS_ERR_INVALID_ARG, "shared_fused_combine: null pointer");
+    const size_t need = metis_workspace_size(METIS_OP_SHARED, T, I_s, H, topk, 0);
+    if (ws_bytes < need)
+        return fail(METIS_ERR_INVALID_ARG, "shared_fused_combine: workspace of %zu bytes, need %zu", ws_bytes, need);
+    if (!aligned(x_bf16, 16) || !aligned(w_sup_bf16, 16) || !aligned(w_sdn_bf16, 16) ||
+        !aligned(o_routed_bf16, 16) || !aligned(y_bf16, 16) || !aligned(workspace, 16) ||
+        !aligned(slot_to_row, 4) || !aligned(topk_w, 4))
+        return fail(METIS_ERR_INVALID_ARG,
+                    "shared_fused_combine: x, weights, o, y and the workspace 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    __nv_bfloat16* hs = static_cast<__nv_bfloat16*>(workspace);
+    int rc = launch_bf16_gemm(static_cast<const __nv_bfloat16*>(x_bf16),
+                              static_cast<const __nv_bfloat16*>(w_sup_bf16), hs, static_cast<int>(T),
+                              static_cast<int>(I_s), static_cast<int>(H), nullptr, nullptr, nullptr, 0, st);
+    if (rc) return rc;
+    return launch_bf16_gemm(hs, static_cast<const __nv_bfloat16*>(w_sdn_bf16),
+                            static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(T), static_cast<int>(H),
+                            static_cast<int>(I_s), static_cast<const __nv_bfloat16*>(o_routed_bf16),
+                            slot_to_row, topk_w, static_cast<int>(topk), st);
+}
+

@@ -294,6 +294,9 @@ extern "C" size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, i
             moe_region_offset(0, M_or_T, topk, E, K_or_H, N_or_I, &total);
             return static_cast<size_t>(total);
         }
+        case METIS_OP_SHARED:
+            // the shared expert's hidden rows h_s [T, I_s] BF16
+            return static_cast<size_t>(align256(2 * M_or_T * N_or_I));
         case METIS_OP_MOE_NVFP4: {
             if (topk < 1 || E < 1) return 0;
             int64_t total = 0;

@@ -8,6 +8,8 @@ only the device status word.
     python -m moe_gemm_token_b200.drive decode M [--calls N]
     python -m moe_gemm_token_b200.drive w16 M N K [--calls N]
     python -m moe_gemm_token_b200.drive quant M K [--calls N]
+    python -m moe_gemm_token_b200.drive moe4  [--calls N]
+    python -m moe_gemm_token_b200.drive gemm4 M N K [--calls N]
 
 Each call is enqueued on the current stream; the script synchronises once at
 the end and exits non-zero if the device status word reports an error.
@@ -26,9 +28,14 @@ def _codes(n, k, g):
     return c
 
 
+def _sf(n, g):
+    """E4M3 block scales 2^-3 .. 2^2 (no NaN code), in any layout."""
+    return torch.randint(0x20, 0x48, (n,), dtype=torch.uint8, device="cuda", generator=g)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["moe", "gemm", "fused", "decode", "w16", "quant"])
+    ap.add_argument("op", choices=["moe", "gemm", "fused", "decode", "w16", "quant", "moe4", "gemm4"])
     ap.add_argument("dims", nargs="*", type=int)
     ap.add_argument("--calls", type=int, default=3)
     a = ap.parse_args(argv)
@@ -52,6 +59,35 @@ def main(argv=None):
         ws = torch.empty(metis.metis_workspace_size(metis.METIS_OP_MOE, T, I, H, k, E),
                          dtype=torch.uint8, device=dev)
         call = lambda: metis.metis_moe_fp8_grouped_gemm(x, ids, w, wu, su, wd, sd, y, ws)
+    elif a.op == "moe4":
+        T, H, I, E, k = 4096, 2048, 1024, 64, 8
+        x = torch.randn(T, H, device=dev, generator=g).to(torch.bfloat16)
+        logits = torch.randn(T, E, device=dev, generator=g)
+        logits[:, :4] += 0.93
+        top = torch.topk(logits, k, dim=1)
+        ids = top.indices.to(torch.int32).contiguous()
+        w = torch.softmax(top.values, dim=1).float().contiguous()
+        wu = torch.randint(0, 256, (E, I, H // 2), dtype=torch.uint8, device=dev, generator=g)
+        wd = torch.randint(0, 256, (E, H, I // 2), dtype=torch.uint8, device=dev, generator=g)
+        sfu = _sf(E * I * H // 16, g)
+        sfd = _sf(E * H * I // 16, g)
+        gu = torch.rand(E, device=dev, generator=g) * 1e-3 + 1e-4
+        gd = torch.rand(E, device=dev, generator=g) * 1e-3 + 1e-4
+        y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(metis.metis_workspace_size(metis.METIS_OP_MOE_NVFP4, T, I, H, k, E),
+                         dtype=torch.uint8, device=dev)
+        call = lambda: metis.metis_moe_nvfp4_grouped_gemm(x, ids, w, wu, sfu, gu, wd, sfd, gd, y, ws)
+    elif a.op == "gemm4":
+        M, N, K = a.dims
+        Mp = (M + 127) // 128 * 128
+        qa = torch.randint(0, 256, (Mp, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        sa = _sf(Mp * K // 16, g)
+        ga = torch.rand(M, device=dev, generator=g) + 0.5
+        qb = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        sb = _sf(N * K // 16, g)
+        gb = torch.ones(1, device=dev)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        call = lambda: metis.metis_nvfp4_gemm(qa, sa, ga, qb, sb, gb, y)
     elif a.op in ("gemm", "fused"):
         M, N, K = a.dims
         x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)

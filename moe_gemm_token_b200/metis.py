@@ -32,6 +32,7 @@ METIS_OP_W8A16 = 2
 METIS_OP_MOE = 3
 METIS_OP_LINEAR = 4
 METIS_OP_MOE_NVFP4 = 5
+METIS_OP_SHARED = 6
 METIS_A_F32 = 2
 METIS_SF_ROWMAJOR = 0
 METIS_SF_TILED = 1
@@ -86,6 +87,8 @@ def load():
         "metis_moe_nvfp4_grouped_gemm": ([p, p, p, i64, i64, i64, i64, i64, p, p, p, p, p, p, i32,
                                           p, p, sz, p], i32),
         "metis_moe_nvfp4_workspace_offset": ([i32, i64, i64, i64, i64, i64], i64),
+        "metis_bf16_gemm": ([p, p, p, i64, i64, i64, p], i32),
+        "metis_moe_shared_fused_combine": ([p, i64, i64, i64, p, p, p, p, p, i64, p, p, sz, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -274,4 +277,27 @@ def metis_moe_nvfp4_workspace_offset(region, T, topk, E, H, I):
         region = MOE4_WS[region]
     return int(load().metis_moe_nvfp4_workspace_offset(int(region), int(T), int(topk), int(E),
                                                        int(H), int(I)))
+
+
+# ------------------------------------------------------------ shared expert
+
+def metis_bf16_gemm(x, w, y, stream=None):
+    """y [M, N] = bf16(x [M, K] w [N, K]^T) on the tensor cores."""
+    M, K = x.shape
+    N = w.shape[0]
+    return _check("metis_bf16_gemm", load().metis_bf16_gemm(_p(x), _p(w), _p(y), M, N, K, _s(stream)))
+
+
+def metis_moe_shared_fused_combine(x, w_sup, w_sdn, o_routed, slot_to_row, topk_w, y, workspace,
+                                   stream=None):
+    """y = shared expert(x) + routed combine, the combine fused into the shared
+    down-projection (o_routed / slot_to_row: the routed layer's workspace
+    regions after it ran with y=None)."""
+    T, H = x.shape
+    I_s = w_sup.shape[0]
+    topk = topk_w.shape[1]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    return _check("metis_moe_shared_fused_combine", load().metis_moe_shared_fused_combine(
+        _p(x), T, H, I_s, _p(w_sup), _p(w_sdn), _p(o_routed), _p(slot_to_row), _p(topk_w), topk,
+        _p(y), _p(workspace), ws_bytes, _s(stream)))
 

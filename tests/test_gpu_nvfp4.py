@@ -222,28 +222,31 @@ def run_moe4(m, d, up, dn):
         o=R("O", 2 * Sp * H).view(np.uint16).reshape(Sp, H), y=bf16_host(y))
 
 
-def check_moe4(d, g, up, dn):
+def check_moe4(d, g, up, dn, tokens=None):
     T, k, E, H, I = d["T"], d["topk"], d["E"], d["H"], d["I"]
     ids = d["topk_ids"]
     counts, offsets, s2r, _ = oracle.moe_route(ids, E)
     padded = np.r_[0, np.cumsum((counts + 127) // 128 * 128)].astype(np.int32)
-    exp = ids.reshape(-1)
-    rows = padded[exp] + (s2r - offsets[exp])
+    exp_all = ids.reshape(-1)
+    rows_all = padded[exp_all] + (s2r - offsets[exp_all])
     assert_bytes_equal(g["counts"], counts, "counts")
     assert_bytes_equal(g["offsets"], padded, "padded offsets")
-    assert_bytes_equal(g["s2r"], rows, "slot_to_row")
-    assert_bytes_equal(g["r2s"][rows], np.arange(T * k, dtype=np.int32), "row_to_slot")
+    assert_bytes_equal(g["s2r"], rows_all, "slot_to_row")
+    assert_bytes_equal(g["r2s"][rows_all], np.arange(T * k, dtype=np.int32), "row_to_slot")
     pad = np.ones(padded[-1], bool)
-    pad[rows] = False
+    pad[rows_all] = False
     assert np.all(g["r2s"][:padded[-1]][pad] == -1), "pad rows marked"
     # x in NVFP4, written into every row its token was routed to
     qx, sx, gx = oracle.nvfp4_quant(d["x"], per_row=True)
-    tok = np.arange(T * k) // k
-    assert_bytes_equal(oracle.e2m1_unpack(g["aq"][rows]), qx[tok], "x codes in expert order")
-    assert_bytes_equal(untile_np(g["sfa"], rows, H), sx[tok], "x block scales in expert order")
-    assert_bytes_equal(g["ga"][rows].view(np.uint32), gx[tok].view(np.uint32), "x global scales")
+    tok_all = np.arange(T * k) // k
+    assert_bytes_equal(oracle.e2m1_unpack(g["aq"][rows_all]), qx[tok_all], "x codes in expert order")
+    assert_bytes_equal(untile_np(g["sfa"], rows_all, H), sx[tok_all], "x block scales in expert order")
+    assert_bytes_equal(g["ga"][rows_all].view(np.uint32), gx[tok_all].view(np.uint32), "x global scales")
+    toks = np.arange(T) if tokens is None else np.asarray(tokens)
+    slots = (toks[:, None] * k + np.arange(k)).reshape(-1)
+    rows, exp, tok = rows_all[slots], exp_all[slots], tok_all[slots]
     # up-projection on the GPU's operands
-    h64 = np.empty((T * k, I))
+    h64 = np.empty((slots.size, I))
     for e in np.unique(exp):
         sel = np.nonzero(exp == e)[0]
         _, h64[sel] = oracle.nvfp4_gemm(qx[tok[sel]], sx[tok[sel]], gx[tok[sel]], up[0][e], up[1][e],
@@ -255,16 +258,16 @@ def check_moe4(d, g, up, dn):
     assert_bytes_equal(untile_np(g["sfh"], rows, I), sh, "h block scales")
     assert_bytes_equal(g["gh"][rows].view(np.uint32), gh.view(np.uint32), "h global scales")
     # down-projection on the GPU's codes
-    o64 = np.empty((T * k, H))
+    o64 = np.empty((slots.size, H))
     for e in np.unique(exp):
         sel = np.nonzero(exp == e)[0]
         _, o64[sel] = oracle.nvfp4_gemm(qh[sel], sh[sel], gh[sel], dn[0][e], dn[1][e], dn[2][e])
     assert_close(g["o"][rows], o64, "o")
     # combine on the GPU's o, then the whole layer against the oracle alone
-    _, y64 = oracle.moe_combine(g["o"][rows].reshape(T, k, H), d["topk_w"])
-    assert_close(g["y"], y64, "y (combine)")
-    ref = oracle.moe_forward_nvfp4(d["x"], ids, d["topk_w"], up, dn)
-    assert_close(g["y"], ref["y64"], "y (end to end)")
+    _, y64 = oracle.moe_combine(g["o"][rows].reshape(toks.size, k, H), d["topk_w"][toks])
+    assert_close(g["y"][toks], y64, "y (combine)")
+    ref = oracle.moe_forward_nvfp4(d["x"], ids, d["topk_w"], up, dn, tokens=toks)
+    assert_close(g["y"][toks], ref["y64"], "y (end to end)")
 
 
 @pytest.mark.parametrize("T,H,I,E,k,seed", [(200, 256, 128, 8, 2, 11), (300, 512, 256, 64, 8, 12),
@@ -290,3 +293,45 @@ def test_moe_nvfp4_empty_experts_and_determinism(metis):
     check_moe4(d, g1, up, dn)
     g2 = run_moe4(metis, d, up, dn)
     assert_bytes_equal(g1["y"], g2["y"], "run-to-run")
+
+
+def test_moe_nvfp4_full_size(metis):
+    """The workload the bench times (4096 tokens, hidden 2048, latent 1024,
+    64 experts, top-8, four hot experts), checked on sampled tokens."""
+    d = synth.moe()
+    up, dn = _weights_nvfp4(d["w_up"]), _weights_nvfp4(d["w_down"])
+    g = run_moe4(metis, d, up, dn)
+    ids = d["topk_ids"]
+    rng = np.random.default_rng(1)
+    hot_tok = np.nonzero(np.isin(ids, d["hot_experts"]).any(axis=1))[0]
+    toks = np.unique(np.r_[rng.choice(d["T"], 24, replace=False), hot_tok[:8], 0, d["T"] - 1])
+    check_moe4(d, g, up, dn, tokens=toks)
+
+
+@pytest.mark.parametrize("M,N,K", [(8192, 4096, 4096)])
+def test_nvfp4_gemm_full_size_sampled(metis, M, N, K):
+    """The dense NVFP4 GEMM at a bench size, quantized on the GPU, sampled rows."""
+    d = synth.large_m(M=M, K=K)
+    x = bf16_dev(d["x"])
+    Mp = (M + 127) // 128 * 128
+    qa = torch.empty((Mp, K // 2), dtype=torch.uint8, device="cuda")
+    sa = torch.empty((Mp * K // 16,), dtype=torch.uint8, device="cuda")
+    ga = torch.empty((M,), dtype=torch.float32, device="cuda")
+    metis.metis_quant_nvfp4(x, qa[:M], sa, ga, tiled=True)
+    w = dev(d["w"][:N])
+    qb = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+    sb = torch.empty((N * K // 16,), dtype=torch.uint8, device="cuda")
+    gb = torch.empty((1,), dtype=torch.float32, device="cuda")
+    metis.metis_quant_nvfp4(w, qb, sb, gb, rows_per_scale=N, tiled=True)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_nvfp4_gemm(qa, sa, ga, qb, sb, gb, y)
+    assert metis.metis_check_device_status() == 0
+    rows = np.unique(np.r_[np.random.default_rng(2).choice(M, 30, replace=False), 0, M - 1])
+    qa_r, sa_r, ga_r = oracle.nvfp4_quant(d["x"][rows], per_row=True)
+    qb_r, sb_r, gb_r = oracle.nvfp4_quant(d["w"][:N], per_row=False)
+    assert_bytes_equal(oracle.e2m1_unpack(qa.cpu().numpy()[rows]), qa_r, "A codes")
+    assert_bytes_equal(untile_np(sa.cpu().numpy(), rows, K), sa_r, "A scales")
+    assert_bytes_equal(gb.cpu().numpy().view(np.uint32), gb_r.view(np.uint32), "B global scale")
+    _, y64 = oracle.nvfp4_gemm(qa_r, sa_r, ga_r, qb_r, sb_r, gb_r[0])
+    assert_close(bf16_host(y)[rows], y64, "y")
+
