@@ -600,7 +600,35 @@ def secondary_figures(metis, dev, pk):
     tf = 2 * 2 * T * k * H * I / t / 1e12
     out["moe_4096tok_64e_top8"] = {"us": t * 1e6, "tok/s": T / t, "TFLOP/s": tf,
                                    "frac_of_fp8_peak": tf / peak8}
-    del wu, wd, wsp
+    # the layer with its shared expert (BF16, latent 1024): the routed layer
+    # with y = NULL, then the shared expert with the routed combine fused into
+    # its down-projection's epilogue
+    Is = 1024
+    wsu = (torch.randn(Is, H, device=dev, generator=g) * 0.03).to(torch.bfloat16)
+    wsd = (torch.randn(H, Is, device=dev, generator=g) * 0.03).to(torch.bfloat16)
+    wss = torch.empty(metis.metis_workspace_size(metis.METIS_OP_SHARED, T, Is, H, k, 0),
+                      dtype=torch.uint8, device=dev)
+    o_off = metis.metis_moe_workspace_offset("O", T, k, E, H, I)
+    r_off = metis.metis_moe_workspace_offset("SLOT_TO_ROW", T, k, E, H, I)
+    o_reg = wsp[o_off:].view(torch.bfloat16)
+    s2r_reg = wsp[r_off:r_off + 4 * T * k].view(torch.int32)
+
+    def shared():
+        metis.metis_moe_shared_fused_combine(x, wsu, wsd, o_reg, s2r_reg, w, y, wss)
+
+    def layer():
+        metis.metis_moe_fp8_grouped_gemm(x, ids, w, wu, su, wd, sd, None, wsp)
+        shared()
+    hs = torch.empty(T, Is, dtype=torch.bfloat16, device=dev)
+    t_l = timeit(layer, 20)
+    t_s = timeit(shared, 20)
+    t_g = timeit(lambda: metis.metis_bf16_gemm(x, wsu, hs), 20)
+    out["moe_with_shared_4096tok_64e_top8"] = {
+        "us": t_l * 1e6, "tok/s": T / t_l, "shared_fused_combine_us": t_s * 1e6,
+        "bf16_gemm_4096x1024x2048_us": t_g * 1e6,
+        "bf16_gemm_TFLOP/s": 2 * T * Is * H / t_g / 1e12,
+        "bf16_gemm_frac_of_bf16_peak": 2 * T * Is * H / t_g / 1e12 / pk["bf16_tflops"]}
+    del wu, wd, wsp, o_reg, s2r_reg
     # the same routed-expert layer with NVFP4 experts (E2M1 codes, E4M3 scale
     # per 16, FP32 scale per expert; inputs rounded to NVFP4 per token)
     peak4 = pk["bf16_tflops"] * FP4_PER_BF16

@@ -191,9 +191,15 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, cons
     }
 }
 
+// L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned address.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // The W16 epilogue chunk: y = bf16(acc), staged as above; with the fused
 // combine each 8-column piece then gets the token's routed outputs added,
-// y = bf16(s + sum_j w_j o_j) in FP32, j ascending (all loads issued first).
+// y = bf16(s + sum_j w_j o_j) in FP32, j ascending. Two rows are handled at
+// a time, so 2 * topk loads are in flight per lane.
 __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, const Tile& ti, int q,
                                                 int lane, uint8_t* stg, const int2* cb,
                                                 const Params& p) {
@@ -208,41 +214,62 @@ __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, 
     __syncwarp();
     const int n = ti.n0 + c * 32 + (lane & 3) * 8;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int rr = (lane >> 2) + 8 * i;
-        uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
-        const int row = ti.a_row0 + q * 32 + rr;
-        if (row >= ti.row_end || n >= p.N) continue;
+    for (int i0 = 0; i0 < 4; i0 += 2) {
+        uint4 val[2];
+        bool live[2];
+        uint4 ov[2][COMB_K];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int rr = (lane >> 2) + 8 * (i0 + u);
+            val[u] = *reinterpret_cast<const uint4*>(stg + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
+            live[u] = ti.a_row0 + q * 32 + rr < ti.row_end && n < p.N;
+        }
         if (p.o != nullptr) {
-            const int2* e = cb + rr * COMB_K;
-            uint4 ov[COMB_K];
+            // every load of both rows before the first add (the (row, weight)
+            // pairs are read from shared memory where they are used)
 #pragma unroll
-            for (int j = 0; j < COMB_K; ++j)
-                if (j < p.topk && e[j].x >= 0)
-                    ov[j] = *reinterpret_cast<const uint4*>(p.o + static_cast<size_t>(e[j].x) * p.N + n);
-            const uint32_t sv[4] = {val.x, val.y, val.z, val.w};
-            float a[8];
+            for (int u = 0; u < 2; ++u) {
+                const int2* e = cb + ((lane >> 2) + 8 * (i0 + u)) * COMB_K;
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                a[2 * h] = bf16_lo(sv[h]);
-                a[2 * h + 1] = bf16_hi(sv[h]);
-            }
-#pragma unroll
-            for (int j = 0; j < COMB_K; ++j) {
-                if (j < p.topk && e[j].x >= 0) {
-                    const float wj = __int_as_float(e[j].y);
-                    const uint32_t ow[4] = {ov[j].x, ov[j].y, ov[j].z, ov[j].w};
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        a[2 * h] = fmaf(wj, bf16_lo(ow[h]), a[2 * h]);
-                        a[2 * h + 1] = fmaf(wj, bf16_hi(ow[h]), a[2 * h + 1]);
-                    }
+                for (int j = 0; j < COMB_K; ++j) {
+                    const int r = e[j].x;
+                    if (live[u] && j < p.topk && r >= 0)
+                        ov[u][j] = *reinterpret_cast<const uint4*>(p.o + static_cast<size_t>(r) * p.N + n);
                 }
             }
-            val = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
-                             pack_bf16x2(a[6], a[7]));
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int2* e = cb + ((lane >> 2) + 8 * (i0 + u)) * COMB_K;
+                const uint32_t sv[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
+                float a[8];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    a[2 * h] = bf16_lo(sv[h]);
+                    a[2 * h + 1] = bf16_hi(sv[h]);
+                }
+#pragma unroll
+                for (int j = 0; j < COMB_K; ++j) {
+                    const int2 ej = e[j];
+                    if (live[u] && j < p.topk && ej.x >= 0) {
+                        const float wj = __int_as_float(ej.y);
+                        const uint32_t ow[4] = {ov[u][j].x, ov[u][j].y, ov[u][j].z, ov[u][j].w};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            a[2 * h] = fmaf(wj, bf16_lo(ow[h]), a[2 * h]);
+                            a[2 * h + 1] = fmaf(wj, bf16_hi(ow[h]), a[2 * h + 1]);
+                        }
+                    }
+                }
+                val[u] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                                    pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
+            }
         }
-        *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.N + n) = val;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int rr = (lane >> 2) + 8 * (i0 + u);
+            const int row = ti.a_row0 + q * 32 + rr;
+            if (live[u]) *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.N + n) = val[u];
+        }
     }
 }
 
@@ -579,10 +606,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (p.o != nullptr) {
                     const int row = ti.a_row0 + q * 32 + lane;
                     int2* mine = comb + ((warp - 2) * 32 + lane) * COMB_K;
+                    // this warp's columns of the routed rows go to L2 now, while
+                    // the tile's MMAs run
+                    const int col0 = ti.n0 + c0 * 32;
+                    const int ncol = min(CPW * 32, p.N - col0);
                     for (int j = 0; j < p.topk; ++j) {
                         const size_t sidx = static_cast<size_t>(row) * p.topk + j;
-                        mine[j] = row < ti.row_end ? make_int2(p.s2r[sidx], __float_as_int(p.topk_w[sidx]))
-                                                   : make_int2(-1, 0);
+                        const int2 v = row < ti.row_end ? make_int2(p.s2r[sidx], __float_as_int(p.topk_w[sidx]))
+                                                        : make_int2(-1, 0);
+                        mine[j] = v;
+                        if (v.x >= 0 && ncol > 0)
+                            prefetch_l2(p.o + static_cast<size_t>(v.x) * p.N + col0, static_cast<uint32_t>(ncol) * 2u);
                     }
                     __syncwarp();
                 }

@@ -10,6 +10,8 @@ only the device status word.
     python -m moe_gemm_token_b200.drive quant M K [--calls N]
     python -m moe_gemm_token_b200.drive moe4  [--calls N]
     python -m moe_gemm_token_b200.drive gemm4 M N K [--calls N]
+    python -m moe_gemm_token_b200.drive shared [--calls N]
+    python -m moe_gemm_token_b200.drive bf16 M N K [--calls N]
 
 Each call is enqueued on the current stream; the script synchronises once at
 the end and exits non-zero if the device status word reports an error.
@@ -35,7 +37,7 @@ def _sf(n, g):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["moe", "gemm", "fused", "decode", "w16", "quant", "moe4", "gemm4"])
+    ap.add_argument("op", choices=["moe", "gemm", "fused", "decode", "w16", "quant", "moe4", "gemm4", "shared", "bf16"])
     ap.add_argument("dims", nargs="*", type=int)
     ap.add_argument("--calls", type=int, default=3)
     a = ap.parse_args(argv)
@@ -43,7 +45,7 @@ def main(argv=None):
     g = torch.Generator(device="cuda")
     g.manual_seed(7)
     dev = "cuda"
-    if a.op == "moe":
+    if a.op in ("moe", "shared"):
         T, H, I, E, k = 4096, 2048, 1024, 64, 8
         x = torch.randn(T, H, device=dev, generator=g).to(torch.bfloat16)
         logits = torch.randn(T, E, device=dev, generator=g)
@@ -59,6 +61,21 @@ def main(argv=None):
         ws = torch.empty(metis.metis_workspace_size(metis.METIS_OP_MOE, T, I, H, k, E),
                          dtype=torch.uint8, device=dev)
         call = lambda: metis.metis_moe_fp8_grouped_gemm(x, ids, w, wu, su, wd, sd, y, ws)
+        if a.op == "shared":
+            # routed layer with y = NULL, then the BF16 shared expert (latent
+            # 1024) with the routed combine fused into its down-projection
+            wsu = (torch.randn(1024, H, device=dev, generator=g) * 0.03).to(torch.bfloat16)
+            wsd = (torch.randn(H, 1024, device=dev, generator=g) * 0.03).to(torch.bfloat16)
+            wss = torch.empty(metis.metis_workspace_size(metis.METIS_OP_SHARED, T, 1024, H, k, 0),
+                              dtype=torch.uint8, device=dev)
+            o_off = metis.metis_moe_workspace_offset("O", T, k, E, H, I)
+            r_off = metis.metis_moe_workspace_offset("SLOT_TO_ROW", T, k, E, H, I)
+            o_reg = ws[o_off:].view(torch.bfloat16)
+            s2r = ws[r_off:r_off + 4 * T * k].view(torch.int32)
+
+            def call():
+                metis.metis_moe_fp8_grouped_gemm(x, ids, w, wu, su, wd, sd, None, ws)
+                metis.metis_moe_shared_fused_combine(x, wsu, wsd, o_reg, s2r, w, y, wss)
     elif a.op == "moe4":
         T, H, I, E, k = 4096, 2048, 1024, 64, 8
         x = torch.randn(T, H, device=dev, generator=g).to(torch.bfloat16)
@@ -77,6 +94,12 @@ def main(argv=None):
         ws = torch.empty(metis.metis_workspace_size(metis.METIS_OP_MOE_NVFP4, T, I, H, k, E),
                          dtype=torch.uint8, device=dev)
         call = lambda: metis.metis_moe_nvfp4_grouped_gemm(x, ids, w, wu, sfu, gu, wd, sfd, gd, y, ws)
+    elif a.op == "bf16":
+        M, N, K = a.dims
+        x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+        wb = (torch.randn(N, K, device=dev, generator=g) * 0.03).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        call = lambda: metis.metis_bf16_gemm(x, wb, y)
     elif a.op == "gemm4":
         M, N, K = a.dims
         Mp = (M + 127) // 128 * 128
