@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
     __shared__ int part[SCAN_THREADS];  // [g][e]: sums, then prefix over g
     __shared__ int warp_tot[32];
     __shared__ int excl_e[MAX_E];
+    __shared__ int cnt_e[MAX_E];
     int Ep = 1;
     while (Ep < E) Ep <<= 1;
     const int G = SCAN_THREADS / Ep;
@@ -125,11 +126,18 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
         counts[threadIdx.x] = total;
         offsets[threadIdx.x] = excl;
         excl_e[threadIdx.x] = excl;
+        cnt_e[threadIdx.x] = total;
         if (threadIdx.x == E - 1) offsets[E] = excl + ptotal;
-        if (r2s_pad)
-            for (int r = excl + total; r < excl + ptotal; ++r) r2s_pad[r] = -1;
     }
     __syncthreads();
+    // pad rows (fewer than pad per expert) marked -1, by all threads
+    if (r2s_pad) {
+        for (int i = threadIdx.x; i < E * pad; i += SCAN_THREADS) {
+            const int ee = i / pad, k = i - ee * pad;
+            const int c = cnt_e[ee];
+            if (k < (c + pad - 1) / pad * pad - c) r2s_pad[excl_e[ee] + c + k] = -1;
+        }
+    }
     // chunk bases: this thread's run of chunks, from its expert's offset plus
     // the counts of the runs before it
     if (e < E) {

@@ -126,8 +126,12 @@ struct QuantArgs {
     int64_t pad_rows;         // tiled, no gather: rows [R, pad_rows) get zero scales
 };
 
-template <typename T>
+// NBL > 0 (BF16 rows with K <= 512 NBL): lane l keeps blocks l, l + 32, ...
+// of the row in registers, so the row is read from memory once; NBL = 0
+// reads it twice (amax pass, then codes).
+template <typename T, int NBL>
 __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArgs a) {
+    static_assert(NBL == 0 || sizeof(T) == 2, "register-resident rows are BF16");
     grid_dependency_wait();  // the rows may be the previous kernel's output
     grid_launch_dependents();
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -145,16 +149,50 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
     if (a.row_valid && a.row_valid[r] < 0) return;
     const T* row = static_cast<const T*>(a.x) + r * a.ldx;
     const int nb = static_cast<int>(a.K / 16);
+    uint4 raw[NBL > 0 ? NBL : 1][2];
+    if constexpr (NBL > 0) {
+#pragma unroll
+        for (int i = 0; i < NBL; ++i) {
+            const int b = lane + 32 * i;
+            if (b < nb) {
+                raw[i][0] = ld_nc_v4(row + 16 * b);
+                raw[i][1] = ld_nc_v4(row + 16 * b + 8);
+            } else {
+                raw[i][0] = raw[i][1] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    } else {
+        raw[0][0] = raw[0][1] = make_uint4(0u, 0u, 0u, 0u);  // unused
+    }
+    auto unpack = [&](int i, float (&v)[16]) {
+        const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
+                               raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            v[2 * h] = bf16_lo(w[h]);
+            v[2 * h + 1] = bf16_hi(w[h]);
+        }
+    };
     float amax;
     if (a.gamax) {
         amax = a.gamax[r / a.rps];
     } else {
         float m = 0.0f;
-        for (int b = lane; b < nb; b += 32) {
-            float v[16];
-            load16(row + 16 * b, v);
+        if constexpr (NBL > 0) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+            for (int i = 0; i < NBL; ++i) {
+                float v[16];
+                unpack(i, v);
+#pragma unroll
+                for (int h = 0; h < 16; ++h) m = fmaxf(m, fabsf(v[h]));
+            }
+        } else {
+            for (int b = lane; b < nb; b += 32) {
+                float v[16];
+                load16(row + 16 * b, v);
+#pragma unroll
+                for (int h = 0; h < 16; ++h) m = fmaxf(m, fabsf(v[h]));
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -162,12 +200,11 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
     }
     const float inv_g = amax > 0.0f ? fminf(__fdiv_rn(2688.0f, amax), 3.402823466e38f) : 0.0f;
     const int ndst = a.dst_rows ? a.topk : 1;
-    for (int b0 = 0; b0 < nb; b0 += 32) {
+    // one pass over 32 blocks (512 elements); v holds this lane's block b0 + lane
+    auto block_pass = [&](int b0, const float (&v)[16]) {
         const int b = b0 + lane;
         uint32_t lo = 0, hi = 0, sbc = 0;
         if (b < nb) {
-            float v[16];
-            load16(row + 16 * b, v);
             float bm = 0.0f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) bm = fmaxf(bm, fabsf(v[i]));
@@ -194,6 +231,23 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
                 *reinterpret_cast<uint32_t*>(a.sf + off) = s4;
             }
             if (b0 == 0 && lane == 0 && !a.gamax) a.g[dr] = __fdiv_rn(amax, 2688.0f);
+        }
+    };
+    if constexpr (NBL > 0) {
+#pragma unroll
+        for (int i = 0; i < NBL; ++i) {
+            if (32 * i >= nb) break;  // warp-uniform
+            float v[16];
+            unpack(i, v);
+            block_pass(32 * i, v);
+        }
+    } else {
+        for (int b0 = 0; b0 < nb; b0 += 32) {
+            float v[16];
+#pragma unroll
+            for (int h = 0; h < 16; ++h) v[h] = 0.0f;
+            if (b0 + lane < nb) load16(row + 16 * (b0 + lane), v);
+            block_pass(b0, v);
         }
     }
 }
@@ -272,10 +326,21 @@ int launch_nvfp4_quant(const T* x, int64_t R, int64_t K, int64_t ldx, int64_t rp
         a.gamax = g;
     }
     const int64_t rows = a.pad_rows;
-    if ((rc = cuda_check(launch_pdl(nvfp4_quant_kernel<T>, dim3(static_cast<unsigned>((rows + QWARPS - 1) / QWARPS)),
-                                    dim3(QWARPS * 32), 0, st, 1, a),
-                         "nvfp4 quant launch")))
-        return rc;
+    const dim3 grid(static_cast<unsigned>((rows + QWARPS - 1) / QWARPS));
+    auto go = [&](auto kernel) {
+        return cuda_check(launch_pdl(kernel, grid, dim3(QWARPS * 32), 0, st, 1, a), "nvfp4 quant launch");
+    };
+    // BF16 rows of up to 4096 elements stay in registers (one read of x)
+    if constexpr (sizeof(T) == 2) {
+        if (rps == 1 && K <= 512) rc = go(nvfp4_quant_kernel<T, 1>);
+        else if (rps == 1 && K <= 1024) rc = go(nvfp4_quant_kernel<T, 2>);
+        else if (rps == 1 && K <= 2048) rc = go(nvfp4_quant_kernel<T, 4>);
+        else if (rps == 1 && K <= 4096) rc = go(nvfp4_quant_kernel<T, 8>);
+        else rc = go(nvfp4_quant_kernel<T, 0>);
+    } else {
+        rc = go(nvfp4_quant_kernel<T, 0>);
+    }
+    if (rc) return rc;
     if (rps > 1) {
         const int64_t sets = R / rps;
         nvfp4_finish_scales_kernel<<<static_cast<unsigned>((sets + 255) / 256), 256, 0, st>>>(g, sets);
