@@ -364,32 +364,22 @@ namespace nvfp4 {
 
 constexpr int BKB = 128;        // code bytes per row per k-block (256 elements)
 constexpr int KCH = 4;          // 64-element MMA chunks per k-block
-constexpr int ROWS = 128;       // rows of A per tile (TMEM lanes)
+constexpr int ROWS = 128;       // rows of A per CTA per tile (TMEM lanes)
 constexpr int BN = 256;         // output columns per tile
-constexpr int STAGES = 3;
 constexpr int EPI_WARPS = 16;   // four per TMEM lane quadrant
-constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int SCALE_WARP = 2 + EPI_WARPS;   // first of the warps copying scale factors into TMEM
+constexpr int SCALE_WARPS = 4;              // each copies one of a k-block's four 64-element chunks
+constexpr int THREADS = 64 + EPI_WARPS * 32 + SCALE_WARPS * 32;
 constexpr int ATOM = 512;       // one tiled scale atom: 128 rows x 4 scales
-constexpr int A_STAGE = ROWS * BKB;
-constexpr int B_STAGE = BN * BKB;
-constexpr int SFA_STAGE = KCH * ATOM;
-constexpr int SFB_STAGE = 2 * KCH * ATOM;   // two 128-row halves of B
-constexpr int A_OFF = 0;
-constexpr int B_OFF = A_OFF + STAGES * A_STAGE;
-constexpr int SFA_OFF = B_OFF + STAGES * B_STAGE;
-constexpr int SFB_OFF = SFA_OFF + STAGES * SFA_STAGE;
-constexpr int TILES = SFB_OFF + STAGES * SFB_STAGE;
+constexpr int SFA_STAGE = KCH * ATOM;       // this CTA's 128 rows of A
+constexpr int SFB_STAGE = 2 * KCH * ATOM;   // both 128-row halves of B (every CTA)
 constexpr int STAGING = EPI_WARPS * 32 * 64;    // a 32 x 32 BF16 block per epilogue warp
-constexpr int NUM_BARS = 2 * STAGES + 3;        // full, empty, tfull, tempty, drain
-constexpr int BAR_OFF = TILES + STAGING;
-constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
-constexpr int GROUP_OFF = MISC_OFF + 16;
 constexpr int MAX_GROUPS = 1024;
-constexpr size_t BYTES_DENSE = 1024 + GROUP_OFF;
-constexpr size_t BYTES_GROUPED = BYTES_DENSE + 3 * (MAX_GROUPS + 1) * 4;
 constexpr int TMEM_COLS = 512;
 constexpr int SF_COL = BN;      // two scale buffers of 48 columns after the accumulator
 constexpr int SF_BUF = 48;      // SFA: 4 chunks x 4 columns; SFB: 4 chunks x 8 columns
+constexpr int SF_BUFS = 4;      // scale buffers in TMEM (the scale warp runs ahead of the MMAs)
+constexpr int SF_ROW = 256;     // the scale buffers seen by TMA as rows of 256 bytes
 
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format
 // 1), K-major, UE4M3 scales (bit 23 clear), dense K = 64, N >> 3 at bit 17,
@@ -398,6 +388,31 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
     return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
            (static_cast<uint32_t>(m >> 4) << 24);
 }
+
+// Shared-memory layout of the one-CTA (CTAS = 1, 128 x 256 tiles) and the
+// CTA-pair (CTAS = 2, 256 x 256 tiles: each CTA holds 128 rows of A, 128 rows
+// of B and the scales of all 256 rows of B) kernels.
+template <int CTAS, bool GROUPED>
+struct Lay {
+    static constexpr int B_ROWS = BN / CTAS;
+    static constexpr int A_STAGE = ROWS * BKB;
+    static constexpr int B_STAGE = B_ROWS * BKB;
+    static constexpr int STAGES = CTAS == 2 ? (GROUPED ? 4 : 5) : 3;
+    static constexpr int A_OFF = 0;
+    static constexpr int B_OFF = A_OFF + STAGES * A_STAGE;
+    static constexpr int SFA_OFF = B_OFF + STAGES * B_STAGE;
+    static constexpr int SFB_OFF = SFA_OFF + STAGES * SFA_STAGE;
+    static constexpr int TILES = SFB_OFF + STAGES * SFB_STAGE;
+    // full, empty, tfull, tempty, drain, scale buffers full/empty, scale drain
+    static constexpr int NUM_BARS = 2 * STAGES + 3 + 2 * SF_BUFS + SCALE_WARPS;
+    static constexpr int BAR_OFF = TILES + STAGING;
+    static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+    static constexpr int GROUP_OFF = MISC_OFF + 16;
+    static constexpr size_t BYTES = 1024 + GROUP_OFF + (GROUPED ? 3 * (MAX_GROUPS + 1) * 4 : 0);
+    static constexpr uint32_t IDESC = idesc_nvf4(ROWS * CTAS, BN);
+    // CTA pair: both CTAs' loads of a stage counted on the even CTA's barrier
+    static constexpr uint32_t PAIR_TX = CTAS * (A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE);
+};
 
 // Shared-memory descriptor of one scale atom as the tcgen05.cp source: 32
 // rows of 16 bytes, no swizzle, 8-row core matrices 128 bytes apart.
@@ -410,9 +425,15 @@ __device__ __forceinline__ uint64_t sf_atom_desc(uint32_t saddr) {
 }
 
 // Copies one 512-byte atom into TMEM columns [taddr, taddr + 4) of every lane
-// quadrant: lane l of each quadrant gets bytes 16 l .. 16 l + 15.
+// quadrant: lane l of each quadrant gets bytes 16 l .. 16 l + 15. The pair
+// form, issued by the even CTA, copies each CTA's atom at this shared-memory
+// offset into its own TMEM.
 __device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+__device__ __forceinline__ void sf_copy_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
                  : "memory");
 }
 
@@ -426,8 +447,21 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
         : "memory");
 }
+// The CTA pair's block-scaled MMA (M = 256: 128 rows of A per CTA, B rows
+// split between the CTAs, each CTA's TMEM holding its own rows of D, its own
+// A scales and all of B's scales).
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
 
-// Non-tensor bulk copy global -> shared, completing on an mbarrier.
+// Non-tensor bulk copy global -> shared, completing on an mbarrier of this CTA.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -449,11 +483,15 @@ struct GemmParams {
 };
 
 struct Tile {
-    int a_row0, row_end, b_row0, n0, group;
+    int a_row0, row_end, b_row0, b_base, n0, group;
 };
 
+// Tile t -> rows and columns; a tile is 128 * CTAS rows of A (this CTA's
+// 128 at rank * 128) by BN columns.
+template <int CTAS>
 struct Sched {
     int num_n, num_m, total, N, M;
+    uint32_t rank;
     const int* g_tile;   // grouped: prefix sums of tiles per group (smem)
     const int* g_row;    // grouped: first rows (smem)
     const int* g_cnt;    // grouped: rows per group (smem)
@@ -462,9 +500,9 @@ struct Sched {
         Tile ti;
         if (g_tile == nullptr) {
             const int mb = t % num_m, nb = t / num_m;
-            ti.a_row0 = mb * ROWS;
+            ti.a_row0 = mb * ROWS * CTAS + static_cast<int>(rank) * ROWS;
             ti.row_end = M;
-            ti.b_row0 = nb * BN;
+            ti.b_base = nb * BN;
             ti.n0 = nb * BN;
             ti.group = 0;
         } else {
@@ -475,14 +513,15 @@ struct Sched {
             }
             const int e = lo;
             const int local = t - g_tile[e];
-            const int mt = (g_cnt[e] + ROWS - 1) / ROWS;
+            const int mt = (g_cnt[e] + ROWS * CTAS - 1) / (ROWS * CTAS);
             const int mb = local % mt, nb = local / mt;
-            ti.a_row0 = g_row[e] + mb * ROWS;
+            ti.a_row0 = g_row[e] + mb * ROWS * CTAS + static_cast<int>(rank) * ROWS;
             ti.row_end = g_row[e] + g_cnt[e];
-            ti.b_row0 = e * N + nb * BN;
+            ti.b_base = e * N + nb * BN;
             ti.n0 = nb * BN;
             ti.group = e;
         }
+        ti.b_row0 = ti.b_base + static_cast<int>(rank) * (BN / CTAS);
         return ti;
     }
 };
@@ -519,27 +558,35 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, cons
     }
 }
 
-template <bool GROUPED>
+template <int CTAS, bool GROUPED>
 __global__ void __launch_bounds__(THREADS, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                   const GemmParams p) {
+    using L = Lay<CTAS, GROUPED>;
+    constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* staging = smem + TILES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);
-    int* g_tile = reinterpret_cast<int*>(smem + GROUP_OFF);
+    uint8_t* staging = smem + L::TILES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+    int* g_tile = reinterpret_cast<int*>(smem + L::GROUP_OFF);
     int* g_row = g_tile + (MAX_GROUPS + 1);
     int* g_cnt = g_row + (MAX_GROUPS + 1);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
+    const uint32_t rank = CTAS == 2 ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
     auto full = [&](int s) { return smem_u32(&bars[s]); };
     auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
     const uint32_t tfull = smem_u32(&bars[2 * STAGES]);
     const uint32_t tempty = smem_u32(&bars[2 * STAGES + 1]);
     const uint32_t drain = smem_u32(&bars[2 * STAGES + 2]);
+    auto sf_full = [&](int b) { return smem_u32(&bars[2 * STAGES + 3 + b]); };
+    auto sf_empty = [&](int b) { return smem_u32(&bars[2 * STAGES + 3 + SF_BUFS + b]); };
+    const uint32_t sdrain = smem_u32(&bars[2 * STAGES + 3 + 2 * SF_BUFS]);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -547,27 +594,43 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             mbar_init(empty(s), 1);
         }
         mbar_init(tfull, 1);
-        mbar_init(tempty, EPI_WARPS);
+        mbar_init(tempty, CTAS * EPI_WARPS);
         mbar_init(drain, 1);
+        for (int b = 0; b < SF_BUFS; ++b) {
+            mbar_init(sf_full(b), SCALE_WARPS);
+            mbar_init(sf_empty(b), 1);
+        }
+        for (int w = 0; w < SCALE_WARPS; ++w) mbar_init(sdrain + 8 * w, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if constexpr (CTAS == 2) {
+            tma_prefetch_desc(&tmSFA);
+            tma_prefetch_desc(&tmSFB);
+        }
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (CTAS == 2) {
+            tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+            tmem_relinquish();
+        }
     }
 
     // operands, scales and offsets may come from the previous kernel (PDL)
     grid_launch_dependents();
     grid_dependency_wait();
 
-    Sched sc;
+    Sched<CTAS> sc;
     sc.N = p.N;
     sc.M = p.M;
     sc.E = p.E;
+    sc.rank = rank;
     sc.num_n = (p.N + BN - 1) / BN;
+    constexpr int TROWS = ROWS * CTAS;   // rows of A per tile
     if constexpr (GROUPED) {
         if (warp == 0) {
             const int per = (p.E + 31) / 32;
@@ -575,7 +638,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             int local = 0;
             for (int i = 0; i < per; ++i) {
                 const int e = g0 + i;
-                if (e < p.E) local += ((p.counts[e] + ROWS - 1) / ROWS) * sc.num_n;
+                if (e < p.E) local += ((p.counts[e] + TROWS - 1) / TROWS) * sc.num_n;
             }
             int incl = local;
 #pragma unroll
@@ -590,7 +653,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     g_tile[e] = run;
                     g_row[e] = p.offsets[e];
                     g_cnt[e] = p.counts[e];
-                    run += ((p.counts[e] + ROWS - 1) / ROWS) * sc.num_n;
+                    run += ((p.counts[e] + TROWS - 1) / TROWS) * sc.num_n;
                 }
             }
             if (lane == 31) g_tile[p.E] = incl;
@@ -603,18 +666,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         sc.g_tile = nullptr;
         sc.g_row = nullptr;
         sc.g_cnt = nullptr;
-        sc.num_m = (p.M + ROWS - 1) / ROWS;
+        sc.num_m = (p.M + TROWS - 1) / TROWS;
         sc.total = sc.num_m * sc.num_n;
     }
     __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CTAS == 2) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     if constexpr (GROUPED) sc.total = g_tile[p.E];
     const uint32_t tmem_base = *tmem_slot;
     const int kch_total = p.K / 64;             // 64-element chunks per row
     const int num_kb = (kch_total + KCH - 1) / KCH;
-    constexpr uint32_t IDESC = idesc_nvf4(ROWS, BN);
+    const int first = CTAS == 2 ? static_cast<int>(blockIdx.x / 2) : static_cast<int>(blockIdx.x);
+    const int stride = CTAS == 2 ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -622,10 +686,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_phase = 0;
-            for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+            for (int t = first; t < sc.total && !*abort_flag; t += stride) {
                 const Tile ti = sc.get(t);
                 const int64_t rb_a = ti.a_row0 / ROWS;
-                const int64_t rb_b0 = ti.b_row0 / ROWS;
+                const int64_t rb_b0 = ti.b_base / ROWS;
                 // the second 128-row half of B exists only when n0 + 128 < N;
                 // otherwise its scale atoms repeat the first half's (the
                 // columns it feeds are never stored)
@@ -635,38 +699,59 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                         *abort_flag = 1;
                         break;
                     }
-                    const int nk = min(KCH, kch_total - kb * KCH);
-                    const uint32_t sfb = static_cast<uint32_t>(nk * ATOM);
-                    mbar_arrive_expect_tx(full(stage), A_STAGE + B_STAGE + 3 * sfb);
-                    tma_load_2d(smem_u32(smem + A_OFF + stage * A_STAGE), &tmA, kb * BKB, ti.a_row0, full(stage));
-                    tma_load_2d(smem_u32(smem + B_OFF + stage * B_STAGE), &tmB, kb * BKB, ti.b_row0, full(stage));
                     const int64_t c0 = static_cast<int64_t>(kb) * KCH;
-                    bulk_load(smem_u32(smem + SFA_OFF + stage * SFA_STAGE),
-                              p.sfa + (rb_a * kch_total + c0) * ATOM, sfb, full(stage));
-                    bulk_load(smem_u32(smem + SFB_OFF + stage * SFB_STAGE),
-                              p.sfb + (rb_b0 * kch_total + c0) * ATOM, sfb, full(stage));
-                    bulk_load(smem_u32(smem + SFB_OFF + stage * SFB_STAGE + KCH * ATOM),
-                              p.sfb + (rb_b1 * kch_total + c0) * ATOM, sfb, full(stage));
+                    const uint32_t sa = smem_u32(smem + L::A_OFF + stage * L::A_STAGE);
+                    const uint32_t sb = smem_u32(smem + L::B_OFF + stage * L::B_STAGE);
+                    const uint32_t ssa = smem_u32(smem + L::SFA_OFF + stage * SFA_STAGE);
+                    const uint32_t ssb = smem_u32(smem + L::SFB_OFF + stage * SFB_STAGE);
+                    if constexpr (CTAS == 2) {
+                        // whole boxes (4 atoms each, past the last chunk too:
+                        // later atoms or zero fill) so that the byte count is fixed
+                        const uint32_t fl = mapa_shared(full(stage), 0);
+                        constexpr int RPA = ATOM / SF_ROW;  // 256-byte rows per atom
+                        if (leader) mbar_arrive_expect_tx(full(stage), L::PAIR_TX);
+                        tma_load_2d_pair(sa, &tmA, kb * BKB, ti.a_row0, fl);
+                        tma_load_2d_pair(sb, &tmB, kb * BKB, ti.b_row0, fl);
+                        tma_load_2d_pair(ssa, &tmSFA, 0, static_cast<int32_t>((rb_a * kch_total + c0) * RPA), fl);
+                        tma_load_2d_pair(ssb, &tmSFB, 0, static_cast<int32_t>((rb_b0 * kch_total + c0) * RPA), fl);
+                        tma_load_2d_pair(ssb + KCH * ATOM, &tmSFB, 0,
+                                         static_cast<int32_t>((rb_b1 * kch_total + c0) * RPA), fl);
+                    } else {
+                        const int nk = min(KCH, kch_total - kb * KCH);
+                        const uint32_t sfb = static_cast<uint32_t>(nk * ATOM);
+                        mbar_arrive_expect_tx(full(stage), L::A_STAGE + L::B_STAGE + 3 * sfb);
+                        tma_load_2d(sa, &tmA, kb * BKB, ti.a_row0, full(stage));
+                        tma_load_2d(sb, &tmB, kb * BKB, ti.b_row0, full(stage));
+                        bulk_load(ssa, p.sfa + (rb_a * kch_total + c0) * ATOM, sfb, full(stage));
+                        bulk_load(ssb, p.sfb + (rb_b0 * kch_total + c0) * ATOM, sfb, full(stage));
+                        bulk_load(ssb + KCH * ATOM, p.sfb + (rb_b1 * kch_total + c0) * ATOM, sfb, full(stage));
+                    }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
             if (*abort_flag) {
-                // let the copies in flight land before the CTA exits
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued & (1u << s))
-                        mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
+                // let the copies in flight land before the CTA exits (the odd
+                // CTA's copies complete on the even CTA's barriers: wait a while)
+                if (leader) {
+                    for (int s = 0; s < STAGES; ++s)
+                        if (issued & (1u << s))
+                            mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
+                } else {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 100000ull) {}
+                }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             // --------------------------------------------------------- MMA issuer
             int stage = 0;
             uint32_t phase = 0;
             uint32_t acc_phase = 0;
             uint32_t kglob = 0;
-            for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+            for (int t = first; t < sc.total && !*abort_flag; t += stride) {
                 if (!mbar_wait(tempty, acc_phase ^ 1u, p.timeout_ns, p.status)) {
                     *abort_flag = 1;
                     break;
@@ -680,27 +765,36 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     }
                     tc_fence_after();
                     const int nk = min(KCH, kch_total - kb * KCH);
-                    const uint32_t sfa_t = tmem_base + SF_COL + SF_BUF * (kglob & 1u);
+                    // this k-block's scales, copied into TMEM by the scale warp
+                    const uint32_t buf = kglob % SF_BUFS;
+                    if (!mbar_wait(sf_full(buf), (kglob / SF_BUFS) & 1u, p.timeout_ns, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfa_t = tmem_base + SF_COL + SF_BUF * buf;
                     const uint32_t sfb_t = sfa_t + 16;
-                    const uint32_t sa = smem_u32(smem + SFA_OFF + stage * SFA_STAGE);
-                    const uint32_t sb = smem_u32(smem + SFB_OFF + stage * SFB_STAGE);
+                    const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + L::A_OFF + stage * L::A_STAGE));
+                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + L::B_OFF + stage * L::B_STAGE));
 #pragma unroll
                     for (int c = 0; c < KCH; ++c) {
                         if (c < nk) {
-                            sf_copy(sfa_t + 4 * c, sf_atom_desc(sa + c * ATOM));
-                            sf_copy(sfb_t + 8 * c, sf_atom_desc(sb + c * ATOM));
-                            sf_copy(sfb_t + 8 * c + 4, sf_atom_desc(sb + (KCH + c) * ATOM));
+                            const uint32_t acc = (kb > 0 || c > 0) ? 1u : 0u;
+                            if constexpr (CTAS == 2)
+                                mma_nvf4_pair(tmem_base, adesc + 2 * c, bdesc + 2 * c, L::IDESC, sfa_t + 4 * c,
+                                              sfb_t + 8 * c, acc);
+                            else
+                                mma_nvf4(tmem_base, adesc + 2 * c, bdesc + 2 * c, L::IDESC, sfa_t + 4 * c,
+                                         sfb_t + 8 * c, acc);
                         }
                     }
-                    const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + A_OFF + stage * A_STAGE));
-                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + B_OFF + stage * B_STAGE));
-#pragma unroll
-                    for (int c = 0; c < KCH; ++c) {
-                        if (c < nk)
-                            mma_nvf4(tmem_base, adesc + 2 * c, bdesc + 2 * c, IDESC, sfa_t + 4 * c,
-                                     sfb_t + 8 * c, (kb > 0 || c > 0) ? 1u : 0u);
+                    if constexpr (CTAS == 2) {
+                        mma_commit_pair_mc(empty(stage), 0x3);
+                        mma_commit_pair(sf_empty(buf));
+                    } else {
+                        mma_commit(empty(stage));
+                        mma_commit(sf_empty(buf));
                     }
-                    mma_commit(empty(stage));
                     ++kglob;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -708,11 +802,67 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     *abort_flag = 1;
                     break;
                 }
-                mma_commit(tfull);
+                if constexpr (CTAS == 2) mma_commit_pair_mc(tfull, 0x3);
+                else mma_commit(tfull);
                 acc_phase ^= 1u;
             }
-            mma_commit(drain);
+            if constexpr (CTAS == 2) mma_commit_pair(drain);
+            else mma_commit(drain);
             mbar_wait(drain, 0, p.timeout_ns, p.status);
+        }
+    } else if (warp >= SCALE_WARP) {
+        const int part = warp - SCALE_WARP;   // chunks [part * KCH / SCALE_WARPS, ...)
+        if (lane == 0 && leader) {
+            // ------------------------------------------------- scale-factor copies
+            // Each stage's scale atoms go into the next TMEM scale buffer as
+            // soon as the stage has landed and the buffer's previous MMAs are
+            // done, so that the copies overlap the MMA thread's work.
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t kglob = 0;
+            for (int t = first; t < sc.total && !*abort_flag; t += stride) {
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    const uint32_t buf = kglob % SF_BUFS;
+                    if (!mbar_wait(full(stage), phase, p.timeout_ns, p.status) ||
+                        !mbar_wait(sf_empty(buf), ((kglob / SF_BUFS) & 1u) ^ 1u, p.timeout_ns, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nk = min(KCH, kch_total - kb * KCH);
+                    const uint32_t sfa_t = tmem_base + SF_COL + SF_BUF * buf;
+                    const uint32_t sfb_t = sfa_t + 16;
+                    const uint32_t sa = smem_u32(smem + L::SFA_OFF + stage * SFA_STAGE);
+                    const uint32_t sb = smem_u32(smem + L::SFB_OFF + stage * SFB_STAGE);
+#pragma unroll
+                    for (int c = 0; c < KCH; ++c) {
+                        if (c < nk && c / (KCH / SCALE_WARPS) == part) {
+                            if constexpr (CTAS == 2) {
+                                sf_copy_pair(sfa_t + 4 * c, sf_atom_desc(sa + c * ATOM));
+                                sf_copy_pair(sfb_t + 8 * c, sf_atom_desc(sb + c * ATOM));
+                                sf_copy_pair(sfb_t + 8 * c + 4, sf_atom_desc(sb + (KCH + c) * ATOM));
+                            } else {
+                                sf_copy(sfa_t + 4 * c, sf_atom_desc(sa + c * ATOM));
+                                sf_copy(sfb_t + 8 * c, sf_atom_desc(sb + c * ATOM));
+                                sf_copy(sfb_t + 8 * c + 4, sf_atom_desc(sb + (KCH + c) * ATOM));
+                            }
+                        }
+                    }
+                    if constexpr (CTAS == 2) mma_commit_pair(sf_full(buf));
+                    else mma_commit(sf_full(buf));
+                    ++kglob;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) {
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+            // every copy issued by this thread completes before TMEM is released
+            if constexpr (CTAS == 2) mma_commit_pair(sdrain + 8 * part);
+            else mma_commit(sdrain + 8 * part);
+            mbar_wait(sdrain + 8 * part, 0, p.timeout_ns, p.status);
         }
     } else {
         // -------------------------------------------------------------- epilogue
@@ -720,7 +870,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int part = (warp - 2) >> 2;    // columns 64 part .. 64 part + 63
         uint8_t* stg = staging + (warp - 2) * (32 * 64);
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < sc.total && !*abort_flag; t += gridDim.x) {
+        for (int t = first; t < sc.total && !*abort_flag; t += stride) {
             const Tile ti = sc.get(t);
             const int row = ti.a_row0 + q * 32 + lane;
             const float ga = row < ti.row_end ? p.ga[row] : 0.0f;
@@ -739,7 +889,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             // the whole accumulator has been read by this warp: release it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty);
+            if (lane == 0) {
+                if constexpr (CTAS == 2) mbar_arrive_cluster(mapa_shared(tempty, 0));
+                else mbar_arrive(tempty);
+            }
             store_chunk(va, 2 * part, ti, q, lane, ga, gb, stg, p.y, p.N);
             store_chunk(vb, 2 * part + 1, ti, q, lane, ga, gb, stg, p.y, p.N);
             acc_phase ^= 1u;
@@ -748,20 +901,22 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
     __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CTAS == 2) cluster_sync_all(); else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        if constexpr (CTAS == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 
-template <bool GROUPED>
-int prepare_gemm(const DeviceInfo& di, size_t smem) {
+template <int CTAS, bool GROUPED>
+int prepare_gemm(const DeviceInfo& di) {
     static bool done[64];
+    const size_t smem = Lay<CTAS, GROUPED>::BYTES;
     if (static_cast<size_t>(di.max_smem_optin) < smem)
         return fail(METIS_ERR_UNSUPPORTED, "nvfp4 gemm needs %zu bytes of shared memory", smem);
     if (!done[di.device]) {
-        int rc = cuda_check(cudaFuncSetAttribute(nvfp4_gemm_kernel<GROUPED>,
+        int rc = cuda_check(cudaFuncSetAttribute(nvfp4_gemm_kernel<CTAS, GROUPED>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(smem)),
                             "cudaFuncSetAttribute(nvfp4 gemm)");
@@ -771,10 +926,38 @@ int prepare_gemm(const DeviceInfo& di, size_t smem) {
     return METIS_OK;
 }
 
+// Co-resident CTA pairs of the 2-CTA kernel (cached per device).
+template <bool GROUPED>
+int max_pairs(const DeviceInfo& di, int* out) {
+    static int cached[64];
+    if (!cached[di.device]) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (di.num_sms / 2), 1, 1);
+        cfg.blockDim = dim3(THREADS, 1, 1);
+        cfg.dynamicSmemBytes = Lay<2, GROUPED>::BYTES;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<2, GROUPED>, &cfg),
+                            "cudaOccupancyMaxActiveClusters(nvfp4)");
+        if (rc) return rc;
+        if (n < 1) return fail(METIS_ERR_UNSUPPORTED, "no CTA pair of the nvfp4 gemm fits an SM pair");
+        cached[di.device] = n;
+    }
+    *out = cached[di.device];
+    return METIS_OK;
+}
+
 }  // namespace nvfp4
 
 // y = NVFP4 GEMM. a_rows: rows of A's code buffer (a multiple of 128);
 // b_rows: rows of B ([groups * N]). offsets/counts null: dense with M rows.
+// CTA pairs (256-row tiles) for the grouped GEMM and for M > 128.
 // Arguments validated by the caller.
 int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, int64_t a_rows,
                       const uint8_t* qb, const uint8_t* sfb, const float* gb, int64_t b_rows,
@@ -784,13 +967,6 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
-    CUtensorMap ta, tb;
-    if ((rc = make_tmap_2d(&ta, qa, 1, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(a_rows),
-                           static_cast<uint64_t>(K / 2), BKB, ROWS, true)))
-        return rc;
-    if ((rc = make_tmap_2d(&tb, qb, 1, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(b_rows),
-                           static_cast<uint64_t>(K / 2), BKB, BN, true)))
-        return rc;
     GemmParams p{};
     p.sfa = sfa;
     p.ga = ga;
@@ -806,20 +982,47 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
     if ((rc = device_status_word(&p.status))) return rc;
     p.timeout_ns = watchdog_ns();
     const bool grouped = offsets != nullptr;
-    const size_t smem = grouped ? BYTES_GROUPED : BYTES_DENSE;
-    int grid = di.num_sms;
-    if (!grouped) {
-        const int64_t tiles = ((static_cast<int64_t>(M) + ROWS - 1) / ROWS) * ((N + BN - 1) / BN);
-        if (tiles == 0) return METIS_OK;
-        grid = static_cast<int>(tiles < di.num_sms ? tiles : di.num_sms);
+    const bool pair = grouped || M > ROWS;
+    const uint32_t b_box = pair ? BN / 2 : BN;
+    CUtensorMap ta, tb, tsa, tsb;
+    if ((rc = make_tmap_2d(&ta, qa, 1, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(a_rows),
+                           static_cast<uint64_t>(K / 2), BKB, ROWS, true)))
+        return rc;
+    if ((rc = make_tmap_2d(&tb, qb, 1, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(b_rows),
+                           static_cast<uint64_t>(K / 2), BKB, b_box, true)))
+        return rc;
+    // the tiled scales as rows of 256 bytes (two per atom), 4 atoms per box
+    if ((rc = make_tmap_2d(&tsa, sfa, 1, SF_ROW, static_cast<uint64_t>(a_rows) * (K / 16) / SF_ROW, SF_ROW,
+                           SF_ROW, KCH * ATOM / SF_ROW, false)))
+        return rc;
+    if ((rc = make_tmap_2d(&tsb, sfb, 1, SF_ROW, static_cast<uint64_t>(b_rows) * (K / 16) / SF_ROW, SF_ROW,
+                           SF_ROW, KCH * ATOM / SF_ROW, false)))
+        return rc;
+    if (pair) {
+        int pairs = 0;
+        int clusters = 0;
+        if (grouped) {
+            if ((rc = prepare_gemm<2, true>(di))) return rc;
+            if ((rc = max_pairs<true>(di, &pairs))) return rc;
+            clusters = pairs;
+            return cuda_check(launch_pdl(nvfp4_gemm_kernel<2, true>, dim3(2 * clusters), dim3(THREADS),
+                                         Lay<2, true>::BYTES, st, 2, ta, tb, tsa, tsb, p),
+                              "nvfp4 grouped gemm (CTA pair) launch");
+        }
+        if ((rc = prepare_gemm<2, false>(di))) return rc;
+        if ((rc = max_pairs<false>(di, &pairs))) return rc;
+        const int64_t tiles = ((static_cast<int64_t>(M) + 2 * ROWS - 1) / (2 * ROWS)) * ((N + BN - 1) / BN);
+        clusters = static_cast<int>(tiles < pairs ? tiles : pairs);
+        return cuda_check(launch_pdl(nvfp4_gemm_kernel<2, false>, dim3(2 * clusters), dim3(THREADS),
+                                     Lay<2, false>::BYTES, st, 2, ta, tb, tsa, tsb, p),
+                          "nvfp4 gemm (CTA pair) launch");
     }
-    if (grouped) {
-        if ((rc = prepare_gemm<true>(di, smem))) return rc;
-        return cuda_check(launch_pdl(nvfp4_gemm_kernel<true>, dim3(grid), dim3(THREADS), smem, st, 1, ta, tb, p),
-                          "nvfp4 grouped gemm launch");
-    }
-    if ((rc = prepare_gemm<false>(di, smem))) return rc;
-    return cuda_check(launch_pdl(nvfp4_gemm_kernel<false>, dim3(grid), dim3(THREADS), smem, st, 1, ta, tb, p),
+    const int64_t tiles = ((static_cast<int64_t>(M) + ROWS - 1) / ROWS) * ((N + BN - 1) / BN);
+    if (tiles == 0) return METIS_OK;
+    const int grid = static_cast<int>(tiles < di.num_sms ? tiles : di.num_sms);
+    if ((rc = prepare_gemm<1, false>(di))) return rc;
+    return cuda_check(launch_pdl(nvfp4_gemm_kernel<1, false>, dim3(grid), dim3(THREADS), Lay<1, false>::BYTES,
+                                 st, 1, ta, tb, tsa, tsb, p),
                       "nvfp4 gemm launch");
 }
 
