@@ -131,7 +131,16 @@ struct QuantArgs {
 // reads it twice (amax pass, then codes).
 template <typename T, int NBL>
 __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArgs a) {
+    static_assert(QWARPS * 32 == 256, "one thread per E4M3 code builds the reciprocal table");
     static_assert(NBL == 0 || sizeof(T) == 2, "register-resident rows are BF16");
+    // 1 / D(code) for every E4M3 block-scale code (0 for a zero scale): the
+    // same IEEE division, once per code instead of once per block
+    __shared__ float inv_scale[256];
+    {
+        const float d = e4m3_to_f32(threadIdx.x);
+        inv_scale[threadIdx.x] = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+    }
+    __syncthreads();
     grid_dependency_wait();  // the rows may be the previous kernel's output
     grid_launch_dependents();
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -209,8 +218,7 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
 #pragma unroll
             for (int i = 0; i < 16; ++i) bm = fmaxf(bm, fabsf(v[i]));
             sbc = f32x2_to_e4m3x2(__fdiv_rn(__fmul_rn(bm, inv_g), 6.0f), 0.0f) & 0xFFu;
-            const float ds = e4m3_to_f32(sbc);
-            const float inv_s = ds > 0.0f ? __fdiv_rn(1.0f, ds) : 0.0f;
+            const float inv_s = inv_scale[sbc];
             float w[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) w[i] = __fmul_rn(__fmul_rn(v[i], inv_g), inv_s);

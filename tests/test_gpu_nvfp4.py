@@ -96,6 +96,25 @@ def test_quant_nvfp4_extremes(metis):
     assert_bytes_equal(oracle.e2m1_unpack(q), qr, "codes")
 
 
+def test_quant_nvfp4_strided_rows(metis):
+    """Rows with a leading dimension larger than K (BF16 and FP32)."""
+    R, K, pad = 37, 320, 64
+    d = synth.linear(9, R, K, 8, row_magnitude_log10=(-2, 2))
+    qr, sr, gr = oracle.nvfp4_quant(d["x"], per_row=True)
+    big = np.zeros((R, K + pad), dtype=np.uint16)
+    big[:, :K] = d["x"]
+    q, sf, g = _quant_gpu(metis, bf16_dev(big)[:, :K])
+    assert_bytes_equal(g.view(np.uint32), gr.view(np.uint32), "global scales (BF16)")
+    assert_bytes_equal(sf.reshape(R, K // 16), sr, "block scales (BF16)")
+    assert_bytes_equal(oracle.e2m1_unpack(q), qr, "codes (BF16)")
+    f = oracle.bf16_to_float(d["x"])
+    bigf = np.zeros((R, K + pad), dtype=np.float32)
+    bigf[:, :K] = f
+    q, sf, g = _quant_gpu(metis, dev(bigf)[:, :K])
+    assert_bytes_equal(oracle.e2m1_unpack(q), qr, "codes (FP32)")
+    assert_bytes_equal(g.view(np.uint32), gr.view(np.uint32), "global scales (FP32)")
+
+
 @pytest.mark.parametrize("E,N,K,seed", [(3, 128, 256, 7), (2, 384, 2048, 8)])
 def test_quant_nvfp4_weight_sets_tiled(metis, E, N, K, seed):
     """FP32 expert weights [E*N, K], one global scale per expert, tiled scales."""
