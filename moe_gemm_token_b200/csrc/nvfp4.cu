@@ -126,53 +126,16 @@ struct QuantArgs {
     int64_t pad_rows;         // tiled, no gather: rows [R, pad_rows) get zero scales
 };
 
-// NBL > 0 (BF16 rows with K <= 512 NBL): lane l keeps blocks l, l + 32, ...
-// of the row in registers, so the row is read from memory once; NBL = 0
-// reads it twice (amax pass, then codes).
+// One row's quantization by one warp. NBL > 0 (BF16 rows with K <= 512 NBL):
+// the row is already in registers, lane l holding blocks l, l + 32, ... in
+// raw; NBL = 0 reads it twice (amax pass, then codes).
 template <typename T, int NBL>
-__global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArgs a) {
-    static_assert(QWARPS * 32 == 256, "one thread per E4M3 code builds the reciprocal table");
-    static_assert(NBL == 0 || sizeof(T) == 2, "register-resident rows are BF16");
-    // 1 / D(code) for every E4M3 block-scale code (0 for a zero scale): the
-    // same IEEE division, once per code instead of once per block
-    __shared__ float inv_scale[256];
-    {
-        const float d = e4m3_to_f32(threadIdx.x);
-        inv_scale[threadIdx.x] = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
-    }
-    __syncthreads();
-    grid_dependency_wait();  // the rows may be the previous kernel's output
-    grid_launch_dependents();
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t r = static_cast<int64_t>(blockIdx.x) * QWARPS + warp;
-    const int64_t kc = a.K / 64;
-    if (r >= a.R) {
-        // zero scales for the pad rows of the last 128-row atom
-        if (a.tiled && r < a.pad_rows) {
-            for (int64_t c = lane; c < kc; c += 32)
-                *reinterpret_cast<uint32_t*>(a.sf + tiled_sf_offset(r, c, kc)) = 0u;
-        }
-        return;
-    }
-    if (a.nrows && r >= *a.nrows) return;
-    if (a.row_valid && a.row_valid[r] < 0) return;
+__device__ __forceinline__ void quant_row(const QuantArgs& a, int64_t r, int lane,
+                                          const uint4 (&raw)[NBL > 0 ? NBL : 1][2],
+                                          const float* inv_scale) {
     const T* row = static_cast<const T*>(a.x) + r * a.ldx;
     const int nb = static_cast<int>(a.K / 16);
-    uint4 raw[NBL > 0 ? NBL : 1][2];
-    if constexpr (NBL > 0) {
-#pragma unroll
-        for (int i = 0; i < NBL; ++i) {
-            const int b = lane + 32 * i;
-            if (b < nb) {
-                raw[i][0] = ld_nc_v4(row + 16 * b);
-                raw[i][1] = ld_nc_v4(row + 16 * b + 8);
-            } else {
-                raw[i][0] = raw[i][1] = make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-    } else {
-        raw[0][0] = raw[0][1] = make_uint4(0u, 0u, 0u, 0u);  // unused
-    }
+    const int64_t kc = a.K / 64;
     auto unpack = [&](int i, float (&v)[16]) {
         const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
                                raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
@@ -182,6 +145,22 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
             v[2 * h + 1] = bf16_hi(w[h]);
         }
     };
+    // register-resident rows: each block's maximum, taken once for both the
+    // row amax and the block scale
+    float bmax[NBL > 0 ? NBL : 1];
+    if constexpr (NBL > 0) {
+#pragma unroll
+        for (int i = 0; i < NBL; ++i) {
+            float v[16];
+            unpack(i, v);
+            float bm = 0.0f;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) bm = fmaxf(bm, fabsf(v[h]));
+            bmax[i] = bm;
+        }
+    } else {
+        bmax[0] = 0.0f;
+    }
     float amax;
     if (a.gamax) {
         amax = a.gamax[r / a.rps];
@@ -189,12 +168,7 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
         float m = 0.0f;
         if constexpr (NBL > 0) {
 #pragma unroll
-            for (int i = 0; i < NBL; ++i) {
-                float v[16];
-                unpack(i, v);
-#pragma unroll
-                for (int h = 0; h < 16; ++h) m = fmaxf(m, fabsf(v[h]));
-            }
+            for (int i = 0; i < NBL; ++i) m = fmaxf(m, bmax[i]);
         } else {
             for (int b = lane; b < nb; b += 32) {
                 float v[16];
@@ -210,13 +184,11 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
     const float inv_g = amax > 0.0f ? fminf(__fdiv_rn(2688.0f, amax), 3.402823466e38f) : 0.0f;
     const int ndst = a.dst_rows ? a.topk : 1;
     // one pass over 32 blocks (512 elements); v holds this lane's block b0 + lane
-    auto block_pass = [&](int b0, const float (&v)[16]) {
+    // and bm its maximum magnitude
+    auto block_pass = [&](int b0, const float (&v)[16], float bm) {
         const int b = b0 + lane;
         uint32_t lo = 0, hi = 0, sbc = 0;
         if (b < nb) {
-            float bm = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) bm = fmaxf(bm, fabsf(v[i]));
             sbc = f32x2_to_e4m3x2(__fdiv_rn(__fmul_rn(bm, inv_g), 6.0f), 0.0f) & 0xFFu;
             const float inv_s = inv_scale[sbc];
             float w[16];
@@ -247,7 +219,7 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
             if (32 * i >= nb) break;  // warp-uniform
             float v[16];
             unpack(i, v);
-            block_pass(32 * i, v);
+            block_pass(32 * i, v, bmax[i]);
         }
     } else {
         for (int b0 = 0; b0 < nb; b0 += 32) {
@@ -255,7 +227,70 @@ __global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArg
 #pragma unroll
             for (int h = 0; h < 16; ++h) v[h] = 0.0f;
             if (b0 + lane < nb) load16(row + 16 * (b0 + lane), v);
-            block_pass(b0, v);
+            float bm = 0.0f;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) bm = fmaxf(bm, fabsf(v[h]));
+            block_pass(b0, v, bm);
+        }
+    }
+}
+
+// RPW rows per warp (rows r0 .. r0 + RPW - 1): with NBL > 0 every row's loads
+// are issued before the first row is encoded, so a warp waits on memory once.
+template <typename T, int NBL, int RPW>
+__global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArgs a) {
+    static_assert(QWARPS * 32 == 256, "one thread per E4M3 code builds the reciprocal table");
+    static_assert(NBL == 0 || sizeof(T) == 2, "register-resident rows are BF16");
+    static_assert(NBL > 0 || RPW == 1, "two-pass rows are one per warp");
+    // 1 / D(code) for every E4M3 block-scale code (0 for a zero scale): the
+    // same IEEE division, once per code instead of once per block
+    __shared__ float inv_scale[256];
+    {
+        const float d = e4m3_to_f32(threadIdx.x);
+        inv_scale[threadIdx.x] = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+    }
+    __syncthreads();
+    grid_dependency_wait();  // the rows may be the previous kernel's output
+    grid_launch_dependents();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t r0 = (static_cast<int64_t>(blockIdx.x) * QWARPS + warp) * RPW;
+    const int64_t kc = a.K / 64;
+    const int nb = static_cast<int>(a.K / 16);
+    uint4 raw[RPW][NBL > 0 ? NBL : 1][2];
+    bool live[RPW];
+    // rows below R are inside the buffer: their loads go out before the
+    // validity checks' own loads come back (a skipped row is read, not used)
+#pragma unroll
+    for (int u = 0; u < RPW; ++u) {
+        const int64_t r = r0 + u;
+#pragma unroll
+        for (int i = 0; i < (NBL > 0 ? NBL : 1); ++i) {
+            const int b = lane + 32 * i;
+            if (NBL > 0 && r < a.R && b < nb) {
+                const T* row = static_cast<const T*>(a.x) + r * a.ldx;
+                raw[u][i][0] = ld_nc_v4(row + 16 * b);
+                raw[u][i][1] = ld_nc_v4(row + 16 * b + 8);
+            } else {
+                raw[u][i][0] = raw[u][i][1] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < RPW; ++u) {
+        const int64_t r = r0 + u;
+        live[u] = r < a.R && !(a.nrows && r >= *a.nrows) && !(a.row_valid && a.row_valid[r] < 0);
+    }
+#pragma unroll
+    for (int u = 0; u < RPW; ++u) {
+        const int64_t r = r0 + u;
+        if (r >= a.R) {
+            // zero scales for the pad rows of the last 128-row atom
+            if (a.tiled && r < a.pad_rows) {
+                for (int64_t c = lane; c < kc; c += 32)
+                    *reinterpret_cast<uint32_t*>(a.sf + tiled_sf_offset(r, c, kc)) = 0u;
+            }
+        } else if (live[u]) {
+            quant_row<T, NBL>(a, r, lane, raw[u], inv_scale);
         }
     }
 }
@@ -334,19 +369,20 @@ int launch_nvfp4_quant(const T* x, int64_t R, int64_t K, int64_t ldx, int64_t rp
         a.gamax = g;
     }
     const int64_t rows = a.pad_rows;
-    const dim3 grid(static_cast<unsigned>((rows + QWARPS - 1) / QWARPS));
-    auto go = [&](auto kernel) {
+    auto go = [&](auto kernel, int rpw) {
+        const dim3 grid(static_cast<unsigned>((rows + QWARPS * rpw - 1) / (QWARPS * rpw)));
         return cuda_check(launch_pdl(kernel, grid, dim3(QWARPS * 32), 0, st, 1, a), "nvfp4 quant launch");
     };
-    // BF16 rows of up to 4096 elements stay in registers (one read of x)
+    // BF16 rows of up to 4096 elements stay in registers (one read of x);
+    // rows of up to 1024 go two to a warp
     if constexpr (sizeof(T) == 2) {
-        if (rps == 1 && K <= 512) rc = go(nvfp4_quant_kernel<T, 1>);
-        else if (rps == 1 && K <= 1024) rc = go(nvfp4_quant_kernel<T, 2>);
-        else if (rps == 1 && K <= 2048) rc = go(nvfp4_quant_kernel<T, 4>);
-        else if (rps == 1 && K <= 4096) rc = go(nvfp4_quant_kernel<T, 8>);
-        else rc = go(nvfp4_quant_kernel<T, 0>);
+        if (rps == 1 && K <= 512) rc = go(nvfp4_quant_kernel<T, 1, 2>, 2);
+        else if (rps == 1 && K <= 1024) rc = go(nvfp4_quant_kernel<T, 2, 2>, 2);
+        else if (rps == 1 && K <= 2048) rc = go(nvfp4_quant_kernel<T, 4, 1>, 1);
+        else if (rps == 1 && K <= 4096) rc = go(nvfp4_quant_kernel<T, 8, 1>, 1);
+        else rc = go(nvfp4_quant_kernel<T, 0, 1>, 1);
     } else {
-        rc = go(nvfp4_quant_kernel<T, 0>);
+        rc = go(nvfp4_quant_kernel<T, 0, 1>, 1);
     }
     if (rc) return rc;
     if (rps > 1) {

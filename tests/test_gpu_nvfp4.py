@@ -299,6 +299,14 @@ def test_moe_nvfp4_parity(metis, T, H, I, E, k, seed):
     check_moe4(d, g, up, dn)
 
 
+def test_moe_nvfp4_many_experts(metis):
+    """256 experts (group tables and pad marking at larger E), top-4."""
+    d = synth.moe(seed=19, T=96, H=128, I=128, E=256, topk=4, hot=4, load_ratio=2.0)
+    up, dn = _weights_nvfp4(d["w_up"]), _weights_nvfp4(d["w_down"])
+    g = run_moe4(metis, d, up, dn)
+    check_moe4(d, g, up, dn)
+
+
 def test_moe_nvfp4_empty_experts_and_determinism(metis):
     d = synth.moe(seed=16, T=64, H=128, I=128, E=16, topk=2, hot=0, load_ratio=1.0)
     ids = d["topk_ids"]
