@@ -60,7 +60,7 @@ extern "C" {
 typedef enum {
     METIS_OK = 0,
     METIS_ERR_INVALID_ARG = -1, /* bad pointer, size, alignment or layout */
-    METIS_ERR_UNSUPPORTED = -2, /* valid request this build does not implement */
+    METIS_ERR_UNSUPPORTED = -2, /* valid request the library does not implement */
     METIS_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed */
     METIS_ERR_TIMEOUT = -4      /* a device-side bounded wait ran out */
 } metis_status;
