@@ -27,7 +27,7 @@ def has_cuda():
 
 @pytest.fixture(scope="session")
 def metis():
-    """The CUDA library's Python binding, on a GPU machine only (never a fallback)."""
+    """The CUDA library's Python binding, on a machine with a GPU only (never a fallback)."""
     if not has_cuda():
         pytest.fail("GPU test collected on a machine without CUDA; run with -m 'not gpu'")
     from moe_gemm_token_b200 import metis as m
