@@ -182,3 +182,23 @@ def test_nvfp4_workspace_layout(lib):
     for o, s, nxt in zip(offs, sizes, offs[1:] + [total]):
         assert o + s <= nxt
     assert metis.metis_moe_nvfp4_workspace_offset(12, T, k, E, H, I) == -1
+
+
+def test_shared_expert_host_validation_without_gpu(lib):
+    p = ctypes.c_void_p(0x1000)
+    null = None
+    E = metis.METIS_ERR_INVALID_ARG
+    # BF16 GEMM: N or K not a multiple of 8, misaligned y, M = 0 is a no-op
+    assert lib.metis_bf16_gemm(p, p, p, 4, 12, 16, null) == E
+    assert lib.metis_bf16_gemm(p, p, p, 4, 16, 12, null) == E
+    assert lib.metis_bf16_gemm(p, p, ctypes.c_void_p(0x1008), 4, 16, 16, null) == E
+    assert lib.metis_bf16_gemm(p, p, p, 0, 16, 16, null) == metis.METIS_OK
+    # fused shared combine: topk > 8, H not a multiple of 16, workspace too small
+    need = metis.metis_workspace_size(metis.METIS_OP_SHARED, 8, 64, 128, 2, 0)
+    assert need == 8 * 64 * 2 or need >= 8 * 64 * 2
+    args = lambda T, H, Is, k, ws: (p, T, H, Is, p, p, p, p, p, k, p, p, ws, null)
+    assert lib.metis_moe_shared_fused_combine(*args(8, 128, 64, 9, need)) == E
+    assert lib.metis_moe_shared_fused_combine(*args(8, 120, 64, 2, need)) == E
+    assert lib.metis_moe_shared_fused_combine(*args(8, 128, 64, 2, need - 16)) == E
+    assert b"workspace" in lib.metis_last_error()
+    assert lib.metis_moe_shared_fused_combine(*args(0, 128, 64, 2, 0)) == metis.METIS_OK
