@@ -381,6 +381,18 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                  : "memory");
 }
 
+// Relaxed arrives (no release fence): for handing over tensor-memory state
+// whose accesses are already completed (tcgen05.wait::ld / ::st) and ordered
+// by tcgen05.fence::before_thread_sync, where a release would also wait for
+// the thread's earlier global stores.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
 // TMA load into this CTA's shared memory whose completion is counted on an
 // mbarrier that may live in either CTA of the pair (cta_group::2). No multicast.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, int32_t x,

@@ -931,11 +931,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             tmem_ld_32x32b_x32(tbase + 32, vb);
             tmem_ld_wait();
             // the whole accumulator has been read by this warp: release it
+            // (relaxed: a release would first wait for this warp's stores of
+            // the previous tile, holding up the next tile's MMAs)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if constexpr (CTAS == 2) mbar_arrive_cluster(mapa_shared(tempty, 0));
-                else mbar_arrive(tempty);
+                if constexpr (CTAS == 2) mbar_arrive_cluster_relaxed(mapa_shared(tempty, 0));
+                else mbar_arrive_relaxed(tempty);
             }
             store_chunk(va, 2 * part, ti, q, lane, ga, gb, stg, p.y, p.N);
             store_chunk(vb, 2 * part + 1, ti, q, lane, ga, gb, stg, p.y, p.N);
