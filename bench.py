@@ -555,7 +555,9 @@ def secondary_figures(metis, dev, pk):
             "fused_quant_us": t_f * 1e6, "fused_quant_TFLOP/s": fl / t_f / 1e12}
         del x, xq, b, y
     # the default maths for many tokens: the same 4096-token chain through
-    # W8A16 on the tensor cores (weights widened to BF16), no quantizers
+    # W8A16 (weights widened exactly to BF16), no quantizers. metis_linear
+    # widens each layer's weights into the workspace and runs the BF16
+    # CTA-pair GEMM; metis_w8a16_gemm widens them inside its kernel.
     T, K1, N1 = M_TOK, K_HID, N_FF
     xd = torch.randn(T, K1, device=dev, generator=g).to(torch.bfloat16)
     w1c, w2c = codes(N1, K1), codes(K1, N1)
@@ -563,19 +565,27 @@ def secondary_figures(metis, dev, pk):
     s2c = torch.rand(K1, device=dev, generator=g) * 1e-3
     h1 = torch.empty(T, N1, dtype=torch.bfloat16, device=dev)
     h2 = torch.empty(T, K1, dtype=torch.bfloat16, device=dev)
+    wsw = torch.empty(metis.metis_workspace_size(metis.METIS_OP_W8A16_WIDENED, T, N1, K1),
+                      dtype=torch.uint8, device=dev)
 
     def chain16():
+        metis.metis_linear(xd, w1c, s1c, h1, fast_math=False, workspace=wsw)
+        metis.metis_linear(h1, w2c, s2c, h2, fast_math=False, workspace=wsw)
+
+    def chain16_in_kernel():
         metis.metis_w8a16_gemm(xd, w1c, s1c, h1)
         metis.metis_w8a16_gemm(h1, w2c, s2c, h2)
     t = timeit(chain16, 10)
-    t1 = timeit(lambda: metis.metis_w8a16_gemm(xd, w1c, s1c, h1), 10)
+    t1 = timeit(lambda: metis.metis_linear(xd, w1c, s1c, h1, fast_math=False, workspace=wsw), 10)
+    t_in = timeit(chain16_in_kernel, 10)
     fl = 2 * T * K1 * N1
     peak16 = pk["bf16_tflops"]
     out["prefill_default_maths_4096tok"] = {
         "us": t * 1e6, "tok/s": T / t, "TFLOP/s": 2 * fl / t / 1e12,
         "frac_of_bf16_peak": 2 * fl / t / 1e12 / peak16,
-        "layer1_us": t1 * 1e6, "layer1_TFLOP/s": fl / t1 / 1e12}
-    del xd, w1c, w2c, h1, h2
+        "layer1_us": t1 * 1e6, "layer1_TFLOP/s": fl / t1 / 1e12,
+        "in_kernel_widening_us": t_in * 1e6, "in_kernel_widening_TFLOP/s": 2 * fl / t_in / 1e12}
+    del xd, w1c, w2c, h1, h2, wsw
     # routed experts: 4096 tokens, hidden 2048, latent 1024, 64 experts, top-8
     T, H, I, E, k = 4096, 2048, 1024, 64, 8
     x = torch.randn(T, H, device=dev, generator=g).to(torch.bfloat16)

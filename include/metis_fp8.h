@@ -153,6 +153,21 @@ METIS_API int metis_fp8_gemm(const void* a, int a_kind, float* s_tok, const uint
 METIS_API int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
                      int64_t M, int64_t N, int64_t K, metis_stream_t stream);
 
+/* The same default maths for many tokens through a workspace: the weights are
+ * first widened exactly to BF16 [N, K] in `workspace` by an HBM-bound pass
+ * (E4M3 NaN codes widen to NaN), then multiplied by the BF16 CTA-pair
+ * tensor-core GEMM with s_w applied to the FP32 sum in its epilogue:
+ *   y[m, n] = bf16_rn( fl32( s_w[n] * sum_k x[m, k] * D(wq[n, k]) ) ).
+ * Faster than metis_w8a16_gemm's in-kernel widening once the token count
+ * amortises the pass (metis_linear uses it for M >= 512).
+ *   workspace: metis_workspace_size(METIS_OP_W8A16_WIDENED, M, N, K, 0, 0)
+ *   bytes, 16-byte aligned; overwritten.
+ *   Requires K % 16 == 0, K >= 16, N % 8 == 0, N >= 8, M >= 0; x, wq, y
+ *   16-byte aligned, s_w 4-byte aligned. */
+METIS_API int metis_w8a16_gemm_widened(const void* x_bf16, const uint8_t* wq, const float* s_w,
+                                       void* y_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
+                                       size_t ws_bytes, metis_stream_t stream);
+
 /* Router top-k feeding the routed-expert layer. The cards keep "the routers
  * and their balance bias" in FP32 and route each token to a few experts
  * ("Lernex/Metis-1.6-Logos-FP8", "What is in FP8"; four per token in
@@ -252,6 +267,8 @@ METIS_API int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int6
  *   METIS_OP_FP8_GEMM_FUSED: (M, N, K) of metis_fp8_gemm with a_kind = METIS_A_BF16.
  *   METIS_OP_MOE:            (T, I, H, topk, E) of metis_moe_fp8_grouped_gemm.
  *   METIS_OP_LINEAR:         (M, N, K) of metis_linear with fast_math != 0.
+ *   METIS_OP_W8A16_WIDENED:  (M, N, K) of metis_w8a16_gemm_widened, and of
+ *                            metis_linear's default maths for many tokens.
  *   Other ops need none (0). Returns 0 for invalid arguments. */
 #define METIS_OP_FP8_GEMM 0
 #define METIS_OP_FP8_GEMM_FUSED 1
@@ -259,6 +276,7 @@ METIS_API int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int6
 #define METIS_OP_MOE 3
 #define METIS_OP_LINEAR 4
 #define METIS_OP_SHARED 6       /* metis_moe_shared_fused_combine: (T, I_s, H, topk, 0) */
+#define METIS_OP_W8A16_WIDENED 7 /* metis_w8a16_gemm_widened: 2 * N * K bytes */
 METIS_API size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, int64_t K_or_H,
                             int64_t topk, int64_t E);
 
@@ -293,10 +311,14 @@ METIS_API int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk
  * (metis_w8a16_gemm); more tokens take the fast-math W8A8 path when
  * fast_math != 0 (metis_quant_fp8_per_token into the workspace, then
  * metis_fp8_gemm with a_kind = METIS_A_E4M3), and the default maths
- * (metis_w8a16_gemm, tensor-core path) otherwise.
+ * otherwise.
  * s_tok [M] receives the per-token scales on the fast-math path; `workspace`
  * holds the E4M3 codes: metis_workspace_size(METIS_OP_LINEAR, M, N, K, 0, 0)
- * bytes, 16-byte aligned (0 for M <= 8). */
+ * bytes, 16-byte aligned (0 for M <= 8).
+ * Default maths with M >= 512: when `workspace` (16-byte aligned) holds
+ * metis_workspace_size(METIS_OP_W8A16_WIDENED, M, N, K, 0, 0) bytes,
+ * metis_w8a16_gemm_widened runs; otherwise metis_w8a16_gemm (in-kernel
+ * widening). Both compute the same products with FP32 accumulation. */
 METIS_API int metis_linear(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
                  int64_t M, int64_t N, int64_t K, int fast_math, float* s_tok,
                  void* workspace, size_t ws_bytes, metis_stream_t stream);

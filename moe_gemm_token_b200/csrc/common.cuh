@@ -79,11 +79,16 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
                       __nv_bfloat16* y, const int32_t* offsets, const int32_t* counts, int E, int M,
                       int N, int K, cudaStream_t st);
 
-// BF16 GEMM y = bf16(a b^T) (gemm_fp8.cu); o non-null fuses the routed
-// combine: y[t] = bf16(bf16(a b^T)[t] + sum_j topk_w[t*topk+j] o[s2r[t*topk+j]]).
+// BF16 GEMM y = bf16(a b^T) (gemm_fp8.cu); s_b non-null scales column n:
+// y = bf16(fl32((a b^T)[., n] * s_b[n])); o non-null fuses the routed combine:
+// y[t] = bf16(bf16(a b^T)[t] + sum_j topk_w[t*topk+j] o[s2r[t*topk+j]]).
 int launch_bf16_gemm(const __nv_bfloat16* a, const __nv_bfloat16* b, __nv_bfloat16* y, int M, int N,
-                     int K, const __nv_bfloat16* o, const int32_t* s2r, const float* topk_w, int topk,
-                     cudaStream_t st);
+                     int K, const float* s_b, const __nv_bfloat16* o, const int32_t* s2r,
+                     const float* topk_w, int topk, cudaStream_t st);
+
+// Exact E4M3 -> BF16 widening of n bytes (w16_gemm.cu); n a multiple of 16,
+// both buffers 16-byte aligned.
+int launch_widen_e4m3(const uint8_t* w, __nv_bfloat16* out, int64_t n, cudaStream_t st);
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -480,6 +485,50 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// Four E4M3 bytes -> two BF16 pairs (bytes 0,1 and 2,3), exactly. The byte
+// s.eeee.mmm is placed in a BF16 as s | eeee.mmm << 4, which for e > 0 is
+// 2^(e-127) (1 + m/8) and for e = 0 the BF16 subnormal m/8 * 2^-126; one
+// BF16 multiply by 2^120 (exact; subnormal inputs are kept) gives the E4M3
+// value, 2^(e-7) (1 + m/8) or m * 2^-9. prmt's sign-replicating selectors
+// put each byte's sign in bit 15 of its half. NaN codes (e = 15, m = 7) come
+// out as +-480 here; widen_e4m3x16 repairs them.
+__device__ __forceinline__ void widen_e4m3x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    uint32_t p0, p1;
+    asm("prmt.b32 %0, %1, 0, 0x9180;" : "=r"(p0) : "r"(w));
+    asm("prmt.b32 %0, %1, 0, 0xB3A2;" : "=r"(p1) : "r"(w));
+    const uint32_t u0 = (p0 << 4) & 0x87F087F0u;
+    const uint32_t u1 = (p1 << 4) & 0x87F087F0u;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(u0), "r"(0x7B807B80u));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(u1), "r"(0x7B807B80u));
+}
+
+// Sixteen E4M3 bytes -> eight BF16 pairs, element 2i in the low half of o[i].
+// A byte whose low 7 bits are all set (E4M3 NaN) becomes a BF16 NaN of the
+// same sign.
+__device__ __forceinline__ void widen_e4m3x16(const uint4& v, uint32_t (&o)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) widen_e4m3x4(w[i], o[2 * i], o[2 * i + 1]);
+    // 0x80 in every byte whose low 7 bits are 0x7F (no carry crosses a byte)
+    uint32_t nan = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) nan |= (w[i] & 0x7F7F7F7Fu) + 0x01010101u;
+    if (nan & 0x80808080u) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t byte = (w[i] >> (8 * b)) & 0xFFu;
+                if ((byte & 0x7Fu) == 0x7Fu) {
+                    uint32_t& word = o[2 * i + (b >> 1)];
+                    const int sh = 16 * (b & 1);
+                    word = (word & ~(0xFFFFu << sh)) | (((byte << 8) | 0x7FC0u) << sh);
+                }
+            }
+        }
+    }
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -196,16 +196,25 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// The W16 epilogue chunk: y = bf16(acc), staged as above; with the fused
-// combine each 8-column piece then gets the token's routed outputs added,
+// The W16 epilogue chunk: y = bf16(acc), or bf16(acc * sw[n]) with per-column
+// scales (SCALED), staged as above; without scales the fused
+// combine may then add the token's routed outputs to each 8-column piece,
 // y = bf16(s + sum_j w_j o_j) in FP32, j ascending. Two rows are handled at
 // a time, so 2 * topk loads are in flight per lane.
+template <bool SCALED>
 __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, const Tile& ti, int q,
-                                                int lane, uint8_t* stg, const int2* cb,
+                                                int lane, const float* sw, uint8_t* stg, const int2* cb,
                                                 const Params& p) {
     uint32_t pk[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+    for (int j = 0; j < 16; ++j) {
+        float lo = __uint_as_float(v[2 * j]), hi = __uint_as_float(v[2 * j + 1]);
+        if constexpr (SCALED) {
+            lo = __fmul_rn(lo, sw[c * 32 + 2 * j]);
+            hi = __fmul_rn(hi, sw[c * 32 + 2 * j + 1]);
+        }
+        pk[j] = pack_bf16x2(lo, hi);
+    }
     __syncwarp();
 #pragma unroll
     for (int pc = 0; pc < 4; ++pc)
@@ -224,7 +233,7 @@ __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, 
             val[u] = *reinterpret_cast<const uint4*>(stg + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
             live[u] = ti.a_row0 + q * 32 + rr < ti.row_end && n < p.N;
         }
-        if (p.o != nullptr) {
+        if (!SCALED && p.o != nullptr) {
             // every load of both rows before the first add (the (row, weight)
             // pairs are read from shared memory where they are used)
 #pragma unroll
@@ -273,7 +282,7 @@ __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, 
     }
 }
 
-template <int CTAS, bool GROUPED, bool ABF16, int BN, bool W16 = false>
+template <int CTAS, bool GROUPED, bool ABF16, int BN, bool W16 = false, bool SCALED = false>
 __global__ void __launch_bounds__(Layout<CTAS, ABF16, BN, W16>::THREADS_, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
@@ -602,8 +611,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const Tile ti = sc.get(t);
             const int2* cb = comb + (warp - 2) * 32 * COMB_K;
             if constexpr (W16) {
-                // the fused combine's (row, weight) pairs of this warp's 32 rows
-                if (p.o != nullptr) {
+                if constexpr (SCALED) {
+                    // per-column scales (the default maths' s_w)
+                    if (et < BN / 2) {
+                        const int n = ti.n0 + 2 * et;
+                        sw_smem[acc * BN + 2 * et] = n < p.N ? p.s_b[n] : 0.0f;
+                        sw_smem[acc * BN + 2 * et + 1] = n + 1 < p.N ? p.s_b[n + 1] : 0.0f;
+                    }
+                } else if (p.o != nullptr) {
+                    // the fused combine's (row, weight) pairs of this warp's 32 rows
                     const int row = ti.a_row0 + q * 32 + lane;
                     int2* mine = comb + ((warp - 2) * 32 + lane) * COMB_K;
                     // this warp's columns of the routed rows go to L2 now, while
@@ -660,7 +676,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         else mbar_arrive(tempty(acc));
                     }
                 }
-                if constexpr (W16) store_chunk_w16(cur, c0 + i, ti, q, lane, stg, cb, p);
+                if constexpr (W16) store_chunk_w16<SCALED>(cur, c0 + i, ti, q, lane, sw, stg, cb, p);
                 else store_chunk(cur, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N);
                 if (i + 1 < CPW) tmem_ld_wait();
             }
@@ -679,13 +695,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
 }
 
-template <int CTAS, bool GROUPED, bool ABF16 = false, int BN = BN_MAX, bool W16 = false>
+template <int CTAS, bool GROUPED, bool ABF16 = false, int BN = BN_MAX, bool W16 = false, bool SCALED = false>
 int prepare(const DeviceInfo& di, size_t smem) {
     static bool done[64];
     if (static_cast<size_t>(di.max_smem_optin) < smem)
         return fail(METIS_ERR_UNSUPPORTED, "fp8 gemm needs %zu bytes of shared memory", smem);
     if (!done[di.device]) {
-        int rc = cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED, ABF16, BN, W16>,
+        int rc = cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED, ABF16, BN, W16, SCALED>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(smem)),
                             "cudaFuncSetAttribute(fp8 gemm)");
@@ -696,7 +712,7 @@ int prepare(const DeviceInfo& di, size_t smem) {
 }
 
 // Co-resident CTA pairs of the 2-CTA kernel (cached per device).
-template <bool ABF16 = false, int BN = BN_MAX, bool GROUPED = false, bool W16 = false>
+template <bool ABF16 = false, int BN = BN_MAX, bool GROUPED = false, bool W16 = false, bool SCALED = false>
 int max_pairs(const DeviceInfo& di, int* out) {
     static int cached[64];
     if (!cached[di.device]) {
@@ -713,7 +729,7 @@ int max_pairs(const DeviceInfo& di, int* out) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, GROUPED, ABF16, BN, W16>, &cfg),
+        int rc = cuda_check(cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<2, GROUPED, ABF16, BN, W16, SCALED>, &cfg),
                             "cudaOccupancyMaxActiveClusters");
         if (rc) return rc;
         if (n < 1) return fail(METIS_ERR_UNSUPPORTED, "no CTA pair of the fp8 gemm fits an SM pair");
@@ -852,40 +868,53 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
 // BF16 x BF16 GEMM y = bf16(a b^T) on the tcgen05 pipeline (CTA pairs for
 // M > 128), optionally with the routed combine fused into the epilogue (o
 // non-null). Arguments validated by the caller.
+namespace gemm {
+
+template <bool SCALED>
+int launch_w16(const __nv_bfloat16* a, const __nv_bfloat16* b, const Params& p, int M, int N, int K,
+               const DeviceInfo& di, cudaStream_t st) {
+    int rc;
+    const int num_n = (N + BN_MAX - 1) / BN_MAX;
+    CUtensorMap ta, tb;
+    if ((rc = make_tmap_2d(&ta, a, 2, K, M, static_cast<uint64_t>(K) * 2, BK / 2, ROWS, true))) return rc;
+    if (M > ROWS) {
+        using L = Layout<2, false, BN_MAX, true>;
+        if ((rc = prepare<2, false, false, BN_MAX, true, SCALED>(di, L::BYTES_DENSE))) return rc;
+        int pairs = 0;
+        if ((rc = max_pairs<false, BN_MAX, false, true, SCALED>(di, &pairs))) return rc;
+        if ((rc = make_tmap_2d(&tb, b, 2, K, N, static_cast<uint64_t>(K) * 2, BK / 2, L::B_ROWS, true)))
+            return rc;
+        const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
+        const int clusters = tiles < pairs ? tiles : pairs;
+        return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, false, BN_MAX, true, SCALED>, dim3(2 * clusters),
+                                     dim3(L::THREADS_), L::BYTES_DENSE, st, 2, ta, tb, p),
+                          "bf16 gemm (CTA pair) launch");
+    }
+    using L = Layout<1, false, BN_MAX, true>;
+    if ((rc = prepare<1, false, false, BN_MAX, true, SCALED>(di, L::BYTES_DENSE))) return rc;
+    if ((rc = make_tmap_2d(&tb, b, 2, K, N, static_cast<uint64_t>(K) * 2, BK / 2, L::B_ROWS, true))) return rc;
+    const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
+    const int grid = tiles < di.num_sms ? tiles : di.num_sms;
+    return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, false, BN_MAX, true, SCALED>, dim3(grid),
+                                 dim3(L::THREADS_), L::BYTES_DENSE, st, 1, ta, tb, p),
+                      "bf16 gemm launch");
+}
+
+}  // namespace gemm
+
 int launch_bf16_gemm(const __nv_bfloat16* a, const __nv_bfloat16* b, __nv_bfloat16* y, int M, int N,
-                     int K, const __nv_bfloat16* o, const int32_t* s2r, const float* topk_w, int topk,
-                     cudaStream_t st) {
+                     int K, const float* s_b, const __nv_bfloat16* o, const int32_t* s2r, const float* topk_w,
+                     int topk, cudaStream_t st) {
     using namespace gemm;
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
-    Params p{nullptr, nullptr, nullptr, y, nullptr, M, N, K, 1, status, watchdog_ns(), o, s2r, topk_w, topk};
-    const int num_n = (N + BN_MAX - 1) / BN_MAX;
-    CUtensorMap ta, tb;
-    if ((rc = make_tmap_2d(&ta, a, 2, K, M, static_cast<uint64_t>(K) * 2, BK / 2, ROWS, true))) return rc;
-    if (M > ROWS) {
-        using L = Layout<2, false, BN_MAX, true>;
-        if ((rc = prepare<2, false, false, BN_MAX, true>(di, L::BYTES_DENSE))) return rc;
-        int pairs = 0;
-        if ((rc = max_pairs<false, BN_MAX, false, true>(di, &pairs))) return rc;
-        if ((rc = make_tmap_2d(&tb, b, 2, K, N, static_cast<uint64_t>(K) * 2, BK / 2, L::B_ROWS, true)))
-            return rc;
-        const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
-        const int clusters = tiles < pairs ? tiles : pairs;
-        return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, false, BN_MAX, true>, dim3(2 * clusters),
-                                     dim3(L::THREADS_), L::BYTES_DENSE, st, 2, ta, tb, p),
-                          "bf16 gemm (CTA pair) launch");
-    }
-    using L = Layout<1, false, BN_MAX, true>;
-    if ((rc = prepare<1, false, false, BN_MAX, true>(di, L::BYTES_DENSE))) return rc;
-    if ((rc = make_tmap_2d(&tb, b, 2, K, N, static_cast<uint64_t>(K) * 2, BK / 2, L::B_ROWS, true))) return rc;
-    const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
-    const int grid = tiles < di.num_sms ? tiles : di.num_sms;
-    return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, false, BN_MAX, true>, dim3(grid), dim3(L::THREADS_),
-                                 L::BYTES_DENSE, st, 1, ta, tb, p),
-                      "bf16 gemm launch");
+    if (s_b != nullptr && o != nullptr)
+        return fail(METIS_ERR_INVALID_ARG, "bf16 gemm: per-column scales and the fused combine are exclusive");
+    Params p{nullptr, nullptr, s_b, y, nullptr, M, N, K, 1, status, watchdog_ns(), o, s2r, topk_w, topk};
+    return s_b != nullptr ? launch_w16<true>(a, b, p, M, N, K, di, st) : launch_w16<false>(a, b, p, M, N, K, di, st);
 }
 
 }  // namespace metis
@@ -905,7 +934,8 @@ extern "C" int metis_bf16_gemm(const void* x_bf16, const void* w_bf16, void* y_b
         return fail(METIS_ERR_INVALID_ARG, "bf16_gemm: x, w and y must be 16-byte aligned");
     return launch_bf16_gemm(static_cast<const __nv_bfloat16*>(x_bf16), static_cast<const __nv_bfloat16*>(w_bf16),
                             static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(M), static_cast<int>(N),
-                            static_cast<int>(K), nullptr, nullptr, nullptr, 0, static_cast<cudaStream_t>(stream));
+                            static_cast<int>(K), nullptr, nullptr, nullptr, nullptr, 0,
+                            static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int metis_fp8_gemm(const void* a, int a_kind, float* s_tok, const uint8_t* wq,

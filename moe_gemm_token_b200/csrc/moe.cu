@@ -634,11 +634,11 @@ extern "C" int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int
     __nv_bfloat16* hs = static_cast<__nv_bfloat16*>(workspace);
     int rc = launch_bf16_gemm(static_cast<const __nv_bfloat16*>(x_bf16),
                               static_cast<const __nv_bfloat16*>(w_sup_bf16), hs, static_cast<int>(T),
-                              static_cast<int>(I_s), static_cast<int>(H), nullptr, nullptr, nullptr, 0, st);
+                              static_cast<int>(I_s), static_cast<int>(H), nullptr, nullptr, nullptr, nullptr, 0, st);
     if (rc) return rc;
     return launch_bf16_gemm(hs, static_cast<const __nv_bfloat16*>(w_sdn_bf16),
                             static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(T), static_cast<int>(H),
-                            static_cast<int>(I_s), static_cast<const __nv_bfloat16*>(o_routed_bf16),
+                            static_cast<int>(I_s), nullptr, static_cast<const __nv_bfloat16*>(o_routed_bf16),
                             slot_to_row, topk_w, static_cast<int>(topk), st);
 }
 

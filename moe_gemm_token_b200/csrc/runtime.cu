@@ -294,6 +294,9 @@ extern "C" size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, i
             moe_region_offset(0, M_or_T, topk, E, K_or_H, N_or_I, &total);
             return static_cast<size_t>(total);
         }
+        case METIS_OP_W8A16_WIDENED:
+            // the weights widened to BF16 [N, K]
+            return M_or_T < 1 ? 0 : static_cast<size_t>(align256(2 * N_or_I * K_or_H));
         case METIS_OP_SHARED:
             // the shared expert's hidden rows h_s [T, I_s] BF16
             return static_cast<size_t>(align256(2 * M_or_T * N_or_I));
@@ -320,13 +323,26 @@ extern "C" int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t top
     return moe_region_offset(region, T, topk, E, H, I, nullptr);
 }
 
+// Fewest tokens for which metis_linear's default maths widens the weights
+// into the workspace. Measured on B200 for N x K = 6144 x 2048, 2048 x 6144
+// and 14336 x 4096: at 256 tokens the in-kernel widening was faster for two
+// of the three (19.8 vs 24.3 us, 59 vs 73 us), at 512 the widened weights won
+// for all three (24.9 vs 32.9 us, 42.0 vs 44.8 us, 96.8 vs 110 us).
+constexpr int64_t kWidenMinTokens = 512;
+
 extern "C" int metis_linear(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
                             int64_t M, int64_t N, int64_t K, int fast_math, float* s_tok,
                             void* workspace, size_t ws_bytes, metis_stream_t stream) {
     clear_error();
     // M <= 8 tokens always take the default maths; more tokens take it unless fast_math
-    if ((M >= 1 && M <= 8) || (M > 8 && !fast_math))
+    if (M >= 1 && M <= 8) return metis_w8a16_gemm(x_bf16, wq, s_w, y_bf16, M, N, K, stream);
+    if (M > 8 && !fast_math) {
+        // enough tokens and room for the widened weights: the BF16 CTA-pair GEMM
+        if (M >= kWidenMinTokens && workspace && aligned(workspace, 16) &&
+            ws_bytes >= metis_workspace_size(METIS_OP_W8A16_WIDENED, M, N, K, 0, 0))
+            return metis_w8a16_gemm_widened(x_bf16, wq, s_w, y_bf16, M, N, K, workspace, ws_bytes, stream);
         return metis_w8a16_gemm(x_bf16, wq, s_w, y_bf16, M, N, K, stream);
+    }
     if (M > 0 && M * K > 0 && K % 16 == 0) {
         const size_t need = metis_workspace_size(METIS_OP_LINEAR, M, N, K, 0, 0);
         if (!workspace || ws_bytes < need || !aligned(workspace, 16))

@@ -363,4 +363,82 @@ int launch_w8a16_tensor(const __nv_bfloat16* x, const uint8_t* wq, const float* 
                       "w8a16 tensor-core GEMM launch");
 }
 
+namespace w16 {
+
+// Exact E4M3 -> BF16 widening of a weight matrix into a workspace, HBM-bound:
+// 1 byte read and 2 written per element, four 16-byte loads in flight per
+// thread. The BF16 copy is left in L2 for the GEMM that follows.
+__global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint4* __restrict__ w, uint4* __restrict__ out,
+                                                          int64_t n16) {
+    // the workspace may still be read by the previous kernel (the previous
+    // layer's GEMM): wait for it before writing
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = ld_w16(reinterpret_cast<const uint8_t*>(w + i + u * stride));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            uint32_t o[8];
+            widen_e4m3x16(v[u], o);
+            out[2 * (i + u * stride)] = make_uint4(o[0], o[1], o[2], o[3]);
+            out[2 * (i + u * stride) + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+    }
+    for (; i < n16; i += stride) {
+        uint32_t o[8];
+        widen_e4m3x16(ld_w16(reinterpret_cast<const uint8_t*>(w + i)), o);
+        out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+        out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+}  // namespace w16
+
+int launch_widen_e4m3(const uint8_t* w, __nv_bfloat16* out, int64_t n, cudaStream_t st) {
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc) return rc;
+    const int64_t n16 = n / 16;
+    if (n16 == 0) return METIS_OK;
+    int64_t blocks = (n16 + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(di.num_sms) * 8;  // 8 resident 256-thread blocks per SM
+    if (blocks > cap) blocks = cap;
+    return cuda_check(launch_pdl(w16::widen_e4m3_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, 1,
+                                 reinterpret_cast<const uint4*>(w), reinterpret_cast<uint4*>(out), n16),
+                      "e4m3 widening launch");
+}
+
 }  // namespace metis
+
+using namespace metis;
+
+extern "C" int metis_w8a16_gemm_widened(const void* x_bf16, const uint8_t* wq, const float* s_w,
+                                        void* y_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
+                                        size_t ws_bytes, metis_stream_t stream) {
+    clear_error();
+    if (M < 0 || M > 0x7fffffff || N < 8 || N % 8 != 0 || N > 0x7fffffff || K < 16 || K % 16 != 0 ||
+        K > 0x7fffffff)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "w8a16_gemm_widened: need M >= 0, N >= 8 with N %% 8 == 0, K >= 16 with K %% 16 == 0 "
+                    "(M=%lld N=%lld K=%lld)", (long long)M, (long long)N, (long long)K);
+    if (M == 0) return METIS_OK;
+    if (!x_bf16 || !wq || !s_w || !y_bf16) return fail(METIS_ERR_INVALID_ARG, "w8a16_gemm_widened: null pointer");
+    if (!aligned(x_bf16, 16) || !aligned(wq, 16) || !aligned(s_w, 4) || !aligned(y_bf16, 16))
+        return fail(METIS_ERR_INVALID_ARG, "w8a16_gemm_widened: x, wq and y must be 16-byte aligned");
+    const size_t need = metis_workspace_size(METIS_OP_W8A16_WIDENED, M, N, K, 0, 0);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 16))
+        return fail(METIS_ERR_INVALID_ARG,
+                    "w8a16_gemm_widened: needs a 16-byte aligned workspace of %zu bytes (got %zu)", need,
+                    ws_bytes);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    __nv_bfloat16* wb = static_cast<__nv_bfloat16*>(workspace);
+    int rc = launch_widen_e4m3(wq, wb, N * K, st);
+    if (rc) return rc;
+    return launch_bf16_gemm(static_cast<const __nv_bfloat16*>(x_bf16), wb, static_cast<__nv_bfloat16*>(y_bf16),
+                            static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), s_w, nullptr, nullptr,
+                            nullptr, 0, st);
+}

@@ -33,6 +33,7 @@ METIS_OP_MOE = 3
 METIS_OP_LINEAR = 4
 METIS_OP_MOE_NVFP4 = 5
 METIS_OP_SHARED = 6
+METIS_OP_W8A16_WIDENED = 7
 METIS_A_F32 = 2
 METIS_SF_ROWMAJOR = 0
 METIS_SF_TILED = 1
@@ -73,6 +74,7 @@ def load():
         "metis_quant_fp8_per_channel": ([p, i64, i64, i64, p, i64, p, p], i32),
         "metis_fp8_gemm": ([p, i32, p, p, p, p, i64, i64, i64, p, sz, p], i32),
         "metis_w8a16_gemm": ([p, p, p, p, i64, i64, i64, p], i32),
+        "metis_w8a16_gemm_widened": ([p, p, p, p, i64, i64, i64, p, sz, p], i32),
         "metis_moe_route_topk": ([p, p, i64, i64, i64, p, p, p], i32),
         "metis_moe_fp8_grouped_gemm": ([p, p, p, i64, i64, i64, i64, i64, p, p, p, p, i32, p, p,
                                         sz, p], i32),
@@ -175,6 +177,16 @@ def metis_w8a16_gemm(x, wq, s_w, y, stream=None):
         _p(x), _p(wq), _p(s_w), _p(y), M, N, K, _s(stream)))
 
 
+def metis_w8a16_gemm_widened(x, wq, s_w, y, workspace, stream=None):
+    """y [M, N] = W8A16(x, wq) with the weights widened to BF16 into `workspace`
+    first (metis_workspace_size(METIS_OP_W8A16_WIDENED, M, N, K) bytes)."""
+    M, K = x.shape
+    N = wq.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    return _check("metis_w8a16_gemm_widened", load().metis_w8a16_gemm_widened(
+        _p(x), _p(wq), _p(s_w), _p(y), M, N, K, _p(workspace), ws_bytes, _s(stream)))
+
+
 def metis_moe_route_topk(logits, topk_ids, topk_w, bias=None, stream=None):
     """Router top-k: logits [T, E] FP32 (+ bias [E]) -> topk_ids [T, k], topk_w [T, k]."""
     T, E = logits.shape
@@ -222,7 +234,8 @@ def metis_moe_workspace_offset(region, T, topk, E, H, I):
 
 def metis_linear(x, wq, s_w, y, fast_math=True, s_tok=None, workspace=None, stream=None):
     """Dispatch rule: M <= 8 -> W8A16; otherwise W8A8 with fast_math (per-token
-    quantizer into `workspace`, then the E4M3 GEMM) and W8A16 without."""
+    quantizer into `workspace`, then the E4M3 GEMM) and W8A16 without (the
+    widened-weights GEMM when M >= 512 and `workspace` holds the BF16 weights)."""
     M, K = x.shape
     N = wq.shape[0]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -85,6 +85,20 @@ def test_host_validation_without_gpu(lib):
     assert lib.metis_w8a16_gemm(p, p, p, p, 9, 128, 250, null) == metis.METIS_ERR_INVALID_ARG
     assert lib.metis_w8a16_gemm(p, p, p, p, 4, 128, 16384, null) == metis.METIS_ERR_INVALID_ARG
     assert lib.metis_w8a16_gemm(p, p, p, p, 4, 128, 264, null) == metis.METIS_ERR_INVALID_ARG
+    # W8A16 through widened weights: N % 8, K % 16, the workspace of 2 N K bytes
+    need_w = lib.metis_workspace_size(metis.METIS_OP_W8A16_WIDENED, 300, 6144, 2048, 0, 0)
+    assert need_w == 2 * 6144 * 2048
+    assert lib.metis_workspace_size(metis.METIS_OP_W8A16_WIDENED, 0, 6144, 2048, 0, 0) == 0
+    assert lib.metis_w8a16_gemm_widened(p, p, p, p, 300, 100, 256, p, 1 << 30, null) == \
+        metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_w8a16_gemm_widened(p, p, p, p, 300, 128, 250, p, 1 << 30, null) == \
+        metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_w8a16_gemm_widened(p, p, p, p, 300, 6144, 2048, p, need_w - 16, null) == \
+        metis.METIS_ERR_INVALID_ARG
+    assert b"workspace" in lib.metis_last_error()
+    assert lib.metis_w8a16_gemm_widened(p, p, p, p, 300, 6144, 2048, ctypes.c_void_p(0x1008), need_w,
+                                        null) == metis.METIS_ERR_INVALID_ARG
+    assert lib.metis_w8a16_gemm_widened(p, p, p, p, 0, 6144, 2048, p, 0, null) == metis.METIS_OK
     # MoE: activation, topk > E, H % 16, small workspace
     assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 2, 4, 64, 32, p, p, p, p, 1, p, p, 1 << 30,
                                           null) == metis.METIS_ERR_UNSUPPORTED

@@ -80,9 +80,11 @@ def test_prefill_chain_full_size(metis):
     assert_close(bf16_host(y2)[rows], y2_64, "layer 2")
 
 
-def test_prefill_chain_default_maths_full_size(metis):
+@pytest.mark.parametrize("widened", [False, True])
+def test_prefill_chain_default_maths_full_size(metis, widened):
     """The same 4096-token chain through the default maths (metis_linear
-    without fast-math: W8A16, weights widened to BF16 on the tensor cores)."""
+    without fast-math: W8A16, weights widened to BF16 in the kernel, or first
+    into a workspace for the BF16 CTA-pair GEMM)."""
     d = synth.prefill_chain()
     M, K, N = d["M"], d["K"], d["N"]
     w1, s1, w1r, s1r = _weights(metis, d["w1"])
@@ -90,8 +92,12 @@ def test_prefill_chain_default_maths_full_size(metis):
     y1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     y2 = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
     s_tok = torch.empty((M,), dtype=torch.float32, device="cuda")
-    metis.metis_linear(bf16_dev(d["x"]), w1, s1, y1, fast_math=False, s_tok=s_tok)
-    metis.metis_linear(y1, w2, s2, y2, fast_math=False, s_tok=s_tok)
+    ws = None
+    if widened:
+        n = metis.metis_workspace_size(metis.METIS_OP_W8A16_WIDENED, M, N, K)
+        ws = torch.empty((n,), dtype=torch.uint8, device="cuda")
+    metis.metis_linear(bf16_dev(d["x"]), w1, s1, y1, fast_math=False, s_tok=s_tok, workspace=ws)
+    metis.metis_linear(y1, w2, s2, y2, fast_math=False, s_tok=s_tok, workspace=ws)
     assert metis.metis_check_device_status() == 0
     rows = _sample_rows(M, d["x"])
     _, y1_64 = oracle.gemm_w8a16(d["x"][rows], w1r, s1r)

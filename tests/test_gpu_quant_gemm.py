@@ -265,6 +265,136 @@ def test_w8a16_tensor_core_exact_products(metis):
     assert_bytes_equal(bf16_host(y), yr, "w8a16 tensor exact")
 
 
+def test_w8a16_tensor_core_nan_codes(metis):
+    """E4M3 NaN weight codes (0x7F, 0xFF) widen to NaN: every output of those
+    channels is NaN, and every other output matches the oracle."""
+    M, N, K = 272, 520, 192
+    d = synth.linear(77, M, K, N, outlier_channels=0, outlier_scale=1.0)
+    wq_r, sw_r = oracle.quant_per_channel(d["w"])
+    wq_r = wq_r.copy()
+    wq_r[3, 5] = 0x7F
+    wq_r[300, 191] = 0xFF
+    wq_r[519, 0] = 0x7F
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_w8a16_gemm(bf16_dev(d["x"]), dev(wq_r), dev(sw_r), y)
+    assert metis.metis_check_device_status() == 0
+    got = bf16_host(y)
+    nan = (got & 0x7FFF) > 0x7F80
+    assert np.array_equal(np.nonzero(nan.any(axis=0))[0], [3, 300, 519])
+    assert nan[:, [3, 300, 519]].all()
+    keep = np.setdiff1d(np.arange(N), [3, 300, 519])
+    _, y64 = oracle.gemm_w8a16(d["x"], wq_r[keep], sw_r[keep])
+    assert_close(got[:, keep], y64, "w8a16 tensor, finite channels")
+
+
+def _widened_ws(metis, M, N, K):
+    n = metis.metis_workspace_size(metis.METIS_OP_W8A16_WIDENED, M, N, K)
+    return torch.zeros((n,), dtype=torch.uint8, device="cuda")
+
+
+def test_w8a16_widening_is_exact_for_every_code(metis):
+    """The widening pass writes the BF16 value of every E4M3 code exactly
+    (subnormals included) and a same-signed NaN for 0x7F and 0xFF."""
+    N, K = 16, 256
+    # every code in every row, at a different column per row
+    codes = ((np.arange(K)[None, :] + 17 * np.arange(N)[:, None]) % 256).astype(np.uint8)
+    ws = _widened_ws(metis, 9, N, K)
+    x = torch.zeros((9, K), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((9, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_w8a16_gemm_widened(x, dev(codes), dev(np.ones(N, np.float32)), y, ws)
+    assert metis.metis_check_device_status() == 0
+    wb = ws[:2 * N * K].view(torch.int16).view(N, K).cpu().numpy().view(np.uint16)
+    want = oracle.e4m3_decode(codes)
+    isnan = np.isnan(want)
+    assert np.array_equal(isnan, (codes & 0x7F) == 0x7F)
+    got = oracle.bf16_to_float(wb).astype(np.float64)
+    assert np.array_equal(got[~isnan], want[~isnan])
+    assert np.array_equal(np.signbit(got[~isnan]), np.signbit(want[~isnan]))  # -0 stays -0
+    assert np.all(np.isnan(got[isnan]))
+    assert np.array_equal(np.signbit(got[isnan]), (codes[isnan] & 0x80) != 0)
+
+
+@pytest.mark.parametrize("M,N,K", [(9, 264, 512), (256, 256, 128), (300, 6144, 2048), (513, 136, 4096),
+                                   (1000, 520, 1040), (129, 8, 16)])
+def test_w8a16_widened_parity(metis, M, N, K):
+    """The default maths through widened weights and the BF16 CTA-pair GEMM
+    (per-channel scale in its epilogue), ragged in M, N and K."""
+    d = synth.linear(M * 5 + N + 3 * K, M, K, N, outlier_channels=2, outlier_scale=20.0)
+    wq, s_w = _prep_weights(metis, d["w"])
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_w8a16_gemm_widened(bf16_dev(d["x"]), wq, s_w, y, _widened_ws(metis, M, N, K))
+    assert metis.metis_check_device_status() == 0
+    wq_r, sw_r = oracle.quant_per_channel(d["w"])
+    _, y64 = oracle.gemm_w8a16(d["x"], wq_r, sw_r)
+    assert_close(bf16_host(y), y64, f"w8a16 widened {M}x{N}x{K}")
+
+
+def test_w8a16_widened_exact_products(metis):
+    """Subnormal and small normal weight codes, small-integer x, unit scales:
+    every product and partial sum is exact in FP32, so the BF16 outputs equal
+    the oracle's bit for bit."""
+    rng = np.random.default_rng(19)
+    M, N, K = 300, 264, 320
+    codes = (rng.integers(1, 8, (N, K)) | (rng.integers(0, 2, (N, K)) << 7)).astype(np.uint8)
+    codes[:, ::5] = 0x38  # 1.0
+    codes[::3, 1::7] = 0xC0  # -2.0
+    x = synth.f32_to_bf16_bits(rng.integers(-4, 5, (M, K)).astype(np.float32))
+    s_w = np.ones(N, np.float32)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_w8a16_gemm_widened(bf16_dev(x), dev(codes), dev(s_w), y, _widened_ws(metis, M, N, K))
+    assert metis.metis_check_device_status() == 0
+    yr, _ = oracle.gemm_w8a16(x, codes, s_w)
+    assert np.any(yr != 0)
+    assert_bytes_equal(bf16_host(y), yr, "w8a16 widened exact")
+
+
+def test_w8a16_widened_nan_codes(metis):
+    M, N, K = 272, 520, 192
+    d = synth.linear(78, M, K, N)
+    wq_r, sw_r = oracle.quant_per_channel(d["w"])
+    wq_r = wq_r.copy()
+    wq_r[3, 5] = 0x7F
+    wq_r[300, 191] = 0xFF
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    metis.metis_w8a16_gemm_widened(bf16_dev(d["x"]), dev(wq_r), dev(sw_r), y, _widened_ws(metis, M, N, K))
+    assert metis.metis_check_device_status() == 0
+    got = bf16_host(y)
+    nan = (got & 0x7FFF) > 0x7F80
+    assert np.array_equal(np.nonzero(nan.any(axis=0))[0], [3, 300])
+    assert nan[:, [3, 300]].all()
+    keep = np.setdiff1d(np.arange(N), [3, 300])
+    _, y64 = oracle.gemm_w8a16(d["x"], wq_r[keep], sw_r[keep])
+    assert_close(got[:, keep], y64, "w8a16 widened, finite channels")
+
+
+@pytest.mark.parametrize("M", [300, 512, 700])
+def test_linear_default_maths_dispatch(metis, M):
+    """metis_linear without fast-math: M >= 512 with a large enough workspace
+    runs the widened-weights GEMM, otherwise the in-kernel widening; each is
+    bit-identical to its direct call."""
+    N, K = 384, 512
+    d = synth.linear(M + 11, M, K, N)
+    wq, s_w = _prep_weights(metis, d["w"])
+    x = bf16_dev(d["x"])
+    ws = _widened_ws(metis, M, N, K)
+    y_lin = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    y_dir = torch.empty_like(y_lin)
+    metis.metis_linear(x, wq, s_w, y_lin, fast_math=False, workspace=ws)
+    if M >= 512:
+        metis.metis_w8a16_gemm_widened(x, wq, s_w, y_dir, _widened_ws(metis, M, N, K))
+    else:
+        metis.metis_w8a16_gemm(x, wq, s_w, y_dir)
+    assert metis.metis_check_device_status() == 0
+    assert torch.equal(y_lin.view(torch.int16), y_dir.view(torch.int16))
+    # without a workspace the in-kernel path runs at any M
+    y_in = torch.empty_like(y_lin)
+    metis.metis_linear(x, wq, s_w, y_in, fast_math=False)
+    y_ref = torch.empty_like(y_lin)
+    metis.metis_w8a16_gemm(x, wq, s_w, y_ref)
+    torch.cuda.synchronize()
+    assert torch.equal(y_in.view(torch.int16), y_ref.view(torch.int16))
+
+
 def test_w8a16_subnormal_weights_and_wide_x(metis):
     """Weight rows with many E4M3 subnormal codes and tokens whose elements
     span many binades: the widening and the per-token shift stay exact."""
