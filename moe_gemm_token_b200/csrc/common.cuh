@@ -493,7 +493,7 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
 // BF16 multiply by 2^120 (exact; subnormal inputs are kept) gives the E4M3
 // value, 2^(e-7) (1 + m/8) or m * 2^-9. prmt's sign-replicating selectors
 // put each byte's sign in bit 15 of its half. NaN codes (e = 15, m = 7) come
-// out as +-480 here; widen_e4m3x16 repairs them.
+// out as +-480 here; widen_e4m3x8 repairs them.
 __device__ __forceinline__ void widen_e4m3x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
     uint32_t p0, p1;
     asm("prmt.b32 %0, %1, 0, 0x9180;" : "=r"(p0) : "r"(w));
@@ -504,30 +504,29 @@ __device__ __forceinline__ void widen_e4m3x4(uint32_t w, uint32_t& lo, uint32_t&
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(u1), "r"(0x7B807B80u));
 }
 
-// Sixteen E4M3 bytes -> eight BF16 pairs, element 2i in the low half of o[i].
+// Eight E4M3 bytes -> four BF16 pairs, element 2i in the low half of word i.
 // A byte whose low 7 bits are all set (E4M3 NaN) becomes a BF16 NaN of the
-// same sign.
-__device__ __forceinline__ void widen_e4m3x16(const uint4& v, uint32_t (&o)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) widen_e4m3x4(w[i], o[2 * i], o[2 * i + 1]);
-    // 0x80 in every byte whose low 7 bits are 0x7F (no carry crosses a byte)
-    uint32_t nan = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) nan |= (w[i] & 0x7F7F7F7Fu) + 0x01010101u;
+// same sign (a rarely taken branch).
+__device__ __forceinline__ void widen_e4m3x8(const uint2& v, uint4& o) {
+    widen_e4m3x4(v.x, o.x, o.y);
+    widen_e4m3x4(v.y, o.z, o.w);
+    const uint32_t nan = ((v.x & 0x7F7F7F7Fu) + 0x01010101u) | ((v.y & 0x7F7F7F7Fu) + 0x01010101u);
     if (nan & 0x80808080u) {
+        uint32_t r[4] = {o.x, o.y, o.z, o.w};
+        const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2; ++i) {
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const uint32_t byte = (w[i] >> (8 * b)) & 0xFFu;
                 if ((byte & 0x7Fu) == 0x7Fu) {
-                    uint32_t& word = o[2 * i + (b >> 1)];
+                    uint32_t& word = r[2 * i + (b >> 1)];
                     const int sh = 16 * (b & 1);
                     word = (word & ~(0xFFFFu << sh)) | (((byte << 8) | 0x7FC0u) << sh);
                 }
             }
         }
+        o = make_uint4(r[0], r[1], r[2], r[3]);
     }
 }
 

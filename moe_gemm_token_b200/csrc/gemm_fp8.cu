@@ -56,6 +56,7 @@ constexpr int TMEM_COLS = 2 * BN_MAX;
 constexpr int MAX_GROUPS = 1024;
 
 constexpr int CONV_WARPS = 8;                  // fused-quantization converter warps
+constexpr int RASTER_M = 16;  // row blocks per raster group of the dense schedule
 constexpr int COMB_K = 8;                      // fused combine: routed slots per token
 constexpr int ASTG_SLOT = ROWS * BK * 2;       // one BF16 A tile (two 64-column boxes)
 
@@ -126,8 +127,14 @@ struct Sched {
     __device__ __forceinline__ Tile get(int t) const {
         Tile ti;
         if (g_tile == nullptr) {
-            const int mb = t % num_m;
-            const int nb = t / num_m;
+            // groups of RASTER_M row blocks, row block fastest inside a group:
+            // the tiles running together share a few row blocks of A and
+            // column blocks of B in L2
+            const int per_group = RASTER_M * num_n;
+            const int g = t / per_group, r = t - g * per_group;
+            const int gm = min(RASTER_M, num_m - g * RASTER_M);
+            const int mb = g * RASTER_M + r % gm;
+            const int nb = r / gm;
             ti.a_row0 = mb * ROWS * CTAS + static_cast<int>(rank) * ROWS;
             ti.row_end = M;
             ti.b_row0 = nb * BN + static_cast<int>(rank) * (BN / CTAS);

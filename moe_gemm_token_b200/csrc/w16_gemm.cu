@@ -366,33 +366,35 @@ int launch_w8a16_tensor(const __nv_bfloat16* x, const uint8_t* wq, const float* 
 namespace w16 {
 
 // Exact E4M3 -> BF16 widening of a weight matrix into a workspace, HBM-bound:
-// 1 byte read and 2 written per element, four 16-byte loads in flight per
-// thread. The BF16 copy is left in L2 for the GEMM that follows.
-__global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint4* __restrict__ w, uint4* __restrict__ out,
-                                                          int64_t n16) {
+// 1 byte read and 2 written per element. A thread widens 8 bytes into one
+// 16-byte store, so a warp reads 256 and writes 512 contiguous bytes per
+// instruction; each thread has WIDEN_BATCH loads in flight (grid-strided)
+// before it widens and stores them. The BF16 copy stays in L2 for the GEMM
+// that follows.
+constexpr int WIDEN_BATCH = 8;
+
+__global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint2* __restrict__ w, uint4* __restrict__ out,
+                                                          int64_t n8) {
     // the workspace may still be read by the previous kernel (the previous
     // layer's GEMM): wait for it before writing
     grid_dependency_wait();
     grid_launch_dependents();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    for (; i + 3 * stride < n16; i += 4 * stride) {
-        uint4 v[4];
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += WIDEN_BATCH * stride) {
+        uint2 v[WIDEN_BATCH];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = ld_w16(reinterpret_cast<const uint8_t*>(w + i + u * stride));
+        for (int u = 0; u < WIDEN_BATCH; ++u)
+            if (i + u * stride < n8) v[u] = __ldg(w + i + u * stride);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            uint32_t o[8];
-            widen_e4m3x16(v[u], o);
-            out[2 * (i + u * stride)] = make_uint4(o[0], o[1], o[2], o[3]);
-            out[2 * (i + u * stride) + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+        for (int u = 0; u < WIDEN_BATCH; ++u) {
+            const int64_t c = i + u * stride;
+            if (c < n8) {
+                uint4 o;
+                widen_e4m3x8(v[u], o);
+                out[c] = o;
+            }
         }
-    }
-    for (; i < n16; i += stride) {
-        uint32_t o[8];
-        widen_e4m3x16(ld_w16(reinterpret_cast<const uint8_t*>(w + i)), o);
-        out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
-        out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
 }
 
@@ -402,13 +404,14 @@ int launch_widen_e4m3(const uint8_t* w, __nv_bfloat16* out, int64_t n, cudaStrea
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
-    const int64_t n16 = n / 16;
-    if (n16 == 0) return METIS_OK;
-    int64_t blocks = (n16 + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(di.num_sms) * 8;  // 8 resident 256-thread blocks per SM
+    const int64_t n8 = n / 8;
+    if (n8 == 0) return METIS_OK;
+    // WIDEN_BATCH chunks per thread, at most 8 resident 256-thread blocks per SM
+    int64_t blocks = (n8 + w16::WIDEN_BATCH * 256 - 1) / (w16::WIDEN_BATCH * 256);
+    const int64_t cap = static_cast<int64_t>(di.num_sms) * 8;
     if (blocks > cap) blocks = cap;
     return cuda_check(launch_pdl(w16::widen_e4m3_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, 1,
-                                 reinterpret_cast<const uint4*>(w), reinterpret_cast<uint4*>(out), n16),
+                                 reinterpret_cast<const uint2*>(w), reinterpret_cast<uint4*>(out), n8),
                       "e4m3 widening launch");
 }
 

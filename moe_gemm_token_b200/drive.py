@@ -7,6 +7,7 @@ only the device status word.
     python -m moe_gemm_token_b200.drive fused M N K [--calls N]
     python -m moe_gemm_token_b200.drive decode M [--calls N]
     python -m moe_gemm_token_b200.drive w16 M N K [--calls N]
+    python -m moe_gemm_token_b200.drive w16w M N K [--calls N]
     python -m moe_gemm_token_b200.drive quant M K [--calls N]
     python -m moe_gemm_token_b200.drive moe4  [--calls N]
     python -m moe_gemm_token_b200.drive gemm4 M N K [--calls N]
@@ -37,7 +38,8 @@ def _sf(n, g):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["moe", "gemm", "fused", "decode", "w16", "quant", "moe4", "gemm4", "shared", "bf16"])
+    ap.add_argument("op", choices=["moe", "gemm", "fused", "decode", "w16", "w16w", "quant", "moe4", "gemm4", "shared",
+                                   "bf16"])
     ap.add_argument("dims", nargs="*", type=int)
     ap.add_argument("--calls", type=int, default=3)
     a = ap.parse_args(argv)
@@ -126,13 +128,18 @@ def main(argv=None):
             ws = torch.empty(metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, M, N, K, 0, 0),
                              dtype=torch.uint8, device=dev)
             call = lambda: metis.metis_fp8_gemm(x, metis.METIS_A_BF16, s, b, sb, y, workspace=ws)
-    elif a.op == "w16":
+    elif a.op in ("w16", "w16w"):
         M, N, K = a.dims
         x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
         wq = _codes(N, K, g)
         sw = torch.rand(N, device=dev, generator=g) * 1e-3
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        call = lambda: metis.metis_w8a16_gemm(x, wq, sw, y)
+        if a.op == "w16":
+            call = lambda: metis.metis_w8a16_gemm(x, wq, sw, y)
+        else:  # weights widened into a workspace, then the BF16 CTA-pair GEMM
+            ws = torch.empty(metis.metis_workspace_size(metis.METIS_OP_W8A16_WIDENED, M, N, K),
+                             dtype=torch.uint8, device=dev)
+            call = lambda: metis.metis_w8a16_gemm_widened(x, wq, sw, y, ws)
     elif a.op == "decode":
         (M,) = a.dims
         N, K = 14336, 4096

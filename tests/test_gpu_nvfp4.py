@@ -162,7 +162,8 @@ def _gemm_gpu(m, qa, sa, ga, qb, sb, gb):
 
 
 @pytest.mark.parametrize("M,N,K,seed", [(1, 128, 64, 0), (130, 256, 256, 1), (300, 384, 320, 2),
-                                        (257, 512, 2048, 3), (64, 128, 4096, 4), (517, 1024, 1024, 5)])
+                                        (257, 512, 2048, 3), (64, 128, 4096, 4), (517, 1024, 1024, 5),
+                                        (4500, 384, 256, 6)])
 def test_nvfp4_gemm_parity_quantized(metis, M, N, K, seed):
     d = synth.linear(seed, M, K, N, outlier_channels=min(4, K), outlier_scale=10.0,
                      row_magnitude_log10=(-2, 2))

@@ -89,7 +89,7 @@ def _prep_weights(metis, w):
 
 
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 272), (1, 8, 16), (129, 264, 1040),
-                                   (520, 784, 1024), (257, 1024, 2048)])
+                                   (520, 784, 1024), (257, 1024, 2048), (4500, 520, 256)])
 def test_fp8_gemm_parity(metis, M, N, K):
     d = synth.linear(M * 7 + N, M, K, N, outlier_channels=4, outlier_scale=20.0, zero_rows=(M // 3,))
     wq, s_w = _prep_weights(metis, d["w"])
@@ -315,7 +315,7 @@ def test_w8a16_widening_is_exact_for_every_code(metis):
 
 
 @pytest.mark.parametrize("M,N,K", [(9, 264, 512), (256, 256, 128), (300, 6144, 2048), (513, 136, 4096),
-                                   (1000, 520, 1040), (129, 8, 16)])
+                                   (1000, 520, 1040), (129, 8, 16), (4500, 264, 256)])
 def test_w8a16_widened_parity(metis, M, N, K):
     """The default maths through widened weights and the BF16 CTA-pair GEMM
     (per-channel scale in its epilogue), ragged in M, N and K."""

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("M,N,K,seed", [(1, 8, 8, 0), (130, 256, 256, 1), (300, 384, 328, 2),
-                                        (512, 1024, 2048, 3), (77, 136, 1000, 4)])
+                                        (512, 1024, 2048, 3), (77, 136, 1000, 4), (4500, 264, 128, 5)])
 def test_bf16_gemm_parity(metis, M, N, K, seed):
     rng = np.random.default_rng(seed)
     x = synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
