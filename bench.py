@@ -229,6 +229,29 @@ class ClockSampler:
 
 # --------------------------------------------------------------- metis arm
 
+def moe_floor_us(T, H, I, E, k, hbm_gbs, peak_tflops, fp4):
+    """Lower bound on the routed-expert layer's time: for each HBM-heavy
+    kernel the larger of its algorithmic bytes over the measured HBM
+    bandwidth and its FLOPs over the tensor peak, summed (the latency-bound
+    routing kernels count as zero). Bytes per kernel, with S = T * k slots:
+    quantizer of x (x read, codes + scales written into S rows), grouped
+    up-projection (codes of x, expert weights, h written), quantizer of h,
+    grouped down-projection (codes of h, weights, o written), combine (o read,
+    y written). Codes are 1 byte per element in FP8 and half a byte plus one
+    E4M3 scale per 16 in NVFP4."""
+    S = T * k
+    code = (lambda n: n / 2 + n / 16) if fp4 else (lambda n: n)
+    fl = 2.0 * S * I * H
+    kernels = [
+        (2 * T * H + code(S * H) + 4 * S, 0.0),                  # quantize x into expert rows
+        (code(S * H) + code(E * I * H) + 2 * S * I, fl),         # up-projection
+        (2 * S * I + code(S * I) + 4 * S, 0.0),                  # quantize h
+        (code(S * I) + code(E * H * I) + 2 * S * H, fl),         # down-projection
+        (2 * S * H + 8 * S + 2 * T * H, 0.0),                    # weighted combine
+    ]
+    return sum(max(b / (hbm_gbs * 1e9), f / (peak_tflops * 1e12)) for b, f in kernels) * 1e6
+
+
 def gemm_traffic_from_profile():
     """DRAM bytes per GEMM launch from the committed ncu summary, if it was
     taken on the current kernel source (else None)."""
@@ -608,8 +631,10 @@ def secondary_figures(metis, dev, pk):
                                            "GB/s": (T * E * 4 + T * k * 8) / t_r / 1e9}
     t = timeit(lambda: metis.metis_moe_fp8_grouped_gemm(x, ids, w, wu, su, wd, sd, y, wsp), 20)
     tf = 2 * 2 * T * k * H * I / t / 1e12
+    floor = moe_floor_us(T, H, I, E, k, hbm, peak8, fp4=False)
     out["moe_4096tok_64e_top8"] = {"us": t * 1e6, "tok/s": T / t, "TFLOP/s": tf,
-                                   "frac_of_fp8_peak": tf / peak8}
+                                   "frac_of_fp8_peak": tf / peak8, "floor_us": floor,
+                                   "frac_of_floor": floor / (t * 1e6)}
     # the layer with its shared expert (BF16, latent 1024): the routed layer
     # with y = NULL, then the shared expert with the routed combine fused into
     # its down-projection's epilogue
@@ -655,8 +680,10 @@ def secondary_figures(metis, dev, pk):
     t = timeit(lambda: metis.metis_moe_nvfp4_grouped_gemm(x, ids, w, wu4, sfu, gu, wd4, sfd, gd,
                                                           y, ws4), 20)
     tf = 2 * 2 * T * k * H * I / t / 1e12
+    floor = moe_floor_us(T, H, I, E, k, hbm, peak4, fp4=True)
     out["moe_nvfp4_4096tok_64e_top8"] = {"us": t * 1e6, "tok/s": T / t, "TFLOP/s": tf,
-                                         "frac_of_fp4_peak": tf / peak4}
+                                         "frac_of_fp4_peak": tf / peak4, "floor_us": floor,
+                                         "frac_of_floor": floor / (t * 1e6)}
     del wu4, wd4, sfu, sfd, ws4
     # dense NVFP4 GEMM (codes and tiled scales resident, 2 rotating B > L2 at the large size)
     for (M, K) in [(8192, 4096), (16384, 8192)]:
