@@ -40,6 +40,13 @@ namespace nvfp4 {
 // Eight binary32 values -> eight E2M1 codes, round-to-nearest-even and
 // saturating to +-6 (cvt.rn.satfinite.e2m1x2 puts its first source in the
 // high nibble); v[0] lands in bits 0..3 of the result.
+// Elementwise maximum of two BF16 pairs (a NaN operand yields the other).
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float* v) {
     uint32_t r;
     asm("{\n\t"
@@ -146,17 +153,18 @@ __device__ __forceinline__ void quant_row(const QuantArgs& a, int64_t r, int lan
         }
     };
     // register-resident rows: each block's maximum, taken once for both the
-    // row amax and the block scale
+    // row amax and the block scale, on the packed BF16 pairs (sign cleared,
+    // then max.bf16x2, which like fmaxf ignores a NaN operand)
     float bmax[NBL > 0 ? NBL : 1];
     if constexpr (NBL > 0) {
 #pragma unroll
         for (int i = 0; i < NBL; ++i) {
-            float v[16];
-            unpack(i, v);
-            float bm = 0.0f;
+            const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
+                                   raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
+            uint32_t m2 = w[0] & 0x7FFF7FFFu;
 #pragma unroll
-            for (int h = 0; h < 16; ++h) bm = fmaxf(bm, fabsf(v[h]));
-            bmax[i] = bm;
+            for (int h = 1; h < 8; ++h) m2 = bf16x2_max(m2, w[h] & 0x7FFF7FFFu);
+            bmax[i] = fmaxf(bf16_lo(m2), bf16_hi(m2));
         }
     } else {
         bmax[0] = 0.0f;
@@ -182,7 +190,11 @@ __device__ __forceinline__ void quant_row(const QuantArgs& a, int64_t r, int lan
         amax = m;
     }
     const float inv_g = amax > 0.0f ? fminf(__fdiv_rn(2688.0f, amax), 3.402823466e38f) : 0.0f;
+    const float g_row = __fdiv_rn(amax, 2688.0f);
     const int ndst = a.dst_rows ? a.topk : 1;
+    // the destination rows, loaded once per row: lane j holds destination j
+    // (up to 32 of them; more are read from memory where they are used)
+    const int my_dst = (a.dst_rows && lane < ndst) ? a.dst_rows[r * a.topk + lane] : -1;
     // one pass over 32 blocks (512 elements); v holds this lane's block b0 + lane
     // and bm its maximum magnitude
     auto block_pass = [&](int b0, const float (&v)[16], float bm) {
@@ -203,14 +215,18 @@ __device__ __forceinline__ void quant_row(const QuantArgs& a, int64_t r, int lan
         s4 |= __shfl_down_sync(0xffffffffu, sbc, 2) << 16;
         s4 |= __shfl_down_sync(0xffffffffu, sbc, 3) << 24;
         for (int j = 0; j < ndst; ++j) {
-            const int64_t dr = a.dst_rows ? a.dst_rows[r * a.topk + j] : r;
+            int64_t dr = r;
+            if (a.dst_rows) {
+                const int d = __shfl_sync(0xffffffffu, my_dst, j & 31);
+                dr = j < 32 ? d : a.dst_rows[r * a.topk + j];
+            }
             if (dr < 0 || b >= nb) continue;
             *reinterpret_cast<uint2*>(a.q + dr * (a.K / 2) + 8 * b) = make_uint2(lo, hi);
             if ((lane & 3) == 0) {
                 const int64_t off = a.tiled ? tiled_sf_offset(dr, b / 4, kc) : dr * (a.K / 16) + b;
                 *reinterpret_cast<uint32_t*>(a.sf + off) = s4;
             }
-            if (b0 == 0 && lane == 0 && !a.gamax) a.g[dr] = __fdiv_rn(amax, 2688.0f);
+            if (b0 == 0 && lane == 0 && !a.gamax) a.g[dr] = g_row;
         }
     };
     if constexpr (NBL > 0) {
@@ -238,7 +254,7 @@ __device__ __forceinline__ void quant_row(const QuantArgs& a, int64_t r, int lan
 // RPW rows per warp (rows r0 .. r0 + RPW - 1): with NBL > 0 every row's loads
 // are issued before the first row is encoded, so a warp waits on memory once.
 template <typename T, int NBL, int RPW>
-__global__ void __launch_bounds__(QWARPS * 32) nvfp4_quant_kernel(const QuantArgs a) {
+__global__ void __launch_bounds__(QWARPS * 32, (NBL > 0 && NBL <= 4) ? 4 : 1) nvfp4_quant_kernel(const QuantArgs a) {
     static_assert(QWARPS * 32 == 256, "one thread per E4M3 code builds the reciprocal table");
     static_assert(NBL == 0 || sizeof(T) == 2, "register-resident rows are BF16");
     static_assert(NBL > 0 || RPW == 1, "two-pass rows are one per warp");
