@@ -553,7 +553,7 @@ def secondary_figures(metis, dev, pk):
     # large-M W8A8 GEMM from BF16 activations (per-token magnitudes
     # log-uniform in [1e-2, 1e2]): the GEMM alone, the separate quantizer +
     # GEMM (the product path), and the fused-quantization variant
-    for (M, K) in [(8192, 4096), (16384, 8192)]:
+    for (M, K) in [(8192, 4096), (16384, 4096), (8192, 8192), (16384, 8192)]:
         mag = torch.exp(torch.empty(M, 1, device=dev).uniform_(-4.6052, 4.6052, generator=g))
         x = (torch.randn(M, K, device=dev, generator=g) * mag).to(torch.bfloat16)
         b = codes(K, K)

@@ -129,7 +129,7 @@ def test_moe_full_size(metis):
     check_moe(d, g, tokens=toks)
 
 
-@pytest.mark.parametrize("M,K", [(8192, 4096), (16384, 8192)])
+@pytest.mark.parametrize("M,K", [(8192, 4096), (16384, 4096), (8192, 8192), (16384, 8192)])
 def test_large_m_full_size(metis, M, K):
     d = synth.large_m(M=M, K=K)
     N = K
@@ -144,6 +144,16 @@ def test_large_m_full_size(metis, M, K):
     xq_r, st_r = oracle.quant_per_token(d["x"])
     assert_bytes_equal(xq.cpu().numpy(), xq_r, "codes")
     assert_bytes_equal(st.cpu().numpy().view(np.uint32), st_r.view(np.uint32), "scales")
-    rows = _sample_rows(M, d["x"], n=32)
+    rows = _sample_rows(M, d["x"], n=256)  # 256 sampled rows and the extreme ones
     _, y64 = oracle.gemm_w8a8(xq_r, st_r, wq_r, s_r, rows=rows)
     assert_close(bf16_host(y)[rows], y64, f"large M {M}x{K}")
+    # the fused-quantization prologue on the same input: the same scales and,
+    # bit for bit, the same output as quantizer + E4M3 GEMM
+    st_f = torch.empty_like(st)
+    y_f = torch.empty_like(y)
+    ws = torch.empty((metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, M, N, K),),
+                     dtype=torch.uint8, device="cuda")
+    metis.metis_fp8_gemm(x_dev, metis.METIS_A_BF16, st_f, wq, s_w, y_f, workspace=ws)
+    assert metis.metis_check_device_status() == 0
+    assert_bytes_equal(st_f.cpu().numpy().view(np.uint32), st_r.view(np.uint32), "fused scales")
+    assert torch.equal(y_f.view(torch.int16), y.view(torch.int16)), "fused prologue differs"
