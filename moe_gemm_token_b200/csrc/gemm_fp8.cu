@@ -23,20 +23,25 @@
 //             and 128 rows of B (16 + 16 KB per 128-deep k-block, 6 stages),
 //             so each SM streams half of the B tile it would need alone. Both
 //             CTAs' TMA loads complete on the even CTA's mbarrier; its MMA
-//             commits are multicast to both CTAs. Dense GEMMs with M > 128.
+//             commits are multicast to both CTAs. Dense GEMMs with M > 128,
+//             and the grouped GEMM of the routed experts for K >= 2048.
 //   CTAS = 1  one CTA computes 128 x 256 (4 stages of 16 + 32 KB). Used for
-//             the grouped GEMM of the routed experts (rows of A grouped by
-//             expert, B = [E * N, K], tile schedule built on the device from
-//             the expert offsets) and for small M.
+//             small M and for the grouped GEMM with K < 2048 (the routed
+//             down-projection), where it measured faster than pairs.
+// Grouped: rows of A grouped by expert, B = [E * N, K], the tile schedule
+// built on the device from the expert offsets. Dense: tiles in groups of
+// RASTER_M row blocks, row block fastest inside a group.
 // Fused quantization (ABF16): A arrives as BF16. An amax pre-pass has written
 // each row's 448/amax; the producer TMA-loads BF16 A tiles into a 2-slot
 // staging ring, and 8 converter warps turn each into the swizzled E4M3 tile
 // the MMA reads (x * (448/amax), cvt.rn.satfinite: the standalone quantizer's
 // bytes), so the codes never go through HBM.
 // BF16 operands (W16): the same pipeline with BF16 A and B tiles (64 elements
-// = 128 bytes per k-block row, tcgen05.mma kind::f16), no scales; used by the
-// shared expert ("Lernex/Metis-1.6-Praxis" card, "Architecture": one shared
-// expert beside the routed ones; kept in BF16 by the FP8 cards). Its
+// = 128 bytes per k-block row, tcgen05.mma kind::f16). Without scales it is
+// the shared expert's GEMM ("Lernex/Metis-1.6-Praxis" card, "Architecture":
+// one shared expert beside the routed ones; kept in BF16 by the FP8 cards);
+// with per-column scales (SCALED) it is the default maths on weights widened
+// to BF16 beforehand: y = bf16(acc * s_w[n]). The shared expert's
 // down-projection can add the routed experts' weighted outputs in the
 // epilogue: y[t] = bf16(s[t] + sum_j w[t,j] o[row(t,j)]) with s the BF16
 // product, so the routed combine needs no kernel and s never reaches HBM.

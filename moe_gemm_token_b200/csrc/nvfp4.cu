@@ -11,24 +11,34 @@
 //                        8 bytes of packed codes, and every fourth lane writes
 //                        the 4 scales of its 64-element chunk as one word, in
 //                        row-major or in the tensor cores' tiled layout.
-//   nvfp4_gemm_kernel    persistent, warp-specialised block-scaled GEMM,
-//                        128 x 256 tiles, 576 threads per CTA:
-//                          warp 0      TMA of the A and B code tiles (128-byte
-//                                      swizzle) and bulk copies of the tiled
-//                                      scale atoms into a 3-stage ring;
-//                          warp 1      TMEM owner; one lane copies each
-//                                      stage's scale atoms into TMEM
-//                                      (tcgen05.cp 32x128b.warpx4) and issues
-//                                      tcgen05.mma kind::mxf4nvf4 block16;
-//                          warps 2-17  epilogue: four warps per TMEM lane
-//                                      quadrant, 64 columns each, read the
-//                                      whole accumulator at once, release it,
-//                                      then scale (g_a[row] * g_b), round to
-//                                      BF16 and store through a swizzled
-//                                      staging block.
+//   nvfp4_gemm_kernel    persistent, warp-specialised block-scaled GEMM
+//                        (tcgen05.mma kind::mxf4nvf4 block16, K = 64 per
+//                        instruction), 704 threads per CTA. CTA pairs
+//                        (cta_group::2, 256 x 256 tiles) for the grouped GEMM
+//                        and for M > 128; one CTA (128 x 256) otherwise.
+//                          warp 0       TMA of the A and B code tiles (128-byte
+//                                       swizzle) and of the stage's tiled scale
+//                                       atoms (pairs: TMA through a 256-byte-row
+//                                       view, completing on the even CTA's
+//                                       barrier; one CTA: bulk copies) into a
+//                                       ring of 5 (pairs, dense), 4 (pairs,
+//                                       grouped) or 3 (one CTA) stages;
+//                          warp 1       TMEM owner; one lane of the even CTA
+//                                       issues the MMAs;
+//                          warps 2-17   epilogue: four warps per TMEM lane
+//                                       quadrant, 64 columns each, read the
+//                                       whole accumulator at once, hand it back
+//                                       with a relaxed arrive, then scale
+//                                       (g_a[row] * g_b), round to BF16 and
+//                                       store through a swizzled staging block;
+//                          warps 18-21  one per 64-element chunk: copy the
+//                                       chunk's scale atoms of each stage into
+//                                       TMEM (tcgen05.cp 32x128b.warpx4), into
+//                                       the next of four 48-column buffers.
 //                        TMEM: one 256-column FP32 accumulator (the scale
-//                        factors need columns too, so two accumulators do not
-//                        fit in 512) and two 48-column scale buffers.
+//                        buffers need columns too, so two accumulators do not
+//                        fit in 512). Dense tiles run in groups of RASTER_M row
+//                        blocks; grouped tiles follow the padded expert offsets.
 #include "common.cuh"
 #include "../../include/metis_nvfp4.h"
 
