@@ -519,11 +519,24 @@ def secondary_figures(metis, dev, pk):
     out = {}
     hbm = pk["hbm_gbs"]
     peak8 = pk["bf16_tflops"] * FP8_PER_BF16
+    # the tiny linear layer (16 tokens, 256 -> 512): launch-latency bound,
+    # quantizer + E4M3 GEMM per call
+    xt = torch.randn(16, 256, device=dev, generator=g).to(torch.bfloat16)
+    wt, swt = codes(512, 256), torch.rand(512, device=dev, generator=g) * 1e-3
+    xqt = torch.empty(16, 256, dtype=torch.uint8, device=dev)
+    stt = torch.empty(16, device=dev)
+    yt = torch.empty(16, 512, dtype=torch.bfloat16, device=dev)
+
+    def tiny():
+        metis.metis_quant_fp8_per_token(xt, xqt, stt)
+        metis.metis_fp8_gemm(xqt, 0, stt, wt, swt, yt)
+    out["tiny_linear_16x512x256"] = {"us": timeit(tiny, 200) * 1e6}
+    del xt, wt, swt, xqt, stt, yt
     # decode: 4 rotating weight sets (235 MB > L2)
     N, K = 14336, 4096
     ws = [codes(N, K) for _ in range(4)]
     sw = torch.rand(N, device=dev, generator=g) * 1e-3
-    for M in (1, 8):
+    for M in (1, 2, 4, 8):
         x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         i = [0]
@@ -632,9 +645,12 @@ def secondary_figures(metis, dev, pk):
     t = timeit(lambda: metis.metis_moe_fp8_grouped_gemm(x, ids, w, wu, su, wd, sd, y, wsp), 20)
     tf = 2 * 2 * T * k * H * I / t / 1e12
     floor = moe_floor_us(T, H, I, E, k, hbm, peak8, fp4=False)
+    load = torch.bincount(ids.flatten().long(), minlength=E).float()
     out["moe_4096tok_64e_top8"] = {"us": t * 1e6, "tok/s": T / t, "TFLOP/s": tf,
                                    "frac_of_fp8_peak": tf / peak8, "floor_us": floor,
-                                   "frac_of_floor": floor / (t * 1e6)}
+                                   "frac_of_floor": floor / (t * 1e6),
+                                   "hot_expert_load_ratio": float(load[:4].mean() / load.mean()),
+                                   "rows_per_expert_min_max": [int(load.min()), int(load.max())]}
     # the layer with its shared expert (BF16, latent 1024): the routed layer
     # with y = NULL, then the shared expert with the routed combine fused into
     # its down-projection's epilogue
