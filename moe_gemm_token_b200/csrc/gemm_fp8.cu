@@ -680,12 +680,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (i + 1 < CPW) {
                     tmem_ld_32x32b_x32(tbase + (c0 + i + 1) * 32, nxt);
                 } else {
-                    // every column of this accumulator has been read: release it
+                    // every column of this accumulator has been read (and the
+                    // reads waited for): hand it back without a release, which
+                    // would also wait for this warp's earlier global stores
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        if constexpr (CTAS == 2) mbar_arrive_cluster(mapa_shared(tempty(acc), 0));
-                        else mbar_arrive(tempty(acc));
+                        if constexpr (CTAS == 2) mbar_arrive_cluster_relaxed(mapa_shared(tempty(acc), 0));
+                        else mbar_arrive_relaxed(tempty(acc));
                     }
                 }
                 if constexpr (W16) store_chunk_w16<SCALED>(cur, c0 + i, ti, q, lane, sw, stg, cb, p);
@@ -816,9 +818,8 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     Params p{s_a, nullptr, s_b, y, offsets, rows, N, K, E, status, watchdog_ns()};
     CUtensorMap ta, tb;
     if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, ROWS, true))) return rc;
-    if (K < 2048) {
-        // short k-loops: 128-row single-CTA tiles (measured faster for the
-        // routed down-projection, K = 1024, than CTA pairs)
+    if (K < 1024) {
+        // short k-loops: 128-row single-CTA tiles
         using L = Layout<1>;
         if ((rc = prepare<1, true>(di, L::BYTES_GROUPED))) return rc;
         if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
