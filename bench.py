@@ -35,7 +35,9 @@ sys.path.insert(0, ROOT)
 METRIC = "FP8 W8A8 GEMM TFLOP/s & % FP8 peak; 4096-tok prefill tok/s; decode GB/s %HBM"
 M_TOK, K_HID, N_FF = 4096, 2048, 6144
 SETS = 4
-EV_EVERY = 20  # GEMM timing events on every 20th step of the timed graph
+ISO_CALLS = 200  # layer-1 GEMM launches per graph in the isolated roofline timing
+NOMINAL_FP8_TFLOPS = 4500.0  # dense FP8 tensor peak of a B200 (nominal, for context)
+NOMINAL_HBM_GBS = 8000.0  # HBM3e bandwidth of a B200 (nominal, for context)
 FP8_PER_BF16 = 2.0  # nominal dense FP8 : BF16 tensor throughput (4.5 : 2.25 PFLOP/s)
 FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -49,6 +51,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["metis", "reference"], default="metis")
     ap.add_argument("--no-secondary", action="store_true", help="skip the context figures")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--ref-budget", type=float, default=150.0,
+                    help="seconds of oracle work in the reference arm (warm-up + timed steps)")
     return ap.parse_args()
 
 
@@ -121,6 +125,15 @@ def cpu_baseline(budget_s, batch=256):
                       f"2048->6144, quantize, GEMM 6144->2048), float64 oracle, {dt:.1f} s"}
 
 
+def bench_config(world):
+    """The workload of the JSON line, identical in both arms."""
+    return {"workload": "prefill_chain_4096tok_2048x6144x2048", "global_batch": world * M_TOK,
+            "tokens_per_gpu": M_TOK, "layers": "2048->6144 then 6144->2048, no activation",
+            "step": "quantize+GEMM+quantize+GEMM", "parallelism": f"replicas x{world}",
+            "timed_as": "one CUDA graph of the K steps",
+            "l2": f"{SETS} rotating layer sets (x, W1, W2), 169 MB > 126 MB L2"}
+
+
 def run_reference(args):
     rank, world, _ = env_rank()
     if rank != 0:
@@ -132,7 +145,7 @@ def run_reference(args):
     t0 = time.perf_counter()
     oracle_prefill_tokens(d, wq, np.arange(8))
     per_tok = (time.perf_counter() - t0) / 8
-    budget = 150.0  # seconds for warm-up + timed steps
+    budget = args.ref_budget  # seconds for warm-up + timed steps
     per_step = max(1, min(M_TOK, int(budget / max(1, args.steps + args.warmup) / per_tok)))
     step_tokens = lambda i: (np.arange(per_step) + i * per_step) % M_TOK
     for i in range(args.warmup):
@@ -147,10 +160,10 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "prefill_chain_4096tok_2048x6144x2048", "tokens_per_step": per_step,
-                   "note": "each step is a bounded sample of the 4096-token batch"},
+        "config": bench_config(world),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": os.cpu_count(), "kind": "oracle",
-                         "sample": f"{per_step} tokens per step of the prefill chain"},
+                         "sample": f"each step a bounded sample of {per_step} of the {M_TOK} tokens of "
+                                   f"the prefill chain (float64 oracle, rows are independent)"},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -252,24 +265,32 @@ def moe_floor_us(T, H, I, E, k, hbm_gbs, peak_tflops, fp4):
     return sum(max(b / (hbm_gbs * 1e9), f / (peak_tflops * 1e12)) for b, f in kernels) * 1e6
 
 
+GEMM_COUNTERS = os.path.join(ROOT, "profiles", "fp8_gemm_prefill_4096x6144x2048.json")
+GEMM_SOURCES = [os.path.join(ROOT, "moe_gemm_token_b200", "csrc", f) for f in ("gemm_fp8.cu", "common.cuh")]
+
+
+def gemm_source_sha():
+    """sha256[:16] of the sources the prefill GEMM kernel is compiled from."""
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
 def gemm_traffic_from_profile():
-    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "fp8_gemm_prefill_4096x6144x2048.md")
-    src = os.path.join(ROOT, "moe_gemm_token_b200", "csrc", "gemm_fp8.cu")
-    if not os.path.exists(path):
+    """DRAM bytes per layer-1 GEMM launch (dram__bytes_read.sum +
+    dram__bytes_write.sum) from the committed ncu counters, if they were taken
+    on the current kernel sources (else None)."""
+    try:
+        with open(GEMM_COUNTERS) as f:
+            c = json.load(f)
+    except (OSError, ValueError):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    vals = {}
-    for line in open(path):
-        if ": " in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(": ", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel source sha256[:16]") != sha:
+    if c.get("kernel_sources_sha256_16") != gemm_source_sha():
         return None
     try:
-        return float(vals["dram bytes per launch"])
-    except (KeyError, ValueError):
+        return float(c["dram_bytes_read"]) + float(c["dram_bytes_write"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -335,21 +356,18 @@ def run_metis(args):
         raise RuntimeError("device status error after warm-up")
 
     # The timed region is one CUDA graph of the K steps (no host launch gaps
-    # between kernels); it is replayed once untimed (upload, warm-up) and once
-    # timed. Timing events inside a graph are nodes of their own and add gaps
-    # (about 4 us each on B200), so the GEMMs are bracketed by events on every
-    # EV_EVERY-th step only.
+    # between kernels, no timing events inside); it is replayed once untimed
+    # (upload, warm-up) and once timed, bracketed by events on the stream it
+    # runs on.
     cap = torch.cuda.Stream(device=dev)
     cap.wait_stream(stream)
-    sampled = [i for i in range(args.steps) if i % EV_EVERY == EV_EVERY // 2] or [0]
-    evs = {i: [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for i in sampled}
     start = torch.cuda.Event(enable_timing=True, external=True)
     end = torch.cuda.Event(enable_timing=True, external=True)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=cap):
         start.record(cap)
         for i in range(args.steps):
-            step(i, cap, evs.get(i))
+            step(i, cap)
         end.record(cap)
     torch.cuda.synchronize()
     graph.replay()
@@ -365,27 +383,84 @@ def run_metis(args):
     elapsed_ms = max_over_ranks(start.elapsed_time(end), dist, dev, world)
     ms_per_step = elapsed_ms / args.steps
     value = job_throughput(world, M_TOK, ms_per_step)
+    del graph
 
-    # ---- roofline of the dominant kernel (the W8A8 GEMM), from the live events
-    g1 = [e[0].elapsed_time(e[1]) for e in evs.values()]
-    g2 = [e[2].elapsed_time(e[3]) for e in evs.values()]
-    gemm_ms = (statistics.mean(g1) + statistics.mean(g2)) / 2
-    flops = 2.0 * M_TOK * K_HID * N_FF
-    achieved = flops / (gemm_ms * 1e-3) / 1e12
+    # ---- roofline of the dominant kernel (the W8A8 GEMM, layer 1 shape)
     pk, pk_kind = peaks()
-    # the GEMM runs inside a long timed region (power-capped clocks): the
-    # sustained tensor figure is its denominator
-    peak = pk["bf16_tflops_sustained"] * FP8_PER_BF16
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": gemm_traffic_from_profile(),
-                "kernel": "fp8_gemm_kernel (tcgen05 kind::f8f6f4, cta_group::2, 256x256 tiles per CTA pair)",
-                "peak_source": f"{pk_kind} bf16 sustained {pk['bf16_tflops_sustained']} TFLOP/s x "
-                               f"{FP8_PER_BF16} (nominal FP8:BF16 dense ratio); burst would be "
-                               f"{pk['bf16_tflops'] * FP8_PER_BF16:.0f}",
-                "gemm_samples": len(g1),
-                "gemm_timing_note": "events inside the graph add a launch gap before each bracketed "
-                                    "GEMM, so these durations (and frac) err low",
-                "gemm_ms": [statistics.mean(g1), statistics.mean(g2)]}
+    flops = 2.0 * M_TOK * K_HID * N_FF
+    burst = pk["bf16_tflops"] * FP8_PER_BF16
+    sustained = pk["bf16_tflops_sustained"] * FP8_PER_BF16
+    # (a) in isolation: ISO_CALLS layer-1 GEMMs in one CUDA graph, rotating
+    # the SETS layer sets (A codes and W1 of every set: 84 MB, plus the 50 MB
+    # output), replayed 3 times between two events on the replay stream. Its
+    # denominator is the burst tensor figure (a kernel timed alone).
+    xq_sets = []
+    for s in sets:
+        q = torch.empty((M_TOK, K_HID), dtype=torch.uint8, device=dev)
+        sc = torch.empty((M_TOK,), dtype=torch.float32, device=dev)
+        metis.metis_quant_fp8_per_token(s["x"], q, sc, stream)
+        xq_sets.append((q, sc))
+    torch.cuda.synchronize()
+
+    def gemm1(i, st):
+        (q, sc), (w1, s1) = xq_sets[i % SETS], sets[i % SETS]["w"][0]
+        metis.metis_fp8_gemm(q, metis.METIS_A_E4M3, sc, w1, s1, y1, stream=st)
+
+    for i in range(2 * SETS):
+        gemm1(i, stream)
+    torch.cuda.synchronize()
+    iso_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(iso_graph, stream=cap):
+        for i in range(ISO_CALLS):
+            gemm1(i, cap)
+    torch.cuda.synchronize()
+    iso_graph.replay()
+    torch.cuda.synchronize()
+    a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    a_ev.record(stream)
+    for _ in range(reps):
+        iso_graph.replay()
+    b_ev.record(stream)
+    torch.cuda.synchronize()
+    iso_ms = a_ev.elapsed_time(b_ev) / (reps * ISO_CALLS)
+    del iso_graph
+    achieved = flops / (iso_ms * 1e-3) / 1e12
+    # (b) inside the step, as a cross-check: a separate replay of the step
+    # graph with events around both GEMMs of every step. An event inside a
+    # graph is a node of its own and adds a launch gap before the bracketed
+    # GEMM, so these durations err low; they do not enter the timed region.
+    n_ev = max(10, min(args.steps, 50))
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(n_ev)]
+    ev_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ev_graph, stream=cap):
+        for i in range(n_ev):
+            step(i, cap, evs[i])
+    torch.cuda.synchronize()
+    ev_graph.replay()
+    torch.cuda.synchronize()
+    ev_graph.replay()
+    torch.cuda.synchronize()
+    g1 = [e[0].elapsed_time(e[1]) for e in evs]
+    g2 = [e[2].elapsed_time(e[3]) for e in evs]
+    del ev_graph
+    in_step = flops / (statistics.median(g1) * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                "frac": achieved / burst, "traffic": gemm_traffic_from_profile(),
+                "kernel": "fp8_gemm_kernel (tcgen05 kind::f8f6f4, cta_group::2, 256x256 tiles per CTA pair), "
+                          "M=4096 N=6144 K=2048",
+                "peak_source": f"{pk_kind} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP8_PER_BF16} "
+                               f"(nominal FP8:BF16 dense ratio)",
+                "timed_as": f"{ISO_CALLS} GEMM launches per CUDA graph, {SETS} rotating input sets, "
+                            f"{reps} replays between events",
+                "us_per_launch": iso_ms * 1e3,
+                "frac_of_sustained": achieved / sustained,
+                "frac_of_nominal_fp8": achieved / NOMINAL_FP8_TFLOPS,
+                "in_step": {"achieved": in_step, "frac": in_step / burst, "gemm_samples": len(g1),
+                            "layer1_us_median": statistics.median(g1) * 1e3,
+                            "layer2_us_median": statistics.median(g2) * 1e3,
+                            "note": "events inside a step graph (not the timed one); each adds a "
+                                    "launch gap before the GEMM, so these figures err low"}}
 
     # ---- end to end through the C ABI with host buffers. Every step uploads
     # its input from pinned host memory, runs the two layers through
@@ -461,11 +536,7 @@ def run_metis(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
             "data": "synthetic",
-            "config": {"workload": "prefill_chain_4096tok_2048x6144x2048", "global_batch": world * M_TOK,
-                       "tokens_per_gpu": M_TOK, "layers": "2048->6144 then 6144->2048, no activation",
-                       "step": "quantize+GEMM+quantize+GEMM", "parallelism": f"replicas x{world}",
-                       "timed_as": "one CUDA graph of the K steps; GEMM events on every 20th step",
-                       "l2": f"{SETS} rotating layer sets (x, W1, W2), 169 MB > 126 MB L2"},
+            "config": bench_config(world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(), "secondary": secondary,
@@ -547,21 +618,25 @@ def secondary_figures(metis, dev, pk):
         t = timeit(f, 200)
         byt = N * K + 4 * N + 2 * M * K + 2 * M * N
         out[f"decode_w8a16_M{M}"] = {"us": t * 1e6, "GB/s": byt / t / 1e9,
-                                     "frac_of_measured_hbm": byt / t / 1e9 / hbm}
+                                     "frac_of_measured_hbm": byt / t / 1e9 / hbm,
+                                     "frac_of_nominal_hbm": byt / t / 1e9 / NOMINAL_HBM_GBS}
     del ws
     # quantizer at the prefill and large-M shapes (2 rotating inputs > L2)
-    for (M, K) in [(4096, 2048), (16384, 8192)]:
-        xs = [torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16) for _ in range(2)]
+    for (M, K) in [(4096, 2048), (4096, 6144), (16384, 8192)]:
+        # enough rotating inputs that they cannot stay in the 126 MB L2
+        n_in = max(2, -(-2 * 126 * 2 ** 20 // (2 * M * K)) + 1)
+        xs = [torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16) for _ in range(n_in)]
         xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
         s = torch.empty(M, device=dev)
         i = [0]
 
         def f():
-            i[0] ^= 1
+            i[0] = (i[0] + 1) % n_in
             metis.metis_quant_fp8_per_token(xs[i[0]], xq, s)
         t = timeit(f, 100)
         out[f"quant_{M}x{K}"] = {"us": t * 1e6, "GB/s": (3 * M * K + 4 * M) / t / 1e9,
-                                 "frac_of_measured_hbm": (3 * M * K + 4 * M) / t / 1e9 / hbm}
+                                 "frac_of_measured_hbm": (3 * M * K + 4 * M) / t / 1e9 / hbm,
+                                 "frac_of_nominal_hbm": (3 * M * K + 4 * M) / t / 1e9 / NOMINAL_HBM_GBS}
         del xs
     # large-M W8A8 GEMM from BF16 activations (per-token magnitudes
     # log-uniform in [1e-2, 1e2]): the GEMM alone, the separate quantizer +
@@ -587,6 +662,7 @@ def secondary_figures(metis, dev, pk):
         t_f = timeit(lambda: metis.metis_fp8_gemm(x, 1, sa, b, sb, y, workspace=wsf), 10)
         out[f"gemm_{M}x{K}x{K}"] = {
             "us": t_g * 1e6, "TFLOP/s": fl / t_g / 1e12, "frac_of_fp8_peak": fl / t_g / 1e12 / peak8,
+            "frac_of_nominal_fp8": fl / t_g / 1e12 / NOMINAL_FP8_TFLOPS,
             "quant+gemm_us": t_s * 1e6, "quant+gemm_TFLOP/s": fl / t_s / 1e12,
             "fused_quant_us": t_f * 1e6, "fused_quant_TFLOP/s": fl / t_f / 1e12}
         del x, xq, b, y

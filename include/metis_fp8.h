@@ -86,8 +86,9 @@ METIS_API int metis_watchdog_selftest(uint64_t limit_ns, metis_stream_t stream);
 
 /* Reads (and, if `clear` != 0, clears) the sticky device error word on the
  * current device, synchronising `stream` first. Returns METIS_OK,
- * METIS_ERR_TIMEOUT if a kernel's bounded wait ran out, or METIS_ERR_CUDA.
- * This is the one entry point that synchronises. */
+ * METIS_ERR_TIMEOUT if a kernel's bounded wait ran out, METIS_ERR_INVALID_ARG
+ * if a routed-expert layer met a routing id outside [0, E) (that slot was
+ * dropped), or METIS_ERR_CUDA. This is the one entry point that synchronises. */
 METIS_API int metis_check_device_status(metis_stream_t stream, int clear);
 
 /* Sets the per-wait limit of the device watchdog in nanoseconds (default
@@ -188,8 +189,9 @@ METIS_API int metis_moe_route_topk(const float* logits, const float* bias, int64
  * the routed experts are FP8 with per-channel scales and per-token
  * activations). Steps, all on the device, no host synchronisation:
  * routing histogram -> exclusive prefix sum -> stable permutation of the
- * slots (t, j) by expert -> per-token quantization of x (once per token,
- * written into the expert-contiguous rows of its slots) -> grouped up-projection (W8A8) ->
+ * slots (t, j) by expert -> per-token quantization of x (once per token, in
+ * token order) -> grouped up-projection (W8A8; its operand rows gathered by
+ * token in the GEMM's TMA producer, never copied per slot) ->
  * per-row re-quantization -> grouped down-projection (W8A8) -> weighted
  * un-permute y[t] = sum_j topk_w[t,j] o[t,j] (FP32, j ascending) -> BF16.
  *   x [T, H] BF16, topk_ids [T, topk] int32 in [0, E), topk_w [T, topk] FP32,
@@ -198,8 +200,12 @@ METIS_API int metis_moe_route_topk(const float* logits, const float* bias, int64
  *   and leaves o and the routing in the workspace for
  *   metis_moe_shared_fused_combine (no combine kernel runs).
  *   act must be METIS_ACT_NONE (the cards do not state the experts' activation).
- *   Requires H % 16 == 0, I % 16 == 0, 16 <= H <= 16384, I >= 16, 1 <= topk <= E <= 1024;
- *   ids outside [0, E) are a caller error (not checked on the device).
+ *   Requires H % 16 == 0, I % 16 == 0, 16 <= H <= 16384, I >= 16, 1 <= topk <= E <= 1024.
+ *   Ids outside [0, E) are checked on the device (the ids stay on the GPU, so
+ *   the host cannot see them): such a slot is dropped from the layer (its
+ *   SLOT_TO_ROW entry is -1 and it adds nothing to y[t]; the token's other
+ *   slots are unaffected) and the sticky device error word records it, so the
+ *   next metis_check_device_status() returns METIS_ERR_INVALID_ARG.
  *   Needs `workspace` of metis_workspace_size(METIS_OP_MOE, T, I, H, topk, E)
  *   bytes (256-byte aligned); its regions are given by metis_moe_workspace_offset. */
 #define METIS_ACT_NONE 0
@@ -219,9 +225,12 @@ METIS_API int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* topk
  * library, which each GPU that loads the library keeps until the process exits.
  *   - Problems whose metis_workspace_size(METIS_OP_MOE, ...) exceeds 16 MiB are
  *     rejected with METIS_ERR_INVALID_ARG before anything is launched (about
- *     200 tokens at top-8 with H = 2048, I = 1024).
- *   - The first call on each device looks up the array's device address; make
- *     that first call before any stream capture.
+ *     280 tokens at top-8 with H = 2048, I = 1024).
+ *   - y must not be NULL: the routed outputs would otherwise stay in the
+ *     built-in array, which the caller cannot address (METIS_ERR_INVALID_ARG).
+ *   - The first call on each device (and the first after a cudaDeviceReset,
+ *     which moves the array) looks up the array's device address; make that
+ *     first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents (nothing in it needs to start at zero). Calls that may
  *     overlap on the GPU, e.g. on two streams, race on it: serialise them. */
@@ -286,8 +295,9 @@ METIS_API size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, in
  *   METIS_MOE_WS_OFFSETS     int32 [E + 1]  exclusive prefix sum of COUNTS
  *   METIS_MOE_WS_SLOT_TO_ROW int32 [S]      row of slot s = t*topk + j in expert order
  *   METIS_MOE_WS_ROW_TO_SLOT int32 [S]      inverse permutation
- *   METIS_MOE_WS_AQ          E4M3  [S, H]   per-token codes of x, one row per slot, expert order
- *   METIS_MOE_WS_SA          FP32  [S]      their per-token scales
+ *   METIS_MOE_WS_AQ          E4M3  [T, H]   per-token codes of x, token order (the up-projection
+ *                                           gathers expert t's rows from it by token)
+ *   METIS_MOE_WS_SA          FP32  [T]      their per-token scales
  *   METIS_MOE_WS_H           BF16  [S, I]   up-projection output, expert order
  *   METIS_MOE_WS_HQ          E4M3  [S, I]   its per-row codes
  *   METIS_MOE_WS_SH          FP32  [S]      their scales

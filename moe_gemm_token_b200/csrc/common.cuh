@@ -33,6 +33,10 @@ int current_device_info(DeviceInfo* out);
 
 // Device address of the sticky error word of the current device.
 int device_status_word(uint32_t** out);
+// Unique id of the calling thread's current CUDA context (made current first):
+// device addresses of __device__ variables looked up in one context are
+// cached under this id and looked up again when it changes.
+int current_context_id(uint64_t* out);
 // Per-wait watchdog limit (ns) for kernels launched now.
 uint64_t watchdog_ns();
 

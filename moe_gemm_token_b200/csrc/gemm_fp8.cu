@@ -112,6 +112,16 @@ struct Params {
     const int32_t* s2r;      // [rows of A * topk]; negative: slot dropped
     const float* topk_w;     // [rows of A * topk]
     int topk;
+    // dense tail pieces: tiles past `full` are cut into `split` column pieces,
+    // whose B rows come through the second tensor map (box of BN/split/CTAS rows)
+    int full;
+    int split;
+    // grouped, gathered A (a_rows non-null): row r of the grouped operand is
+    // row a_rows[r] / a_div of the tensor behind tmA (and of s_a), fetched by
+    // 4-row TMA gathers; rows at or past the group's end read row 0
+    const int32_t* a_rows;
+    int a_div;
+    int a_src_rows;  // rows of the tensor behind tmA
 };
 
 struct Tile {
@@ -120,11 +130,14 @@ struct Tile {
     int b_row0;   // first row of B loaded by this CTA
     int n0;       // first output column
     int group;
+    int bn;       // output columns of this tile: BN, or BN / split for a piece of the tail
 };
 
 template <int CTAS, int BN>
 struct Sched {
     int num_n, num_m, total, E, N, M;
+    int full;   // dense: tiles [0, full) are whole; each later tile is cut into `split` pieces
+    int split;  // dense: 1 (no cut), 2 or 4 column pieces per tail tile
     uint32_t rank;
     const int* g_tile;  // grouped: prefix sums of tiles per group [E + 1] (smem)
     const int* g_row;   // grouped: row offsets [E + 1] (smem)
@@ -132,6 +145,18 @@ struct Sched {
     __device__ __forceinline__ Tile get(int t) const {
         Tile ti;
         if (g_tile == nullptr) {
+            // The last tiles of a persistent grid whose tile count is not a
+            // multiple of the CTA pairs would leave most pairs idle in the
+            // final wave: those tiles are cut into `split` column pieces
+            // (BN / split columns each), one piece per pair.
+            int q = 0;
+            ti.bn = BN;
+            if (t >= full) {
+                const int u = t - full;
+                t = full + u / split;
+                q = u - (u / split) * split;
+                ti.bn = BN / split;
+            }
             // groups of RASTER_M row blocks, row block fastest inside a group:
             // the tiles running together share a few row blocks of A and
             // column blocks of B in L2
@@ -142,8 +167,8 @@ struct Sched {
             const int nb = r / gm;
             ti.a_row0 = mb * ROWS * CTAS + static_cast<int>(rank) * ROWS;
             ti.row_end = M;
-            ti.b_row0 = nb * BN + static_cast<int>(rank) * (BN / CTAS);
-            ti.n0 = nb * BN;
+            ti.n0 = nb * BN + q * ti.bn;
+            ti.b_row0 = ti.n0 + static_cast<int>(rank) * (ti.bn / CTAS);
             ti.group = 0;
         } else {
             int lo = 0, hi = E;  // e with g_tile[e] <= t < g_tile[e + 1]
@@ -162,6 +187,7 @@ struct Sched {
             ti.b_row0 = e * N + nb * BN + static_cast<int>(rank) * (BN / CTAS);
             ti.n0 = nb * BN;
             ti.group = e;
+            ti.bn = BN;
         }
         return ti;
     }
@@ -206,6 +232,28 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, cons
 // L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned address.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Four 128-byte rows (rows r0..r3 of a 2-D tensor whose map has a one-row
+// box, starting at column x) into 512 consecutive bytes of shared memory, in
+// the map's swizzle; completion counted on the mbarrier. No multicast.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, int32_t x, int32_t r0,
+                                            int32_t r1, int32_t r2, int32_t r3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+// The same into this CTA's shared memory, completing on an mbarrier of either
+// CTA of the pair (cta_group::2). No multicast.
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* m, int32_t x, int32_t r0,
+                                                 int32_t r1, int32_t r2, int32_t r3, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
 }
 
 // The W16 epilogue chunk: y = bf16(acc), or bf16(acc * sw[n]) with per-column
@@ -297,7 +345,7 @@ __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, 
 template <int CTAS, bool GROUPED, bool ABF16, int BN, bool W16 = false, bool SCALED = false>
 __global__ void __launch_bounds__(Layout<CTAS, ABF16, BN, W16>::THREADS_, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const Params p) {
+                const __grid_constant__ CUtensorMap tmBq, const Params p) {
     using L = Layout<CTAS, ABF16, BN, W16>;
     constexpr int STAGES = L::STAGES;
     constexpr int EPI = L::EPI;
@@ -350,6 +398,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (p.split > 1) tma_prefetch_desc(&tmBq);
     }
     if (warp == 1) {
         if constexpr (CTAS == 2) {
@@ -373,6 +422,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     sc.E = p.E;
     sc.rank = rank;
     sc.num_n = (p.N + BN - 1) / BN;
+    sc.split = p.split > 1 ? p.split : 1;
+    sc.full = p.split > 1 ? p.full : 0x7fffffff;
     if constexpr (GROUPED) {
         // prefix sums of row offsets and of tiles per group, by warp 0
         if (warp == 0) {
@@ -415,6 +466,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         sc.g_row = nullptr;
         sc.num_m = (p.M + ROWS * CTAS - 1) / (ROWS * CTAS);
         sc.total = sc.num_m * sc.num_n;
+        if (sc.split > 1) sc.total = sc.full + (sc.total - sc.full) * sc.split;
     }
     __syncwarp();
     tc_fence_before();
@@ -427,7 +479,69 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const int stride = CTAS == 2 ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (GROUPED && !ABF16 && !W16 && p.a_rows != nullptr) {
+            // ------------------------------------------ producer, gathered A
+            // Each lane fetches 4 of the CTA's 128 A rows per k-block with one
+            // TMA gather (row r of the group is source row a_rows[r] / a_div);
+            // lane 0 waits for the stage and loads B.
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_phase = 0;
+            for (int t = first; t < sc.total; t += stride) {
+                // the flag is read once for the whole warp (the loop holds warp-wide shuffles)
+                if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+                const Tile ti = sc.get(t);
+                int src[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = ti.a_row0 + lane * 4 + i;
+                    int v = r < ti.row_end ? p.a_rows[r] / p.a_div : 0;
+                    src[i] = min(max(v, 0), p.a_src_rows - 1);
+                }
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (lane == 0) ok = mbar_wait(empty(stage), phase ^ 1u, p.timeout_ns, p.status);
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    if (!ok) break;
+                    const uint32_t dst = smem_u32(sA + stage * L::A_STAGE) + lane * 4 * BK;
+                    if constexpr (CTAS == 2) {
+                        const uint32_t fl = mapa_shared(full(stage), 0);
+                        if (lane == 0) {
+                            if (leader) mbar_arrive_expect_tx(full(stage), CTAS * (L::A_STAGE + L::B_STAGE));
+                            tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * L::KE, ti.b_row0, fl);
+                        }
+                        __syncwarp();
+                        tma_gather4_pair(dst, &tmA, kb * L::KE, src[0], src[1], src[2], src[3], fl);
+                    } else {
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(full(stage), L::A_STAGE + L::B_STAGE);
+                            tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * L::KE, ti.b_row0, full(stage));
+                        }
+                        __syncwarp();
+                        tma_gather4(dst, &tmA, kb * L::KE, src[0], src[1], src[2], src[3], full(stage));
+                    }
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) {
+                    if (lane == 0) *abort_flag = 1;
+                    break;
+                }
+            }
+            __syncwarp();
+            if (lane == 0 && *abort_flag) {
+                // let the copies in flight land before the CTA exits
+                if (leader) {
+                    for (int s = 0; s < STAGES; ++s)
+                        if (issued & (1u << s))
+                            mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
+                } else {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 100000ull) {}
+                }
+            }
+        } else if (lane == 0) {
             // ---------------------------------------------------------- producer
             int stage = 0;
             uint32_t phase = 0;
@@ -462,14 +576,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         tma_load_2d(dst + ASTG_SLOT / 2, &tmA, kb * BK + BK / 2, ti.a_row0, bfull(slot));
                         if (++slot == L::ASTG) { slot = 0; sphase ^= 1u; }
                     } else if constexpr (CTAS == 2) {
+                        // a tail piece loads only its BN/split columns' rows of B
+                        const bool piece = ti.bn != BN;
+                        const uint32_t b_bytes = piece ? static_cast<uint32_t>(ti.bn / CTAS) * BK : L::B_STAGE;
                         const uint32_t fl = mapa_shared(full(stage), 0);
-                        if (leader) mbar_arrive_expect_tx(full(stage), CTAS * (L::A_STAGE + L::B_STAGE));
+                        if (leader) mbar_arrive_expect_tx(full(stage), CTAS * (L::A_STAGE + b_bytes));
                         tma_load_2d_pair(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * L::KE, ti.a_row0, fl);
-                        tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * L::KE, ti.b_row0, fl);
+                        tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), piece ? &tmBq : &tmB, kb * L::KE,
+                                         ti.b_row0, fl);
                     } else {
-                        mbar_arrive_expect_tx(full(stage), L::A_STAGE + L::B_STAGE);
+                        const bool piece = ti.bn != BN;
+                        const uint32_t b_bytes = piece ? static_cast<uint32_t>(ti.bn) * BK : L::B_STAGE;
+                        mbar_arrive_expect_tx(full(stage), L::A_STAGE + b_bytes);
                         tma_load_2d(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * L::KE, ti.a_row0, full(stage));
-                        tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * L::KE, ti.b_row0, full(stage));
+                        tma_load_2d(smem_u32(sB + stage * L::B_STAGE), piece ? &tmBq : &tmB, kb * L::KE,
+                                    ti.b_row0, full(stage));
                     }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -505,6 +626,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                // tail pieces of the dense schedule are narrower (N = BN / split)
+                uint32_t idesc = L::IDESC;
+                if constexpr (!GROUPED && !W16 && !ABF16) {
+                    const int bn = sc.get(t).bn;
+                    if (bn != BN) idesc = idesc_e4m3_f32(ROWS * CTAS, bn);
+                }
                 bool ok = true;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(full(stage), phase, p.timeout_ns, p.status)) {
@@ -520,13 +647,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         // (32 bytes: 32 E4M3 or 16 BF16 elements per instruction)
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
                         if constexpr (W16 && CTAS == 2)
-                            mma_f16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
+                            mma_f16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
                         else if constexpr (W16)
-                            mma_f16_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
+                            mma_f16_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
                         else if constexpr (CTAS == 2)
-                            mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
+                            mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
                         else
-                            mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, L::IDESC, accum);
+                            mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
                     }
                     if constexpr (CTAS == 2) mma_commit_pair_mc(empty(stage), 0x3);
                     else mma_commit(empty(stage));
@@ -656,7 +783,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (et < BN / 2) reinterpret_cast<float2*>(sw_smem + acc * BN)[et] = v;
             }
             const int row = ti.a_row0 + q * 32 + lane;
-            const float rs = (!W16 && row < ti.row_end) ? p.s_a[row] : 0.0f;
+            float rs = 0.0f;
+            if (!W16 && row < ti.row_end)
+                rs = (GROUPED && p.a_rows != nullptr) ? p.s_a[p.a_rows[row] / p.a_div] : p.s_a[row];
             // all epilogue threads have written their scales (bounded wait)
             mbar_arrive(epi_sync(acc));
             if (!mbar_wait(epi_sync(acc), acc_phase, p.timeout_ns, p.status) ||
@@ -668,31 +797,44 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const float* sw = sw_smem + acc * BN;
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-            // chunks c0 .. c0 + CPW - 1, the next one loading while this one is
-            // stored; the accumulator is released once the last load completed
-            uint32_t va[32], vb[32];
-            tmem_ld_32x32b_x32(tbase + c0 * 32, va);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < CPW; ++i) {
-                uint32_t(&cur)[32] = (i & 1) ? vb : va;
-                uint32_t(&nxt)[32] = (i & 1) ? va : vb;
-                if (i + 1 < CPW) {
-                    tmem_ld_32x32b_x32(tbase + (c0 + i + 1) * 32, nxt);
-                } else {
-                    // every column of this accumulator has been read (and the
-                    // reads waited for): hand it back without a release, which
-                    // would also wait for this warp's earlier global stores
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if constexpr (CTAS == 2) mbar_arrive_cluster_relaxed(mapa_shared(tempty(acc), 0));
-                        else mbar_arrive_relaxed(tempty(acc));
-                    }
+            // hand the accumulator back once every read of it has completed,
+            // without a release fence (which would also wait for this warp's
+            // earlier global stores)
+            auto hand_back = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (CTAS == 2) mbar_arrive_cluster_relaxed(mapa_shared(tempty(acc), 0));
+                    else mbar_arrive_relaxed(tempty(acc));
                 }
-                if constexpr (W16) store_chunk_w16<SCALED>(cur, c0 + i, ti, q, lane, sw, stg, cb, p);
-                else store_chunk(cur, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N);
-                if (i + 1 < CPW) tmem_ld_wait();
+            };
+            uint32_t va[32], vb[32];
+            if (!GROUPED && !W16 && !ABF16 && ti.bn != BN) {
+                // a narrow tail piece: this warp's chunks that fall inside it,
+                // one at a time
+                const int nval = min(CPW, max(0, (ti.bn - c0 * 32 + 31) / 32));
+                for (int i = 0; i < nval; ++i) {
+                    tmem_ld_32x32b_x32(tbase + (c0 + i) * 32, va);
+                    tmem_ld_wait();
+                    if (i + 1 == nval) hand_back();
+                    store_chunk(va, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N);
+                }
+                if (nval == 0) hand_back();
+            } else {
+                // chunks c0 .. c0 + CPW - 1, the next one loading while this
+                // one is stored
+                tmem_ld_32x32b_x32(tbase + c0 * 32, va);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < CPW; ++i) {
+                    uint32_t(&cur)[32] = (i & 1) ? vb : va;
+                    uint32_t(&nxt)[32] = (i & 1) ? va : vb;
+                    if (i + 1 < CPW) tmem_ld_32x32b_x32(tbase + (c0 + i + 1) * 32, nxt);
+                    else hand_back();
+                    if constexpr (W16) store_chunk_w16<SCALED>(cur, c0 + i, ti, q, lane, sw, stg, cb, p);
+                    else store_chunk(cur, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N);
+                    if (i + 1 < CPW) tmem_ld_wait();
+                }
             }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
@@ -753,13 +895,28 @@ int max_pairs(const DeviceInfo& di, int* out) {
     return METIS_OK;
 }
 
+// The persistent grid runs `tiles` whole tiles on `workers` CTAs (pairs): the
+// last tiles % workers of them form a final wave that keeps few workers busy
+// (4096 x 6144 on 74 pairs: 384 tiles, 14 in the last wave). When that wave
+// would occupy at most a quarter (half) of the workers, each of its tiles is
+// cut into 4 (2) column pieces of BN/4 (BN/2) columns, one piece per worker,
+// so the final wave ends in a fraction of a tile's time.
+inline int tail_split(int tiles, int workers) {
+    if (tiles <= workers) return 1;
+    const int r = tiles % workers;
+    if (r == 0) return 1;
+    if (4 * r <= workers) return 4;
+    if (2 * r <= workers) return 2;
+    return 1;
+}
+
 // Dense E4M3 GEMM with BN-column tiles: CTA pairs (256-row tiles) for
-// M > 128, single CTAs otherwise.
+// M > 128, single CTAs otherwise; the final partial wave in column pieces.
 template <int BN>
-int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, const Params& p,
+int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, Params p,
                  int M, int N, int K, cudaStream_t st) {
     int rc;
-    CUtensorMap tb;
+    CUtensorMap tb, tbq;
     const int num_n = (N + BN - 1) / BN;
     if (M > ROWS) {
         using L = Layout<2, false, BN>;
@@ -769,8 +926,14 @@ int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, 
         if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
         const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
         const int clusters = tiles < pairs ? tiles : pairs;
+        p.split = tail_split(tiles, clusters);
+        p.full = tiles - (p.split > 1 ? tiles % clusters : 0);
+        tbq = tb;
+        if (p.split > 1 &&
+            (rc = make_tmap_2d(&tbq, b, 1, K, N, K, BK, static_cast<uint32_t>(L::B_ROWS / p.split), true)))
+            return rc;
         return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, false, BN>, dim3(2 * clusters), dim3(L::THREADS_),
-                                     L::BYTES_DENSE, st, 2, ta, tb, p),
+                                     L::BYTES_DENSE, st, 2, ta, tb, tbq, p),
                           "fp8 gemm (CTA pair) launch");
     }
     using L = Layout<1, false, BN>;
@@ -778,8 +941,14 @@ int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, 
     if ((rc = make_tmap_2d(&tb, b, 1, K, N, K, BK, L::B_ROWS, true))) return rc;
     const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
+    p.split = tail_split(tiles, grid);
+    p.full = tiles - (p.split > 1 ? tiles % grid : 0);
+    tbq = tb;
+    if (p.split > 1 &&
+        (rc = make_tmap_2d(&tbq, b, 1, K, N, K, BK, static_cast<uint32_t>(L::B_ROWS / p.split), true)))
+        return rc;
     return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, false, BN>, dim3(grid), dim3(L::THREADS_),
-                                 L::BYTES_DENSE, st, 1, ta, tb, p),
+                                 L::BYTES_DENSE, st, 1, ta, tb, tbq, p),
                       "fp8 gemm launch");
 }
 
@@ -807,7 +976,7 @@ int launch_fp8_gemm_dense(const uint8_t* a, const float* s_a, const uint8_t* b, 
 // [e*N, (e+1)*N). `rows` is the row count of A and y (offsets[E] <= rows).
 int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b, const float* s_b,
                             __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
-                            int K, cudaStream_t st) {
+                            int K, cudaStream_t st, const int32_t* a_rows, int a_div, int a_src_rows) {
     using namespace gemm;
     if (E > MAX_GROUPS) return fail(METIS_ERR_UNSUPPORTED, "grouped gemm: E=%d > %d", E, MAX_GROUPS);
     DeviceInfo di;
@@ -817,7 +986,15 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     if ((rc = device_status_word(&status))) return rc;
     Params p{s_a, nullptr, s_b, y, offsets, rows, N, K, E, status, watchdog_ns()};
     CUtensorMap ta, tb;
-    if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, ROWS, true))) return rc;
+    if (a_rows != nullptr) {
+        // A gathered by rows from a [a_src_rows, K] tensor: one-row boxes
+        p.a_rows = a_rows;
+        p.a_div = a_div;
+        p.a_src_rows = a_src_rows;
+        if ((rc = make_tmap_2d(&ta, a, 1, K, a_src_rows, K, BK, 1, true))) return rc;
+    } else if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, ROWS, true))) {
+        return rc;
+    }
     if (K < 1024) {
         // short k-loops: 128-row single-CTA tiles
         using L = Layout<1>;
@@ -825,7 +1002,7 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
         if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
             return rc;
         return cuda_check(launch_pdl(fp8_gemm_kernel<1, true, false, BN_MAX>, dim3(di.num_sms), dim3(L::THREADS_),
-                                     L::BYTES_GROUPED, st, 1, ta, tb, p),
+                                     L::BYTES_GROUPED, st, 1, ta, tb, tb, p),
                           "grouped fp8 gemm launch");
     }
     // CTA pairs on 256-row tiles: each SM streams half of B (routed
@@ -837,7 +1014,7 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
         return rc;
     return cuda_check(launch_pdl(fp8_gemm_kernel<2, true, false, BN_MAX>, dim3(2 * pairs), dim3(L::THREADS_),
-                                 L::BYTES_GROUPED, st, 2, ta, tb, p),
+                                 L::BYTES_GROUPED, st, 2, ta, tb, tb, p),
                       "grouped fp8 gemm (CTA pair) launch");
 }
 
@@ -865,7 +1042,7 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
         const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
         const int clusters = tiles < pairs ? tiles : pairs;
         return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, true, BN_MAX>, dim3(2 * clusters), dim3(L::THREADS_),
-                                     L::BYTES_DENSE, st, 2, ta, tb, p),
+                                     L::BYTES_DENSE, st, 2, ta, tb, tb, p),
                           "fused fp8 gemm (CTA pair) launch");
     }
     using L = Layout<1, true>;
@@ -874,7 +1051,7 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
     const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
     return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, true, BN_MAX>, dim3(grid), dim3(L::THREADS_),
-                                 L::BYTES_DENSE, st, 1, ta, tb, p),
+                                 L::BYTES_DENSE, st, 1, ta, tb, tb, p),
                       "fused fp8 gemm launch");
 }
 
@@ -900,7 +1077,7 @@ int launch_w16(const __nv_bfloat16* a, const __nv_bfloat16* b, const Params& p, 
         const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
         const int clusters = tiles < pairs ? tiles : pairs;
         return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, false, BN_MAX, true, SCALED>, dim3(2 * clusters),
-                                     dim3(L::THREADS_), L::BYTES_DENSE, st, 2, ta, tb, p),
+                                     dim3(L::THREADS_), L::BYTES_DENSE, st, 2, ta, tb, tb, p),
                           "bf16 gemm (CTA pair) launch");
     }
     using L = Layout<1, false, BN_MAX, true>;
@@ -909,7 +1086,7 @@ int launch_w16(const __nv_bfloat16* a, const __nv_bfloat16* b, const Params& p, 
     const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
     return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, false, BN_MAX, true, SCALED>, dim3(grid),
-                                 dim3(L::THREADS_), L::BYTES_DENSE, st, 1, ta, tb, p),
+                                 dim3(L::THREADS_), L::BYTES_DENSE, st, 1, ta, tb, tb, p),
                       "bf16 gemm launch");
 }
 

@@ -8,9 +8,10 @@
 //   2. prefix sums: per-expert offsets and per-(chunk, expert) bases
 //   3. stable ranks: row of slot s = t*topk + j in expert order, via warp
 //      match + per-warp counts (no atomics decide the order)
-//   4. per-token quantization of x, each token once, its codes and scale
-//      written straight into the expert-ordered rows it was routed to
-//   5. grouped up-projection (tcgen05 W8A8 GEMM, tile schedule from offsets)
+//   4. per-token quantization of x, each token once, in token order
+//   5. grouped up-projection (tcgen05 W8A8 GEMM, tile schedule from offsets),
+//      whose producer gathers each expert's A rows from the token-order codes
+//      with 4-row TMA gathers (token = row_to_slot[row] / topk)
 //   6. per-row re-quantization of h
 //   7. grouped down-projection
 //   8. weighted un-permute y[t] = sum_j w[t,j] * o[row(t,j)], FP32, j ascending.
@@ -23,7 +24,8 @@ namespace metis {
 
 int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b, const float* s_b,
                             __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
-                            int K, cudaStream_t st);
+                            int K, cudaStream_t st, const int32_t* a_rows = nullptr, int a_div = 1,
+                            int a_src_rows = 0);
 int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
                           int64_t* total);
 int64_t moe4_padded_rows(int64_t T, int64_t topk, int64_t E);
@@ -320,6 +322,22 @@ __global__ void __launch_bounds__(ROUTE_WARPS * 32) route_topk_kernel(const floa
     }
 }
 
+// Shape and mode checks of the FP8 routed-expert layer, shared by its two
+// entry points (run before any size is computed from T * topk).
+int check_moe_shape(int act, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I) {
+    if (act != METIS_ACT_NONE)
+        return fail(METIS_ERR_UNSUPPORTED, "moe: act=%d; only METIS_ACT_NONE is built", act);
+    if (T < 0 || T > (1ll << 30) || topk < 1 || E < topk || E > MAX_E)
+        return fail(METIS_ERR_INVALID_ARG, "moe: need 0 <= T <= 2^30 and 1 <= topk <= E <= %d "
+                    "(T=%lld topk=%lld E=%lld)", MAX_E, (long long)T, (long long)topk, (long long)E);
+    if (H < 16 || I < 16 || H % 16 || I % 16 || H > 16384 || I > (1 << 20))
+        return fail(METIS_ERR_INVALID_ARG,
+                    "moe: need 16 <= H <= 16384 and I >= 16, both multiples of 16 (H=%lld I=%lld)",
+                    (long long)H, (long long)I);
+    if (T * topk > (1ll << 30)) return fail(METIS_ERR_INVALID_ARG, "moe: T*topk too large");
+    return METIS_OK;
+}
+
 }  // namespace moe
 }  // namespace metis
 
@@ -334,17 +352,9 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
                                           metis_stream_t stream) {
     using namespace moe;
     clear_error();
-    if (act != METIS_ACT_NONE)
-        return fail(METIS_ERR_UNSUPPORTED, "moe: act=%d; only METIS_ACT_NONE is built", act);
-    if (T < 0 || topk < 1 || E < topk || E > MAX_E)
-        return fail(METIS_ERR_INVALID_ARG, "moe: need T >= 0 and 1 <= topk <= E <= %d (T=%lld topk=%lld E=%lld)",
-                    MAX_E, (long long)T, (long long)topk, (long long)E);
-    if (H < 16 || I < 16 || H % 16 || I % 16 || H > 16384 || I > (1 << 20))
-        return fail(METIS_ERR_INVALID_ARG,
-                    "moe: need 16 <= H <= 16384 and I >= 16, both multiples of 16 (H=%lld I=%lld)",
-                    (long long)H, (long long)I);
+    int rc = check_moe_shape(act, T, topk, E, H, I);
+    if (rc) return rc;
     const int64_t S = T * topk;
-    if (S > (1ll << 30)) return fail(METIS_ERR_INVALID_ARG, "moe: T*topk too large");
     const size_t need = metis_workspace_size(METIS_OP_MOE, T, I, H, topk, E);
     if (T == 0) return METIS_OK;
     if (!x_bf16 || !topk_ids || !topk_w || !w_up || !s_up || !w_down || !s_down || !workspace)
@@ -356,8 +366,7 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
         return fail(METIS_ERR_INVALID_ARG,
                     "moe: workspace must be 256-byte aligned; x, weights, scales and y 16-byte aligned");
     DeviceInfo di;
-    int rc = current_device_info(&di);
-    if (rc) return rc;
+    if ((rc = current_device_info(&di))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     auto region = [&](int r) { return ws + moe_region_offset(r, T, topk, E, H, I, nullptr); };
@@ -387,11 +396,15 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     rank_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
                                      s2r, r2s);
     if ((rc = cuda_check(cudaGetLastError(), "moe routing launch"))) return rc;
+    // x quantized once per token, in token order; the up-projection gathers
+    // each expert's rows from it by token (row r holds slot row_to_slot[r],
+    // token row_to_slot[r] / topk), so the codes are never copied per slot
     if ((rc = launch_quant_rows<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_bf16), T, H, H, aq, H,
-                                               sa, st, s2r, static_cast<int>(topk))))
+                                               sa, st, nullptr, 1)))
         return rc;
     if ((rc = launch_fp8_gemm_grouped(aq, sa, w_up, s_up, h, offsets, static_cast<int>(E),
-                                      static_cast<int>(S), static_cast<int>(I), static_cast<int>(H), st)))
+                                      static_cast<int>(S), static_cast<int>(I), static_cast<int>(H), st,
+                                      r2s, static_cast<int>(topk), static_cast<int>(T))))
         return rc;
     if ((rc = launch_quant_rows<__nv_bfloat16>(h, S, I, I, hq, I, sh, st, nullptr, 1))) return rc;
     if ((rc = launch_fp8_gemm_grouped(hq, sh, w_down, s_down, o, offsets, static_cast<int>(E),
@@ -428,19 +441,27 @@ static __device__ __align__(256) uint8_t g_moe_static_scratch[kMoeStaticScratchB
 
 std::mutex g_static_scratch_mu;
 void* g_static_scratch_ptr[64];
+uint64_t g_static_scratch_ctx[64];  // context id the cached address belongs to
 
+// Device address of the scratch array on the current device. Looked up with
+// cudaGetSymbolAddress the first time a device (or a new context of it, after
+// cudaDeviceReset) is seen, with that device current; cached per device and
+// context id after that.
 int static_scratch_address(void** out) {
     int dev = 0;
     int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
     if (rc) return rc;
     if (dev < 0 || dev >= 64) return fail(METIS_ERR_UNSUPPORTED, "device %d", dev);
+    uint64_t ctx = 0;
+    if ((rc = current_context_id(&ctx))) return rc;
     std::lock_guard<std::mutex> lk(g_static_scratch_mu);
-    if (!g_static_scratch_ptr[dev]) {
+    if (!g_static_scratch_ptr[dev] || g_static_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
         rc = cuda_check(cudaGetSymbolAddress(&p, g_moe_static_scratch),
                         "cudaGetSymbolAddress(static MoE scratch)");
         if (rc) return rc;
         g_static_scratch_ptr[dev] = p;
+        g_static_scratch_ctx[dev] = ctx;
     }
     *out = g_static_scratch_ptr[dev];
     return METIS_OK;
@@ -455,7 +476,15 @@ extern "C" int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int3
                                                   const uint8_t* w_down, const float* s_down,
                                                   int act, void* y_bf16, metis_stream_t stream) {
     clear_error();
+    // the same checks as the workspace entry point, first, so that an
+    // unsupported mode or a bad shape is reported as such
+    int rc = moe::check_moe_shape(act, T, topk, E, H, I);
+    if (rc) return rc;
     if (T == 0) return METIS_OK;
+    // o would stay in the built-in array, which the caller cannot address
+    if (!y_bf16)
+        return fail(METIS_ERR_INVALID_ARG, "moe_noalloc: y is required (the routed outputs cannot be "
+                    "left in the built-in scratch array for a later combine)");
     const size_t need = metis_workspace_size(METIS_OP_MOE, T, I, H, topk, E);
     if (need > kMoeStaticScratchBytes)
         return fail(METIS_ERR_INVALID_ARG,
@@ -463,8 +492,7 @@ extern "C" int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int3
                     "holds %zu (16 MiB); use metis_moe_fp8_grouped_gemm with a caller workspace",
                     need, kMoeStaticScratchBytes);
     void* scratch = nullptr;
-    int rc = static_scratch_address(&scratch);
-    if (rc) return rc;
+    if ((rc = static_scratch_address(&scratch))) return rc;
     return metis_moe_fp8_grouped_gemm(x_bf16, topk_ids, topk_w, T, topk, E, H, I, w_up, s_up,
                                       w_down, s_down, act, y_bf16, scratch,
                                       kMoeStaticScratchBytes, stream);

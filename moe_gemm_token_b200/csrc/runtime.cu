@@ -19,7 +19,14 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 DeviceInfo g_info[kMaxDevices];
 uint32_t* g_status_ptr[kMaxDevices];
+uint64_t g_status_ctx[kMaxDevices];  // context id the cached status address belongs to
 uint64_t g_watchdog_ns = 2000000000ull;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
 
 // Sticky error word, one per device that loads the library.
 __device__ uint32_t g_device_status;
@@ -82,17 +89,53 @@ int current_device_info(DeviceInfo* out) {
     return METIS_OK;
 }
 
+int current_context_id(uint64_t* out) {
+    std::call_once(g_ctx_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+        fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_id = reinterpret_cast<CtxGetIdFn>(fn);
+    });
+    if (!g_ctx_current || !g_ctx_id) return fail(METIS_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId are unavailable");
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS) return fail(METIS_ERR_CUDA, "cuCtxGetCurrent failed");
+    if (ctx == nullptr) {
+        // no CUDA call on this thread yet: cudaSetDevice makes the device's
+        // primary context current (CUDA 12)
+        int dev = 0;
+        int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+        if (rc) return rc;
+        if ((rc = cuda_check(cudaSetDevice(dev), "cudaSetDevice"))) return rc;
+        if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+            return fail(METIS_ERR_CUDA, "no current CUDA context");
+    }
+    unsigned long long id = 0;
+    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return fail(METIS_ERR_CUDA, "cuCtxGetId failed");
+    *out = static_cast<uint64_t>(id);
+    return METIS_OK;
+}
+
 int device_status_word(uint32_t** out) {
     int dev = 0;
     int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
     if (rc) return rc;
     if (dev < 0 || dev >= kMaxDevices) return fail(METIS_ERR_UNSUPPORTED, "device %d", dev);
+    uint64_t ctx = 0;
+    if ((rc = current_context_id(&ctx))) return rc;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_status_ptr[dev]) {
+    // a module's __device__ variables move when its context is re-created
+    // (cudaDeviceReset): the cached address is valid for one context only
+    if (!g_status_ptr[dev] || g_status_ctx[dev] != ctx) {
         void* p = nullptr;
         rc = cuda_check(cudaGetSymbolAddress(&p, g_device_status), "cudaGetSymbolAddress(status)");
         if (rc) return rc;
         g_status_ptr[dev] = static_cast<uint32_t*>(p);
+        g_status_ctx[dev] = ctx;
     }
     *out = g_status_ptr[dev];
     return METIS_OK;
@@ -166,14 +209,13 @@ int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_
         4 * (E + 1),  // OFFSETS
         4 * S,        // SLOT_TO_ROW
         4 * S,        // ROW_TO_SLOT
-        S * H,        // AQ
-        4 * S,        // SA
+        T * H,        // AQ: codes of x, token order
+        4 * T,        // SA: their scales
         2 * S * I,    // H
         S * I,        // HQ
         4 * S,        // SH
         2 * S * H,    // O
     };
-    (void)T;
     int64_t off = 0, at = -1;
     for (int r = 0; r < 10; ++r) {
         if (r == region) at = off;

@@ -59,3 +59,33 @@ def test_reference_arm_runs_on_rank_zero_only():
                        env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_line_matches_the_metis_config():
+    """The reference arm prints one line on rank 0 with the metis arm's
+    config, metric, unit and direction (the oracle on a bounded sample)."""
+    import json
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0", "--ref-budget", "0.5"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.bench_config(1)
+    assert line["metric"] == bench.METRIC and line["unit"] == "tok/s" and line["higher_is_better"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gemm_traffic_needs_counters_of_the_current_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu counters only while the
+    kernel sources hash to the value recorded with them."""
+    import json
+    p = tmp_path / "c.json"
+    monkeypatch.setattr(bench, "GEMM_COUNTERS", str(p))
+    p.write_text(json.dumps({"kernel_sources_sha256_16": bench.gemm_source_sha(),
+                             "dram_bytes_read": 100, "dram_bytes_write": 23}))
+    assert bench.gemm_traffic_from_profile() == 123.0
+    p.write_text(json.dumps({"kernel_sources_sha256_16": "0" * 16,
+                             "dram_bytes_read": 100, "dram_bytes_write": 23}))
+    assert bench.gemm_traffic_from_profile() is None

@@ -1,7 +1,9 @@
 """GPU parity at the full sizes of the five workloads, in the launch
-configuration the benchmark times. Bytes are compared in full; BF16 outputs on
-sampled rows (tokens) that the oracle computes one by one, always including
-the extreme rows (zero rows, largest and smallest magnitudes, hot experts)."""
+configuration the benchmark times. Bytes are compared in full. BF16 outputs
+are compared in full for the tiny layer, the 4096-token prefill chain (both
+maths), decode and the 4096-token routed-expert layer; for the large-M sweep
+(up to 2.2 TFLOP per GEMM) on 256 sampled rows that the oracle computes one by
+one, always including the extreme rows (largest and smallest magnitudes)."""
 import numpy as np
 import pytest
 import torch
@@ -68,16 +70,18 @@ def test_prefill_chain_full_size(metis):
     assert metis.metis_check_device_status() == 0
     xq1r, st1r = oracle.quant_per_token(d["x"])
     assert_bytes_equal(xq1.cpu().numpy(), xq1r, "layer-1 codes")
-    rows = _sample_rows(M, d["x"])
-    _, y1_64 = oracle.gemm_w8a8(xq1r, st1r, w1r, s1r, rows=rows)
+    assert_bytes_equal(st1.cpu().numpy().view(np.uint32), st1r.view(np.uint32), "layer-1 scales")
+    # every token of both layers
+    _, y1_64 = oracle.gemm_w8a8(xq1r, st1r, w1r, s1r)
     y1h = bf16_host(y1)
-    assert_close(y1h[rows], y1_64, "layer 1")
+    assert_close(y1h, y1_64, "layer 1")
+    del y1_64
     # layer 2 starts from the GPU's own layer-1 output
     xq2r, st2r = oracle.quant_per_token(y1h)
     assert_bytes_equal(xq2.cpu().numpy(), xq2r, "layer-2 codes")
     assert_bytes_equal(st2.cpu().numpy().view(np.uint32), st2r.view(np.uint32), "layer-2 scales")
-    _, y2_64 = oracle.gemm_w8a8(xq2r, st2r, w2r, s2r, rows=rows)
-    assert_close(bf16_host(y2)[rows], y2_64, "layer 2")
+    _, y2_64 = oracle.gemm_w8a8(xq2r, st2r, w2r, s2r)
+    assert_close(bf16_host(y2), y2_64, "layer 2")
 
 
 @pytest.mark.parametrize("widened", [False, True])
@@ -99,12 +103,13 @@ def test_prefill_chain_default_maths_full_size(metis, widened):
     metis.metis_linear(bf16_dev(d["x"]), w1, s1, y1, fast_math=False, s_tok=s_tok, workspace=ws)
     metis.metis_linear(y1, w2, s2, y2, fast_math=False, s_tok=s_tok, workspace=ws)
     assert metis.metis_check_device_status() == 0
-    rows = _sample_rows(M, d["x"])
-    _, y1_64 = oracle.gemm_w8a16(d["x"][rows], w1r, s1r)
+    # every token of both layers
+    _, y1_64 = oracle.gemm_w8a16(d["x"], w1r, s1r)
     y1h = bf16_host(y1)
-    assert_close(y1h[rows], y1_64, "layer 1 (default maths)")
-    _, y2_64 = oracle.gemm_w8a16(y1h[rows], w2r, s2r)
-    assert_close(bf16_host(y2)[rows], y2_64, "layer 2 (default maths)")
+    assert_close(y1h, y1_64, "layer 1 (default maths)")
+    del y1_64
+    _, y2_64 = oracle.gemm_w8a16(y1h, w2r, s2r)
+    assert_close(bf16_host(y2), y2_64, "layer 2 (default maths)")
 
 
 @pytest.mark.parametrize("M", [1, 2, 4, 8])
@@ -119,14 +124,10 @@ def test_decode_full_size(metis, M):
 
 
 def test_moe_full_size(metis):
+    """All 4096 tokens (32768 routed slots), every stage."""
     d = synth.moe()
     g = run_moe(metis, d)
-    hot = d["hot_experts"]
-    ids = d["topk_ids"]
-    rng = np.random.default_rng(1)
-    hot_tok = np.nonzero(np.isin(ids, hot).any(axis=1))[0]
-    toks = np.unique(np.r_[rng.choice(d["T"], 24, replace=False), hot_tok[:8], 0, d["T"] - 1])
-    check_moe(d, g, tokens=toks)
+    check_moe(d, g)
 
 
 @pytest.mark.parametrize("M,K", [(8192, 4096), (16384, 4096), (8192, 8192), (16384, 8192)])

@@ -38,7 +38,7 @@ def run_moe(metis, d):
     out = dict(
         counts=R("COUNTS", (E,), torch.int32), offsets=R("OFFSETS", (E + 1,), torch.int32),
         s2r=R("SLOT_TO_ROW", (S,), torch.int32), r2s=R("ROW_TO_SLOT", (S,), torch.int32),
-        aq=R("AQ", (S, H), torch.uint8), sa=R("SA", (S,), torch.float32),
+        aq=R("AQ", (T, H), torch.uint8), sa=R("SA", (T,), torch.float32),
         h=R("H", (S, I), torch.int16).view(np.uint16), hq=R("HQ", (S, I), torch.uint8),
         sh=R("SH", (S,), torch.float32), o=R("O", (S, H), torch.int16).view(np.uint16),
         y=bf16_host(y), wq_up=wq_up, s_up=s_up, wq_dn=wq_dn, s_dn=s_dn)
@@ -54,17 +54,17 @@ def check_moe(d, g, tokens=None):
     assert_bytes_equal(g["offsets"], offsets, "offsets")
     assert_bytes_equal(g["s2r"], s2r, "slot_to_row")
     assert_bytes_equal(g["r2s"], r2s, "row_to_slot")
-    # per-token codes of x, written into every row the token was routed to
+    # per-token codes of x, once per token, in token order
     xq, sx = oracle.quant_per_token(d["x"])
-    tok_of_row = r2s // k
-    assert_bytes_equal(g["aq"], xq[tok_of_row], "x codes in expert order")
-    assert_bytes_equal(g["sa"].view(np.uint32), sx[tok_of_row].view(np.uint32), "x scales in expert order")
+    assert_bytes_equal(g["aq"], xq, "x codes")
+    assert_bytes_equal(g["sa"].view(np.uint32), sx.view(np.uint32), "x scales")
     slots = np.arange(T * k) if tokens is None else \
         (np.asarray(tokens)[:, None] * k + np.arange(k)).reshape(-1)
     rows = s2r[slots]
     exp = ids.reshape(-1)[slots]
-    # up-projection on the GPU's gathered operands
-    _, h64 = oracle.moe_expert_gemm(g["aq"][rows], g["sa"][rows], g["wq_up"], g["s_up"], exp)
+    tok = slots // k
+    # up-projection of each slot's token codes (which the GEMM gathers by row)
+    _, h64 = oracle.moe_expert_gemm(g["aq"][tok], g["sa"][tok], g["wq_up"], g["s_up"], exp)
     assert_close(g["h"][rows], h64, "h")
     # re-quantization of the GPU's h: bit-exact
     hq, sh = oracle.quant_per_token(g["h"][rows])
@@ -170,3 +170,45 @@ def test_route_topk_feeds_the_layer(metis):
     ref = oracle.moe_forward(d["x"], ids_r, w_r.astype(np.float32), g["wq_up"], g["s_up"], g["wq_dn"],
                              g["s_dn"])
     assert_close(g["y"], ref["y64"], "layer fed by the GPU router")
+
+
+def test_moe_out_of_range_ids_are_dropped_and_reported(metis):
+    """Routing ids stay on the GPU, so the host cannot check them: an id
+    outside [0, E) drops that slot (its SLOT_TO_ROW entry is -1 and it adds
+    nothing to y), sets the sticky status word (reported as
+    METIS_ERR_INVALID_ARG) and leaves every other slot as the oracle computes
+    it. The reference: the same layer with the bad slot's weight set to 0 (and
+    any valid id in its place, which only moves rows within an expert)."""
+    d = synth.moe(seed=28, T=128, H=256, I=128, E=8, topk=2, hot=2, load_ratio=2.0)
+    E = d["E"]
+    ids = d["topk_ids"].copy()
+    bad = [(5, 1, E), (77, 0, E + 3), (100, 1, -1)]
+    for t, j, v in bad:
+        ids[t, j] = v
+    d_bad = dict(d, topk_ids=ids)
+    metis.metis_check_device_status()  # start clean
+    T, H, I, k = d["T"], d["H"], d["I"], d["topk"]
+    up = [oracle.quant_per_channel(d["w_up"][e]) for e in range(E)]
+    dn = [oracle.quant_per_channel(d["w_down"][e]) for e in range(E)]
+    wq_up = np.stack([u[0] for u in up]); s_up = np.stack([u[1] for u in up])
+    wq_dn = np.stack([u[0] for u in dn]); s_dn = np.stack([u[1] for u in dn])
+    ws = torch.zeros((metis.metis_workspace_size(metis.METIS_OP_MOE, T, I, H, k, E),),
+                     dtype=torch.uint8, device="cuda")
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    metis.metis_moe_fp8_grouped_gemm(bf16_dev(d_bad["x"]), dev(ids), dev(d["topk_w"]), dev(wq_up),
+                                     dev(s_up), dev(wq_dn), dev(s_dn), y, ws)
+    assert metis.metis_check_device_status(clear=False) == metis.METIS_ERR_INVALID_ARG
+    assert metis.metis_check_device_status(clear=True) == metis.METIS_ERR_INVALID_ARG
+    assert metis.metis_check_device_status() == 0  # cleared
+    s2r = _region(metis, ws, "SLOT_TO_ROW", (T * k,), torch.int32, T, k, E, H, I).cpu().numpy()
+    for t, j, _ in bad:
+        assert s2r[t * k + j] == -1
+    counts = _region(metis, ws, "COUNTS", (E,), torch.int32, T, k, E, H, I).cpu().numpy()
+    assert counts.sum() == T * k - len(bad)
+    ids_ref = ids.copy()
+    w_ref = d["topk_w"].copy()
+    for t, j, _ in bad:
+        ids_ref[t, j] = (ids[t, 1 - j] + 1) % E  # any valid expert other than the token's other one
+        w_ref[t, j] = 0.0
+    ref = oracle.moe_forward(d["x"], ids_ref, w_ref, wq_up, s_up, wq_dn, s_dn)
+    assert_close(bf16_host(y), ref["y64"], "y with dropped slots")

@@ -89,7 +89,12 @@ def _prep_weights(metis, w):
 
 
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 272), (1, 8, 16), (129, 264, 1040),
-                                   (520, 784, 1024), (257, 1024, 2048), (4500, 520, 256)])
+                                   (520, 784, 1024), (257, 1024, 2048), (4500, 520, 256),
+                                   # the final partial wave cut into column pieces on 74 CTA
+                                   # pairs: 384 tiles (14 in the last wave, quarters); 320
+                                   # tiles with a 64-column last tile column (24, halves);
+                                   # 76 tiles with ragged M and N (2, quarters)
+                                   (4096, 6144, 256), (2560, 8000, 512), (1000, 4808, 256)])
 def test_fp8_gemm_parity(metis, M, N, K):
     d = synth.linear(M * 7 + N, M, K, N, outlier_channels=4, outlier_scale=20.0, zero_rows=(M // 3,))
     wq, s_w = _prep_weights(metis, d["w"])
@@ -107,11 +112,12 @@ def test_fp8_gemm_parity(metis, M, N, K):
     assert_close(bf16_host(y), y64, f"y {M}x{N}x{K}")
 
 
-def test_fp8_gemm_exact_integer_products(metis):
+@pytest.mark.parametrize("M,N,K", [(200, 272, 512), (4096, 6144, 64)])
+def test_fp8_gemm_exact_integer_products(metis, M, N, K):
     """Codes whose products and sums are small integers: the FP32 accumulation
-    is exact, so with unit scales the output equals the oracle's BF16 bits."""
+    is exact, so with unit scales the output equals the oracle's BF16 bits
+    (4096 x 6144: every column piece of the final wave lands where it belongs)."""
     rng = np.random.default_rng(11)
-    M, N, K = 200, 272, 512
     vals = np.array([0x38, 0x40, 0x44, 0xB8, 0xC0, 0x00, 0x30], np.uint8)  # 1,2,3,-1,-2,0,0.5
     a = vals[rng.integers(0, vals.size, (M, K))]
     b = vals[rng.integers(0, vals.size, (N, K))]
