@@ -624,20 +624,21 @@ def secondary_figures(metis, dev, pk):
     # quantizer at the prefill and large-M shapes (2 rotating inputs > L2)
     for (M, K) in [(4096, 2048), (4096, 6144), (16384, 8192)]:
         # enough rotating inputs that they cannot stay in the 126 MB L2
-        n_in = max(2, -(-2 * 126 * 2 ** 20 // (2 * M * K)) + 1)
+        # (inputs and outputs: an output rewritten every call would stay in L2)
+        n_in = max(2, -(-2 * 126 * 2 ** 20 // (3 * M * K)) + 1)
         xs = [torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16) for _ in range(n_in)]
-        xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        xqs = [torch.empty(M, K, dtype=torch.uint8, device=dev) for _ in range(n_in)]
         s = torch.empty(M, device=dev)
         i = [0]
 
         def f():
             i[0] = (i[0] + 1) % n_in
-            metis.metis_quant_fp8_per_token(xs[i[0]], xq, s)
+            metis.metis_quant_fp8_per_token(xs[i[0]], xqs[i[0]], s)
         t = timeit(f, 100)
         out[f"quant_{M}x{K}"] = {"us": t * 1e6, "GB/s": (3 * M * K + 4 * M) / t / 1e9,
                                  "frac_of_measured_hbm": (3 * M * K + 4 * M) / t / 1e9 / hbm,
                                  "frac_of_nominal_hbm": (3 * M * K + 4 * M) / t / 1e9 / NOMINAL_HBM_GBS}
-        del xs
+        del xs, xqs
     # large-M W8A8 GEMM from BF16 activations (per-token magnitudes
     # log-uniform in [1e-2, 1e2]): the GEMM alone, the separate quantizer +
     # GEMM (the product path), and the fused-quantization variant

@@ -189,9 +189,8 @@ METIS_API int metis_moe_route_topk(const float* logits, const float* bias, int64
  * the routed experts are FP8 with per-channel scales and per-token
  * activations). Steps, all on the device, no host synchronisation:
  * routing histogram -> exclusive prefix sum -> stable permutation of the
- * slots (t, j) by expert -> per-token quantization of x (once per token, in
- * token order) -> grouped up-projection (W8A8; its operand rows gathered by
- * token in the GEMM's TMA producer, never copied per slot) ->
+ * slots (t, j) by expert -> per-token quantization of x (once per token,
+ * written into the expert-contiguous rows of its slots) -> grouped up-projection (W8A8) ->
  * per-row re-quantization -> grouped down-projection (W8A8) -> weighted
  * un-permute y[t] = sum_j topk_w[t,j] o[t,j] (FP32, j ascending) -> BF16.
  *   x [T, H] BF16, topk_ids [T, topk] int32 in [0, E), topk_w [T, topk] FP32,
@@ -225,7 +224,7 @@ METIS_API int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* topk
  * library, which each GPU that loads the library keeps until the process exits.
  *   - Problems whose metis_workspace_size(METIS_OP_MOE, ...) exceeds 16 MiB are
  *     rejected with METIS_ERR_INVALID_ARG before anything is launched (about
- *     280 tokens at top-8 with H = 2048, I = 1024).
+ *     200 tokens at top-8 with H = 2048, I = 1024).
  *   - y must not be NULL: the routed outputs would otherwise stay in the
  *     built-in array, which the caller cannot address (METIS_ERR_INVALID_ARG).
  *   - The first call on each device (and the first after a cudaDeviceReset,
@@ -250,7 +249,9 @@ METIS_API int metis_moe_fp8_grouped_gemm_noalloc(const void* x_bf16, const int32
 METIS_API int metis_bf16_gemm(const void* x_bf16, const void* w_bf16, void* y_bf16, int64_t M,
                               int64_t N, int64_t K, metis_stream_t stream);
 
-/* The shared expert with the routed combine fused into its down-projection.
+/* The shared expert joined to the routed combine: its two BF16 projections
+ * run as tensor-core GEMMs, and one combine pass adds its output s to the
+ * routed weighted sum (reading o, s and the routing once, writing y once).
  * Reading of the cards (they print no formula): the shared expert runs on
  * every token with weight 1, with the two projections of a routed expert (no
  * activation), and the layer output adds its BF16 output s to the routed
@@ -264,7 +265,7 @@ METIS_API int metis_bf16_gemm(const void* x_bf16, const void* w_bf16, void* y_bf
  *   ran with y = NULL (o rows of H BF16 values).
  *   Requires H and I_s multiples of 16 (H <= 16384), 1 <= topk <= 8; needs
  *   `workspace` of metis_workspace_size(METIS_OP_SHARED, T, I_s, H, topk, 0)
- *   bytes (16-byte aligned) for h_s. */
+ *   bytes (256-byte aligned) for h_s [T, I_s] and s [T, H]. */
 METIS_API int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int64_t H, int64_t I_s,
                                              const void* w_sup_bf16, const void* w_sdn_bf16,
                                              const void* o_routed_bf16, const int32_t* slot_to_row,
@@ -295,9 +296,8 @@ METIS_API size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, in
  *   METIS_MOE_WS_OFFSETS     int32 [E + 1]  exclusive prefix sum of COUNTS
  *   METIS_MOE_WS_SLOT_TO_ROW int32 [S]      row of slot s = t*topk + j in expert order
  *   METIS_MOE_WS_ROW_TO_SLOT int32 [S]      inverse permutation
- *   METIS_MOE_WS_AQ          E4M3  [T, H]   per-token codes of x, token order (the up-projection
- *                                           gathers expert t's rows from it by token)
- *   METIS_MOE_WS_SA          FP32  [T]      their per-token scales
+ *   METIS_MOE_WS_AQ          E4M3  [S, H]   per-token codes of x, one row per slot, expert order
+ *   METIS_MOE_WS_SA          FP32  [S]      their per-token scales
  *   METIS_MOE_WS_H           BF16  [S, I]   up-projection output, expert order
  *   METIS_MOE_WS_HQ          E4M3  [S, I]   its per-row codes
  *   METIS_MOE_WS_SH          FP32  [S]      their scales

@@ -46,6 +46,12 @@ int make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t co
                  uint64_t rows, uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows,
                  bool swizzle128);
 
+// The same for 2-byte elements with the 64-byte swizzle (16-byte pieces of
+// each 64-byte row XOR-ed with bits 7-8 of the shared-memory address); for
+// TMA stores of 32 x 32 BF16 blocks staged in that layout.
+int make_tmap_2d_sw64(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                      uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows);
+
 // Encodes a 3-D tiled TMA descriptor of byte elements: dims {d0, d1, d2},
 // byte strides of dims 1 and 2 {s1, s2} (multiples of 16), box {b0, b1, b2}.
 int make_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
@@ -84,11 +90,9 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
                       int N, int K, cudaStream_t st);
 
 // BF16 GEMM y = bf16(a b^T) (gemm_fp8.cu); s_b non-null scales column n:
-// y = bf16(fl32((a b^T)[., n] * s_b[n])); o non-null fuses the routed combine:
-// y[t] = bf16(bf16(a b^T)[t] + sum_j topk_w[t*topk+j] o[s2r[t*topk+j]]).
+// y = bf16(fl32((a b^T)[., n] * s_b[n])).
 int launch_bf16_gemm(const __nv_bfloat16* a, const __nv_bfloat16* b, __nv_bfloat16* y, int M, int N,
-                     int K, const float* s_b, const __nv_bfloat16* o, const int32_t* s2r,
-                     const float* topk_w, int topk, cudaStream_t st);
+                     int K, const float* s_b, cudaStream_t st);
 
 // Exact E4M3 -> BF16 widening of n bytes (w16_gemm.cu); n a multiple of 16,
 // both buffers 16-byte aligned.

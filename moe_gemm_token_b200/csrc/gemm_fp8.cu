@@ -41,10 +41,10 @@
 // the shared expert's GEMM ("Lernex/Metis-1.6-Praxis" card, "Architecture":
 // one shared expert beside the routed ones; kept in BF16 by the FP8 cards);
 // with per-column scales (SCALED) it is the default maths on weights widened
-// to BF16 beforehand: y = bf16(acc * s_w[n]). The shared expert's
-// down-projection can add the routed experts' weighted outputs in the
-// epilogue: y[t] = bf16(s[t] + sum_j w[t,j] o[row(t,j)]) with s the BF16
-// product, so the routed combine needs no kernel and s never reaches HBM.
+// to BF16 beforehand: y = bf16(acc * s_w[n]).
+// Dense tiles whose count leaves a final wave that keeps at most a quarter of
+// the CTA pairs busy have that wave's tiles cut into four column pieces, one
+// per pair (an MMA of N = 64 and a B box of a quarter of the rows).
 // Every mbarrier wait is bounded by the device watchdog: on a timeout the CTA
 // sets the sticky error word, stops issuing work, drains what it issued,
 // frees TMEM and returns.
@@ -62,7 +62,6 @@ constexpr int MAX_GROUPS = 1024;
 
 constexpr int CONV_WARPS = 8;                  // fused-quantization converter warps
 constexpr int RASTER_M = 16;  // row blocks per raster group of the dense schedule
-constexpr int COMB_K = 8;                      // fused combine: routed slots per token
 constexpr int ASTG_SLOT = ROWS * BK * 2;       // one BF16 A tile (two 64-column boxes)
 
 template <int CTAS, bool ABF16 = false, int BN = BN_MAX, bool W16 = false>
@@ -82,11 +81,9 @@ struct Layout {
     static constexpr int TILES = STAGES * (A_STAGE + B_STAGE) + ASTG * ASTG_SLOT;
     static constexpr int STAGING = EPI * 32 * 64;  // a 32 x 32 BF16 block per epilogue warp
     static constexpr int SW = 2 * BN * 4;                // per-channel scales, double-buffered
-    static constexpr int COMB = W16 ? EPI * 32 * COMB_K * 8 : 0;  // (row, weight) per routed slot
     // full, empty, tfull[2], tempty[2], drain, epilogue sync[2], staging full/empty
     static constexpr int NUM_BARS = 2 * STAGES + 7 + 2 * ASTG;
-    static constexpr int COMB_OFF = TILES + STAGING + SW;
-    static constexpr int BAR_OFF = COMB_OFF + COMB;
+    static constexpr int BAR_OFF = TILES + STAGING + SW;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int GROUP_OFF = MISC_OFF + 16;
     static constexpr size_t BYTES_DENSE = 1024 + GROUP_OFF;
@@ -107,21 +104,10 @@ struct Params {
     int E;                   // groups (1 for dense)
     uint32_t* status;
     uint64_t timeout_ns;
-    // W16 fused combine (o null: none): y[t] += sum_j topk_w[t*topk+j] * o[s2r[t*topk+j]]
-    const __nv_bfloat16* o;  // routed outputs [rows, N]
-    const int32_t* s2r;      // [rows of A * topk]; negative: slot dropped
-    const float* topk_w;     // [rows of A * topk]
-    int topk;
     // dense tail pieces: tiles past `full` are cut into `split` column pieces,
     // whose B rows come through the second tensor map (box of BN/split/CTAS rows)
     int full;
     int split;
-    // grouped, gathered A (a_rows non-null): row r of the grouped operand is
-    // row a_rows[r] / a_div of the tensor behind tmA (and of s_a), fetched by
-    // 4-row TMA gathers; rows at or past the group's end read row 0
-    const int32_t* a_rows;
-    int a_div;
-    int a_src_rows;  // rows of the tensor behind tmA
 };
 
 struct Tile {
@@ -197,25 +183,47 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// One 32-column chunk of the epilogue: scale, round, stage in the warp's
-// swizzled block (16-byte pieces of each 64-byte row XOR-ed with (row>>1)&3,
-// so both the row-wise writes and the piece-wise reads are conflict-free),
-// then write 8 rows x 64 bytes per instruction.
-__device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, const Tile& ti, int q,
-                                            int lane, float rs, const float* sw,
-                                            uint8_t* stg, __nv_bfloat16* y, int N) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const float lo = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * j]), rs), sw[c * 32 + 2 * j]);
-        const float hi = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * j + 1]), rs), sw[c * 32 + 2 * j + 1]);
-        pk[j] = pack_bf16x2(lo, hi);
-    }
+// Bulk tensor store of a shared-memory box to global memory (completion
+// tracked per thread by bulk groups); and the group waits.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of every committed store have been read
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed store has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Writes one 32 x 32 BF16 block of the output (lane = row, pk = its 32
+// values as packed pairs): staged in the warp's swizzled block (16-byte pieces
+// of each 64-byte row XOR-ed with (row>>1)&3, which is the 64-byte TMA
+// swizzle, so the row-wise writes and the piece-wise reads are conflict-free),
+// then stored by one TMA store when all 32 rows belong to the tile's group
+// (the map clips columns past N), else by the lanes, 8 rows x 64 bytes per
+// instruction, rows at or past row_end skipped.
+__device__ __forceinline__ void put_block(const uint32_t (&pk)[16], int c, const Tile& ti, int q, int lane,
+                                          uint8_t* stg, __nv_bfloat16* y, int N, const CUtensorMap* tmY) {
+    // the previous block's store has read the staging block
+    if (lane == 0) bulk_wait_read();
     __syncwarp();
 #pragma unroll
     for (int pc = 0; pc < 4; ++pc)
         *reinterpret_cast<uint4*>(stg + lane * 64 + ((pc ^ ((lane >> 1) & 3)) * 16)) =
             make_uint4(pk[4 * pc], pk[4 * pc + 1], pk[4 * pc + 2], pk[4 * pc + 3]);
+    const int row0 = ti.a_row0 + q * 32;
+    if (ti.n0 + c * 32 >= N) return;  // a block wholly past the last column: nothing to store
+    if (row0 + 32 <= ti.row_end) {
+        fence_proxy_async_shared();  // the staging writes, to the TMA engine
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmY, smem_u32(stg), ti.n0 + c * 32, row0);
+            bulk_commit();
+        }
+        return;
+    }
     __syncwarp();
     const int n = ti.n0 + c * 32 + (lane & 3) * 8;
 #pragma unroll
@@ -223,48 +231,32 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, cons
         const int rr = (lane >> 2) + 8 * i;
         const uint4 val =
             *reinterpret_cast<const uint4*>(stg + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
-        const int row = ti.a_row0 + q * 32 + rr;
+        const int row = row0 + rr;
         if (row < ti.row_end && n < N)
             *reinterpret_cast<uint4*>(y + static_cast<size_t>(row) * N + n) = val;
     }
 }
 
-// L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned address.
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// Four 128-byte rows (rows r0..r3 of a 2-D tensor whose map has a one-row
-// box, starting at column x) into 512 consecutive bytes of shared memory, in
-// the map's swizzle; completion counted on the mbarrier. No multicast.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, int32_t x, int32_t r0,
-                                            int32_t r1, int32_t r2, int32_t r3, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-// The same into this CTA's shared memory, completing on an mbarrier of either
-// CTA of the pair (cta_group::2). No multicast.
-__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* m, int32_t x, int32_t r0,
-                                                 int32_t r1, int32_t r2, int32_t r3, uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
+// One 32-column chunk of the epilogue: y = bf16(acc * s_a[row] * s_b[n]).
+__device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, const Tile& ti, int q,
+                                            int lane, float rs, const float* sw,
+                                            uint8_t* stg, __nv_bfloat16* y, int N, const CUtensorMap* tmY) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float lo = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * j]), rs), sw[c * 32 + 2 * j]);
+        const float hi = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * j + 1]), rs), sw[c * 32 + 2 * j + 1]);
+        pk[j] = pack_bf16x2(lo, hi);
+    }
+    put_block(pk, c, ti, q, lane, stg, y, N, tmY);
 }
 
 // The W16 epilogue chunk: y = bf16(acc), or bf16(acc * sw[n]) with per-column
-// scales (SCALED), staged as above; without scales the fused
-// combine may then add the token's routed outputs to each 8-column piece,
-// y = bf16(s + sum_j w_j o_j) in FP32, j ascending. Two rows are handled at
-// a time, so 2 * topk loads are in flight per lane.
+// scales (SCALED).
 template <bool SCALED>
 __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, const Tile& ti, int q,
-                                                int lane, const float* sw, uint8_t* stg, const int2* cb,
-                                                const Params& p) {
+                                                int lane, const float* sw, uint8_t* stg, const Params& p,
+                                                const CUtensorMap* tmY) {
     uint32_t pk[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -275,77 +267,14 @@ __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, 
         }
         pk[j] = pack_bf16x2(lo, hi);
     }
-    __syncwarp();
-#pragma unroll
-    for (int pc = 0; pc < 4; ++pc)
-        *reinterpret_cast<uint4*>(stg + lane * 64 + ((pc ^ ((lane >> 1) & 3)) * 16)) =
-            make_uint4(pk[4 * pc], pk[4 * pc + 1], pk[4 * pc + 2], pk[4 * pc + 3]);
-    __syncwarp();
-    const int n = ti.n0 + c * 32 + (lane & 3) * 8;
-#pragma unroll
-    for (int i0 = 0; i0 < 4; i0 += 2) {
-        uint4 val[2];
-        bool live[2];
-        uint4 ov[2][COMB_K];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int rr = (lane >> 2) + 8 * (i0 + u);
-            val[u] = *reinterpret_cast<const uint4*>(stg + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
-            live[u] = ti.a_row0 + q * 32 + rr < ti.row_end && n < p.N;
-        }
-        if (!SCALED && p.o != nullptr) {
-            // every load of both rows before the first add (the (row, weight)
-            // pairs are read from shared memory where they are used)
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int2* e = cb + ((lane >> 2) + 8 * (i0 + u)) * COMB_K;
-#pragma unroll
-                for (int j = 0; j < COMB_K; ++j) {
-                    const int r = e[j].x;
-                    if (live[u] && j < p.topk && r >= 0)
-                        ov[u][j] = *reinterpret_cast<const uint4*>(p.o + static_cast<size_t>(r) * p.N + n);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int2* e = cb + ((lane >> 2) + 8 * (i0 + u)) * COMB_K;
-                const uint32_t sv[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
-                float a[8];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    a[2 * h] = bf16_lo(sv[h]);
-                    a[2 * h + 1] = bf16_hi(sv[h]);
-                }
-#pragma unroll
-                for (int j = 0; j < COMB_K; ++j) {
-                    const int2 ej = e[j];
-                    if (live[u] && j < p.topk && ej.x >= 0) {
-                        const float wj = __int_as_float(ej.y);
-                        const uint32_t ow[4] = {ov[u][j].x, ov[u][j].y, ov[u][j].z, ov[u][j].w};
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            a[2 * h] = fmaf(wj, bf16_lo(ow[h]), a[2 * h]);
-                            a[2 * h + 1] = fmaf(wj, bf16_hi(ow[h]), a[2 * h + 1]);
-                        }
-                    }
-                }
-                val[u] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
-                                    pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int rr = (lane >> 2) + 8 * (i0 + u);
-            const int row = ti.a_row0 + q * 32 + rr;
-            if (live[u]) *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.N + n) = val[u];
-        }
-    }
+    put_block(pk, c, ti, q, lane, stg, p.y, p.N, tmY);
 }
 
 template <int CTAS, bool GROUPED, bool ABF16, int BN, bool W16 = false, bool SCALED = false>
 __global__ void __launch_bounds__(Layout<CTAS, ABF16, BN, W16>::THREADS_, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmBq, const Params p) {
+                const __grid_constant__ CUtensorMap tmBq, const __grid_constant__ CUtensorMap tmY,
+                const Params p) {
     using L = Layout<CTAS, ABF16, BN, W16>;
     constexpr int STAGES = L::STAGES;
     constexpr int EPI = L::EPI;
@@ -359,7 +288,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
-    int2* comb = reinterpret_cast<int2*>(smem + L::COMB_OFF);
     int* g_tile = reinterpret_cast<int*>(smem + L::GROUP_OFF);
     int* g_row = g_tile + (MAX_GROUPS + 1);
 
@@ -398,6 +326,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmY);
         if (p.split > 1) tma_prefetch_desc(&tmBq);
     }
     if (warp == 1) {
@@ -479,69 +408,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const int stride = CTAS == 2 ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
 
     if (warp == 0) {
-        if (GROUPED && !ABF16 && !W16 && p.a_rows != nullptr) {
-            // ------------------------------------------ producer, gathered A
-            // Each lane fetches 4 of the CTA's 128 A rows per k-block with one
-            // TMA gather (row r of the group is source row a_rows[r] / a_div);
-            // lane 0 waits for the stage and loads B.
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t issued = 0, issued_phase = 0;
-            for (int t = first; t < sc.total; t += stride) {
-                // the flag is read once for the whole warp (the loop holds warp-wide shuffles)
-                if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
-                const Tile ti = sc.get(t);
-                int src[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = ti.a_row0 + lane * 4 + i;
-                    int v = r < ti.row_end ? p.a_rows[r] / p.a_div : 0;
-                    src[i] = min(max(v, 0), p.a_src_rows - 1);
-                }
-                bool ok = true;
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (lane == 0) ok = mbar_wait(empty(stage), phase ^ 1u, p.timeout_ns, p.status);
-                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                    if (!ok) break;
-                    const uint32_t dst = smem_u32(sA + stage * L::A_STAGE) + lane * 4 * BK;
-                    if constexpr (CTAS == 2) {
-                        const uint32_t fl = mapa_shared(full(stage), 0);
-                        if (lane == 0) {
-                            if (leader) mbar_arrive_expect_tx(full(stage), CTAS * (L::A_STAGE + L::B_STAGE));
-                            tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * L::KE, ti.b_row0, fl);
-                        }
-                        __syncwarp();
-                        tma_gather4_pair(dst, &tmA, kb * L::KE, src[0], src[1], src[2], src[3], fl);
-                    } else {
-                        if (lane == 0) {
-                            mbar_arrive_expect_tx(full(stage), L::A_STAGE + L::B_STAGE);
-                            tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, kb * L::KE, ti.b_row0, full(stage));
-                        }
-                        __syncwarp();
-                        tma_gather4(dst, &tmA, kb * L::KE, src[0], src[1], src[2], src[3], full(stage));
-                    }
-                    issued |= 1u << stage;
-                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                }
-                if (!ok) {
-                    if (lane == 0) *abort_flag = 1;
-                    break;
-                }
-            }
-            __syncwarp();
-            if (lane == 0 && *abort_flag) {
-                // let the copies in flight land before the CTA exits
-                if (leader) {
-                    for (int s = 0; s < STAGES; ++s)
-                        if (issued & (1u << s))
-                            mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
-                } else {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (globaltimer_ns() - t0 < 100000ull) {}
-                }
-            }
-        } else if (lane == 0) {
+        if (lane == 0) {
             // ---------------------------------------------------------- producer
             int stage = 0;
             uint32_t phase = 0;
@@ -748,7 +615,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         uint32_t acc_phase = 0;
         for (int t = first; t < sc.total && !*abort_flag; t += stride) {
             const Tile ti = sc.get(t);
-            const int2* cb = comb + (warp - 2) * 32 * COMB_K;
             if constexpr (W16) {
                 if constexpr (SCALED) {
                     // per-column scales (the default maths' s_w)
@@ -757,23 +623,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         sw_smem[acc * BN + 2 * et] = n < p.N ? p.s_b[n] : 0.0f;
                         sw_smem[acc * BN + 2 * et + 1] = n + 1 < p.N ? p.s_b[n + 1] : 0.0f;
                     }
-                } else if (p.o != nullptr) {
-                    // the fused combine's (row, weight) pairs of this warp's 32 rows
-                    const int row = ti.a_row0 + q * 32 + lane;
-                    int2* mine = comb + ((warp - 2) * 32 + lane) * COMB_K;
-                    // this warp's columns of the routed rows go to L2 now, while
-                    // the tile's MMAs run
-                    const int col0 = ti.n0 + c0 * 32;
-                    const int ncol = min(CPW * 32, p.N - col0);
-                    for (int j = 0; j < p.topk; ++j) {
-                        const size_t sidx = static_cast<size_t>(row) * p.topk + j;
-                        const int2 v = row < ti.row_end ? make_int2(p.s2r[sidx], __float_as_int(p.topk_w[sidx]))
-                                                        : make_int2(-1, 0);
-                        mine[j] = v;
-                        if (v.x >= 0 && ncol > 0)
-                            prefetch_l2(p.o + static_cast<size_t>(v.x) * p.N + col0, static_cast<uint32_t>(ncol) * 2u);
-                    }
-                    __syncwarp();
                 }
             } else {
                 // per-channel scales of this tile into shared memory
@@ -783,9 +632,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (et < BN / 2) reinterpret_cast<float2*>(sw_smem + acc * BN)[et] = v;
             }
             const int row = ti.a_row0 + q * 32 + lane;
-            float rs = 0.0f;
-            if (!W16 && row < ti.row_end)
-                rs = (GROUPED && p.a_rows != nullptr) ? p.s_a[p.a_rows[row] / p.a_div] : p.s_a[row];
+            const float rs = (!W16 && row < ti.row_end) ? p.s_a[row] : 0.0f;
             // all epilogue threads have written their scales (bounded wait)
             mbar_arrive(epi_sync(acc));
             if (!mbar_wait(epi_sync(acc), acc_phase, p.timeout_ns, p.status) ||
@@ -817,7 +664,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     tmem_ld_32x32b_x32(tbase + (c0 + i) * 32, va);
                     tmem_ld_wait();
                     if (i + 1 == nval) hand_back();
-                    store_chunk(va, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N);
+                    store_chunk(va, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N, &tmY);
                 }
                 if (nval == 0) hand_back();
             } else {
@@ -831,14 +678,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     uint32_t(&nxt)[32] = (i & 1) ? va : vb;
                     if (i + 1 < CPW) tmem_ld_32x32b_x32(tbase + (c0 + i + 1) * 32, nxt);
                     else hand_back();
-                    if constexpr (W16) store_chunk_w16<SCALED>(cur, c0 + i, ti, q, lane, sw, stg, cb, p);
-                    else store_chunk(cur, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N);
+                    if constexpr (W16) store_chunk_w16<SCALED>(cur, c0 + i, ti, q, lane, sw, stg, p, &tmY);
+                    else store_chunk(cur, c0 + i, ti, q, lane, rs, sw, stg, p.y, p.N, &tmY);
                     if (i + 1 < CPW) tmem_ld_wait();
                 }
             }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        // this warp's output stores have completed before the CTA exits
+        if (lane == 0) bulk_wait_all();
     }
 
     __syncwarp();
@@ -898,16 +747,15 @@ int max_pairs(const DeviceInfo& di, int* out) {
 // The persistent grid runs `tiles` whole tiles on `workers` CTAs (pairs): the
 // last tiles % workers of them form a final wave that keeps few workers busy
 // (4096 x 6144 on 74 pairs: 384 tiles, 14 in the last wave). When that wave
-// would occupy at most a quarter (half) of the workers, each of its tiles is
-// cut into 4 (2) column pieces of BN/4 (BN/2) columns, one piece per worker,
-// so the final wave ends in a fraction of a tile's time.
+// would occupy at most a quarter of the workers, each of its tiles is cut into
+// 4 column pieces of BN/4 columns, one piece per worker. Measured on B200:
+// 4096 x 6144 x 2048 45.4 against 45.9 us; halves for a final wave of up to
+// half the workers measured slower (2560 x 8000 x 2048: 43.2 against 39.2 us),
+// so only quarters are cut.
 inline int tail_split(int tiles, int workers) {
     if (tiles <= workers) return 1;
     const int r = tiles % workers;
-    if (r == 0) return 1;
-    if (4 * r <= workers) return 4;
-    if (2 * r <= workers) return 2;
-    return 1;
+    return (r > 0 && 4 * r <= workers) ? 4 : 1;
 }
 
 // Dense E4M3 GEMM with BN-column tiles: CTA pairs (256-row tiles) for
@@ -916,8 +764,9 @@ template <int BN>
 int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, Params p,
                  int M, int N, int K, cudaStream_t st) {
     int rc;
-    CUtensorMap tb, tbq;
+    CUtensorMap tb, tbq, ty;
     const int num_n = (N + BN - 1) / BN;
+    if ((rc = make_tmap_2d_sw64(&ty, p.y, 2, N, M, static_cast<uint64_t>(N) * 2, 32, 32))) return rc;
     if (M > ROWS) {
         using L = Layout<2, false, BN>;
         if ((rc = prepare<2, false, false, BN>(di, L::BYTES_DENSE))) return rc;
@@ -933,7 +782,7 @@ int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, 
             (rc = make_tmap_2d(&tbq, b, 1, K, N, K, BK, static_cast<uint32_t>(L::B_ROWS / p.split), true)))
             return rc;
         return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, false, BN>, dim3(2 * clusters), dim3(L::THREADS_),
-                                     L::BYTES_DENSE, st, 2, ta, tb, tbq, p),
+                                     L::BYTES_DENSE, st, 2, ta, tb, tbq, ty, p),
                           "fp8 gemm (CTA pair) launch");
     }
     using L = Layout<1, false, BN>;
@@ -948,7 +797,7 @@ int launch_dense(const DeviceInfo& di, const CUtensorMap& ta, const uint8_t* b, 
         (rc = make_tmap_2d(&tbq, b, 1, K, N, K, BK, static_cast<uint32_t>(L::B_ROWS / p.split), true)))
         return rc;
     return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, false, BN>, dim3(grid), dim3(L::THREADS_),
-                                 L::BYTES_DENSE, st, 1, ta, tb, tbq, p),
+                                 L::BYTES_DENSE, st, 1, ta, tb, tbq, ty, p),
                       "fp8 gemm launch");
 }
 
@@ -976,7 +825,7 @@ int launch_fp8_gemm_dense(const uint8_t* a, const float* s_a, const uint8_t* b, 
 // [e*N, (e+1)*N). `rows` is the row count of A and y (offsets[E] <= rows).
 int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b, const float* s_b,
                             __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
-                            int K, cudaStream_t st, const int32_t* a_rows, int a_div, int a_src_rows) {
+                            int K, cudaStream_t st) {
     using namespace gemm;
     if (E > MAX_GROUPS) return fail(METIS_ERR_UNSUPPORTED, "grouped gemm: E=%d > %d", E, MAX_GROUPS);
     DeviceInfo di;
@@ -985,16 +834,9 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
     Params p{s_a, nullptr, s_b, y, offsets, rows, N, K, E, status, watchdog_ns()};
-    CUtensorMap ta, tb;
-    if (a_rows != nullptr) {
-        // A gathered by rows from a [a_src_rows, K] tensor: one-row boxes
-        p.a_rows = a_rows;
-        p.a_div = a_div;
-        p.a_src_rows = a_src_rows;
-        if ((rc = make_tmap_2d(&ta, a, 1, K, a_src_rows, K, BK, 1, true))) return rc;
-    } else if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, ROWS, true))) {
-        return rc;
-    }
+    CUtensorMap ta, tb, ty;
+    if ((rc = make_tmap_2d(&ta, a, 1, K, rows, K, BK, ROWS, true))) return rc;
+    if ((rc = make_tmap_2d_sw64(&ty, y, 2, N, rows, static_cast<uint64_t>(N) * 2, 32, 32))) return rc;
     if (K < 1024) {
         // short k-loops: 128-row single-CTA tiles
         using L = Layout<1>;
@@ -1002,7 +844,7 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
         if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
             return rc;
         return cuda_check(launch_pdl(fp8_gemm_kernel<1, true, false, BN_MAX>, dim3(di.num_sms), dim3(L::THREADS_),
-                                     L::BYTES_GROUPED, st, 1, ta, tb, tb, p),
+                                     L::BYTES_GROUPED, st, 1, ta, tb, tb, ty, p),
                           "grouped fp8 gemm launch");
     }
     // CTA pairs on 256-row tiles: each SM streams half of B (routed
@@ -1014,7 +856,7 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
         return rc;
     return cuda_check(launch_pdl(fp8_gemm_kernel<2, true, false, BN_MAX>, dim3(2 * pairs), dim3(L::THREADS_),
-                                 L::BYTES_GROUPED, st, 2, ta, tb, tb, p),
+                                 L::BYTES_GROUPED, st, 2, ta, tb, tb, ty, p),
                       "grouped fp8 gemm (CTA pair) launch");
 }
 
@@ -1031,8 +873,9 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
     if ((rc = device_status_word(&status))) return rc;
     Params p{s_a, inv, s_b, y, nullptr, M, N, K, 1, status, watchdog_ns()};
     const int num_n = (N + BN_MAX - 1) / BN_MAX;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, ty;
     if ((rc = make_tmap_2d(&ta, a, 2, K, M, static_cast<uint64_t>(K) * 2, BK / 2, ROWS, true))) return rc;
+    if ((rc = make_tmap_2d_sw64(&ty, y, 2, N, M, static_cast<uint64_t>(N) * 2, 32, 32))) return rc;
     if (M > ROWS) {
         using L = Layout<2, true>;
         if ((rc = prepare<2, false, true>(di, L::BYTES_DENSE))) return rc;
@@ -1042,7 +885,7 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
         const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
         const int clusters = tiles < pairs ? tiles : pairs;
         return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, true, BN_MAX>, dim3(2 * clusters), dim3(L::THREADS_),
-                                     L::BYTES_DENSE, st, 2, ta, tb, tb, p),
+                                     L::BYTES_DENSE, st, 2, ta, tb, tb, ty, p),
                           "fused fp8 gemm (CTA pair) launch");
     }
     using L = Layout<1, true>;
@@ -1051,13 +894,12 @@ int launch_fp8_gemm_fused(const __nv_bfloat16* a, const float* s_a, const float*
     const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
     return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, true, BN_MAX>, dim3(grid), dim3(L::THREADS_),
-                                 L::BYTES_DENSE, st, 1, ta, tb, tb, p),
+                                 L::BYTES_DENSE, st, 1, ta, tb, tb, ty, p),
                       "fused fp8 gemm launch");
 }
 
 // BF16 x BF16 GEMM y = bf16(a b^T) on the tcgen05 pipeline (CTA pairs for
-// M > 128), optionally with the routed combine fused into the epilogue (o
-// non-null). Arguments validated by the caller.
+// M > 128). Arguments validated by the caller.
 namespace gemm {
 
 template <bool SCALED>
@@ -1065,8 +907,9 @@ int launch_w16(const __nv_bfloat16* a, const __nv_bfloat16* b, const Params& p, 
                const DeviceInfo& di, cudaStream_t st) {
     int rc;
     const int num_n = (N + BN_MAX - 1) / BN_MAX;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, ty;
     if ((rc = make_tmap_2d(&ta, a, 2, K, M, static_cast<uint64_t>(K) * 2, BK / 2, ROWS, true))) return rc;
+    if ((rc = make_tmap_2d_sw64(&ty, p.y, 2, N, M, static_cast<uint64_t>(N) * 2, 32, 32))) return rc;
     if (M > ROWS) {
         using L = Layout<2, false, BN_MAX, true>;
         if ((rc = prepare<2, false, false, BN_MAX, true, SCALED>(di, L::BYTES_DENSE))) return rc;
@@ -1077,7 +920,7 @@ int launch_w16(const __nv_bfloat16* a, const __nv_bfloat16* b, const Params& p, 
         const int tiles = ((M + 2 * ROWS - 1) / (2 * ROWS)) * num_n;
         const int clusters = tiles < pairs ? tiles : pairs;
         return cuda_check(launch_pdl(fp8_gemm_kernel<2, false, false, BN_MAX, true, SCALED>, dim3(2 * clusters),
-                                     dim3(L::THREADS_), L::BYTES_DENSE, st, 2, ta, tb, tb, p),
+                                     dim3(L::THREADS_), L::BYTES_DENSE, st, 2, ta, tb, tb, ty, p),
                           "bf16 gemm (CTA pair) launch");
     }
     using L = Layout<1, false, BN_MAX, true>;
@@ -1086,24 +929,21 @@ int launch_w16(const __nv_bfloat16* a, const __nv_bfloat16* b, const Params& p, 
     const int tiles = ((M + ROWS - 1) / ROWS) * num_n;
     const int grid = tiles < di.num_sms ? tiles : di.num_sms;
     return cuda_check(launch_pdl(fp8_gemm_kernel<1, false, false, BN_MAX, true, SCALED>, dim3(grid),
-                                 dim3(L::THREADS_), L::BYTES_DENSE, st, 1, ta, tb, tb, p),
+                                 dim3(L::THREADS_), L::BYTES_DENSE, st, 1, ta, tb, tb, ty, p),
                       "bf16 gemm launch");
 }
 
 }  // namespace gemm
 
 int launch_bf16_gemm(const __nv_bfloat16* a, const __nv_bfloat16* b, __nv_bfloat16* y, int M, int N,
-                     int K, const float* s_b, const __nv_bfloat16* o, const int32_t* s2r, const float* topk_w,
-                     int topk, cudaStream_t st) {
+                     int K, const float* s_b, cudaStream_t st) {
     using namespace gemm;
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
-    if (s_b != nullptr && o != nullptr)
-        return fail(METIS_ERR_INVALID_ARG, "bf16 gemm: per-column scales and the fused combine are exclusive");
-    Params p{nullptr, nullptr, s_b, y, nullptr, M, N, K, 1, status, watchdog_ns(), o, s2r, topk_w, topk};
+    Params p{nullptr, nullptr, s_b, y, nullptr, M, N, K, 1, status, watchdog_ns()};
     return s_b != nullptr ? launch_w16<true>(a, b, p, M, N, K, di, st) : launch_w16<false>(a, b, p, M, N, K, di, st);
 }
 
@@ -1124,8 +964,7 @@ extern "C" int metis_bf16_gemm(const void* x_bf16, const void* w_bf16, void* y_b
         return fail(METIS_ERR_INVALID_ARG, "bf16_gemm: x, w and y must be 16-byte aligned");
     return launch_bf16_gemm(static_cast<const __nv_bfloat16*>(x_bf16), static_cast<const __nv_bfloat16*>(w_bf16),
                             static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(M), static_cast<int>(N),
-                            static_cast<int>(K), nullptr, nullptr, nullptr, nullptr, 0,
-                            static_cast<cudaStream_t>(stream));
+                            static_cast<int>(K), nullptr, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int metis_fp8_gemm(const void* a, int a_kind, float* s_tok, const uint8_t* wq,

@@ -8,10 +8,9 @@
 //   2. prefix sums: per-expert offsets and per-(chunk, expert) bases
 //   3. stable ranks: row of slot s = t*topk + j in expert order, via warp
 //      match + per-warp counts (no atomics decide the order)
-//   4. per-token quantization of x, each token once, in token order
-//   5. grouped up-projection (tcgen05 W8A8 GEMM, tile schedule from offsets),
-//      whose producer gathers each expert's A rows from the token-order codes
-//      with 4-row TMA gathers (token = row_to_slot[row] / topk)
+//   4. per-token quantization of x, each token once, its codes and scale
+//      written straight into the expert-ordered rows it was routed to
+//   5. grouped up-projection (tcgen05 W8A8 GEMM, tile schedule from offsets)
 //   6. per-row re-quantization of h
 //   7. grouped down-projection
 //   8. weighted un-permute y[t] = sum_j w[t,j] * o[row(t,j)], FP32, j ascending.
@@ -24,8 +23,7 @@ namespace metis {
 
 int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b, const float* s_b,
                             __nv_bfloat16* y, const int32_t* offsets, int E, int rows, int N,
-                            int K, cudaStream_t st, const int32_t* a_rows = nullptr, int a_div = 1,
-                            int a_src_rows = 0);
+                            int K, cudaStream_t st);
 int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_t H, int64_t I,
                           int64_t* total);
 int64_t moe4_padded_rows(int64_t T, int64_t topk, int64_t E);
@@ -194,23 +192,34 @@ __global__ void __launch_bounds__(CHUNK) rank_kernel(const int32_t* __restrict__
     }
 }
 
-// y[t, n..n+7] = bf16( sum_j w[t, j] * o[slot_to_row[t*topk + j], n..n+7] ).
+// y[t, n..n+7] = bf16( s[t, n..n+7] + sum_j w[t, j] * o[slot_to_row[t*topk + j], n..n+7] ),
+// s the shared expert's BF16 output (null: 0).
 // HBM-bound: the row indices and weights of the token are read first, then
 // every row load is issued before the first add (for topk <= COMBINE_MAXK),
-// so a thread has topk 16-byte loads in flight. The sum runs over j in
-// ascending order in FP32 either way.
+// so a thread has topk 16-byte loads in flight. The sum starts from s and runs
+// over j in ascending order in FP32 either way.
 constexpr int COMBINE_MAXK = 8;
 __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const float* __restrict__ w,
                                                       const int32_t* __restrict__ slot_to_row,
                                                       int T, int topk, int H,
-                                                      __nv_bfloat16* __restrict__ y) {
+                                                      __nv_bfloat16* __restrict__ y,
+                                                      const __nv_bfloat16* __restrict__ s) {
     const int groups = H / 8;
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= static_cast<int64_t>(T) * groups) return;
     const int t = static_cast<int>(idx / groups);
     const int n = static_cast<int>(idx - static_cast<int64_t>(t) * groups) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (s != nullptr) {
+        const uint4 v = *reinterpret_cast<const uint4*>(s + static_cast<size_t>(t) * H + n);
+        const uint32_t sv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = bf16_lo(sv[i]);
+            acc[2 * i + 1] = bf16_hi(sv[i]);
+        }
+    }
     auto add = [&](float wj, const uint4& c) {
         const uint32_t v[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
@@ -396,15 +405,15 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     rank_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
                                      s2r, r2s);
     if ((rc = cuda_check(cudaGetLastError(), "moe routing launch"))) return rc;
-    // x quantized once per token, in token order; the up-projection gathers
-    // each expert's rows from it by token (row r holds slot row_to_slot[r],
-    // token row_to_slot[r] / topk), so the codes are never copied per slot
+    // x quantized once per token, its codes and scale written straight into
+    // every expert-ordered row the token was routed to (gathering the rows
+    // inside the GEMM with 4-row TMA gathers instead measured 3x slower for
+    // the up-projection: 205 against 66 us)
     if ((rc = launch_quant_rows<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_bf16), T, H, H, aq, H,
-                                               sa, st, nullptr, 1)))
+                                               sa, st, s2r, static_cast<int>(topk))))
         return rc;
     if ((rc = launch_fp8_gemm_grouped(aq, sa, w_up, s_up, h, offsets, static_cast<int>(E),
-                                      static_cast<int>(S), static_cast<int>(I), static_cast<int>(H), st,
-                                      r2s, static_cast<int>(topk), static_cast<int>(T))))
+                                      static_cast<int>(S), static_cast<int>(I), static_cast<int>(H), st)))
         return rc;
     if ((rc = launch_quant_rows<__nv_bfloat16>(h, S, I, I, hq, I, sh, st, nullptr, 1))) return rc;
     if ((rc = launch_fp8_gemm_grouped(hq, sh, w_down, s_down, o, offsets, static_cast<int>(E),
@@ -414,7 +423,7 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
     const int64_t work = T * (H / 8);
     combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
         o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
-        static_cast<__nv_bfloat16*>(y_bf16));
+        static_cast<__nv_bfloat16*>(y_bf16), nullptr);
     return cuda_check(cudaGetLastError(), "moe combine launch");
 }
 
@@ -622,22 +631,28 @@ extern "C" int metis_moe_nvfp4_grouped_gemm(const void* x_bf16, const int32_t* t
     const int64_t work = T * (H / 8);
     combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
         o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
-        static_cast<__nv_bfloat16*>(y_bf16));
+        static_cast<__nv_bfloat16*>(y_bf16), nullptr);
     return cuda_check(cudaGetLastError(), "moe_nvfp4 combine launch");
 }
 
 // ---------------------------------------------------------------------------
-// The shared expert with the routed combine in its down-projection's epilogue
-// ("Lernex/Metis-1.6-Praxis" card, "Architecture": one shared expert beside
-// the routed ones in every layer; the FP8 cards keep it in BF16):
-//   h_s = bf16(x W_sup^T)                      (BF16 tcgen05 GEMM)
-//   y   = bf16(bf16(h_s W_sdn^T) + sum_j w_j o_j)  (same GEMM, combine fused)
+// The shared expert joined to the routed combine ("Lernex/Metis-1.6-Praxis"
+// card, "Architecture": one shared expert beside the routed ones in every
+// layer; the FP8 cards keep it in BF16):
+//   h_s = bf16(x W_sup^T)                       (BF16 tcgen05 GEMM)
+//   s   = bf16(h_s W_sdn^T)                     (BF16 tcgen05 GEMM, into the workspace)
+//   y   = bf16(s + sum_j w_j o_j)               (the combine kernel, FP32, j ascending)
+// The combine adds s in the same pass that sums the routed rows, before the
+// one final rounding. (Adding the routed rows inside the down-projection's
+// epilogue instead measured slower on B200: its per-thread gathers of the
+// routed rows made the epilogue issue-bound.)
 extern "C" int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int64_t H, int64_t I_s,
                                               const void* w_sup_bf16, const void* w_sdn_bf16,
                                               const void* o_routed_bf16,
                                               const int32_t* slot_to_row, const float* topk_w,
                                               int64_t topk, void* y_bf16, void* workspace,
                                               size_t ws_bytes, metis_stream_t stream) {
+    using namespace moe;
     clear_error();
     if (T < 0 || T > (1ll << 28) || topk < 1 || topk > 8)
         return fail(METIS_ERR_INVALID_ARG, "shared_fused_combine: need T >= 0 and 1 <= topk <= 8 "
@@ -654,19 +669,24 @@ extern "C" int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int
     if (ws_bytes < need)
         return fail(METIS_ERR_INVALID_ARG, "shared_fused_combine: workspace of %zu bytes, need %zu", ws_bytes, need);
     if (!aligned(x_bf16, 16) || !aligned(w_sup_bf16, 16) || !aligned(w_sdn_bf16, 16) ||
-        !aligned(o_routed_bf16, 16) || !aligned(y_bf16, 16) || !aligned(workspace, 16) ||
+        !aligned(o_routed_bf16, 16) || !aligned(y_bf16, 16) || !aligned(workspace, 256) ||
         !aligned(slot_to_row, 4) || !aligned(topk_w, 4))
         return fail(METIS_ERR_INVALID_ARG,
-                    "shared_fused_combine: x, weights, o, y and the workspace 16-byte aligned");
+                    "shared_fused_combine: x, weights, o and y 16-byte aligned, the workspace 256-byte aligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     __nv_bfloat16* hs = static_cast<__nv_bfloat16*>(workspace);
+    __nv_bfloat16* s = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) +
+                                                        ((2 * T * I_s + 255) & ~static_cast<int64_t>(255)));
     int rc = launch_bf16_gemm(static_cast<const __nv_bfloat16*>(x_bf16),
                               static_cast<const __nv_bfloat16*>(w_sup_bf16), hs, static_cast<int>(T),
-                              static_cast<int>(I_s), static_cast<int>(H), nullptr, nullptr, nullptr, nullptr, 0, st);
+                              static_cast<int>(I_s), static_cast<int>(H), nullptr, st);
     if (rc) return rc;
-    return launch_bf16_gemm(hs, static_cast<const __nv_bfloat16*>(w_sdn_bf16),
-                            static_cast<__nv_bfloat16*>(y_bf16), static_cast<int>(T), static_cast<int>(H),
-                            static_cast<int>(I_s), nullptr, static_cast<const __nv_bfloat16*>(o_routed_bf16),
-                            slot_to_row, topk_w, static_cast<int>(topk), st);
+    if ((rc = launch_bf16_gemm(hs, static_cast<const __nv_bfloat16*>(w_sdn_bf16), s, static_cast<int>(T),
+                               static_cast<int>(H), static_cast<int>(I_s), nullptr, st)))
+        return rc;
+    const int64_t work = T * (H / 8);
+    combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o_routed_bf16), topk_w, slot_to_row, static_cast<int>(T),
+        static_cast<int>(topk), static_cast<int>(H), static_cast<__nv_bfloat16*>(y_bf16), s);
+    return cuda_check(cudaGetLastError(), "shared combine launch");
 }
-

@@ -284,15 +284,26 @@ __global__ void __launch_bounds__(QWARPS * 32, (NBL > 0 && NBL <= 4) ? 4 : 1) nv
     const int nb = static_cast<int>(a.K / 16);
     uint4 raw[RPW][NBL > 0 ? NBL : 1][2];
     bool live[RPW];
-    // rows below R are inside the buffer: their loads go out before the
-    // validity checks' own loads come back (a skipped row is read, not used)
+    // which rows are real (the routed layer's padded rows are not): lane u
+    // reads row u's validity, one round trip for all RPW rows, so that the
+    // rows that are skipped are never read
+    {
+        bool lv = false;
+        if (lane < RPW) {
+            const int64_t r = r0 + lane;
+            lv = r < a.R && !(a.nrows && r >= *a.nrows) && !(a.row_valid && a.row_valid[r] < 0);
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, lv);
+#pragma unroll
+        for (int u = 0; u < RPW; ++u) live[u] = (m >> u) & 1u;
+    }
 #pragma unroll
     for (int u = 0; u < RPW; ++u) {
         const int64_t r = r0 + u;
 #pragma unroll
         for (int i = 0; i < (NBL > 0 ? NBL : 1); ++i) {
             const int b = lane + 32 * i;
-            if (NBL > 0 && r < a.R && b < nb) {
+            if (NBL > 0 && live[u] && b < nb) {
                 const T* row = static_cast<const T*>(a.x) + r * a.ldx;
                 raw[u][i][0] = ld_nc_v4(row + 16 * b);
                 raw[u][i][1] = ld_nc_v4(row + 16 * b + 8);
@@ -300,11 +311,6 @@ __global__ void __launch_bounds__(QWARPS * 32, (NBL > 0 && NBL <= 4) ? 4 : 1) nv
                 raw[u][i][0] = raw[u][i][1] = make_uint4(0u, 0u, 0u, 0u);
             }
         }
-    }
-#pragma unroll
-    for (int u = 0; u < RPW; ++u) {
-        const int64_t r = r0 + u;
-        live[u] = r < a.R && !(a.nrows && r >= *a.nrows) && !(a.row_valid && a.row_valid[r] < 0);
     }
 #pragma unroll
     for (int u = 0; u < RPW; ++u) {

@@ -180,6 +180,27 @@ int make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t co
     return METIS_OK;
 }
 
+int make_tmap_2d_sw64(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                      uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows) {
+    CUtensorMap probe;
+    int rc = make_tmap_2d(&probe, base, 1, 16, 1, 16, 16, 1, false);  // resolves the encoder
+    if (rc) return rc;
+    if (elem_bytes != 2) return fail(METIS_ERR_INVALID_ARG, "64-byte swizzled tensor map of %d-byte elements", elem_bytes);
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(METIS_ERR_INVALID_ARG,
+                    "cuTensorMapEncodeTiled (64-byte swizzle) failed (%d): cols=%llu rows=%llu pitch=%llu",
+                    static_cast<int>(r), (unsigned long long)cols, (unsigned long long)rows,
+                    (unsigned long long)row_bytes);
+    return METIS_OK;
+}
+
 int make_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                     uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
     CUtensorMap probe;
@@ -209,13 +230,14 @@ int64_t moe_region_offset(int region, int64_t T, int64_t topk, int64_t E, int64_
         4 * (E + 1),  // OFFSETS
         4 * S,        // SLOT_TO_ROW
         4 * S,        // ROW_TO_SLOT
-        T * H,        // AQ: codes of x, token order
-        4 * T,        // SA: their scales
+        S * H,        // AQ
+        4 * S,        // SA
         2 * S * I,    // H
         S * I,        // HQ
         4 * S,        // SH
         2 * S * H,    // O
     };
+    (void)T;
     int64_t off = 0, at = -1;
     for (int r = 0; r < 10; ++r) {
         if (r == region) at = off;
@@ -340,8 +362,8 @@ extern "C" size_t metis_workspace_size(int op, int64_t M_or_T, int64_t N_or_I, i
             // the weights widened to BF16 [N, K]
             return M_or_T < 1 ? 0 : static_cast<size_t>(align256(2 * N_or_I * K_or_H));
         case METIS_OP_SHARED:
-            // the shared expert's hidden rows h_s [T, I_s] BF16
-            return static_cast<size_t>(align256(2 * M_or_T * N_or_I));
+            // the shared expert's hidden rows h_s [T, I_s] and its output s [T, H], BF16
+            return static_cast<size_t>(align256(2 * M_or_T * N_or_I) + align256(2 * M_or_T * K_or_H));
         case METIS_OP_MOE_NVFP4: {
             if (topk < 1 || E < 1) return 0;
             int64_t total = 0;

@@ -71,6 +71,13 @@ __device__ __forceinline__ uint4 ld_w16(const uint8_t* p) {
     return v;
 }
 
+// One 32-byte load (a whole sector) at a 32-byte aligned address.
+__device__ __forceinline__ void ld_w32(const uint8_t* p, uint4& a, uint4& b) {
+    asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+}
+
 // Four E4M3 bytes -> two BF16 pairs (bytes 0,1 and 2,3), exactly: E4M3 ->
 // FP16 (cvt.rn.f16x2.e4m3x2, exact) -> FP32 (exact) -> BF16 (exact, every
 // E4M3 value being a BF16 value). Eight instructions per four elements.
@@ -216,16 +223,26 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
         const int q = warp & 3;
         const int half = (warp - 2) / 4;   // which 32 elements of the k-block
         const int lane_base = q * 32;
+        const bool wide = (p.K % 32) == 0 && (reinterpret_cast<uintptr_t>(p.w) & 31u) == 0;
         int s = 0;
         uint32_t ph = 0;
         for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
             const int row = (t / num_m) * TILE_N + lane_base + lane;  // weight row = output channel
             const bool row_ok = row < p.N;
             const uint8_t* wrow = p.w + static_cast<size_t>(row_ok ? row : 0) * p.K + 32 * half;
+            // a thread's 32 bytes of a k-block are one sector: one 32-byte
+            // load when the rows are 32-byte aligned (K % 32 == 0; two 16-byte
+            // loads of the same sector would each move the whole sector
+            // through L1), two 16-byte loads otherwise and at the end of K
             auto load_kb = [&](int kb, uint4 (&r)[2]) {
+                const int k0 = kb * BKE + 32 * half;
+                if (wide && row_ok && k0 + 32 <= p.K) {
+                    ld_w32(wrow + kb * BKE, r[0], r[1]);
+                    return;
+                }
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int k = kb * BKE + 32 * half + 16 * j;
+                    const int k = k0 + 16 * j;
                     r[j] = (row_ok && k < p.K) ? ld_w16(wrow + kb * BKE + 16 * j) : make_uint4(0, 0, 0, 0);
                 }
             };
@@ -442,6 +459,5 @@ extern "C" int metis_w8a16_gemm_widened(const void* x_bf16, const uint8_t* wq, c
     int rc = launch_widen_e4m3(wq, wb, N * K, st);
     if (rc) return rc;
     return launch_bf16_gemm(static_cast<const __nv_bfloat16*>(x_bf16), wb, static_cast<__nv_bfloat16*>(y_bf16),
-                            static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), s_w, nullptr, nullptr,
-                            nullptr, 0, st);
+                            static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), s_w, st);
 }

@@ -146,8 +146,7 @@ def test_workspace_layout(lib):
     assert offs[0] == 0 and all(o % 256 == 0 for o in offs)
     assert all(b > a for a, b in zip(offs, offs[1:]))
     S = T * k
-    # x codes and scales in token order (AQ [T, H], SA [T]); the rest per slot
-    sizes = [4 * E, 4 * (E + 1), 4 * S, 4 * S, T * H, 4 * T, 2 * S * I, S * I, 4 * S, 2 * S * H]
+    sizes = [4 * E, 4 * (E + 1), 4 * S, 4 * S, S * H, 4 * S, 2 * S * I, S * I, 4 * S, 2 * S * H]
     for o, s, nxt in zip(offs, sizes, offs[1:] + [total]):
         assert o + s <= nxt
     assert metis.metis_moe_workspace_offset(10, T, k, E, H, I) == -1

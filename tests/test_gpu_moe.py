@@ -38,7 +38,7 @@ def run_moe(metis, d):
     out = dict(
         counts=R("COUNTS", (E,), torch.int32), offsets=R("OFFSETS", (E + 1,), torch.int32),
         s2r=R("SLOT_TO_ROW", (S,), torch.int32), r2s=R("ROW_TO_SLOT", (S,), torch.int32),
-        aq=R("AQ", (T, H), torch.uint8), sa=R("SA", (T,), torch.float32),
+        aq=R("AQ", (S, H), torch.uint8), sa=R("SA", (S,), torch.float32),
         h=R("H", (S, I), torch.int16).view(np.uint16), hq=R("HQ", (S, I), torch.uint8),
         sh=R("SH", (S,), torch.float32), o=R("O", (S, H), torch.int16).view(np.uint16),
         y=bf16_host(y), wq_up=wq_up, s_up=s_up, wq_dn=wq_dn, s_dn=s_dn)
@@ -54,17 +54,17 @@ def check_moe(d, g, tokens=None):
     assert_bytes_equal(g["offsets"], offsets, "offsets")
     assert_bytes_equal(g["s2r"], s2r, "slot_to_row")
     assert_bytes_equal(g["r2s"], r2s, "row_to_slot")
-    # per-token codes of x, once per token, in token order
+    # per-token codes of x, written into every row the token was routed to
     xq, sx = oracle.quant_per_token(d["x"])
-    assert_bytes_equal(g["aq"], xq, "x codes")
-    assert_bytes_equal(g["sa"].view(np.uint32), sx.view(np.uint32), "x scales")
+    tok_of_row = r2s // k
+    assert_bytes_equal(g["aq"], xq[tok_of_row], "x codes in expert order")
+    assert_bytes_equal(g["sa"].view(np.uint32), sx[tok_of_row].view(np.uint32), "x scales in expert order")
     slots = np.arange(T * k) if tokens is None else \
         (np.asarray(tokens)[:, None] * k + np.arange(k)).reshape(-1)
     rows = s2r[slots]
     exp = ids.reshape(-1)[slots]
-    tok = slots // k
-    # up-projection of each slot's token codes (which the GEMM gathers by row)
-    _, h64 = oracle.moe_expert_gemm(g["aq"][tok], g["sa"][tok], g["wq_up"], g["s_up"], exp)
+    # up-projection on the GPU's gathered operands
+    _, h64 = oracle.moe_expert_gemm(g["aq"][rows], g["sa"][rows], g["wq_up"], g["s_up"], exp)
     assert_close(g["h"][rows], h64, "h")
     # re-quantization of the GPU's h: bit-exact
     hq, sh = oracle.quant_per_token(g["h"][rows])
@@ -87,7 +87,9 @@ def check_moe(d, g, tokens=None):
 @pytest.mark.parametrize("T,H,I,E,k,seed", [(200, 256, 128, 8, 2, 11), (300, 512, 256, 64, 8, 12),
                                             (37, 128, 272, 5, 3, 13), (1, 64, 32, 4, 4, 14),
                                             (513, 256, 512, 16, 1, 15),
-                                            (96, 2048, 256, 16, 4, 18)])  # K = 2048: CTA-pair tiles
+                                            (96, 2048, 256, 16, 4, 18),   # K = 2048: CTA-pair tiles
+                                            # pairs, I = 1040: 5 column tiles, the last 16 wide
+                                            (150, 1024, 1040, 6, 2, 19)])
 def test_moe_parity(metis, T, H, I, E, k, seed):
     d = synth.moe(seed=seed, T=T, H=H, I=I, E=E, topk=k, hot=min(2, E), load_ratio=2.0)
     g = run_moe(metis, d)

@@ -90,11 +90,11 @@ def _prep_weights(metis, w):
 
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 272), (1, 8, 16), (129, 264, 1040),
                                    (520, 784, 1024), (257, 1024, 2048), (4500, 520, 256),
-                                   # the final partial wave cut into column pieces on 74 CTA
-                                   # pairs: 384 tiles (14 in the last wave, quarters); 320
-                                   # tiles with a 64-column last tile column (24, halves);
-                                   # 76 tiles with ragged M and N (2, quarters)
-                                   (4096, 6144, 256), (2560, 8000, 512), (1000, 4808, 256)])
+                                   # the final partial wave cut into column quarters on 74
+                                   # CTA pairs: 384 tiles (14 in the last wave); 76 tiles with
+                                   # ragged M and N (2); 84 tiles whose last tile column is
+                                   # 64 wide, so two of its quarters fall past N (10)
+                                   (4096, 6144, 256), (1000, 4808, 256), (1536, 3392, 384)])
 def test_fp8_gemm_parity(metis, M, N, K):
     d = synth.linear(M * 7 + N, M, K, N, outlier_channels=4, outlier_scale=20.0, zero_rows=(M // 3,))
     wq, s_w = _prep_weights(metis, d["w"])

@@ -1,9 +1,8 @@
-"""GPU parity of the BF16 GEMM and of the shared expert with the routed
-combine fused into its down-projection ("Lernex/Metis-1.6-Praxis" card,
-"Architecture": one shared expert beside the routed ones; the FP8 cards keep
-it in BF16), against the CPU oracle through the C ABI. BF16 outputs within
-1e-2 * (1 + |ref|); the fused combine with a zero shared expert is bit-exact
-with the routed layer's own combine kernel."""
+"""GPU parity of the BF16 GEMM and of the shared expert joined to the routed
+combine ("Lernex/Metis-1.6-Praxis" card, "Architecture": one shared expert
+beside the routed ones; the FP8 cards keep it in BF16), against the CPU oracle
+through the C ABI. BF16 outputs within 1e-2 * (1 + |ref|); the combine with a
+zero shared expert is bit-exact with the routed layer's own combine kernel."""
 import numpy as np
 import pytest
 import torch
@@ -52,6 +51,10 @@ def _run_fused(metis, d, wu, wd, o_dev, s2r_dev):
                                          dev(d["topk_w"]), y, ws)
     assert metis.metis_check_device_status() == 0
     hs = ws[:2 * T * I_s].view(torch.int16).view(T, I_s).cpu().numpy().view(np.uint16)
+    s_off = (2 * T * I_s + 255) // 256 * 256   # the shared output s [T, H] follows h_s
+    s = ws[s_off:s_off + 2 * T * H].view(torch.int16).view(T, H).cpu().numpy().view(np.uint16)
+    _, s64 = oracle.gemm_bf16(hs, wd)   # s is the GPU's h_s through the down-projection
+    assert_close(s, s64, "shared output s")
     return bf16_host(y), hs
 
 
