@@ -198,6 +198,22 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int32_t
                  : "memory");
 }
 
+// Bulk tensor store of a shared-memory box to global memory, its completion
+// tracked by this thread's bulk groups; and the group waits. A store must not
+// start at a negative coordinate; elements past the tensor's extent are not
+// written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of every committed store have been read
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed store has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Programmatic dependent launch: wait until the grids this launch depends on
 // have completed and their memory is visible; allow dependents to launch.
 __device__ __forceinline__ void grid_dependency_wait() {

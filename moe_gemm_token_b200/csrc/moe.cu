@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
     const int c0 = static_cast<int>(static_cast<int64_t>(g) * C / G);
     const int c1 = static_cast<int>(static_cast<int64_t>(g + 1) * C / G);
     int local = 0;
+    int first[SCAN_BATCH];  // this thread's first batch of counts, kept for the bases pass
     if (e < E) {
         for (int c = c0; c < c1; c += SCAN_BATCH) {
             int v[SCAN_BATCH];
@@ -86,6 +87,10 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
                 v[i] = c + i < c1 ? chunk_counts[static_cast<size_t>(c + i) * E + e] : 0;
 #pragma unroll
             for (int i = 0; i < SCAN_BATCH; ++i) local += v[i];
+            if (c == c0) {
+#pragma unroll
+                for (int i = 0; i < SCAN_BATCH; ++i) first[i] = v[i];
+            }
         }
     }
     part[g * Ep + e] = local;
@@ -144,9 +149,16 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
         int run = excl_e[e] + part[g * Ep + e];
         for (int c = c0; c < c1; c += SCAN_BATCH) {
             int v[SCAN_BATCH];
+            if (c == c0) {
+                // the first batch is still in registers (a run of up to
+                // SCAN_BATCH chunks, the common case, is read once)
 #pragma unroll
-            for (int i = 0; i < SCAN_BATCH; ++i)
-                v[i] = c + i < c1 ? chunk_counts[static_cast<size_t>(c + i) * E + e] : 0;
+                for (int i = 0; i < SCAN_BATCH; ++i) v[i] = first[i];
+            } else {
+#pragma unroll
+                for (int i = 0; i < SCAN_BATCH; ++i)
+                    v[i] = c + i < c1 ? chunk_counts[static_cast<size_t>(c + i) * E + e] : 0;
+            }
 #pragma unroll
             for (int i = 0; i < SCAN_BATCH; ++i) {
                 if (c + i < c1) chunk_counts[static_cast<size_t>(c + i) * E + e] = run;

@@ -617,20 +617,35 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // One 32-column chunk: y = bf16(acc * g_a[row] * g_b), staged in the warp's
-// swizzled 32 x 64-byte block, written as 8 rows x 64 bytes per instruction.
+// swizzled 32 x 64-byte block (the 64-byte TMA swizzle) and written by one TMA
+// store when all 32 rows belong to the tile's group (the map clips columns
+// past N), else as 8 rows x 64 bytes per instruction by the lanes.
 __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], int c, const Tile& ti, int q,
                                             int lane, float ga, float gb, uint8_t* stg,
-                                            __nv_bfloat16* y, int N) {
+                                            __nv_bfloat16* y, int N, const CUtensorMap* tmY) {
     uint32_t pk[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j)
         pk[j] = pack_bf16x2(__fmul_rn(__fmul_rn(__uint_as_float(v[2 * j]), ga), gb),
                             __fmul_rn(__fmul_rn(__uint_as_float(v[2 * j + 1]), ga), gb));
+    // the previous chunk's store has read the staging block
+    if (lane == 0) bulk_wait_read();
     __syncwarp();
 #pragma unroll
     for (int pc = 0; pc < 4; ++pc)
         *reinterpret_cast<uint4*>(stg + lane * 64 + ((pc ^ ((lane >> 1) & 3)) * 16)) =
             make_uint4(pk[4 * pc], pk[4 * pc + 1], pk[4 * pc + 2], pk[4 * pc + 3]);
+    const int row0 = ti.a_row0 + q * 32;
+    if (ti.n0 + c * 32 >= N) return;  // wholly past the last column: nothing to store
+    if (row0 + 32 <= ti.row_end) {
+        fence_proxy_async_shared();  // the staging writes, to the TMA engine
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmY, smem_u32(stg), ti.n0 + c * 32, row0);
+            bulk_commit();
+        }
+        return;
+    }
     __syncwarp();
     const int n = ti.n0 + c * 32 + (lane & 3) * 8;
 #pragma unroll
@@ -648,7 +663,7 @@ template <int CTAS, bool GROUPED>
 __global__ void __launch_bounds__(THREADS, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                  const GemmParams p) {
+                  const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
     using L = Lay<CTAS, GROUPED>;
     constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -691,6 +706,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmY);
         if constexpr (CTAS == 2) {
             tma_prefetch_desc(&tmSFA);
             tma_prefetch_desc(&tmSFB);
@@ -981,10 +997,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 if constexpr (CTAS == 2) mbar_arrive_cluster_relaxed(mapa_shared(tempty, 0));
                 else mbar_arrive_relaxed(tempty);
             }
-            store_chunk(va, 2 * part, ti, q, lane, ga, gb, stg, p.y, p.N);
-            store_chunk(vb, 2 * part + 1, ti, q, lane, ga, gb, stg, p.y, p.N);
+            store_chunk(va, 2 * part, ti, q, lane, ga, gb, stg, p.y, p.N, &tmY);
+            store_chunk(vb, 2 * part + 1, ti, q, lane, ga, gb, stg, p.y, p.N, &tmY);
             acc_phase ^= 1u;
         }
+        // this warp's output stores have completed before the CTA exits
+        if (lane == 0) bulk_wait_all();
     }
 
     __syncwarp();
@@ -1072,7 +1090,11 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
     const bool grouped = offsets != nullptr;
     const bool pair = grouped || M > ROWS;
     const uint32_t b_box = pair ? BN / 2 : BN;
-    CUtensorMap ta, tb, tsa, tsb;
+    CUtensorMap ta, tb, tsa, tsb, ty;
+    // y: [M, N] (dense) or one row per row of A (grouped), BF16
+    if ((rc = make_tmap_2d_sw64(&ty, y, 2, static_cast<uint64_t>(N), static_cast<uint64_t>(grouped ? a_rows : M),
+                                static_cast<uint64_t>(N) * 2, 32, 32)))
+        return rc;
     if ((rc = make_tmap_2d(&ta, qa, 1, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(a_rows),
                            static_cast<uint64_t>(K / 2), BKB, ROWS, true)))
         return rc;
@@ -1094,7 +1116,7 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
             if ((rc = max_pairs<true>(di, &pairs))) return rc;
             clusters = pairs;
             return cuda_check(launch_pdl(nvfp4_gemm_kernel<2, true>, dim3(2 * clusters), dim3(THREADS),
-                                         Lay<2, true>::BYTES, st, 2, ta, tb, tsa, tsb, p),
+                                         Lay<2, true>::BYTES, st, 2, ta, tb, tsa, tsb, ty, p),
                               "nvfp4 grouped gemm (CTA pair) launch");
         }
         if ((rc = prepare_gemm<2, false>(di))) return rc;
@@ -1102,7 +1124,7 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
         const int64_t tiles = ((static_cast<int64_t>(M) + 2 * ROWS - 1) / (2 * ROWS)) * ((N + BN - 1) / BN);
         clusters = static_cast<int>(tiles < pairs ? tiles : pairs);
         return cuda_check(launch_pdl(nvfp4_gemm_kernel<2, false>, dim3(2 * clusters), dim3(THREADS),
-                                     Lay<2, false>::BYTES, st, 2, ta, tb, tsa, tsb, p),
+                                     Lay<2, false>::BYTES, st, 2, ta, tb, tsa, tsb, ty, p),
                           "nvfp4 gemm (CTA pair) launch");
     }
     const int64_t tiles = ((static_cast<int64_t>(M) + ROWS - 1) / ROWS) * ((N + BN - 1) / BN);
@@ -1110,7 +1132,7 @@ int launch_nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga, in
     const int grid = static_cast<int>(tiles < di.num_sms ? tiles : di.num_sms);
     if ((rc = prepare_gemm<1, false>(di))) return rc;
     return cuda_check(launch_pdl(nvfp4_gemm_kernel<1, false>, dim3(grid), dim3(THREADS), Lay<1, false>::BYTES,
-                                 st, 1, ta, tb, tsa, tsb, p),
+                                 st, 1, ta, tb, tsa, tsb, ty, p),
                       "nvfp4 gemm launch");
 }
 
