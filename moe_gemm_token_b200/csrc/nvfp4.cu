@@ -240,12 +240,52 @@ __device__ __forceinline__ void quant_row(const QuantArgs& a, int64_t r, int lan
         }
     };
     if constexpr (NBL > 0) {
+        // register-resident rows: every block of the row is encoded first
+        // (lane l: blocks l, l + 32, ...), then stored to each destination
+        // row with that row's code and scale offsets computed once
+        uint32_t lo[NBL], hi[NBL], s4[NBL];
 #pragma unroll
         for (int i = 0; i < NBL; ++i) {
-            if (32 * i >= nb) break;  // warp-uniform
-            float v[16];
-            unpack(i, v);
-            block_pass(32 * i, v, bmax[i]);
+            lo[i] = hi[i] = s4[i] = 0;
+            if (32 * i >= nb) continue;  // warp-uniform
+            const int b = 32 * i + lane;
+            uint32_t sbc = 0;
+            if (b < nb) {
+                float v[16];
+                unpack(i, v);
+                sbc = f32x2_to_e4m3x2(__fdiv_rn(__fmul_rn(bmax[i], inv_g), 6.0f), 0.0f) & 0xFFu;
+                const float inv_s = inv_scale[sbc];
+                float w[16];
+#pragma unroll
+                for (int h = 0; h < 16; ++h) w[h] = __fmul_rn(__fmul_rn(v[h], inv_g), inv_s);
+                lo[i] = f32x8_to_e2m1x8(w);
+                hi[i] = f32x8_to_e2m1x8(w + 8);
+            }
+            // the scales of the 4 blocks of a 64-element chunk (lanes 4c .. 4c+3)
+            uint32_t s = sbc;
+            s |= __shfl_down_sync(0xffffffffu, sbc, 1) << 8;
+            s |= __shfl_down_sync(0xffffffffu, sbc, 2) << 16;
+            s |= __shfl_down_sync(0xffffffffu, sbc, 3) << 24;
+            s4[i] = s;
+        }
+        for (int j = 0; j < ndst; ++j) {
+            int64_t dr = r;
+            if (a.dst_rows) {
+                const int d = __shfl_sync(0xffffffffu, my_dst, j & 31);
+                dr = j < 32 ? d : a.dst_rows[r * a.topk + j];
+            }
+            if (dr < 0) continue;  // warp-uniform
+            uint8_t* qrow = a.q + dr * (a.K / 2);
+            uint8_t* srow = a.sf + (a.tiled ? tiled_sf_offset(dr, 0, kc) : dr * (a.K / 16));
+#pragma unroll
+            for (int i = 0; i < NBL; ++i) {
+                const int b = 32 * i + lane;
+                if (b >= nb) continue;
+                *reinterpret_cast<uint2*>(qrow + 8 * b) = make_uint2(lo[i], hi[i]);
+                if ((lane & 3) == 0)
+                    *reinterpret_cast<uint32_t*>(srow + (a.tiled ? 512 * (b >> 2) : b)) = s4[i];
+            }
+            if (lane == 0 && !a.gamax) a.g[dr] = g_row;
         }
     } else {
         for (int b0 = 0; b0 < nb; b0 += 32) {
