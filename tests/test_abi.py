@@ -109,6 +109,18 @@ def test_host_validation_without_gpu(lib):
     assert lib.metis_moe_fp8_grouped_gemm(p, p, p, 8, 2, 4, 64, 32, p, p, p, p, 0, p, p, 16,
                                           null) == metis.METIS_ERR_INVALID_ARG
     assert b"workspace" in lib.metis_last_error()
+    # allocation-free routed layer: the same shape checks first (an unsupported
+    # activation is reported as such, absurd T is rejected before any size is
+    # computed), then y is required, then the built-in scratch bounds the size
+    na = lib.metis_moe_fp8_grouped_gemm_noalloc
+    assert na(p, p, p, 4096, 8, 64, 2048, 1024, p, p, p, p, 1, p, null) == metis.METIS_ERR_UNSUPPORTED
+    assert na(p, p, p, 8, 5, 4, 64, 32, p, p, p, p, 0, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert na(p, p, p, 1 << 40, 8, 64, 2048, 1024, p, p, p, p, 0, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert na(p, p, p, 0, 8, 64, 2048, 1024, p, p, p, p, 0, null, null) == metis.METIS_OK  # nothing to do
+    assert na(p, p, p, 16, 8, 64, 2048, 1024, p, p, p, p, 0, null, null) == metis.METIS_ERR_INVALID_ARG
+    assert b"y is required" in lib.metis_last_error()
+    assert na(p, p, p, 4096, 8, 64, 2048, 1024, p, p, p, p, 0, p, null) == metis.METIS_ERR_INVALID_ARG
+    assert b"16 MiB" in lib.metis_last_error()
     # watchdog self-test: the limit must be 1 .. 1e9 ns
     assert lib.metis_watchdog_selftest(0, null) == metis.METIS_ERR_INVALID_ARG
     assert lib.metis_watchdog_selftest(2000000000, null) == metis.METIS_ERR_INVALID_ARG
