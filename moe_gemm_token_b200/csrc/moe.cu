@@ -204,6 +204,116 @@ __global__ void __launch_bounds__(CHUNK) rank_kernel(const int32_t* __restrict__
     }
 }
 
+// The prefix sums and the stable ranks in one kernel, for routing tables that
+// fit in shared memory (C * E <= RS_MAX_TAB counts, E <= RS_MAX_E): every
+// block reads the whole per-chunk count table (a few tens of KB from L2),
+// derives each expert's total, its own chunk's base row and the expert
+// offsets (padded to `pad` rows), and ranks its chunk as rank_kernel does.
+// Block 0 writes counts and offsets; the pad rows of expert e (row_to_slot
+// -1) are marked by block e % gridDim.x. Saves the single-block scan kernel
+// and its launch.
+constexpr int RS_MAX_TAB = 16384;
+constexpr int RS_MAX_E = 256;
+__global__ void __launch_bounds__(CHUNK) rank_scan_kernel(const int32_t* __restrict__ ids, int S, int E,
+                                                          const int32_t* __restrict__ chunk_counts,
+                                                          int32_t* __restrict__ counts,
+                                                          int32_t* __restrict__ offsets, int pad,
+                                                          int32_t* __restrict__ slot_to_row,
+                                                          int32_t* __restrict__ row_to_slot) {
+    constexpr int WARPS = CHUNK / 32;
+    extern __shared__ int tab[];                 // [C][E] counts of every chunk
+    __shared__ int wcnt[WARPS][RS_MAX_E];        // per-warp counts, then exclusive prefix over warps
+    __shared__ int part_tot[CHUNK];              // [g][e] partial totals over chunk groups
+    __shared__ int part_bef[CHUNK];              // [g][e] partial counts of the chunks before this one
+    __shared__ int base_e[RS_MAX_E];             // this chunk's first row of expert e
+    __shared__ int warp_tot[WARPS];
+    const int C = gridDim.x;
+    const int c = blockIdx.x;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    // the count table, and this chunk's warp-level ranks meanwhile
+    if ((C * E & 3) == 0) {
+        const int4* src = reinterpret_cast<const int4*>(chunk_counts);
+        for (int i = threadIdx.x; i < C * E / 4; i += CHUNK) reinterpret_cast<int4*>(tab)[i] = src[i];
+    } else {
+        for (int i = threadIdx.x; i < C * E; i += CHUNK) tab[i] = chunk_counts[i];
+    }
+    for (int i = threadIdx.x; i < WARPS * E; i += CHUNK) wcnt[i / E][i % E] = 0;
+    const int s = c * CHUNK + threadIdx.x;
+    int e = s < S ? ids[s] : -1;
+    if (e >= E) e = -1;
+    const bool ok = e >= 0;
+    if (s < S && !ok) slot_to_row[s] = -1;  // dropped: never written or read again
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(peers & ((1u << lane) - 1u));
+    __syncthreads();
+    if (ok && rank_w == 0) wcnt[warp][e] = __popc(peers);
+    // expert x's total and the count of its slots in chunks before c:
+    // G = CHUNK / Ep groups of threads each sum a run of chunks
+    int Ep = 1;
+    while (Ep < E) Ep <<= 1;
+    const int G = CHUNK / Ep;
+    {
+        const int x = threadIdx.x % Ep, g = threadIdx.x / Ep;
+        const int c0 = g * C / G, c1 = (g + 1) * C / G;
+        int tot = 0, bef = 0;
+        if (x < E)
+            for (int cc = c0; cc < c1; ++cc) {
+                const int v = tab[cc * E + x];
+                tot += v;
+                if (cc < c) bef += v;
+            }
+        part_tot[g * Ep + x] = tot;
+        part_bef[g * Ep + x] = bef;
+    }
+    __syncthreads();
+    // thread t < Ep: expert t's total (padded) and its exclusive prefix over experts
+    int total = 0, before = 0;
+    if (threadIdx.x < Ep) {
+        for (int g = 0; g < G; ++g) {
+            total += part_tot[g * Ep + threadIdx.x];
+            before += part_bef[g * Ep + threadIdx.x];
+        }
+    }
+    const int ptotal = (total + pad - 1) / pad * pad;
+    int incl = ptotal;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    // per-warp exclusive prefix over experts (and warp prefix sums for x)
+    for (int i = threadIdx.x; i < E; i += CHUNK) {
+        int run = 0;
+        for (int w = 0; w < WARPS; ++w) {
+            const int v = wcnt[w][i];
+            wcnt[w][i] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    int wbase = 0;
+    for (int w = 0; w < warp; ++w) wbase += warp_tot[w];
+    if (threadIdx.x < E) {
+        const int excl = wbase + incl - ptotal;  // offset of expert threadIdx.x
+        base_e[threadIdx.x] = excl + before;
+        if (c == 0) {
+            counts[threadIdx.x] = total;
+            offsets[threadIdx.x] = excl;
+            if (threadIdx.x == E - 1) offsets[E] = excl + ptotal;
+        }
+        // pad rows (fewer than pad per expert), expert x by block x % C
+        if (pad > 1 && threadIdx.x % C == c)
+            for (int k = total; k < ptotal; ++k) row_to_slot[excl + k] = -1;
+    }
+    __syncthreads();
+    if (ok) {
+        const int row = base_e[e] + wcnt[warp][e] + rank_w;
+        slot_to_row[s] = row;
+        row_to_slot[row] = s;
+    }
+}
+
 // y[t, n..n+7] = bf16( s[t, n..n+7] + sum_j w[t, j] * o[slot_to_row[t*topk + j], n..n+7] ),
 // s the shared expert's BF16 output (null: 0).
 // HBM-bound: the row indices and weights of the token are read first, then
@@ -359,6 +469,35 @@ int check_moe_shape(int act, int64_t T, int64_t topk, int64_t E, int64_t H, int6
     return METIS_OK;
 }
 
+// Routing: histogram per chunk, then the prefix sums and stable ranks (one
+// fused kernel when the count table fits in shared memory, else a
+// single-block scan followed by the rank kernel). pad > 1: every expert's
+// rows padded to a multiple of pad, pad rows of row_to_slot set to -1.
+int launch_routing(const int32_t* ids, int S, int E, int32_t* chunk_tab, int32_t* counts, int32_t* offsets,
+                   int pad, int32_t* s2r, int32_t* r2s, uint32_t* status, cudaStream_t st) {
+    const int C = (S + CHUNK - 1) / CHUNK;
+    count_kernel<<<C, CHUNK, 0, st>>>(ids, S, E, chunk_tab, status);
+    const size_t tab_bytes = static_cast<size_t>(C) * E * 4;
+    if (static_cast<int64_t>(C) * E <= RS_MAX_TAB && E <= RS_MAX_E) {
+        static bool attr_done[64];
+        int dev = 0;
+        int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+        if (rc) return rc;
+        if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+            if ((rc = cuda_check(cudaFuncSetAttribute(rank_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      RS_MAX_TAB * 4),
+                                 "cudaFuncSetAttribute(rank_scan)")))
+                return rc;
+            attr_done[dev] = true;
+        }
+        rank_scan_kernel<<<C, CHUNK, tab_bytes, st>>>(ids, S, E, chunk_tab, counts, offsets, pad, s2r, r2s);
+    } else {
+        scan_kernel<<<1, SCAN_THREADS, 0, st>>>(chunk_tab, C, E, counts, offsets, pad, pad > 1 ? r2s : nullptr);
+        rank_kernel<<<C, CHUNK, 0, st>>>(ids, S, E, chunk_tab, s2r, r2s);
+    }
+    return cuda_check(cudaGetLastError(), "moe routing launch");
+}
+
 }  // namespace moe
 }  // namespace metis
 
@@ -410,13 +549,9 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
 
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
-    count_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
-                                      status);
-    scan_kernel<<<1, SCAN_THREADS, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets, 1,
-                                            nullptr);
-    rank_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
-                                     s2r, r2s);
-    if ((rc = cuda_check(cudaGetLastError(), "moe routing launch"))) return rc;
+    if ((rc = launch_routing(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab, counts, offsets, 1,
+                             s2r, r2s, status, st)))
+        return rc;
     // x quantized once per token, its codes and scale written straight into
     // every expert-ordered row the token was routed to (gathering the rows
     // inside the GEMM with 4-row TMA gathers instead measured 3x slower for
@@ -620,12 +755,9 @@ extern "C" int metis_moe_nvfp4_grouped_gemm(const void* x_bf16, const int32_t* t
 
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
-    count_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
-                                      status);
-    scan_kernel<<<1, SCAN_THREADS, 0, st>>>(chunk_tab, C, static_cast<int>(E), counts, offsets, 128, r2s);
-    rank_kernel<<<C, CHUNK, 0, st>>>(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab,
-                                     s2r, r2s);
-    if ((rc = cuda_check(cudaGetLastError(), "moe_nvfp4 routing launch"))) return rc;
+    if ((rc = launch_routing(topk_ids, static_cast<int>(S), static_cast<int>(E), chunk_tab, counts, offsets, 128,
+                             s2r, r2s, status, st)))
+        return rc;
     // x: NVFP4 per token, each token once, into the rows it was routed to
     if ((rc = launch_nvfp4_quant(static_cast<const __nv_bfloat16*>(x_bf16), T, H, H, 1, aq, sfa, 1, ga,
                                  s2r, static_cast<int>(topk), nullptr, nullptr, st)))

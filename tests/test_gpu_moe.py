@@ -96,6 +96,17 @@ def test_moe_parity(metis, T, H, I, E, k, seed):
     check_moe(d, g)
 
 
+@pytest.mark.parametrize("T,E,k,seed", [(64, 320, 4, 40), (4096, 160, 8, 41)])
+def test_moe_routing_without_the_fused_scan(metis, T, E, k, seed):
+    """Routing tables too large for the fused prefix-sum and rank kernel (more
+    than 256 experts; more than 16384 per-chunk counts: 128 chunks x 160
+    experts) take the single-block scan and the rank kernel; every stage
+    still matches the oracle."""
+    d = synth.moe(seed=seed, T=T, H=128, I=64, E=E, topk=k, hot=4, load_ratio=2.0)
+    g = run_moe(metis, d)
+    check_moe(d, g)
+
+
 def test_moe_empty_experts(metis):
     """Experts that receive no token produce no tiles; the others are unaffected."""
     d = synth.moe(seed=16, T=64, H=128, I=64, E=16, topk=2, hot=0, load_ratio=1.0)

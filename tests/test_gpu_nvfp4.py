@@ -300,9 +300,12 @@ def test_moe_nvfp4_parity(metis, T, H, I, E, k, seed):
     check_moe4(d, g, up, dn)
 
 
-def test_moe_nvfp4_many_experts(metis):
-    """256 experts (group tables and pad marking at larger E), top-4."""
-    d = synth.moe(seed=19, T=96, H=128, I=128, E=256, topk=4, hot=4, load_ratio=2.0)
+@pytest.mark.parametrize("E,seed", [(256, 19), (320, 20)])
+def test_moe_nvfp4_many_experts(metis, E, seed):
+    """256 experts (group tables and pad marking at larger E; the fused
+    prefix-sum and rank kernel) and 320 (past its 256-expert limit: the
+    single-block scan, which marks the pad rows, then the rank kernel), top-4."""
+    d = synth.moe(seed=seed, T=96, H=128, I=128, E=E, topk=4, hot=4, load_ratio=2.0)
     up, dn = _weights_nvfp4(d["w_up"]), _weights_nvfp4(d["w_down"])
     g = run_moe4(metis, d, up, dn)
     check_moe4(d, g, up, dn)
