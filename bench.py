@@ -418,12 +418,16 @@ def run_metis(args):
     torch.cuda.synchronize()
     a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     reps = 3
-    a_ev.record(stream)
-    for _ in range(reps):
-        iso_graph.replay()
-    b_ev.record(stream)
-    torch.cuda.synchronize()
+    # the SM clock during this window (about 26 ms): under the power cap it
+    # falls while the GEMMs run, and the kernel's time follows it
+    with ClockSampler(local, period=0.002) as iso_clk:
+        a_ev.record(stream)
+        for _ in range(reps):
+            iso_graph.replay()
+        b_ev.record(stream)
+        torch.cuda.synchronize()
     iso_ms = a_ev.elapsed_time(b_ev) / (reps * ISO_CALLS)
+    iso_clocks = iso_clk.summary()
     del iso_graph
     achieved = flops / (iso_ms * 1e-3) / 1e12
     # (b) inside the step, as a cross-check: a separate replay of the step
@@ -454,6 +458,8 @@ def run_metis(args):
                 "timed_as": f"{ISO_CALLS} GEMM launches per CUDA graph, {SETS} rotating input sets, "
                             f"{reps} replays between events",
                 "us_per_launch": iso_ms * 1e3,
+                "clocks": iso_clocks,
+                "kcycles_per_launch": (iso_ms * iso_clocks["sm_mhz"] if iso_clocks.get("sm_mhz") else None),
                 "frac_of_sustained": achieved / sustained,
                 "frac_of_nominal_fp8": achieved / NOMINAL_FP8_TFLOPS,
                 "in_step": {"achieved": in_step, "frac": in_step / burst, "gemm_samples": len(g1),
