@@ -14,6 +14,8 @@
 //   6. per-row re-quantization of h
 //   7. grouped down-projection
 //   8. weighted un-permute y[t] = sum_j w[t,j] * o[row(t,j)], FP32, j ascending.
+#include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -316,71 +318,138 @@ __global__ void __launch_bounds__(CHUNK) rank_scan_kernel(const int32_t* __restr
 
 // y[t, n..n+7] = bf16( s[t, n..n+7] + sum_j w[t, j] * o[slot_to_row[t*topk + j], n..n+7] ),
 // s the shared expert's BF16 output (null: 0).
-// HBM-bound: the row indices and weights of the token are read first, then
-// every row load is issued before the first add (for topk <= COMBINE_MAXK),
-// so a thread has topk 16-byte loads in flight. The sum starts from s and runs
-// over j in ascending order in FP32 either way.
+// HBM-bound. A persistent grid walks the (token, 8-column group) items with
+// a stride of its thread count. For topk <= COMBINE_MAXK a thread issues
+// every row load of its item before the first add (topk 16-byte loads in
+// flight) and reads the next item's row indices and weights while they are
+// in flight, so the index round trip is off the critical path. Three blocks
+// per SM (80 registers a thread): two blocks, unbounded, measured slower.
+// The sum starts from s and runs over j in ascending order in FP32 either
+// way.
 constexpr int COMBINE_MAXK = 8;
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ o,
+__global__ void __launch_bounds__(256, 3) combine_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const float* __restrict__ w,
                                                       const int32_t* __restrict__ slot_to_row,
                                                       int T, int topk, int H,
                                                       __nv_bfloat16* __restrict__ y,
                                                       const __nv_bfloat16* __restrict__ s) {
     const int groups = H / 8;
-    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= static_cast<int64_t>(T) * groups) return;
-    const int t = static_cast<int>(idx / groups);
-    const int n = static_cast<int>(idx - static_cast<int64_t>(t) * groups) * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (s != nullptr) {
-        const uint4 v = *reinterpret_cast<const uint4*>(s + static_cast<size_t>(t) * H + n);
-        const uint32_t sv[4] = {v.x, v.y, v.z, v.w};
+    const int64_t total = static_cast<int64_t>(T) * groups;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    auto start = [&](int64_t i, float (&acc)[8]) {
+        const int t = static_cast<int>(i / groups);
+        const int n = static_cast<int>(i - static_cast<int64_t>(t) * groups) * 8;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc[2 * i] = bf16_lo(sv[i]);
-            acc[2 * i + 1] = bf16_hi(sv[i]);
-        }
-    }
-    auto add = [&](float wj, const uint4& c) {
-        const uint32_t v[4] = {c.x, c.y, c.z, c.w};
+        for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+        if (s != nullptr) {
+            const uint4 v = *reinterpret_cast<const uint4*>(s + static_cast<size_t>(t) * H + n);
+            const uint32_t sv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc[2 * i] = fmaf(wj, bf16_lo(v[i]), acc[2 * i]);
-            acc[2 * i + 1] = fmaf(wj, bf16_hi(v[i]), acc[2 * i + 1]);
-        }
-    };
-    if (topk <= COMBINE_MAXK) {
-        int r[COMBINE_MAXK];
-        float wj[COMBINE_MAXK];
-        uint4 c[COMBINE_MAXK];
-#pragma unroll
-        for (int j = 0; j < COMBINE_MAXK; ++j) {
-            if (j < topk) {
-                r[j] = slot_to_row[static_cast<int64_t>(t) * topk + j];
-                wj[j] = w[static_cast<int64_t>(t) * topk + j];
+            for (int k = 0; k < 4; ++k) {
+                acc[2 * k] = bf16_lo(sv[k]);
+                acc[2 * k + 1] = bf16_hi(sv[k]);
             }
         }
+    };
+    auto add = [&](float (&acc)[8], float wj, const uint4& c) {
+        const uint32_t v[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int j = 0; j < COMBINE_MAXK; ++j)
-            if (j < topk && r[j] >= 0) c[j] = *reinterpret_cast<const uint4*>(o + static_cast<size_t>(r[j]) * H + n);
+        for (int k = 0; k < 4; ++k) {
+            acc[2 * k] = fmaf(wj, bf16_lo(v[k]), acc[2 * k]);
+            acc[2 * k + 1] = fmaf(wj, bf16_hi(v[k]), acc[2 * k + 1]);
+        }
+    };
+    auto finish = [&](int64_t i, const float (&acc)[8]) {
+        const int t = static_cast<int>(i / groups);
+        const int n = static_cast<int>(i - static_cast<int64_t>(t) * groups) * 8;
+        uint4 out;
+        out.x = pack_bf16x2(acc[0], acc[1]);
+        out.y = pack_bf16x2(acc[2], acc[3]);
+        out.z = pack_bf16x2(acc[4], acc[5]);
+        out.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + n) = out;
+    };
+    if (topk <= COMBINE_MAXK) {
+        // row indices (-1: no row) and weights of an item's token
+        auto fetch = [&](int64_t i, int (&r)[COMBINE_MAXK], float (&wj)[COMBINE_MAXK]) {
+            const int64_t t = i / groups;
 #pragma unroll
-        for (int j = 0; j < COMBINE_MAXK; ++j)
-            if (j < topk && r[j] >= 0) add(wj[j], c[j]);
+            for (int j = 0; j < COMBINE_MAXK; ++j) {
+                r[j] = -1;
+                wj[j] = 0.0f;
+                if (j < topk) {
+                    r[j] = slot_to_row[t * topk + j];
+                    wj[j] = w[t * topk + j];
+                }
+            }
+        };
+        int r[COMBINE_MAXK];
+        float wj[COMBINE_MAXK];
+        if (idx < total) fetch(idx, r, wj);
+        while (idx < total) {
+            const int n = static_cast<int>(idx % groups) * 8;
+            uint4 c[COMBINE_MAXK];
+#pragma unroll
+            for (int j = 0; j < COMBINE_MAXK; ++j)
+                if (r[j] >= 0) c[j] = *reinterpret_cast<const uint4*>(o + static_cast<size_t>(r[j]) * H + n);
+            float acc[8];
+            start(idx, acc);
+            const int64_t next = idx + stride;
+            int rn[COMBINE_MAXK];
+            float wn[COMBINE_MAXK];
+            if (next < total) fetch(next, rn, wn);
+#pragma unroll
+            for (int j = 0; j < COMBINE_MAXK; ++j)
+                if (r[j] >= 0) add(acc, wj[j], c[j]);
+            finish(idx, acc);
+            idx = next;
+#pragma unroll
+            for (int j = 0; j < COMBINE_MAXK; ++j) {
+                r[j] = rn[j];
+                wj[j] = wn[j];
+            }
+        }
     } else {
-        for (int j = 0; j < topk; ++j) {
-            const int64_t s = static_cast<int64_t>(t) * topk + j;
-            const int rj = slot_to_row[s];
-            if (rj < 0) continue;
-            add(w[s], *reinterpret_cast<const uint4*>(o + static_cast<size_t>(rj) * H + n));
+        for (; idx < total; idx += stride) {
+            const int64_t t = idx / groups;
+            const int n = static_cast<int>(idx % groups) * 8;
+            float acc[8];
+            start(idx, acc);
+            for (int j = 0; j < topk; ++j) {
+                const int rj = slot_to_row[t * topk + j];
+                if (rj < 0) continue;
+                add(acc, w[t * topk + j], *reinterpret_cast<const uint4*>(o + static_cast<size_t>(rj) * H + n));
+            }
+            finish(idx, acc);
         }
     }
-    uint4 out;
-    out.x = pack_bf16x2(acc[0], acc[1]);
-    out.y = pack_bf16x2(acc[2], acc[3]);
-    out.z = pack_bf16x2(acc[4], acc[5]);
-    out.w = pack_bf16x2(acc[6], acc[7]);
-    *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + n) = out;
+}
+
+// Launches the combine on a persistent grid: as many 256-thread blocks as
+// fit on the device at once (occupancy cached per device), at most one per
+// 256 items.
+int launch_combine(const __nv_bfloat16* o, const float* w, const int32_t* slot_to_row, int64_t T,
+                   int64_t topk, int64_t H, __nv_bfloat16* y, const __nv_bfloat16* s, cudaStream_t st) {
+    DeviceInfo di;
+    int rc;
+    if ((rc = current_device_info(&di))) return rc;
+    static std::atomic<int> per_sm[64];
+    int occ = per_sm[di.device & 63].load(std::memory_order_relaxed);
+    if (occ == 0) {
+        int n = 0;
+        if ((rc = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_kernel, 256, 0),
+                             "combine occupancy")))
+            return rc;
+        occ = n > 0 ? n : 1;
+        per_sm[di.device & 63].store(occ, std::memory_order_relaxed);
+    }
+    const int64_t work = T * (H / 8);
+    const int64_t blocks = std::min<int64_t>((work + 255) / 256, static_cast<int64_t>(di.num_sms) * occ);
+    if (blocks <= 0) return METIS_OK;
+    combine_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(o, w, slot_to_row, static_cast<int>(T),
+                                                                  static_cast<int>(topk), static_cast<int>(H), y, s);
+    return cuda_check(cudaGetLastError(), "moe combine launch");
 }
 
 // Router top-k, one warp per token (the reading of the cards' FP32 router
@@ -567,11 +636,7 @@ extern "C" int metis_moe_fp8_grouped_gemm(const void* x_bf16, const int32_t* top
                                       static_cast<int>(S), static_cast<int>(H), static_cast<int>(I), st)))
         return rc;
     if (!y_bf16) return METIS_OK;  // the caller combines (metis_moe_shared_fused_combine)
-    const int64_t work = T * (H / 8);
-    combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
-        o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
-        static_cast<__nv_bfloat16*>(y_bf16), nullptr);
-    return cuda_check(cudaGetLastError(), "moe combine launch");
+    return launch_combine(o, topk_w, s2r, T, topk, H, static_cast<__nv_bfloat16*>(y_bf16), nullptr, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -772,11 +837,7 @@ extern "C" int metis_moe_nvfp4_grouped_gemm(const void* x_bf16, const int32_t* t
                                 static_cast<int>(E), 0, static_cast<int>(H), static_cast<int>(I), st)))
         return rc;
     if (!y_bf16) return METIS_OK;  // the caller combines (metis_moe_shared_fused_combine)
-    const int64_t work = T * (H / 8);
-    combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
-        o, topk_w, s2r, static_cast<int>(T), static_cast<int>(topk), static_cast<int>(H),
-        static_cast<__nv_bfloat16*>(y_bf16), nullptr);
-    return cuda_check(cudaGetLastError(), "moe_nvfp4 combine launch");
+    return launch_combine(o, topk_w, s2r, T, topk, H, static_cast<__nv_bfloat16*>(y_bf16), nullptr, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -828,9 +889,6 @@ extern "C" int metis_moe_shared_fused_combine(const void* x_bf16, int64_t T, int
     if ((rc = launch_bf16_gemm(hs, static_cast<const __nv_bfloat16*>(w_sdn_bf16), s, static_cast<int>(T),
                                static_cast<int>(H), static_cast<int>(I_s), nullptr, st)))
         return rc;
-    const int64_t work = T * (H / 8);
-    combine_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(o_routed_bf16), topk_w, slot_to_row, static_cast<int>(T),
-        static_cast<int>(topk), static_cast<int>(H), static_cast<__nv_bfloat16*>(y_bf16), s);
-    return cuda_check(cudaGetLastError(), "shared combine launch");
+    return launch_combine(static_cast<const __nv_bfloat16*>(o_routed_bf16), topk_w, slot_to_row, T, topk, H,
+                          static_cast<__nv_bfloat16*>(y_bf16), s, st);
 }
