@@ -567,9 +567,18 @@ def secondary_figures(metis, dev, pk):
         c[(c & 0x7F) == 0x7F] = 0x38
         return c
 
+    clk_samples = []
+
+    def figure_mhz():
+        """Median SM clock over the timed replays since the previous call."""
+        m = statistics.median(clk_samples) if clk_samples else None
+        clk_samples.clear()
+        return m
+
     def timeit(fn, iters):
         """GPU time per call: `iters` calls captured once in a CUDA graph and
-        replayed, so host-side launch overhead does not enter the figure."""
+        replayed, so host-side launch overhead does not enter the figure.
+        The SM clock is sampled during the timed replays (figure_mhz)."""
         for _ in range(5):
             fn()
         torch.cuda.synchronize()
@@ -585,15 +594,23 @@ def secondary_figures(metis, dev, pk):
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = 3
-        a.record()
-        for _ in range(reps):
-            graph.replay()
-        b.record()
-        torch.cuda.synchronize()
+        with ClockSampler(torch.cuda.current_device(), period=0.002) as clk:
+            a.record()
+            for _ in range(reps):
+                graph.replay()
+            b.record()
+            torch.cuda.synchronize()
+        clk_samples.extend(m for m, _ in getattr(clk, "samples", []))
         del graph
         return a.elapsed_time(b) / (reps * iters) * 1e-3
 
-    out = {}
+    class Figures(dict):
+        """Each figure records the median SM clock of its timed replays."""
+
+        def __setitem__(self, key, value):
+            super().__setitem__(key, dict(value, sm_mhz=figure_mhz()))
+
+    out = Figures()
     hbm = pk["hbm_gbs"]
     peak8 = pk["bf16_tflops"] * FP8_PER_BF16
     # the tiny linear layer (16 tokens, 256 -> 512): launch-latency bound,
@@ -645,66 +662,6 @@ def secondary_figures(metis, dev, pk):
                                  "frac_of_measured_hbm": (3 * M * K + 4 * M) / t / 1e9 / hbm,
                                  "frac_of_nominal_hbm": (3 * M * K + 4 * M) / t / 1e9 / NOMINAL_HBM_GBS}
         del xs, xqs
-    # large-M W8A8 GEMM from BF16 activations (per-token magnitudes
-    # log-uniform in [1e-2, 1e2]): the GEMM alone, the separate quantizer +
-    # GEMM (the product path), and the fused-quantization variant
-    for (M, K) in [(8192, 4096), (16384, 4096), (8192, 8192), (16384, 8192)]:
-        mag = torch.exp(torch.empty(M, 1, device=dev).uniform_(-4.6052, 4.6052, generator=g))
-        x = (torch.randn(M, K, device=dev, generator=g) * mag).to(torch.bfloat16)
-        b = codes(K, K)
-        sa = torch.empty(M, device=dev)
-        sb = torch.rand(K, device=dev, generator=g)
-        xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
-        y = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-        wsf = torch.empty(metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, M, K, K, 0, 0),
-                          dtype=torch.uint8, device=dev)
-        metis.metis_quant_fp8_per_token(x, xq, sa)
-
-        def separate():
-            metis.metis_quant_fp8_per_token(x, xq, sa)
-            metis.metis_fp8_gemm(xq, 0, sa, b, sb, y)
-        fl = 2 * M * K * K
-        t_g = timeit(lambda: metis.metis_fp8_gemm(xq, 0, sa, b, sb, y), 20)
-        t_s = timeit(separate, 20)
-        t_f = timeit(lambda: metis.metis_fp8_gemm(x, 1, sa, b, sb, y, workspace=wsf), 10)
-        out[f"gemm_{M}x{K}x{K}"] = {
-            "us": t_g * 1e6, "TFLOP/s": fl / t_g / 1e12, "frac_of_fp8_peak": fl / t_g / 1e12 / peak8,
-            "frac_of_nominal_fp8": fl / t_g / 1e12 / NOMINAL_FP8_TFLOPS,
-            "quant+gemm_us": t_s * 1e6, "quant+gemm_TFLOP/s": fl / t_s / 1e12,
-            "fused_quant_us": t_f * 1e6, "fused_quant_TFLOP/s": fl / t_f / 1e12}
-        del x, xq, b, y
-    # the default maths for many tokens: the same 4096-token chain through
-    # W8A16 (weights widened exactly to BF16), no quantizers. metis_linear
-    # widens each layer's weights into the workspace and runs the BF16
-    # CTA-pair GEMM; metis_w8a16_gemm widens them inside its kernel.
-    T, K1, N1 = M_TOK, K_HID, N_FF
-    xd = torch.randn(T, K1, device=dev, generator=g).to(torch.bfloat16)
-    w1c, w2c = codes(N1, K1), codes(K1, N1)
-    s1c = torch.rand(N1, device=dev, generator=g) * 1e-3
-    s2c = torch.rand(K1, device=dev, generator=g) * 1e-3
-    h1 = torch.empty(T, N1, dtype=torch.bfloat16, device=dev)
-    h2 = torch.empty(T, K1, dtype=torch.bfloat16, device=dev)
-    wsw = torch.empty(metis.metis_workspace_size(metis.METIS_OP_W8A16_WIDENED, T, N1, K1),
-                      dtype=torch.uint8, device=dev)
-
-    def chain16():
-        metis.metis_linear(xd, w1c, s1c, h1, fast_math=False, workspace=wsw)
-        metis.metis_linear(h1, w2c, s2c, h2, fast_math=False, workspace=wsw)
-
-    def chain16_in_kernel():
-        metis.metis_w8a16_gemm(xd, w1c, s1c, h1)
-        metis.metis_w8a16_gemm(h1, w2c, s2c, h2)
-    t = timeit(chain16, 10)
-    t1 = timeit(lambda: metis.metis_linear(xd, w1c, s1c, h1, fast_math=False, workspace=wsw), 10)
-    t_in = timeit(chain16_in_kernel, 10)
-    fl = 2 * T * K1 * N1
-    peak16 = pk["bf16_tflops"]
-    out["prefill_default_maths_4096tok"] = {
-        "us": t * 1e6, "tok/s": T / t, "TFLOP/s": 2 * fl / t / 1e12,
-        "frac_of_bf16_peak": 2 * fl / t / 1e12 / peak16,
-        "layer1_us": t1 * 1e6, "layer1_TFLOP/s": fl / t1 / 1e12,
-        "in_kernel_widening_us": t_in * 1e6, "in_kernel_widening_TFLOP/s": 2 * fl / t_in / 1e12}
-    del xd, w1c, w2c, h1, h2, wsw
     # routed experts: 4096 tokens, hidden 2048, latent 1024, 64 experts, top-8
     T, H, I, E, k = 4096, 2048, 1024, 64, 8
     x = torch.randn(T, H, device=dev, generator=g).to(torch.bfloat16)
@@ -784,6 +741,66 @@ def secondary_figures(metis, dev, pk):
                                          "frac_of_fp4_peak": tf / peak4, "floor_us": floor,
                                          "frac_of_floor": floor / (t * 1e6)}
     del wu4, wd4, sfu, sfd, ws4
+    # large-M W8A8 GEMM from BF16 activations (per-token magnitudes
+    # log-uniform in [1e-2, 1e2]): the GEMM alone, the separate quantizer +
+    # GEMM (the product path), and the fused-quantization variant
+    for (M, K) in [(8192, 4096), (16384, 4096), (8192, 8192), (16384, 8192)]:
+        mag = torch.exp(torch.empty(M, 1, device=dev).uniform_(-4.6052, 4.6052, generator=g))
+        x = (torch.randn(M, K, device=dev, generator=g) * mag).to(torch.bfloat16)
+        b = codes(K, K)
+        sa = torch.empty(M, device=dev)
+        sb = torch.rand(K, device=dev, generator=g)
+        xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        y = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        wsf = torch.empty(metis.metis_workspace_size(metis.METIS_OP_FP8_GEMM_FUSED, M, K, K, 0, 0),
+                          dtype=torch.uint8, device=dev)
+        metis.metis_quant_fp8_per_token(x, xq, sa)
+
+        def separate():
+            metis.metis_quant_fp8_per_token(x, xq, sa)
+            metis.metis_fp8_gemm(xq, 0, sa, b, sb, y)
+        fl = 2 * M * K * K
+        t_g = timeit(lambda: metis.metis_fp8_gemm(xq, 0, sa, b, sb, y), 20)
+        t_s = timeit(separate, 20)
+        t_f = timeit(lambda: metis.metis_fp8_gemm(x, 1, sa, b, sb, y, workspace=wsf), 10)
+        out[f"gemm_{M}x{K}x{K}"] = {
+            "us": t_g * 1e6, "TFLOP/s": fl / t_g / 1e12, "frac_of_fp8_peak": fl / t_g / 1e12 / peak8,
+            "frac_of_nominal_fp8": fl / t_g / 1e12 / NOMINAL_FP8_TFLOPS,
+            "quant+gemm_us": t_s * 1e6, "quant+gemm_TFLOP/s": fl / t_s / 1e12,
+            "fused_quant_us": t_f * 1e6, "fused_quant_TFLOP/s": fl / t_f / 1e12}
+        del x, xq, b, y
+    # the default maths for many tokens: the same 4096-token chain through
+    # W8A16 (weights widened exactly to BF16), no quantizers. metis_linear
+    # widens each layer's weights into the workspace and runs the BF16
+    # CTA-pair GEMM; metis_w8a16_gemm widens them inside its kernel.
+    T, K1, N1 = M_TOK, K_HID, N_FF
+    xd = torch.randn(T, K1, device=dev, generator=g).to(torch.bfloat16)
+    w1c, w2c = codes(N1, K1), codes(K1, N1)
+    s1c = torch.rand(N1, device=dev, generator=g) * 1e-3
+    s2c = torch.rand(K1, device=dev, generator=g) * 1e-3
+    h1 = torch.empty(T, N1, dtype=torch.bfloat16, device=dev)
+    h2 = torch.empty(T, K1, dtype=torch.bfloat16, device=dev)
+    wsw = torch.empty(metis.metis_workspace_size(metis.METIS_OP_W8A16_WIDENED, T, N1, K1),
+                      dtype=torch.uint8, device=dev)
+
+    def chain16():
+        metis.metis_linear(xd, w1c, s1c, h1, fast_math=False, workspace=wsw)
+        metis.metis_linear(h1, w2c, s2c, h2, fast_math=False, workspace=wsw)
+
+    def chain16_in_kernel():
+        metis.metis_w8a16_gemm(xd, w1c, s1c, h1)
+        metis.metis_w8a16_gemm(h1, w2c, s2c, h2)
+    t = timeit(chain16, 10)
+    t1 = timeit(lambda: metis.metis_linear(xd, w1c, s1c, h1, fast_math=False, workspace=wsw), 10)
+    t_in = timeit(chain16_in_kernel, 10)
+    fl = 2 * T * K1 * N1
+    peak16 = pk["bf16_tflops"]
+    out["prefill_default_maths_4096tok"] = {
+        "us": t * 1e6, "tok/s": T / t, "TFLOP/s": 2 * fl / t / 1e12,
+        "frac_of_bf16_peak": 2 * fl / t / 1e12 / peak16,
+        "layer1_us": t1 * 1e6, "layer1_TFLOP/s": fl / t1 / 1e12,
+        "in_kernel_widening_us": t_in * 1e6, "in_kernel_widening_TFLOP/s": 2 * fl / t_in / 1e12}
+    del xd, w1c, w2c, h1, h2, wsw
     # dense NVFP4 GEMM (codes and tiled scales resident, 2 rotating B > L2 at the large size)
     for (M, K) in [(8192, 4096), (16384, 8192)]:
         qa = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
