@@ -96,6 +96,16 @@ def test_moe_parity(metis, T, H, I, E, k, seed):
     check_moe(d, g)
 
 
+@pytest.mark.parametrize("T,H,I,E,k,seed", [(300, 256, 128, 16, 9, 42), (1024, 1024, 128, 16, 10, 43)])
+def test_moe_parity_more_than_eight_experts_per_token(metis, T, H, I, E, k, seed):
+    """More than 8 experts per token take the combine's general loop (the
+    row indices read inside the sum); with 1024 tokens x 128 column groups
+    every thread of the persistent grid walks several items."""
+    d = synth.moe(seed=seed, T=T, H=H, I=I, E=E, topk=k, hot=2, load_ratio=2.0)
+    g = run_moe(metis, d)
+    check_moe(d, g)
+
+
 @pytest.mark.parametrize("T,E,k,seed", [(64, 320, 4, 40), (4096, 160, 8, 41)])
 def test_moe_routing_without_the_fused_scan(metis, T, E, k, seed):
     """Routing tables too large for the fused prefix-sum and rank kernel (more
