@@ -9,38 +9,46 @@
 // Computed as y^T = W x^T so that the widened weights never pass through
 // shared memory: a 128-channel x 128-token tile per CTA, the channels on the
 // 128 TMEM lanes.
-//   warp 0      TMA producer of the x tiles (BF16, 128 tokens x 64 elements,
-//               128-byte swizzle) into an 8-stage shared-memory ring;
+//   warp 0      TMA producer of the x tiles (BF16, 128 tokens x 128
+//               elements as two 64-element boxes, 128-byte swizzle) into a
+//               4-stage shared-memory ring;
 //   warp 1      allocates all 512 TMEM columns (two 128-column FP32
-//               accumulators, eight 32-column weight stages); one lane issues
+//               accumulators, four 64-column weight stages); one lane issues
 //               tcgen05.mma.kind::f16 with A = the widened weights in TMEM and
-//               B = the x tile in shared memory;
+//               B = the x tile in shared memory, 8 MMAs (K = 16) per stage;
 //   warps 2..9  converters, two per TMEM lane quadrant: each thread streams
-//               32 bytes of its weight row per k-block from global memory
-//               (eight k-blocks ahead in registers), widens E4M3 to BF16
+//               64 bytes of its weight row per stage from global memory
+//               (four stages ahead in registers), widens E4M3 to BF16
 //               exactly (through FP16 and FP32: every E4M3 value is a BF16
-//               value) and writes the 16 packed words into its lane of a TMEM
+//               value) and writes the 32 packed words into its lane of a TMEM
 //               weight stage (tcgen05.st);
 //   warps 10..13 epilogue: tcgen05.ld of 32 channels x 32 tokens, x s_w[n],
 //               BF16 RNE, transposed through a 32x32 shared-memory block and
 //               stored as 64-byte token rows.
+// One thread issues every MMA, and a tcgen05.mma of 128 x 128 x 16 takes
+// about as long to issue as twice its tensor time: each stage therefore
+// carries 8 MMAs, and the MMA thread waits on one barrier per stage (the x
+// tile's bytes and the converters' arrivals complete the same barrier) and
+// commits to one (which both the producer and the converters wait on).
 // Every mbarrier wait is bounded by the device watchdog.
 #include "common.cuh"
 
 namespace metis {
 namespace w16 {
 
-constexpr int BKE = 64;          // K elements per k-block (128 bytes of BF16 x)
+constexpr int BKE = 128;         // K elements per stage (two 128-byte rows of BF16 x per token)
+constexpr int BOXE = 64;         // K elements per x box (128 bytes: the swizzle span)
 constexpr int TILE_N = 128;      // channels per tile (TMEM lanes)
 constexpr int TILE_M = 128;      // tokens per tile (accumulator columns)
-constexpr int STAGES = 8;        // x ring and TMEM weight stages
-constexpr int X_STAGE = TILE_M * BKE * 2;  // 16 KB
+constexpr int STAGES = 4;        // x ring and TMEM weight stages
+constexpr int X_BOX = TILE_M * BOXE * 2;   // 16 KB
+constexpr int X_STAGE = 2 * X_BOX;         // 32 KB
 constexpr int A_COLS = BKE / 2;  // TMEM columns per weight stage (two BF16 per column)
 constexpr int ACC_COLS = TILE_M;
-constexpr int TMEM_COLS = 512;   // 2 x 128 accumulator + 8 x 32 weight columns
+constexpr int TMEM_COLS = 512;   // 2 x 128 accumulator + 4 x 64 weight columns
 constexpr int A_COL0 = 2 * ACC_COLS;
-constexpr int CONV_WARPS = 8;   // two per TMEM lane quadrant, each on half of a k-block
-constexpr int PF = 8;           // k-blocks of weight bytes in flight per converter thread
+constexpr int CONV_WARPS = 8;   // two per TMEM lane quadrant, each on half of a stage
+constexpr int PF = 4;           // stages of weight bytes in flight per converter thread
 constexpr int THREADS = 64 + CONV_WARPS * 32 + 4 * 32;
 constexpr uint32_t IDESC = idesc_bf16_f32(TILE_N, TILE_M);
 
@@ -49,8 +57,8 @@ static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
 // shared memory: x ring | epilogue staging (4 warps x 2 KB) | barriers | misc
 constexpr int STG_OFF = STAGES * X_STAGE;
 constexpr int BAR_OFF = STG_OFF + 4 * 2048;
-// xfull[S], xempty[S], afull[S], aempty[S], tfull[2], tempty[2], drain
-constexpr int NUM_BARS = 4 * STAGES + 5;
+// full[S] (x bytes + converter arrivals), empty[S], tfull[2], tempty[2], drain
+constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
 constexpr size_t SMEM_BYTES = 1024 + MISC_OFF + 16;
 
@@ -112,22 +120,19 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);
-    auto xfull = [&](int s) { return smem_u32(&bars[s]); };
-    auto xempty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
-    auto afull = [&](int s) { return smem_u32(&bars[2 * STAGES + s]); };
-    auto aempty = [&](int s) { return smem_u32(&bars[3 * STAGES + s]); };
-    auto tfull = [&](int b) { return smem_u32(&bars[4 * STAGES + b]); };
-    auto tempty = [&](int b) { return smem_u32(&bars[4 * STAGES + 2 + b]); };
-    const uint32_t drain = smem_u32(&bars[4 * STAGES + 4]);
+    auto full = [&](int s) { return smem_u32(&bars[s]); };
+    auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+    auto tfull = [&](int b) { return smem_u32(&bars[2 * STAGES + b]); };
+    auto tempty = [&](int b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
+    const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(xfull(s), 1);
-            mbar_init(xempty(s), 1);
-            mbar_init(afull(s), CONV_WARPS);
-            mbar_init(aempty(s), 1);
+            // the producer's arrival (with the x bytes) and one per converter warp
+            mbar_init(full(s), 1 + CONV_WARPS);
+            mbar_init(empty(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull(b), 1);
@@ -161,12 +166,14 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
             for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
                 const int m0 = (t % num_m) * TILE_M;
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(xempty(s), ph ^ 1u, p.timeout_ns, p.status)) {
+                    if (!mbar_wait(empty(s), ph ^ 1u, p.timeout_ns, p.status)) {
                         *abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(xfull(s), X_STAGE);
-                    tma_load_2d(smem_u32(ring + s * X_STAGE), &tmX, kb * BKE, m0, xfull(s));
+                    mbar_arrive_expect_tx(full(s), X_STAGE);
+                    const uint32_t dst = smem_u32(ring + s * X_STAGE);
+                    tma_load_2d(dst, &tmX, kb * BKE, m0, full(s));
+                    tma_load_2d(dst + X_BOX, &tmX, kb * BKE + BOXE, m0, full(s));
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
             }
@@ -192,19 +199,22 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
                 bool ok = true;
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(xfull(s), ph, p.timeout_ns, p.status) ||
-                        !mbar_wait(afull(s), ph, p.timeout_ns, p.status)) {
+                    if (!mbar_wait(full(s), ph, p.timeout_ns, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(ring + s * X_STAGE));
+                    const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(ring + s * X_STAGE));
+                    const uint64_t bdesc1 = sw128_kmajor_desc(smem_u32(ring + s * X_STAGE + X_BOX));
                     const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
+                    // K = 16 per MMA: 8 TMEM columns of A, 32 bytes along a box row of B
 #pragma unroll
-                    for (int k = 0; k < BKE / 16; ++k)  // K = 16 per MMA: 8 columns, 32 bytes
-                        mma_f16_tmem_a(d_tmem, a_tmem + 8 * k, bdesc + 2 * k, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(xempty(s));
-                    mma_commit(aempty(s));
+                    for (int k = 0; k < BOXE / 16; ++k)
+                        mma_f16_tmem_a(d_tmem, a_tmem + 8 * k, bdesc0 + 2 * k, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int k = 0; k < BOXE / 16; ++k)
+                        mma_f16_tmem_a(d_tmem, a_tmem + 8 * (k + BOXE / 16), bdesc1 + 2 * k, IDESC, 1u);
+                    mma_commit(empty(s));
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) {
@@ -221,7 +231,7 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
     } else if (warp < 2 + CONV_WARPS) {
         // -------------------------------------------------------- converters
         const int q = warp & 3;
-        const int half = (warp - 2) / 4;   // which 32 elements of the k-block
+        const int half = (warp - 2) / 4;   // which 64 elements of the stage
         const int lane_base = q * 32;
         const bool wide = (p.K % 32) == 0 && (reinterpret_cast<uintptr_t>(p.w) & 31u) == 0;
         int s = 0;
@@ -229,25 +239,29 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
         for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
             const int row = (t / num_m) * TILE_N + lane_base + lane;  // weight row = output channel
             const bool row_ok = row < p.N;
-            const uint8_t* wrow = p.w + static_cast<size_t>(row_ok ? row : 0) * p.K + 32 * half;
-            // a thread's 32 bytes of a k-block are one sector: one 32-byte
-            // load when the rows are 32-byte aligned (K % 32 == 0; two 16-byte
+            const uint8_t* wrow = p.w + static_cast<size_t>(row_ok ? row : 0) * p.K + 64 * half;
+            // a thread's 64 bytes of a stage are two sectors: 32-byte loads
+            // when the rows are 32-byte aligned (K % 32 == 0; two 16-byte
             // loads of the same sector would each move the whole sector
-            // through L1), two 16-byte loads otherwise and at the end of K
-            auto load_kb = [&](int kb, uint4 (&r)[2]) {
-                const int k0 = kb * BKE + 32 * half;
-                if (wide && row_ok && k0 + 32 <= p.K) {
-                    ld_w32(wrow + kb * BKE, r[0], r[1]);
-                    return;
-                }
+            // through L1), 16-byte loads otherwise and at the end of K
+            auto load_kb = [&](int kb, uint4 (&r)[4]) {
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int k = k0 + 16 * j;
-                    r[j] = (row_ok && k < p.K) ? ld_w16(wrow + kb * BKE + 16 * j) : make_uint4(0, 0, 0, 0);
+                for (int h = 0; h < 2; ++h) {
+                    const int k0 = kb * BKE + 64 * half + 32 * h;
+                    if (wide && row_ok && k0 + 32 <= p.K) {
+                        ld_w32(wrow + kb * BKE + 32 * h, r[2 * h], r[2 * h + 1]);
+                        continue;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int k = k0 + 16 * j;
+                        r[2 * h + j] = (row_ok && k < p.K) ? ld_w16(wrow + kb * BKE + 32 * h + 16 * j)
+                                                           : make_uint4(0, 0, 0, 0);
+                    }
                 }
             };
-            // PF k-blocks of weight bytes in flight per thread (L2 latency)
-            uint4 buf[PF][2];
+            // PF stages of weight bytes in flight per thread (L2 latency)
+            uint4 buf[PF][4];
 #pragma unroll
             for (int d = 0; d < PF; ++d) load_kb(d, buf[d]);
             bool ok = true;
@@ -256,27 +270,27 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
                 for (int d = 0; d < PF; ++d) {
                     const int kb = kb0 + d;
                     if (kb >= num_kb || !ok) break;
-                    uint32_t words[16];
+                    uint32_t words[32];
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
+                    for (int j = 0; j < 4; ++j) {
                         const uint32_t v[4] = {buf[d][j].x, buf[d][j].y, buf[d][j].z, buf[d][j].w};
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             e4m3x4_to_bf16x2x2(v[i], words[8 * j + 2 * i], words[8 * j + 2 * i + 1]);
                     }
                     load_kb(kb + PF, buf[d]);  // zeros past the end of K
-                    if (!mbar_wait(aempty(s), ph ^ 1u, p.timeout_ns, p.status)) {
+                    if (!mbar_wait(empty(s), ph ^ 1u, p.timeout_ns, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    tmem_st_32x32b_x16(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
-                                           static_cast<uint32_t>(A_COL0 + s * A_COLS + 16 * half),
+                    tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
+                                           static_cast<uint32_t>(A_COL0 + s * A_COLS + 32 * half),
                                        words);
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(afull(s));
+                    if (lane == 0) mbar_arrive(full(s));
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
             }
@@ -371,7 +385,7 @@ int launch_w8a16_tensor(const __nv_bfloat16* x, const uint8_t* wq, const float* 
     if ((rc = device_status_word(&status))) return rc;
     CUtensorMap tx;
     if ((rc = make_tmap_2d(&tx, x, 2, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                           static_cast<uint64_t>(K) * 2, BKE, TILE_M, true)))
+                           static_cast<uint64_t>(K) * 2, BOXE, TILE_M, true)))
         return rc;
     Params p{wq, s_w, y, M, N, K, status, watchdog_ns()};
     const int tiles = ((M + TILE_M - 1) / TILE_M) * ((N + TILE_N - 1) / TILE_N);
