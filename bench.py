@@ -664,6 +664,9 @@ def secondary_figures(metis, dev, pk):
                                  "frac_of_nominal_hbm": (3 * M * K + 4 * M) / t / 1e9 / NOMINAL_HBM_GBS}
         del xs, xqs
     # routed experts: 4096 tokens, hidden 2048, latent 1024, 64 experts, top-8
+    # (a generator of its own, so the workload does not depend on the figures
+    # timed before it)
+    g.manual_seed(3)
     T, H, I, E, k = 4096, 2048, 1024, 64, 8
     x = torch.randn(T, H, device=dev, generator=g).to(torch.bfloat16)
     logits = torch.randn(T, E, device=dev, generator=g)

@@ -160,7 +160,7 @@ METIS_API int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const floa
  * tensor-core GEMM with s_w applied to the FP32 sum in its epilogue:
  *   y[m, n] = bf16_rn( fl32( s_w[n] * sum_k x[m, k] * D(wq[n, k]) ) ).
  * Faster than metis_w8a16_gemm's in-kernel widening once the token count
- * amortises the pass (metis_linear uses it for M >= 512).
+ * amortises the pass (metis_linear uses it for M >= 2048).
  *   workspace: metis_workspace_size(METIS_OP_W8A16_WIDENED, M, N, K, 0, 0)
  *   bytes, 16-byte aligned; overwritten.
  *   Requires K % 16 == 0, K >= 16, N % 8 == 0, N >= 8, M >= 0; x, wq, y
@@ -325,7 +325,7 @@ METIS_API int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t topk
  * s_tok [M] receives the per-token scales on the fast-math path; `workspace`
  * holds the E4M3 codes: metis_workspace_size(METIS_OP_LINEAR, M, N, K, 0, 0)
  * bytes, 16-byte aligned (0 for M <= 8).
- * Default maths with M >= 512: when `workspace` (16-byte aligned) holds
+ * Default maths with M >= 2048: when `workspace` (16-byte aligned) holds
  * metis_workspace_size(METIS_OP_W8A16_WIDENED, M, N, K, 0, 0) bytes,
  * metis_w8a16_gemm_widened runs; otherwise metis_w8a16_gemm (in-kernel
  * widening). Both compute the same products with FP32 accumulation. */

@@ -389,10 +389,12 @@ extern "C" int64_t metis_moe_workspace_offset(int region, int64_t T, int64_t top
 
 // Fewest tokens for which metis_linear's default maths widens the weights
 // into the workspace. Measured on B200 for N x K = 6144 x 2048, 2048 x 6144
-// and 14336 x 4096: at 256 tokens the in-kernel widening was faster for two
-// of the three (19.8 vs 24.3 us, 59 vs 73 us), at 512 the widened weights won
-// for all three (24.9 vs 32.9 us, 42.0 vs 44.8 us, 96.8 vs 110 us).
-constexpr int64_t kWidenMinTokens = 512;
+// and 14336 x 4096 (in-kernel widening against widening pass + BF16 GEMM):
+// at 1536 tokens the in-kernel kernel was faster for the three together
+// (33.3 + 40.9 + 145.7 against 32.2 + 40.8 + 164.2 us), at 2048 they were
+// even (48.0 + 41.7 + 192.3 against 42.2 + 41.8 + 195.3 us), and at 4096 the
+// widened weights won (6144 x 2048: 78.1 against 91.3 us).
+constexpr int64_t kWidenMinTokens = 2048;
 
 extern "C" int metis_linear(const void* x_bf16, const uint8_t* wq, const float* s_w, void* y_bf16,
                             int64_t M, int64_t N, int64_t K, int fast_math, float* s_tok,

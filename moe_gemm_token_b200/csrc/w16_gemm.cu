@@ -7,15 +7,16 @@
 // the only thing rounded).
 //
 // Computed as y^T = W x^T so that the widened weights never pass through
-// shared memory: a 128-channel x 128-token tile per CTA, the channels on the
-// 128 TMEM lanes.
-//   warp 0      TMA producer of the x tiles (BF16, 128 tokens x 128
-//               elements as two 64-element boxes, 128-byte swizzle) into a
-//               4-stage shared-memory ring;
-//   warp 1      allocates all 512 TMEM columns (two 128-column FP32
-//               accumulators, four 64-column weight stages); one lane issues
-//               tcgen05.mma.kind::f16 with A = the widened weights in TMEM and
-//               B = the x tile in shared memory, 8 MMAs (K = 16) per stage;
+// shared memory: a 128-channel x TM-token tile per CTA (TM = 128 or 256),
+// the channels on the 128 TMEM lanes.
+//   warp 0      TMA producer of the x tiles (BF16, TM tokens x 128 elements
+//               as two 64-element boxes, 128-byte swizzle) into a
+//               shared-memory ring (4 stages for TM = 128, 3 for 256);
+//   warp 1      allocates all 512 TMEM columns (FP32 accumulators: two of
+//               128 columns, or one of 256; 64-column weight stages after
+//               them); one lane issues tcgen05.mma.kind::f16 with A = the
+//               widened weights in TMEM and B = the x tile in shared memory,
+//               8 MMAs (K = 16) per stage;
 //   warps 2..9  converters, two per TMEM lane quadrant: each thread streams
 //               64 bytes of its weight row per stage from global memory
 //               (four stages ahead in registers), widens E4M3 to BF16
@@ -27,9 +28,10 @@
 //               stored as 64-byte token rows.
 // One thread issues every MMA, and a tcgen05.mma of 128 x 128 x 16 takes
 // about as long to issue as twice its tensor time: each stage therefore
-// carries 8 MMAs, and the MMA thread waits on one barrier per stage (the x
+// carries 8 MMAs, the MMA thread waits on one barrier per stage (the x
 // tile's bytes and the converters' arrivals complete the same barrier) and
-// commits to one (which both the producer and the converters wait on).
+// commits to one (which both the producer and the converters wait on), and
+// when there are tiles enough the 256-token tiles halve the MMAs per FLOP.
 // Every mbarrier wait is bounded by the device watchdog.
 #include "common.cuh"
 
@@ -39,28 +41,35 @@ namespace w16 {
 constexpr int BKE = 128;         // K elements per stage (two 128-byte rows of BF16 x per token)
 constexpr int BOXE = 64;         // K elements per x box (128 bytes: the swizzle span)
 constexpr int TILE_N = 128;      // channels per tile (TMEM lanes)
-constexpr int TILE_M = 128;      // tokens per tile (accumulator columns)
-constexpr int STAGES = 4;        // x ring and TMEM weight stages
-constexpr int X_BOX = TILE_M * BOXE * 2;   // 16 KB
-constexpr int X_STAGE = 2 * X_BOX;         // 32 KB
 constexpr int A_COLS = BKE / 2;  // TMEM columns per weight stage (two BF16 per column)
-constexpr int ACC_COLS = TILE_M;
-constexpr int TMEM_COLS = 512;   // 2 x 128 accumulator + 4 x 64 weight columns
-constexpr int A_COL0 = 2 * ACC_COLS;
+constexpr int TMEM_COLS = 512;
 constexpr int CONV_WARPS = 8;   // two per TMEM lane quadrant, each on half of a stage
 constexpr int PF = 4;           // stages of weight bytes in flight per converter thread
 constexpr int THREADS = 64 + CONV_WARPS * 32 + 4 * 32;
-constexpr uint32_t IDESC = idesc_bf16_f32(TILE_N, TILE_M);
 
-static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
-
-// shared memory: x ring | epilogue staging (4 warps x 2 KB) | barriers | misc
-constexpr int STG_OFF = STAGES * X_STAGE;
-constexpr int BAR_OFF = STG_OFF + 4 * 2048;
-// full[S] (x bytes + converter arrivals), empty[S], tfull[2], tempty[2], drain
-constexpr int NUM_BARS = 2 * STAGES + 5;
-constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
-constexpr size_t SMEM_BYTES = 1024 + MISC_OFF + 16;
+// Tiles of TM tokens (accumulator columns). TM = 128: two accumulators (the
+// epilogue drains one while the MMAs fill the other) and 4 weight stages.
+// TM = 256: N = 256 MMAs, half as many per FLOP for the one issuing thread;
+// TMEM then holds one accumulator and 3 weight stages, so the epilogue's
+// drain of a tile is not overlapped with the next tile's MMAs.
+template <int TM>
+struct Cfg {
+    static constexpr int ACCS = TM == 128 ? 2 : 1;
+    static constexpr int STAGES = TM == 128 ? 4 : 3;  // x ring and TMEM weight stages
+    static constexpr int X_BOX = TM * BOXE * 2;       // 16 or 32 KB
+    static constexpr int X_STAGE = 2 * X_BOX;
+    static constexpr int A_COL0 = ACCS * TM;          // weight stages after the accumulators
+    static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_N, TM);
+    // shared memory: x ring | epilogue staging (4 warps x 2 KB) | barriers | misc
+    static constexpr int STG_OFF = STAGES * X_STAGE;
+    static constexpr int BAR_OFF = STG_OFF + 4 * 2048;
+    // full[S] (x bytes + converter arrivals), empty[S], tfull[ACCS], tempty[ACCS], drain
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * ACCS + 1;
+    static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+    static constexpr size_t SMEM_BYTES = 1024 + MISC_OFF + 16;
+    static_assert(TM == 128 || TM == 256, "tile width");
+    static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+};
 
 struct Params {
     const uint8_t* w;     // [N, K] E4M3
@@ -110,21 +119,27 @@ __device__ __forceinline__ void e4m3x4_to_bf16x2x2(uint32_t w, uint32_t& lo, uin
         : "r"(w));
 }
 
+template <int TM>
 __global__ void __launch_bounds__(THREADS, 1)
 w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
+    using C = Cfg<TM>;
+    constexpr int STAGES = C::STAGES;
+    constexpr int X_BOX = C::X_BOX;
+    constexpr int X_STAGE = C::X_STAGE;
+    constexpr int A_COL0 = C::A_COL0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* ring = smem;
-    uint8_t* staging = smem + STG_OFF;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);
+    uint8_t* staging = smem + C::STG_OFF;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
     auto full = [&](int s) { return smem_u32(&bars[s]); };
     auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
     auto tfull = [&](int b) { return smem_u32(&bars[2 * STAGES + b]); };
-    auto tempty = [&](int b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
-    const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
+    auto tempty = [&](int b) { return smem_u32(&bars[2 * STAGES + C::ACCS + b]); };
+    const uint32_t drain = smem_u32(&bars[2 * STAGES + 2 * C::ACCS]);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -134,7 +149,7 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
             mbar_init(full(s), 1 + CONV_WARPS);
             mbar_init(empty(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::ACCS; ++b) {
             mbar_init(tfull(b), 1);
             mbar_init(tempty(b), 4);  // the four epilogue warps
         }
@@ -153,7 +168,7 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
     grid_launch_dependents();
     grid_dependency_wait();  // x may be the previous kernel's output
     const uint32_t tmem_base = *tmem_slot;
-    const int num_m = (p.M + TILE_M - 1) / TILE_M;
+    const int num_m = (p.M + TM - 1) / TM;
     const int total = num_m * ((p.N + TILE_N - 1) / TILE_N);
     const int num_kb = (p.K + BKE - 1) / BKE;
     // tiles: token block fastest, so CTAs running together share weight rows
@@ -164,7 +179,7 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
             int s = 0;
             uint32_t ph = 0;
             for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-                const int m0 = (t % num_m) * TILE_M;
+                const int m0 = (t % num_m) * TM;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(empty(s), ph ^ 1u, p.timeout_ns, p.status)) {
                         *abort_flag = 1;
@@ -196,7 +211,7 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * TM);
                 bool ok = true;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(full(s), ph, p.timeout_ns, p.status)) {
@@ -210,10 +225,10 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
                     // K = 16 per MMA: 8 TMEM columns of A, 32 bytes along a box row of B
 #pragma unroll
                     for (int k = 0; k < BOXE / 16; ++k)
-                        mma_f16_tmem_a(d_tmem, a_tmem + 8 * k, bdesc0 + 2 * k, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+                        mma_f16_tmem_a(d_tmem, a_tmem + 8 * k, bdesc0 + 2 * k, C::IDESC, (kb > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
                     for (int k = 0; k < BOXE / 16; ++k)
-                        mma_f16_tmem_a(d_tmem, a_tmem + 8 * (k + BOXE / 16), bdesc1 + 2 * k, IDESC, 1u);
+                        mma_f16_tmem_a(d_tmem, a_tmem + 8 * (k + BOXE / 16), bdesc1 + 2 * k, C::IDESC, 1u);
                     mma_commit(empty(s));
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
@@ -222,8 +237,7 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
                     break;
                 }
                 mma_commit(tfull(acc));
-                acc ^= 1;
-                if (acc == 0) acc_ph ^= 1u;
+                if (++acc == C::ACCS) { acc = 0; acc_ph ^= 1u; }
             }
             mma_commit(drain);
             mbar_wait(drain, 0, p.timeout_ns, p.status);
@@ -306,7 +320,7 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
         int acc = 0;
         uint32_t acc_ph = 0;
         for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-            const int m0 = (t % num_m) * TILE_M;
+            const int m0 = (t % num_m) * TM;
             const int n_lane = (t / num_m) * TILE_N + q * 32 + lane;  // this thread's channel
             const float sw = n_lane < p.N ? p.s_w[n_lane] : 0.0f;
             if (!mbar_wait(tfull(acc), acc_ph, p.timeout_ns, p.status)) {
@@ -315,13 +329,13 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
             }
             tc_fence_after();
             const uint32_t tbase =
-                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_COLS);
+                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * TM);
             const int nq0 = (t / num_m) * TILE_N + q * 32;  // first channel of this warp
-            for (int c = 0; c < TILE_M / 32; ++c) {
+            for (int c = 0; c < TM / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tbase + c * 32, v);
                 tmem_ld_wait();
-                if (c == TILE_M / 32 - 1) {
+                if (c == TM / 32 - 1) {
                     // the accumulator has been read: release it
                     tc_fence_before();
                     __syncwarp();
@@ -346,8 +360,7 @@ w16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
                         *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(m) * p.N + n) = val;
                 }
             }
-            acc ^= 1;
-            if (acc == 0) acc_ph ^= 1u;
+            if (++acc == C::ACCS) { acc = 0; acc_ph ^= 1u; }
         }
     }
 
@@ -372,25 +385,43 @@ int launch_w8a16_tensor(const __nv_bfloat16* x, const uint8_t* wq, const float* 
     if (rc) return rc;
     static bool attr_done[64];
     if (!attr_done[di.device]) {
-        if (static_cast<size_t>(di.max_smem_optin) < SMEM_BYTES)
+        if (static_cast<size_t>(di.max_smem_optin) < Cfg<256>::SMEM_BYTES)
             return fail(METIS_ERR_UNSUPPORTED, "w8a16 tensor-core GEMM needs %zu bytes of shared memory",
-                        SMEM_BYTES);
-        if ((rc = cuda_check(cudaFuncSetAttribute(w16_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  static_cast<int>(SMEM_BYTES)),
+                        Cfg<256>::SMEM_BYTES);
+        if ((rc = cuda_check(cudaFuncSetAttribute(w16_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(Cfg<128>::SMEM_BYTES)),
+                             "cudaFuncSetAttribute(w16 gemm)")))
+            return rc;
+        if ((rc = cuda_check(cudaFuncSetAttribute(w16_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(Cfg<256>::SMEM_BYTES)),
                              "cudaFuncSetAttribute(w16 gemm)")))
             return rc;
         attr_done[di.device] = true;
     }
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
+    Params p{wq, s_w, y, M, N, K, status, watchdog_ns()};
+    // a wave of 256-token tiles takes about 1.25 times as long as one of
+    // 128-token tiles (17.7 against 14.0 us for 6144 x 2048 weights) for
+    // twice the work (the same MMA count, the epilogue not overlapped): take
+    // them unless their fewer, longer waves are slower on this grid
+    const int64_t nn = (N + TILE_N - 1) / TILE_N;
+    const int64_t t128 = (M + 127) / 128 * nn, t256 = (M + 255) / 256 * nn;
+    const int64_t w128 = (t128 + di.num_sms - 1) / di.num_sms, w256 = (t256 + di.num_sms - 1) / di.num_sms;
+    const bool wide = 125 * w256 < 100 * w128;
+    const int tm = wide ? 256 : 128;
     CUtensorMap tx;
     if ((rc = make_tmap_2d(&tx, x, 2, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                           static_cast<uint64_t>(K) * 2, BOXE, TILE_M, true)))
+                           static_cast<uint64_t>(K) * 2, BOXE, tm, true)))
         return rc;
-    Params p{wq, s_w, y, M, N, K, status, watchdog_ns()};
-    const int tiles = ((M + TILE_M - 1) / TILE_M) * ((N + TILE_N - 1) / TILE_N);
-    const int grid = tiles < di.num_sms ? tiles : di.num_sms;
-    return cuda_check(launch_pdl(w16_gemm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, st, 1, tx, p),
+    const int64_t tiles = wide ? t256 : t128;
+    const int grid = static_cast<int>(tiles < di.num_sms ? tiles : di.num_sms);
+    if (wide)
+        return cuda_check(launch_pdl(w16_gemm_kernel<256>, dim3(grid), dim3(THREADS), Cfg<256>::SMEM_BYTES, st,
+                                     1, tx, p),
+                          "w8a16 tensor-core GEMM launch");
+    return cuda_check(launch_pdl(w16_gemm_kernel<128>, dim3(grid), dim3(THREADS), Cfg<128>::SMEM_BYTES, st, 1,
+                                 tx, p),
                       "w8a16 tensor-core GEMM launch");
 }
 

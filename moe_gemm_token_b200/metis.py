@@ -235,7 +235,7 @@ def metis_moe_workspace_offset(region, T, topk, E, H, I):
 def metis_linear(x, wq, s_w, y, fast_math=True, s_tok=None, workspace=None, stream=None):
     """Dispatch rule: M <= 8 -> W8A16; otherwise W8A8 with fast_math (per-token
     quantizer into `workspace`, then the E4M3 GEMM) and W8A16 without (the
-    widened-weights GEMM when M >= 512 and `workspace` holds the BF16 weights)."""
+    widened-weights GEMM when M >= 2048 and `workspace` holds the BF16 weights)."""
     M, K = x.shape
     N = wq.shape[0]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -237,10 +237,13 @@ def test_w8a16_parity(metis, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(9, 264, 512), (64, 256, 128), (100, 520, 272), (128, 128, 64),
-                                   (200, 1000, 1040), (300, 6144, 2048), (513, 136, 4096)])
+                                   (200, 1000, 1040), (300, 6144, 2048), (513, 136, 4096),
+                                   # enough tiles for 256-token tiles (one wave instead of two)
+                                   (1000, 4104, 1040), (1500, 2056, 256)])
 def test_w8a16_tensor_core_parity(metis, M, N, K):
     """M > 8: the default maths on the tensor cores (weights widened to BF16
-    in tensor memory, x BF16 from shared memory), ragged in M, N and K."""
+    in tensor memory, x BF16 from shared memory), ragged in M, N and K, on
+    128-token tiles and (the last two shapes) 256-token tiles."""
     d = synth.linear(M * 3 + N + 7 * K, M, K, N, outlier_channels=2, outlier_scale=20.0)
     wq, s_w = _prep_weights(metis, d["w"])
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -251,13 +254,14 @@ def test_w8a16_tensor_core_parity(metis, M, N, K):
     assert_close(bf16_host(y), y64, f"w8a16 tensor {M}x{N}x{K}")
 
 
-def test_w8a16_tensor_core_exact_products(metis):
+@pytest.mark.parametrize("M,N,K", [(160, 264, 320), (1200, 2056, 384)])
+def test_w8a16_tensor_core_exact_products(metis, M, N, K):
     """Every weight code an E4M3 subnormal or small normal and x small
     integers: products and partial sums are exact in FP32, so the output
     equals the oracle's BF16 bits. A widening that lost subnormals, or a
-    wrong lane/column layout of the weights in tensor memory, fails here."""
+    wrong lane/column layout of the weights in tensor memory, fails here
+    (the second shape on 256-token tiles)."""
     rng = np.random.default_rng(9)
-    M, N, K = 160, 264, 320
     codes = (rng.integers(1, 8, (N, K)) | (rng.integers(0, 2, (N, K)) << 7)).astype(np.uint8)
     codes[:, ::5] = 0x38  # 1.0
     codes[::3, 1::7] = 0xC0  # -2.0
@@ -373,11 +377,14 @@ def test_w8a16_widened_nan_codes(metis):
     assert_close(got[:, keep], y64, "w8a16 widened, finite channels")
 
 
-@pytest.mark.parametrize("M", [300, 512, 700])
+WIDEN_MIN_TOKENS = 2048  # metis_linear widens the weights into the workspace from here
+
+
+@pytest.mark.parametrize("M", [300, 2047, 2048, 2100])
 def test_linear_default_maths_dispatch(metis, M):
-    """metis_linear without fast-math: M >= 512 with a large enough workspace
-    runs the widened-weights GEMM, otherwise the in-kernel widening; each is
-    bit-identical to its direct call."""
+    """metis_linear without fast-math: M >= 2048 with a large enough
+    workspace runs the widened-weights GEMM, otherwise the in-kernel
+    widening; each is bit-identical to its direct call."""
     N, K = 384, 512
     d = synth.linear(M + 11, M, K, N)
     wq, s_w = _prep_weights(metis, d["w"])
@@ -386,7 +393,7 @@ def test_linear_default_maths_dispatch(metis, M):
     y_lin = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     y_dir = torch.empty_like(y_lin)
     metis.metis_linear(x, wq, s_w, y_lin, fast_math=False, workspace=ws)
-    if M >= 512:
+    if M >= WIDEN_MIN_TOKENS:
         metis.metis_w8a16_gemm_widened(x, wq, s_w, y_dir, _widened_ws(metis, M, N, K))
     else:
         metis.metis_w8a16_gemm(x, wq, s_w, y_dir)
