@@ -432,8 +432,10 @@ def run_metis(args):
     achieved = flops / (iso_ms * 1e-3) / 1e12
     # (b) inside the step, as a cross-check: a separate replay of the step
     # graph with events around both GEMMs of every step. An event inside a
-    # graph is a node of its own and adds a launch gap before the bracketed
-    # GEMM, so these durations err low; they do not enter the timed region.
+    # graph is a node of its own: it ends the programmatic overlap of the
+    # GEMM's launch and set-up with the kernel before it, so each bracketed
+    # interval also holds that launch and set-up and these durations err
+    # high; they do not enter the timed region.
     n_ev = max(10, min(args.steps, 50))
     evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(n_ev)]
     ev_graph = torch.cuda.CUDAGraph()
@@ -465,8 +467,9 @@ def run_metis(args):
                 "in_step": {"achieved": in_step, "frac": in_step / burst, "gemm_samples": len(g1),
                             "layer1_us_median": statistics.median(g1) * 1e3,
                             "layer2_us_median": statistics.median(g2) * 1e3,
-                            "note": "events inside a step graph (not the timed one); each adds a "
-                                    "launch gap before the GEMM, so these figures err low"}}
+                            "note": "events inside a step graph (not the timed one); each event node "
+                                    "ends the GEMM's programmatic launch overlap, so the intervals also "
+                                    "hold its launch and set-up and err high"}}
 
     # ---- end to end through the C ABI with host buffers. Every step uploads
     # its input from pinned host memory, runs the two layers through

@@ -64,11 +64,19 @@ constexpr int CONV_WARPS = 8;                  // fused-quantization converter w
 constexpr int RASTER_M = 16;  // row blocks per raster group of the dense schedule
 constexpr int ASTG_SLOT = ROWS * BK * 2;       // one BF16 A tile (two 64-column boxes)
 
-template <int CTAS, bool ABF16 = false, int BN = BN_MAX, bool W16 = false>
+template <int CTAS, bool ABF16 = false, int BN = BN_MAX, bool W16 = false, bool GROUPED = false>
 struct Layout {
     // BF16 k-blocks take twice the MMA time of E4M3 ones: fewer stages suffice
-    static constexpr int STAGES = W16 ? (CTAS == 2 ? 4 : 3)
-                                      : (CTAS == 2 ? (ABF16 ? 4 : 6) : (ABF16 ? 3 : 4));
+    // Dense CTA-pair tiles take two 128-byte k-blocks per ring stage: one
+    // thread issues every MMA of the pair, at about the pipe's own rate, and
+    // each barrier wait and commit it does between MMAs costs throughput
+    // (8 MMAs per wait instead of 4: 4096 x 6144 x 2048 44.9 -> 42.4 us).
+    // The grouped kernel (short k-loops per tile) measured better with the
+    // finer 6-stage ring.
+    static constexpr int KPS = (CTAS == 2 && !ABF16 && !GROUPED) ? 2 : 1;
+    static constexpr int STAGES = KPS == 2 ? 3
+                                           : (W16 ? (CTAS == 2 ? 4 : 3)
+                                                  : (CTAS == 2 ? (ABF16 ? 4 : 6) : (ABF16 ? 3 : 4)));
     static constexpr int ASTG = ABF16 ? 2 : 0;  // BF16 staging slots
     // epilogue warps: two per TMEM lane quadrant, each on half the columns
     // (one per quadrant in the fused variants, whose shared memory and
@@ -76,8 +84,10 @@ struct Layout {
     static constexpr int EPI = ABF16 ? 4 : 8;
     static constexpr int THREADS_ = THREADS + EPI * 32 + (ABF16 ? CONV_WARPS * 32 : 0);
     static constexpr int B_ROWS = BN / CTAS;   // rows of B loaded by one CTA
-    static constexpr int A_STAGE = ROWS * BK;
-    static constexpr int B_STAGE = B_ROWS * BK;
+    static constexpr int A_BOX = ROWS * BK;
+    static constexpr int B_BOX = B_ROWS * BK;
+    static constexpr int A_STAGE = KPS * A_BOX;
+    static constexpr int B_STAGE = KPS * B_BOX;
     static constexpr int TILES = STAGES * (A_STAGE + B_STAGE) + ASTG * ASTG_SLOT;
     static constexpr int STAGING = EPI * 32 * 64;  // a 32 x 32 BF16 block per epilogue warp
     static constexpr int SW = 2 * BN * 4;                // per-channel scales, double-buffered
@@ -257,11 +267,11 @@ __device__ __forceinline__ void store_chunk_w16(const uint32_t (&v)[32], int c, 
 }
 
 template <int CTAS, bool GROUPED, bool ABF16, int BN, bool W16 = false, bool SCALED = false>
-__global__ void __launch_bounds__(Layout<CTAS, ABF16, BN, W16>::THREADS_, 1)
+__global__ void __launch_bounds__(Layout<CTAS, ABF16, BN, W16, GROUPED>::THREADS_, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmBq, const __grid_constant__ CUtensorMap tmY,
                 const Params p) {
-    using L = Layout<CTAS, ABF16, BN, W16>;
+    using L = Layout<CTAS, ABF16, BN, W16, GROUPED>;
     constexpr int STAGES = L::STAGES;
     constexpr int EPI = L::EPI;
     extern __shared__ uint8_t smem_raw[];
@@ -390,6 +400,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     if constexpr (GROUPED) sc.total = g_tile[p.E];
     const uint32_t tmem_base = *tmem_slot;
     const int num_kb = (p.K + L::KE - 1) / L::KE;
+    const int num_st = (num_kb + L::KPS - 1) / L::KPS;  // ring stages per tile
     const int first = CTAS == 2 ? static_cast<int>(blockIdx.x / 2) : static_cast<int>(blockIdx.x);
     const int stride = CTAS == 2 ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
 
@@ -403,7 +414,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             uint32_t issued = 0, issued_phase = 0;
             for (int t = first; t < sc.total && !*abort_flag; t += stride) {
                 const Tile ti = sc.get(t);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int ks = 0; ks < num_st; ++ks) {
+                    const int kb = ks * L::KPS;  // first k-block of the stage
                     if (!mbar_wait(empty(stage), phase ^ 1u, p.timeout_ns, p.status)) {
                         *abort_flag = 1;
                         break;
@@ -430,13 +442,18 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         if (++slot == L::ASTG) { slot = 0; sphase ^= 1u; }
                     } else if constexpr (CTAS == 2) {
                         // a tail piece loads only its BN/split columns' rows of B
+                        // (a k-block past the end of K is zero-filled and not multiplied)
                         const bool piece = ti.bn != BN;
-                        const uint32_t b_bytes = piece ? static_cast<uint32_t>(ti.bn / CTAS) * BK : L::B_STAGE;
+                        const uint32_t b_bytes = piece ? static_cast<uint32_t>(ti.bn / CTAS) * BK : L::B_BOX;
                         const uint32_t fl = mapa_shared(full(stage), 0);
-                        if (leader) mbar_arrive_expect_tx(full(stage), CTAS * (L::A_STAGE + b_bytes));
-                        tma_load_2d_pair(smem_u32(sA + stage * L::A_STAGE), &tmA, kb * L::KE, ti.a_row0, fl);
-                        tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE), piece ? &tmBq : &tmB, kb * L::KE,
-                                         ti.b_row0, fl);
+                        if (leader) mbar_arrive_expect_tx(full(stage), CTAS * L::KPS * (L::A_BOX + b_bytes));
+#pragma unroll
+                        for (int h = 0; h < L::KPS; ++h) {
+                            tma_load_2d_pair(smem_u32(sA + stage * L::A_STAGE + h * L::A_BOX), &tmA,
+                                             (kb + h) * L::KE, ti.a_row0, fl);
+                            tma_load_2d_pair(smem_u32(sB + stage * L::B_STAGE + h * L::B_BOX),
+                                             piece ? &tmBq : &tmB, (kb + h) * L::KE, ti.b_row0, fl);
+                        }
                     } else {
                         const bool piece = ti.bn != BN;
                         const uint32_t b_bytes = piece ? static_cast<uint32_t>(ti.bn) * BK : L::B_STAGE;
@@ -486,14 +503,18 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     if (bn != BN) idesc = idesc_e4m3_f32(ROWS * CTAS, bn);
                 }
                 bool ok = true;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int ks = 0; ks < num_st; ++ks) {
                     if (!mbar_wait(full(stage), phase, p.timeout_ns, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * L::A_STAGE));
-                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * L::B_STAGE));
+#pragma unroll
+                    for (int h = 0; h < L::KPS; ++h) {
+                    const int kb = ks * L::KPS + h;
+                    if (L::KPS > 1 && kb >= num_kb) break;  // the zero-filled k-block past K
+                    const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * L::A_STAGE + h * L::A_BOX));
+                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * L::B_STAGE + h * L::B_BOX));
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) {
                         // advance 32 bytes along K inside the swizzled 128-byte rows
@@ -507,6 +528,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                             mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
                         else
                             mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+                    }
                     }
                     if constexpr (CTAS == 2) mma_commit_pair_mc(empty(stage), 0x3);
                     else mma_commit(empty(stage));
@@ -707,7 +729,7 @@ template <bool ABF16 = false, int BN = BN_MAX, bool GROUPED = false, bool W16 = 
 int max_pairs(const DeviceInfo& di, int* out) {
     static int cached[64];
     if (!cached[di.device]) {
-        using L = Layout<2, ABF16, BN, W16>;
+        using L = Layout<2, ABF16, BN, W16, GROUPED>;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (di.num_sms / 2), 1, 1);
         cfg.blockDim = dim3(L::THREADS_, 1, 1);
@@ -825,7 +847,7 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     if ((rc = make_tmap_2d_sw64(&ty, y, 2, N, rows, static_cast<uint64_t>(N) * 2, 32, 32))) return rc;
     if (K < 1024) {
         // short k-loops: 128-row single-CTA tiles
-        using L = Layout<1>;
+        using L = Layout<1, false, BN_MAX, false, true>;
         if ((rc = prepare<1, true>(di, L::BYTES_GROUPED))) return rc;
         if ((rc = make_tmap_2d(&tb, b, 1, K, static_cast<uint64_t>(E) * N, K, BK, L::B_ROWS, true)))
             return rc;
@@ -835,7 +857,7 @@ int launch_fp8_gemm_grouped(const uint8_t* a, const float* s_a, const uint8_t* b
     }
     // CTA pairs on 256-row tiles: each SM streams half of B (routed
     // up-projection, K = 2048: 72 -> 66 us)
-    using L = Layout<2>;
+    using L = Layout<2, false, BN_MAX, false, true>;
     if ((rc = prepare<2, true>(di, L::BYTES_GROUPED))) return rc;
     int pairs = 0;
     if ((rc = max_pairs<false, BN_MAX, true>(di, &pairs))) return rc;
