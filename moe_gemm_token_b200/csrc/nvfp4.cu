@@ -492,9 +492,8 @@ constexpr int SFB_STAGE = 2 * KCH * ATOM;   // both 128-row halves of B (every C
 constexpr int STAGING = EPI_WARPS * 32 * 64;    // a 32 x 32 BF16 block per epilogue warp
 constexpr int MAX_GROUPS = 1024;
 constexpr int TMEM_COLS = 512;
-constexpr int SF_COL = BN;      // two scale buffers of 48 columns after the accumulator
+constexpr int SF_COL = BN;      // one scale buffer of 48 columns per ring stage after the accumulator
 constexpr int SF_BUF = 48;      // SFA: 4 chunks x 4 columns; SFB: 4 chunks x 8 columns
-constexpr int SF_BUFS = 4;      // scale buffers in TMEM (the scale warp runs ahead of the MMAs)
 constexpr int SF_ROW = 256;     // the scale buffers seen by TMA as rows of 256 bytes
 
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format
@@ -519,8 +518,10 @@ struct Lay {
     static constexpr int SFA_OFF = B_OFF + STAGES * B_STAGE;
     static constexpr int SFB_OFF = SFA_OFF + STAGES * SFA_STAGE;
     static constexpr int TILES = SFB_OFF + STAGES * SFB_STAGE;
-    // full, empty, tfull, tempty, drain, scale buffers full/empty, scale drain
-    static constexpr int NUM_BARS = 2 * STAGES + 3 + 2 * SF_BUFS + SCALE_WARPS;
+    // landed (TMA bytes), full (scales in TMEM), empty, tfull, tempty, drain,
+    // scale drain
+    static constexpr int NUM_BARS = 3 * STAGES + 3 + SCALE_WARPS;
+    static_assert(SF_COL + STAGES * SF_BUF <= TMEM_COLS, "TMEM: accumulator and one scale buffer per stage");
     static constexpr int BAR_OFF = TILES + STAGING;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int GROUP_OFF = MISC_OFF + 16;
@@ -720,27 +721,31 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int lane = threadIdx.x % 32;
     const uint32_t rank = CTAS == 2 ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
+    // A stage's TMA bytes (codes and scale atoms) complete `landed`, which
+    // the scale-copy warps wait on; their copies into the stage's TMEM scale
+    // buffer complete `full`, the one barrier the MMA thread waits on; the
+    // MMA thread's commit to `empty` frees both the shared-memory stage (for
+    // the producer) and the scale buffer (a stage cannot land again before
+    // its previous MMAs are done, so the scale warps need no wait of their
+    // own for it). One wait and one commit per 4 MMAs: one thread issues
+    // them all, at about the tensor pipe's rate.
     auto full = [&](int s) { return smem_u32(&bars[s]); };
     auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
-    const uint32_t tfull = smem_u32(&bars[2 * STAGES]);
-    const uint32_t tempty = smem_u32(&bars[2 * STAGES + 1]);
-    const uint32_t drain = smem_u32(&bars[2 * STAGES + 2]);
-    auto sf_full = [&](int b) { return smem_u32(&bars[2 * STAGES + 3 + b]); };
-    auto sf_empty = [&](int b) { return smem_u32(&bars[2 * STAGES + 3 + SF_BUFS + b]); };
-    const uint32_t sdrain = smem_u32(&bars[2 * STAGES + 3 + 2 * SF_BUFS]);
+    auto landed = [&](int s) { return smem_u32(&bars[2 * STAGES + s]); };
+    const uint32_t tfull = smem_u32(&bars[3 * STAGES]);
+    const uint32_t tempty = smem_u32(&bars[3 * STAGES + 1]);
+    const uint32_t drain = smem_u32(&bars[3 * STAGES + 2]);
+    const uint32_t sdrain = smem_u32(&bars[3 * STAGES + 3]);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full(s), 1);
+            mbar_init(landed(s), 1);
+            mbar_init(full(s), SCALE_WARPS);
             mbar_init(empty(s), 1);
         }
         mbar_init(tfull, 1);
         mbar_init(tempty, CTAS * EPI_WARPS);
         mbar_init(drain, 1);
-        for (int b = 0; b < SF_BUFS; ++b) {
-            mbar_init(sf_full(b), SCALE_WARPS);
-            mbar_init(sf_empty(b), 1);
-        }
         for (int w = 0; w < SCALE_WARPS; ++w) mbar_init(sdrain + 8 * w, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -849,9 +854,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     if constexpr (CTAS == 2) {
                         // whole boxes (4 atoms each, past the last chunk too:
                         // later atoms or zero fill) so that the byte count is fixed
-                        const uint32_t fl = mapa_shared(full(stage), 0);
+                        const uint32_t fl = mapa_shared(landed(stage), 0);
                         constexpr int RPA = ATOM / SF_ROW;  // 256-byte rows per atom
-                        if (leader) mbar_arrive_expect_tx(full(stage), L::PAIR_TX);
+                        if (leader) mbar_arrive_expect_tx(landed(stage), L::PAIR_TX);
                         tma_load_2d_pair(sa, &tmA, kb * BKB, ti.a_row0, fl);
                         tma_load_2d_pair(sb, &tmB, kb * BKB, ti.b_row0, fl);
                         tma_load_2d_pair(ssa, &tmSFA, 0, static_cast<int32_t>((rb_a * kch_total + c0) * RPA), fl);
@@ -861,12 +866,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     } else {
                         const int nk = min(KCH, kch_total - kb * KCH);
                         const uint32_t sfb = static_cast<uint32_t>(nk * ATOM);
-                        mbar_arrive_expect_tx(full(stage), L::A_STAGE + L::B_STAGE + 3 * sfb);
-                        tma_load_2d(sa, &tmA, kb * BKB, ti.a_row0, full(stage));
-                        tma_load_2d(sb, &tmB, kb * BKB, ti.b_row0, full(stage));
-                        bulk_load(ssa, p.sfa + (rb_a * kch_total + c0) * ATOM, sfb, full(stage));
-                        bulk_load(ssb, p.sfb + (rb_b0 * kch_total + c0) * ATOM, sfb, full(stage));
-                        bulk_load(ssb + KCH * ATOM, p.sfb + (rb_b1 * kch_total + c0) * ATOM, sfb, full(stage));
+                        mbar_arrive_expect_tx(landed(stage), L::A_STAGE + L::B_STAGE + 3 * sfb);
+                        tma_load_2d(sa, &tmA, kb * BKB, ti.a_row0, landed(stage));
+                        tma_load_2d(sb, &tmB, kb * BKB, ti.b_row0, landed(stage));
+                        bulk_load(ssa, p.sfa + (rb_a * kch_total + c0) * ATOM, sfb, landed(stage));
+                        bulk_load(ssb, p.sfb + (rb_b0 * kch_total + c0) * ATOM, sfb, landed(stage));
+                        bulk_load(ssb + KCH * ATOM, p.sfb + (rb_b1 * kch_total + c0) * ATOM, sfb, landed(stage));
                     }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -879,7 +884,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 if (leader) {
                     for (int s = 0; s < STAGES; ++s)
                         if (issued & (1u << s))
-                            mbar_wait(full(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
+                            mbar_wait(landed(s), (issued_phase >> s) & 1u, p.timeout_ns, p.status);
                 } else {
                     const uint64_t t0 = globaltimer_ns();
                     while (globaltimer_ns() - t0 < 100000ull) {}
@@ -892,7 +897,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             int stage = 0;
             uint32_t phase = 0;
             uint32_t acc_phase = 0;
-            uint32_t kglob = 0;
             for (int t = first; t < sc.total && !*abort_flag; t += stride) {
                 if (!mbar_wait(tempty, acc_phase ^ 1u, p.timeout_ns, p.status)) {
                     *abort_flag = 1;
@@ -907,14 +911,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     }
                     tc_fence_after();
                     const int nk = min(KCH, kch_total - kb * KCH);
-                    // this k-block's scales, copied into TMEM by the scale warp
-                    const uint32_t buf = kglob % SF_BUFS;
-                    if (!mbar_wait(sf_full(buf), (kglob / SF_BUFS) & 1u, p.timeout_ns, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sfa_t = tmem_base + SF_COL + SF_BUF * buf;
+                    // this stage's scales, copied into its TMEM buffer by the scale warps
+                    const uint32_t sfa_t = tmem_base + SF_COL + SF_BUF * stage;
                     const uint32_t sfb_t = sfa_t + 16;
                     const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + L::A_OFF + stage * L::A_STAGE));
                     const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + L::B_OFF + stage * L::B_STAGE));
@@ -930,14 +928,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                                          sfb_t + 8 * c, acc);
                         }
                     }
-                    if constexpr (CTAS == 2) {
-                        mma_commit_pair_mc(empty(stage), 0x3);
-                        mma_commit_pair(sf_empty(buf));
-                    } else {
-                        mma_commit(empty(stage));
-                        mma_commit(sf_empty(buf));
-                    }
-                    ++kglob;
+                    if constexpr (CTAS == 2) mma_commit_pair_mc(empty(stage), 0x3);
+                    else mma_commit(empty(stage));
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) {
@@ -956,24 +948,21 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int part = warp - SCALE_WARP;   // chunks [part * KCH / SCALE_WARPS, ...)
         if (lane == 0 && leader) {
             // ------------------------------------------------- scale-factor copies
-            // Each stage's scale atoms go into the next TMEM scale buffer as
-            // soon as the stage has landed and the buffer's previous MMAs are
-            // done, so that the copies overlap the MMA thread's work.
+            // Each stage's scale atoms go into the stage's TMEM scale buffer as
+            // soon as the stage has landed (its previous MMAs are then done),
+            // so that the copies overlap the MMA thread's work.
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t kglob = 0;
             for (int t = first; t < sc.total && !*abort_flag; t += stride) {
                 bool ok = true;
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    const uint32_t buf = kglob % SF_BUFS;
-                    if (!mbar_wait(full(stage), phase, p.timeout_ns, p.status) ||
-                        !mbar_wait(sf_empty(buf), ((kglob / SF_BUFS) & 1u) ^ 1u, p.timeout_ns, p.status)) {
+                    if (!mbar_wait(landed(stage), phase, p.timeout_ns, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int nk = min(KCH, kch_total - kb * KCH);
-                    const uint32_t sfa_t = tmem_base + SF_COL + SF_BUF * buf;
+                    const uint32_t sfa_t = tmem_base + SF_COL + SF_BUF * stage;
                     const uint32_t sfb_t = sfa_t + 16;
                     const uint32_t sa = smem_u32(smem + L::SFA_OFF + stage * SFA_STAGE);
                     const uint32_t sb = smem_u32(smem + L::SFB_OFF + stage * SFB_STAGE);
@@ -991,9 +980,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                             }
                         }
                     }
-                    if constexpr (CTAS == 2) mma_commit_pair(sf_full(buf));
-                    else mma_commit(sf_full(buf));
-                    ++kglob;
+                    if constexpr (CTAS == 2) mma_commit_pair(full(stage));
+                    else mma_commit(full(stage));
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) {
