@@ -511,24 +511,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     tc_fence_after();
 #pragma unroll
                     for (int h = 0; h < L::KPS; ++h) {
-                    const int kb = ks * L::KPS + h;
-                    if (L::KPS > 1 && kb >= num_kb) break;  // the zero-filled k-block past K
-                    const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * L::A_STAGE + h * L::A_BOX));
-                    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * L::B_STAGE + h * L::B_BOX));
+                        const int kb = ks * L::KPS + h;
+                        if (L::KPS > 1 && kb >= num_kb) break;  // the zero-filled k-block past K
+                        const uint64_t adesc =
+                            sw128_kmajor_desc(smem_u32(sA + stage * L::A_STAGE + h * L::A_BOX));
+                        const uint64_t bdesc =
+                            sw128_kmajor_desc(smem_u32(sB + stage * L::B_STAGE + h * L::B_BOX));
 #pragma unroll
-                    for (int k = 0; k < BK / 32; ++k) {
-                        // advance 32 bytes along K inside the swizzled 128-byte rows
-                        // (32 bytes: 32 E4M3 or 16 BF16 elements per instruction)
-                        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                        if constexpr (W16 && CTAS == 2)
-                            mma_f16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
-                        else if constexpr (W16)
-                            mma_f16_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
-                        else if constexpr (CTAS == 2)
-                            mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
-                        else
-                            mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
-                    }
+                        for (int k = 0; k < BK / 32; ++k) {
+                            // advance 32 bytes along K inside the swizzled 128-byte rows
+                            // (32 bytes: 32 E4M3 or 16 BF16 elements per instruction)
+                            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                            if constexpr (W16 && CTAS == 2)
+                                mma_f16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+                            else if constexpr (W16)
+                                mma_f16_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+                            else if constexpr (CTAS == 2)
+                                mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+                            else
+                                mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+                        }
                     }
                     if constexpr (CTAS == 2) mma_commit_pair_mc(empty(stage), 0x3);
                     else mma_commit(empty(stage));
