@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/metis_fp8.h"
 
 namespace metis {
@@ -37,6 +39,21 @@ int device_status_word(uint32_t** out);
 // device addresses of __device__ variables looked up in one context are
 // cached under this id and looked up again when it changes.
 int current_context_id(uint64_t* out);
+// Runs `setup` (a kernel attribute to set, say) the first time it is needed
+// on a device in a CUDA context: slots[device] keeps 1 + the id of the
+// context it last ran in, so a context made after cudaDeviceReset runs it
+// again. Returns setup's status.
+template <typename F>
+int once_per_context(std::atomic<uint64_t>* slots, int device, F&& setup) {
+    uint64_t ctx = 0;
+    int rc = current_context_id(&ctx);
+    if (rc) return rc;
+    std::atomic<uint64_t>& s = slots[device & 63];
+    if (s.load(std::memory_order_acquire) == ctx + 1) return 0;
+    if ((rc = setup())) return rc;
+    s.store(ctx + 1, std::memory_order_release);
+    return 0;
+}
 // Per-wait watchdog limit (ns) for kernels launched now.
 uint64_t watchdog_ns();
 

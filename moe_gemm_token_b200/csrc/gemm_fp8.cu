@@ -712,18 +712,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 
 template <int CTAS, bool GROUPED, bool ABF16 = false, int BN = BN_MAX, bool W16 = false, bool SCALED = false>
 int prepare(const DeviceInfo& di, size_t smem) {
-    static bool done[64];
+    static std::atomic<uint64_t> done[64];
     if (static_cast<size_t>(di.max_smem_optin) < smem)
         return fail(METIS_ERR_UNSUPPORTED, "fp8 gemm needs %zu bytes of shared memory", smem);
-    if (!done[di.device]) {
-        int rc = cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED, ABF16, BN, W16, SCALED>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(smem)),
-                            "cudaFuncSetAttribute(fp8 gemm)");
-        if (rc) return rc;
-        done[di.device] = true;
-    }
-    return METIS_OK;
+    return once_per_context(done, di.device, [&] {
+        return cuda_check(cudaFuncSetAttribute(fp8_gemm_kernel<CTAS, GROUPED, ABF16, BN, W16, SCALED>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem)),
+                          "cudaFuncSetAttribute(fp8 gemm)");
+    });
 }
 
 // Co-resident CTA pairs of the 2-CTA kernel (cached per device).

@@ -548,17 +548,16 @@ int launch_routing(const int32_t* ids, int S, int E, int32_t* chunk_tab, int32_t
     count_kernel<<<C, CHUNK, 0, st>>>(ids, S, E, chunk_tab, status);
     const size_t tab_bytes = static_cast<size_t>(C) * E * 4;
     if (static_cast<int64_t>(C) * E <= RS_MAX_TAB && E <= RS_MAX_E) {
-        static bool attr_done[64];
+        static std::atomic<uint64_t> attr_done[64];
         int dev = 0;
         int rc = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
         if (rc) return rc;
-        if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-            if ((rc = cuda_check(cudaFuncSetAttribute(rank_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      RS_MAX_TAB * 4),
-                                 "cudaFuncSetAttribute(rank_scan)")))
-                return rc;
-            attr_done[dev] = true;
-        }
+        rc = once_per_context(attr_done, dev, [] {
+            return cuda_check(cudaFuncSetAttribute(rank_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   RS_MAX_TAB * 4),
+                              "cudaFuncSetAttribute(rank_scan)");
+        });
+        if (rc) return rc;
         rank_scan_kernel<<<C, CHUNK, tab_bytes, st>>>(ids, S, E, chunk_tab, counts, offsets, pad, s2r, r2s);
     } else {
         scan_kernel<<<1, SCAN_THREADS, 0, st>>>(chunk_tab, C, E, counts, offsets, pad, pad > 1 ? r2s : nullptr);

@@ -1057,19 +1057,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
 template <int CTAS, bool GROUPED>
 int prepare_gemm(const DeviceInfo& di) {
-    static bool done[64];
+    static std::atomic<uint64_t> done[64];
     const size_t smem = Lay<CTAS, GROUPED>::BYTES;
     if (static_cast<size_t>(di.max_smem_optin) < smem)
         return fail(METIS_ERR_UNSUPPORTED, "nvfp4 gemm needs %zu bytes of shared memory", smem);
-    if (!done[di.device]) {
-        int rc = cuda_check(cudaFuncSetAttribute(nvfp4_gemm_kernel<CTAS, GROUPED>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(smem)),
-                            "cudaFuncSetAttribute(nvfp4 gemm)");
-        if (rc) return rc;
-        done[di.device] = true;
-    }
-    return METIS_OK;
+    return once_per_context(done, di.device, [&] {
+        return cuda_check(cudaFuncSetAttribute(nvfp4_gemm_kernel<CTAS, GROUPED>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem)),
+                          "cudaFuncSetAttribute(nvfp4 gemm)");
+    });
 }
 
 // Co-resident CTA pairs of the 2-CTA kernel (cached per device).

@@ -383,21 +383,20 @@ int launch_w8a16_tensor(const __nv_bfloat16* x, const uint8_t* wq, const float* 
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
-    static bool attr_done[64];
-    if (!attr_done[di.device]) {
-        if (static_cast<size_t>(di.max_smem_optin) < Cfg<256>::SMEM_BYTES)
-            return fail(METIS_ERR_UNSUPPORTED, "w8a16 tensor-core GEMM needs %zu bytes of shared memory",
-                        Cfg<256>::SMEM_BYTES);
-        if ((rc = cuda_check(cudaFuncSetAttribute(w16_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  static_cast<int>(Cfg<128>::SMEM_BYTES)),
-                             "cudaFuncSetAttribute(w16 gemm)")))
-            return rc;
-        if ((rc = cuda_check(cudaFuncSetAttribute(w16_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  static_cast<int>(Cfg<256>::SMEM_BYTES)),
-                             "cudaFuncSetAttribute(w16 gemm)")))
-            return rc;
-        attr_done[di.device] = true;
-    }
+    static std::atomic<uint64_t> attr_done[64];
+    if (static_cast<size_t>(di.max_smem_optin) < Cfg<256>::SMEM_BYTES)
+        return fail(METIS_ERR_UNSUPPORTED, "w8a16 tensor-core GEMM needs %zu bytes of shared memory",
+                    Cfg<256>::SMEM_BYTES);
+    rc = once_per_context(attr_done, di.device, [] {
+        if (int r = cuda_check(cudaFuncSetAttribute(w16_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    static_cast<int>(Cfg<128>::SMEM_BYTES)),
+                               "cudaFuncSetAttribute(w16 gemm)"))
+            return r;
+        return cuda_check(cudaFuncSetAttribute(w16_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(Cfg<256>::SMEM_BYTES)),
+                          "cudaFuncSetAttribute(w16 gemm)");
+    });
+    if (rc) return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
     Params p{wq, s_w, y, M, N, K, status, watchdog_ns()};

@@ -668,8 +668,8 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc) return rc;
-    static bool attr_done[64];
-    if (!attr_done[di.device]) {
+    static std::atomic<uint64_t> attr_done[64];
+    rc = once_per_context(attr_done, di.device, [&] {
         const int sm = di.max_smem_optin;
         const cudaError_t es[6] = {
             cudaFuncSetAttribute(w8a16_tma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm),
@@ -679,9 +679,10 @@ extern "C" int metis_w8a16_gemm(const void* x_bf16, const uint8_t* wq, const flo
             cudaFuncSetAttribute(w8a16_tma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm),
             cudaFuncSetAttribute(w8a16_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm)};
         for (cudaError_t e : es)
-            if ((rc = cuda_check(e, "cudaFuncSetAttribute(w8a16)"))) return rc;
-        attr_done[di.device] = true;
-    }
+            if (int r = cuda_check(e, "cudaFuncSetAttribute(w8a16)")) return r;
+        return 0;
+    });
+    if (rc) return rc;
     uint32_t* status = nullptr;
     if ((rc = device_status_word(&status))) return rc;
     Args a;
